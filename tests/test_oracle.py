@@ -1,0 +1,374 @@
+"""Pins for the oracle: checks against the FP16 format definition, the
+hand-worked examples in ``tests/golden``, closed-form error bounds and
+ranges, brute force over the whole level-2 domain, and numpy's own integer
+matmul.  None of these re-types the oracle's formulas.
+
+Passages pinned: "QServe: W4A8KV4 Quantization and System Co-design for
+Efficient LLM Serving" (velog notes), Methods 1) Algorithm: QoQ and
+2) System: QServe; same page, Background (no partial-sum dequantization).
+"""
+import os
+from fractions import Fraction
+
+import numpy as np
+import warnings
+import pytest
+
+import synthetic_inputs as si
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_examples.txt")
+
+
+def _golden(kind):
+    rows = []
+    with open(GOLDEN) as f:
+        for line in f:
+            line = line.strip()
+            if not line.startswith(kind + ":"):
+                continue
+            parts = [p.split() for p in line[len(kind) + 1:].split("|")]
+            rows.append(parts)
+    assert rows, kind
+    return rows
+
+
+# ---------------------------------------------------------------------------
+# FP16 conversions
+# ---------------------------------------------------------------------------
+
+def test_fp16_decode_all_patterns(oracle):
+    bits = np.arange(65536, dtype=np.uint16)
+    got = oracle.h2d_array(bits)
+    ref = bits.view(np.float16).astype(np.float64)
+    nan = np.isnan(ref)
+    assert np.isnan(got[nan]).all()
+    assert np.array_equal(got[~nan], ref[~nan])
+    # signed zeros keep their sign
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+
+
+def test_fp16_roundtrip_all_patterns(oracle):
+    bits = np.arange(65536, dtype=np.uint16)
+    vals = bits.view(np.float16)
+    finite = np.isfinite(vals) | np.isinf(vals)
+    back = oracle.d2h_array(vals.astype(np.float64))
+    assert np.array_equal(back[finite], bits[finite])
+    back32 = oracle.f2h_array(vals.astype(np.float32))
+    assert np.array_equal(back32[finite], bits[finite])
+
+
+def test_fp16_ties_go_to_even(oracle):
+    # every exact midpoint between consecutive finite FP16 values, from
+    # binary64 (numpy converts binary64 -> binary16 directly, RNE)
+    pos = np.arange(0, 0x7bff, dtype=np.uint16)
+    lo = pos.view(np.float16).astype(np.float64)
+    hi = (pos + 1).view(np.float16).astype(np.float64)
+    mid = (lo + hi) / 2.0
+    got = oracle.d2h_array(mid)
+    expect = np.where(pos % 2 == 0, pos, pos + 1).astype(np.uint16)
+    assert np.array_equal(got, expect)
+    # just above / below a midpoint rounds away from / toward lo
+    eps = np.abs(mid) * 2.0 ** -40 + 2.0 ** -60
+    assert np.array_equal(oracle.d2h_array(mid + eps), (pos + 1).astype(np.uint16))
+    assert np.array_equal(oracle.d2h_array(mid - eps), pos)
+    assert np.array_equal(oracle.d2h_array(-mid), expect | 0x8000)
+
+
+def test_fp16_random_floats_match_numpy(oracle):
+    rng = np.random.default_rng(123)
+    x = np.concatenate([
+        rng.standard_normal(400_000).astype(np.float32),
+        (rng.standard_normal(200_000) * 1e-5).astype(np.float32),
+        (rng.standard_normal(200_000) * 3e4).astype(np.float32),
+        rng.uniform(-7e4, 7e4, 100_000).astype(np.float32),
+        np.array([65504, 65519.99, 65520, 65536, 1e-8, 2.98e-8, 2.9802322e-08,
+                  5.96e-8, -0.0, 0.0], np.float32),
+    ])
+    with warnings.catch_warnings():
+        warnings.simplefilter("ignore", RuntimeWarning)   # overflow to inf
+        ref = x.astype(np.float16).view(np.uint16)
+        xd = x.astype(np.float64) * (1 + 2.0 ** -30)
+        refd = xd.astype(np.float16).view(np.uint16)
+    assert np.array_equal(oracle.f2h_array(x), ref)
+    assert np.array_equal(oracle.d2h_array(xd), refd)
+
+
+# ---------------------------------------------------------------------------
+# exact integer round-half-even division
+# ---------------------------------------------------------------------------
+
+def test_rne_div_bruteforce(oracle):
+    for b in range(1, 21):
+        for a in range(-300, 301):
+            assert oracle.rne_div(a, b) == round(Fraction(a, b)), (a, b)
+
+
+# ---------------------------------------------------------------------------
+# Level 2 (per group, UINT4 asymmetric)
+# ---------------------------------------------------------------------------
+
+def test_level2_hand_examples(oracle):
+    for w8, sz, q, dq in _golden("level2"):
+        W8 = np.array([[int(v) for v in w8]], np.int8)
+        qq, s2, z = oracle.quant_w_level2(W8, 4)
+        assert [int(s2[0, 0]), int(z[0, 0])] == [int(v) for v in sz], w8
+        assert qq[0].tolist() == [int(v) for v in q], w8
+        d = oracle.dequant_w(qq, s2, z, 4)
+        assert d[0].tolist() == [int(v) for v in dq], w8
+
+
+def _level2_domain_groups(G=128):
+    """Groups covering every (min, max, w) with -119 <= min <= 0 <= max <= 119
+    and min <= w <= max: each group holds min and max plus a slice of the
+    values in between."""
+    groups = []
+    for mn in range(-119, 1):
+        for mx in range(0, 120):
+            vals = np.arange(mn, mx + 1, dtype=np.int16)
+            for start in range(0, len(vals), G - 2):
+                chunk = vals[start:start + G - 2]
+                g = np.full(G, mn, np.int16)
+                g[1] = mx
+                g[2:2 + len(chunk)] = chunk
+                groups.append(g)
+    return np.stack(groups).astype(np.int8)
+
+
+@pytest.fixture(scope="module")
+def level2_domain(oracle):
+    W8 = _level2_domain_groups()
+    q, s2, z = oracle.quant_w_level2(W8, 128)
+    dq = oracle.dequant_w(q, s2, z, 128)
+    return W8, q, s2[:, 0].astype(np.int32), z[:, 0].astype(np.int32), dq
+
+
+def test_level2_bruteforce_half_step_bound(level2_domain):
+    W8, q, s2, z, dq = level2_domain
+    err2 = 2 * np.abs(W8.astype(np.int32) - dq.astype(np.int32))
+    assert (err2 <= s2[:, None]).all()          # |W8 - dq| <= s2 / 2
+
+
+def test_level2_bruteforce_ranges(level2_domain):
+    W8, q, s2, z, dq = level2_domain
+    assert q.min() >= 0 and q.max() <= 15
+    assert z.min() >= 0 and z.max() <= 15
+    assert s2.min() >= 1 and s2.max() <= 16
+    assert (q.astype(np.int32) * s2[:, None]).max() <= 240   # fits a byte lane
+    assert (z * s2).max() <= 240
+    d = dq.astype(np.int32)
+    # dq stays inside INT8: the protective range 119 gives |dq| <= 121
+    assert d.min() == -121 and d.max() == 121
+
+
+def test_level2_bruteforce_scale_is_minimal(level2_domain):
+    W8, q, s2, z, dq = level2_domain
+    w = W8.astype(np.int32)
+    rng_ = np.maximum(w.max(1), 0) - np.minimum(w.min(1), 0)
+    # 15 steps of s2 cover the range, and 15 steps of s2 - 1 do not
+    assert (15 * s2 >= rng_).all()
+    small = s2 > 1
+    assert (15 * (s2[small] - 1) < rng_[small]).all()
+    # lossless whenever the range fits 15 unit steps
+    lossless = rng_ <= 15
+    assert np.array_equal(dq[lossless], W8[lossless])
+
+
+def test_level2_full_range_reduces_to_grid(oracle):
+    # every group spans exactly [-119, 119]: s2 = 16, z = 7 and the result is
+    # the nearest multiple of 16 (ties to even multiple), clipped to 7 steps
+    rng = np.random.default_rng(5)
+    W8 = rng.integers(-119, 120, size=(64, 128)).astype(np.int8)
+    W8[:, 0] = -119
+    W8[:, 1] = 119
+    q, s2, z = oracle.quant_w_level2(W8, 128)
+    assert (s2 == 16).all() and (z == 7).all()
+    dq = oracle.dequant_w(q, s2, z, 128).astype(np.int32)
+    grid = 16 * np.array([[round(Fraction(int(v), 16)) for v in r] for r in W8])
+    assert np.array_equal(dq, np.clip(grid, -112, 128))
+
+
+# ---------------------------------------------------------------------------
+# Level 1 (per output channel, symmetric INT8 with FP16 scale)
+# ---------------------------------------------------------------------------
+
+def test_level1_hand_examples(oracle):
+    for w, s1h, w8 in _golden("level1"):
+        W = np.array([[float(v) for v in w]], np.float16)
+        assert np.array_equal(W.astype(np.float64)[0], [float(v) for v in w])
+        s1, W8 = oracle.quant_w_level1(W)
+        assert int(s1.view(np.uint16)[0]) == int(s1h[0], 16)
+        assert W8[0].tolist() == [int(v) for v in w8]
+
+
+def test_level1_bounds_and_symmetry(oracle):
+    W = si.weights(si.TINY, seed=3)
+    s1, W8 = oracle.quant_w_level1(W)
+    Wf = W.astype(np.float64)
+    s = s1.astype(np.float64)
+    w8 = W8.astype(np.int32)
+    amax = np.abs(Wf).max(1)
+    # the row maximum lands on the edge of the protective range
+    assert (np.abs(w8).max(1) >= 118).all() and np.abs(w8).max() <= 119
+    # sign preserved
+    assert (np.sign(w8) * np.sign(Wf) >= 0).all()
+    # round-trip error: half a step, plus the slack of rounding s1 to FP16
+    slack = np.maximum(amax - 119 * s, 0)
+    err = np.abs(Wf - w8 * s[:, None])
+    assert (err <= s[:, None] / 2 + slack[:, None] + 1e-12).all()
+    assert (slack <= 0.06 * s).all()
+    # the FP16 scale is within half an FP16 step of amax / 119
+    ulp = np.spacing(s1.astype(np.float16)).astype(np.float64)
+    assert (np.abs(s - amax / 119) <= ulp / 2 + 1e-12).all()
+    # negation symmetry and exact power-of-two scaling
+    s1n, W8n = oracle.quant_w_level1(-W)
+    assert np.array_equal(s1n, s1) and np.array_equal(W8n, -W8)
+    s1d, W8d = oracle.quant_w_level1((W.astype(np.float32) * 4).astype(np.float16))
+    assert np.array_equal(s1d.astype(np.float64), 4 * s) and np.array_equal(W8d, W8)
+
+
+def test_level1_tiny_scale_guard(oracle):
+    W = np.zeros((2, 8), np.float16)
+    W[1, 3] = np.float16(2.0 ** -24)           # smallest subnormal
+    s1, W8 = oracle.quant_w_level1(W)
+    assert s1.view(np.uint16).tolist() == [0x3c00, 0x0001]
+    assert W8[1, 3] == 1 and W8[0].tolist() == [0] * 8
+
+
+# ---------------------------------------------------------------------------
+# Per-token activations
+# ---------------------------------------------------------------------------
+
+def test_act_hand_examples(oracle):
+    for x, sxh, x8 in _golden("act"):
+        X = np.array([[float(v) for v in x]], np.float16)
+        X8, sx = oracle.quant_act(X)
+        assert int(sx.view(np.uint16)[0]) == int(sxh[0], 16)
+        assert X8[0].tolist() == [int(v) for v in x8]
+
+
+def test_act_bounds(oracle):
+    X = si.activations(si.TINY, 16, seed=0)
+    X8, sx = oracle.quant_act(X)
+    Xf = X.astype(np.float64)
+    s = sx.astype(np.float64)
+    x8 = X8.astype(np.int32)
+    amax = np.abs(Xf).max(1)
+    assert (np.abs(x8).max(1) >= 126).all() and np.abs(x8).max() <= 127
+    slack = np.maximum(amax - 127 * s, 0)
+    err = np.abs(Xf - x8 * s[:, None])
+    assert (err <= s[:, None] / 2 + slack[:, None] + 1e-12).all()
+    X8n, sxn = oracle.quant_act(-X)
+    assert np.array_equal(X8n, -X8) and np.array_equal(sxn, sx)
+
+
+# ---------------------------------------------------------------------------
+# Integer GEMM and epilogue
+# ---------------------------------------------------------------------------
+
+def test_int_gemm_matches_numpy_int64(oracle):
+    rng = np.random.default_rng(11)
+    for M, N, K in [(1, 1, 1), (3, 5, 7), (17, 33, 256), (16, 128, 512)]:
+        X8 = rng.integers(-127, 128, size=(M, K), dtype=np.int8)
+        dq = rng.integers(-121, 122, size=(N, K), dtype=np.int8)
+        ref = X8.astype(np.int64) @ dq.astype(np.int64).T
+        assert np.array_equal(oracle.int_gemm(X8, dq), ref)
+        ms = rng.integers(0, M, 50)
+        ns = rng.integers(0, N, 50)
+        assert np.array_equal(oracle.int_gemm_at(X8, dq, ms, ns), ref[ms, ns])
+
+
+def test_int_gemm_bruteforce_tiny(oracle):
+    rng = np.random.default_rng(12)
+    X8 = rng.integers(-127, 128, size=(3, 9), dtype=np.int8)
+    dq = rng.integers(-121, 122, size=(4, 9), dtype=np.int8)
+    acc = oracle.int_gemm(X8, dq)
+    for m in range(3):
+        for n in range(4):
+            s = 0
+            for k in range(9):
+                s += int(X8[m, k]) * int(dq[n, k])
+            assert acc[m, n] == s
+
+
+def test_int_gemm_one_hot_columns(oracle):
+    rng = np.random.default_rng(13)
+    K, N = 256, 64
+    dq = rng.integers(-121, 122, size=(N, K), dtype=np.int8)
+    ks = rng.choice(K, 32, replace=False)
+    X8 = np.zeros((32, K), np.int8)
+    X8[np.arange(32), ks] = 1
+    acc = oracle.int_gemm(X8, dq)
+    assert np.array_equal(acc, dq[:, ks].T.astype(np.int32))
+
+
+def test_int_gemm_extreme_fits_int32(oracle):
+    K = 16384
+    X8 = np.full((1, K), -127, np.int8)
+    dq = np.full((2, K), 121, np.int8)
+    dq[1] = -121
+    acc = oracle.int_gemm(X8, dq)
+    assert acc.tolist() == [[-127 * 121 * K, 127 * 121 * K]]
+
+
+def test_epilogue_matches_numpy(oracle):
+    rng = np.random.default_rng(14)
+    M, N = 7, 33
+    acc = rng.integers(-2 ** 27, 2 ** 27, size=(M, N)).astype(np.int32)
+    sx = (rng.uniform(0.5, 1.5, M) * 1e-2).astype(np.float16)
+    s1 = (rng.uniform(0.5, 1.5, N) * 1e-3).astype(np.float16)
+    Y = oracle.epilogue(acc, sx, s1)
+    ref = (acc.astype(np.float64) * sx.astype(np.float64)[:, None]
+           * s1.astype(np.float64)[None, :]).astype(np.float16)
+    assert np.array_equal(Y.view(np.uint16), ref.view(np.uint16))
+
+
+# ---------------------------------------------------------------------------
+# End to end on the small workload: the quantized product stays within the
+# analytic error bound of the unquantized X @ W^T.
+# ---------------------------------------------------------------------------
+
+def test_end_to_end_error_bound_tiny(oracle):
+    L = si.TINY
+    W = si.weights(L, seed=0)
+    X = si.activations(L, 16, seed=0)
+    Wq = oracle.quantize_weights(W, L.group)
+    X8, sx, acc, Y = oracle.w4a8_forward(X, Wq["dq"], Wq["s1"])
+    Xf = X.astype(np.float64)
+    Wf = W.astype(np.float64)
+    s1 = Wq["s1"].astype(np.float64)
+    s2 = np.repeat(Wq["s2"].astype(np.float64), L.group, axis=1)
+    sxf = sx.astype(np.float64)
+    exact = Xf @ Wf.T
+    amax_w = np.abs(Wf).max(1)
+    amax_x = np.abs(Xf).max(1)
+    dW = s1[:, None] * (0.5 + s2 / 2) + np.maximum(amax_w - 119 * s1, 0)[:, None]
+    dX = sxf[:, None] / 2 + np.maximum(amax_x - 127 * sxf, 0)[:, None]
+    bound = (np.abs(Xf) @ dW.T + dX * np.abs(Wf).sum(1)[None, :]
+             + dX * dW.sum(1)[None, :])
+    bound += np.abs(exact) * 2.0 ** -11 + 2.0 ** -24 * 4
+    Yf = Y.astype(np.float64)
+    assert (np.abs(Yf - exact) <= bound).all()
+    # and the result tracks the exact product: 16 levels per group give a
+    # relative error near step / sqrt(12) of the weights, about 12 % here
+    rel = np.linalg.norm(Yf - exact) / np.linalg.norm(exact)
+    assert rel < 0.2
+    # the scaled INT32 accumulator agrees with Y
+    ref = acc.astype(np.float64) * sxf[:, None] * s1[None, :]
+    assert np.array_equal(Y.view(np.uint16), ref.astype(np.float16).view(np.uint16))
+
+
+def test_planted_mistakes_are_caught(oracle):
+    """A transposed operand or a dropped zero term in dq breaks the pins."""
+    L = si.TINY
+    W = si.weights(L, seed=0)
+    Wq = oracle.quantize_weights(W, L.group)
+    q, s2, z = Wq["q"], Wq["s2"], Wq["z"]
+    # dropping the zero term (dq = q*s2) leaves the half-step bound
+    bad = (q.astype(np.int32) * np.repeat(s2, L.group, 1).astype(np.int32))
+    err2 = 2 * np.abs(Wq["W8"].astype(np.int32) - bad)
+    assert not (err2 <= np.repeat(s2, L.group, 1)).all()
+    # a transposed weight operand breaks the one-hot column identity
+    X8 = np.eye(L.K, dtype=np.int8)[:8]
+    acc = oracle.int_gemm(X8, Wq["dq"])
+    assert np.array_equal(acc, Wq["dq"][:, :8].T.astype(np.int32))
+    assert not np.array_equal(acc, Wq["dq"][:8, :].astype(np.int32)[:, :Wq["dq"].shape[0]])
