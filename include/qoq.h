@@ -1,0 +1,208 @@
+/*
+ * qoq.h -- C ABI of the B200 (sm_100a) W4A8 GEMM library with progressive
+ * group quantization (QoQ).
+ *
+ * The method: "QServe: W4A8KV4 Quantization and System Co-design for
+ * Efficient LLM Serving".  Weights are quantized in two levels (Methods,
+ * 1) Algorithm: QoQ): first per output channel to symmetric INT8 with an
+ * FP16 scale s1, inside a protective range, then per group of G input
+ * channels to asymmetric UINT4 codes q with an INT8 group scale s2 and a UINT4
+ * zero z.  Inside the GEMM the codes are turned back into INT8 with
+ * register-level parallelism as dq = q*s2 - z*s2 (Methods, 2) System: QServe,
+ * "subtraction after multiplication"), the products run on INT8 tensor cores
+ * with INT32 accumulation, and the per-token x per-channel FP16 scaling is
+ * applied once after the whole K reduction, so no partial sum is ever
+ * dequantized (Background: the per-group W4A4 main loop that must dequantize
+ * INT32 partial sums; "Part5 LLM部署技术", 3. 实践扩展：QServe（W4A8KV4）).
+ *
+ * Conventions for every entry point:
+ *  - Pointers named as device pointers must point to device memory of the
+ *    current CUDA device; the caller owns all memory.  The library allocates
+ *    no device memory; the only state it keeps between calls is the
+ *    device error word (qoq_device_error) and host-side caches of device
+ *    attributes and of the driver's tensor-map entry point.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *    compute entry point only enqueues work on `stream` and returns without
+ *    synchronizing, except the ones marked "synchronous".
+ *  - Arguments are validated before anything is launched.  A violated
+ *    precondition returns QOQ_ERR_INVALID_ARG or QOQ_ERR_UNSUPPORTED and
+ *    launches nothing.  A CUDA launch or driver error returns QOQ_ERR_CUDA.
+ *    No exception or abort crosses the ABI.
+ *  - FP16 arrays hold IEEE binary16 values (`__half` / `torch.float16`).
+ *    Inputs must be finite; this is not checked on the device.
+ *  - Every device pointer must be 16-byte aligned.
+ *  - Shapes: N % 128 == 0, K % 128 == 0, group in {64, 128}, K % group == 0,
+ *    1 <= M, K <= 133120 (127 * 127 * K stays below 2^31, so INT32
+ *    accumulation cannot overflow).
+ *  - Requires a compute capability 10.0 device (B200); other devices get
+ *    QOQ_ERR_UNSUPPORTED.
+ */
+#ifndef QOQ_H_
+#define QOQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QOQ_API __attribute__((visibility("default")))
+#else
+#define QOQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  QOQ_OK = 0,
+  QOQ_ERR_INVALID_ARG = 1,  /* bad pointer, shape or alignment */
+  QOQ_ERR_UNSUPPORTED = 2,  /* valid but not supported (device, group, size) */
+  QOQ_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+};
+
+/* Human-readable text for a status code (static storage, never NULL). */
+QOQ_API const char* qoq_status_str(int status);
+
+/* Library ABI version (increments on any signature or layout change). */
+QOQ_API int qoq_version(void);
+
+/* Protective range of level 1 (119) and the UINT4 code range (15), so that
+ * callers can check their own offline quantizers against the library. */
+QOQ_API int qoq_protective_range(void);
+
+/* ------------------------------------------------------------------------
+ * Packed weight format
+ *
+ * The packed buffer is a sequence of blocks, one per (n-tile of 128 output
+ * channels, k-tile of 128 input channels), n-tile major: block (nt, kt) starts
+ * at byte (nt * (K/128) + kt) * qoq_packed_block_bytes(group).  A block holds
+ *   codes : 8192 bytes = [j = 0..3][row = 0..127][16 bytes], the 16 bytes
+ *           covering k = 32j .. 32j+31 of that row as four 32-bit words; word
+ *           w (k0 = 32j + 8w) holds in byte b the codes q[k0+b] (low nibble)
+ *           and q[k0+4+b] (high nibble), so one AND gives four codes in K
+ *           order and one shift + AND the next four;
+ *   s2    : 128 * (128/group) bytes = [g = group within tile][row], INT8;
+ *   z     : 64 * (128/group) bytes  = [g][row/2], UINT4 zero of the even row
+ *           in the low nibble and of the odd row in the high nibble.
+ * This is the library's own answer to the pages' "compute-aware weight
+ * reordering" (Methods, 2) System: QServe): each block is one contiguous
+ * bulk copy, and the order matches the dequantizing threads' reads.
+ * ---------------------------------------------------------------------- */
+
+/* Bytes of one (128 x 128) block: 8192 + 192 for group 128, 8192 + 384 for
+ * group 64.  Returns 0 for an unsupported group. */
+QOQ_API size_t qoq_packed_block_bytes(int group);
+
+/* Bytes of the whole packed buffer for an N x K weight (0 if the shape is
+ * invalid). */
+QOQ_API size_t qoq_packed_weight_bytes(int N, int K, int group);
+
+/* ------------------------------------------------------------------------
+ * Offline: progressive group quantization of a weight matrix.
+ *   W      : device, FP16, N x K row-major (the [out, in] layout of a
+ *            linear layer), read only.
+ *   packed : device, qoq_packed_weight_bytes(N, K, group) bytes, written.
+ *   s1     : device, FP16[N], written: per-output-channel level-1 scale.
+ * Level 1: s1[n] = fp16(max_k |W[n,k]| / 119) (1.0 for an all-zero row, the
+ * smallest positive FP16 if the quotient rounds to 0);
+ * W8 = clamp(rne(W / s1), -119, 119) with an IEEE binary32 division.
+ * Level 2, per group: mn = min(0, min W8), mx = max(0, max W8),
+ * s2 = max(1, ceil((mx - mn) / 15)), z = rne(-mn / s2),
+ * q = clamp(rne(W8 / s2) + z, 0, 15) (exact integer round-half-even).
+ * Source: Methods, 1) Algorithm: QoQ and 2) System: QServe (protective
+ * range).  Asynchronous on `stream`.
+ * ---------------------------------------------------------------------- */
+QOQ_API int qoq_quantize_weights(const void* W, int N, int K, int group,
+                         void* packed, void* s1, void* stream);
+
+/* Pack already-quantized codes into the packed format (no quantization).
+ *   q  : device, uint8 N x K, values 0..15;
+ *   s2 : device, int8 N x (K/group), values 1..16;
+ *   z  : device, uint8 N x (K/group), values 0..15;
+ *   packed : device, written.
+ * The caller guarantees |(q - z) * s2| <= 127 (true for every output of
+ * qoq_quantize_weights); values outside the ranges give unspecified codes.
+ * Asynchronous on `stream`. */
+QOQ_API int qoq_pack_codes(const uint8_t* q, const int8_t* s2, const uint8_t* z,
+                   int N, int K, int group, void* packed, void* stream);
+
+/* Debug / inspection: unpack the packed format.  Any of q, s2, z, dq may be
+ * NULL to skip it.  q: uint8 N x K; s2: int8 N x (K/group);
+ * z: uint8 N x (K/group); dq: int8 N x K with dq = q*s2 - z*s2, computed
+ * with the same byte-lane arithmetic as the GEMM main loop.
+ * Asynchronous on `stream`. */
+QOQ_API int qoq_unpack_weights(const void* packed, int N, int K, int group,
+                       uint8_t* q, int8_t* s2, uint8_t* z, int8_t* dq,
+                       void* stream);
+
+/* ------------------------------------------------------------------------
+ * Online: per-token symmetric INT8 activation quantization.
+ *   X  : device, FP16, M x K row-major, read only.
+ *   X8 : device, int8 M x K row-major, written.
+ *   sx : device, FP16[M], written.
+ * sx[m] = fp16(max_k |X[m,k]| / 127) (1.0 for an all-zero row, the smallest
+ * positive FP16 if the quotient rounds to 0);
+ * X8 = clamp(rne(X / sx), -127, 127) with an IEEE binary32 division.
+ * Source: the 8-bit activations of W4A8 (Insight; abstract of the QServe
+ * page); per-token granularity as in the Background's W4A16 / W8A8
+ * families.  Asynchronous on `stream`.
+ * ---------------------------------------------------------------------- */
+QOQ_API int qoq_quantize_act_per_token(const void* X, int M, int K, int8_t* X8,
+                               void* sx, void* stream);
+
+/* ------------------------------------------------------------------------
+ * The hot path: Y = (X8 . dq^T) * sx[m] * s1[n], FP16 out.
+ *   X8     : device, int8 M x K row-major (from qoq_quantize_act_per_token).
+ *   sx     : device, FP16[M].
+ *   packed : device, packed weights (qoq_quantize_weights / qoq_pack_codes).
+ *   s1     : device, FP16[N].
+ *   Y      : device, FP16 M x N row-major, written (rows >= M untouched).
+ * The UINT4 codes are dequantized to INT8 inside the main loop
+ * (dq = q*s2 - z*s2, four byte lanes per 32-bit operation), multiplied on the
+ * INT8 tensor cores (tcgen05, INT32 accumulators in tensor memory), and the
+ * FP16 scaling runs once in the epilogue: Y = fp16_rn(float(acc) *
+ * (float(sx[m]) * float(s1[n]))).  The tile shape and the number of K splits
+ * are chosen per (M, N, K); split partials are summed exactly in INT32 across
+ * a thread-block cluster before the epilogue.  Sources: Methods, 1) and 2);
+ * Background.  Asynchronous on `stream`.
+ * ---------------------------------------------------------------------- */
+QOQ_API int qoq_w4a8_gemm(const int8_t* X8, const void* sx, const void* packed,
+                  const void* s1, int M, int N, int K, int group, void* Y,
+                  void* stream);
+
+/* Debug: the same main loop, storing the raw INT32 accumulator
+ * acc[m, n] = sum_k X8[m,k] * dq[n,k] (device, int32 M x N row-major). */
+QOQ_API int qoq_w4a8_gemm_i32(const int8_t* X8, const void* packed, int M, int N,
+                      int K, int group, int32_t* acc, void* stream);
+
+/* The same GEMM with an explicit launch configuration (tuning and tests).
+ *   tok_tile : token tile (MMA N): 16, 32, 64, 128 or 256, or 0 for auto;
+ *   splits   : K splits per output tile, 1..8 (at most K/128), or 0 for auto.
+ * Exactly one of Y (FP16 output, needs sx and s1) and acc (INT32 output) is
+ * non-NULL.  Asynchronous on `stream`. */
+QOQ_API int qoq_w4a8_gemm_config(const int8_t* X8, const void* sx, const void* packed,
+                         const void* s1, int M, int N, int K, int group,
+                         void* Y, int32_t* acc, int tok_tile, int splits,
+                         void* stream);
+
+/* The launch configuration qoq_w4a8_gemm picks for a shape: token tile,
+ * K splits, CTAs in the grid and pipeline stages.  Host only, no CUDA call
+ * beyond reading the SM count of the current device (148 if none). */
+QOQ_API int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int* splits,
+                  int* ctas, int* stages);
+
+/* ------------------------------------------------------------------------
+ * Device-side error word.  Every wait inside the kernels is bounded; a wait
+ * that runs out sets a bit in this word and the kernel returns early
+ * instead of hanging.  Synchronous (device-wide): reads the word of the
+ * current device and, if `clear` is non-zero, resets it to 0.
+ * Bits: 1 = producer wait, 2 = MMA wait, 4 = dequantizer wait,
+ *       8 = epilogue wait, 16 = cluster reduction.
+ * ---------------------------------------------------------------------- */
+QOQ_API int qoq_device_error(unsigned int* value, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QOQ_H_ */

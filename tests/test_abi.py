@@ -1,0 +1,124 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the public
+header declares, reports sizes and plans, and rejects bad arguments before
+touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import w4a8_quantized_gemm_02_b200 as qoq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qoq.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from w4a8_quantized_gemm_02_b200 import build
+    build.build()
+    return qoq.lib()
+
+
+def header_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"QOQ_API\s+[\w\s\*]+?\b(qoq_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert header_symbols() == sorted(qoq.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in header_symbols():
+        assert hasattr(L, name), name
+        assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+
+
+def test_sizes(L):
+    assert qoq.packed_block_bytes(128) == 8192 + 192
+    assert qoq.packed_block_bytes(64) == 8192 + 384
+    assert qoq.packed_block_bytes(32) == 0
+    assert qoq.packed_weight_bytes(6144, 4096, 128) == 48 * 32 * (8192 + 192)
+    assert qoq.packed_weight_bytes(512, 512, 64) == 4 * 4 * (8192 + 384)
+    assert qoq.packed_weight_bytes(100, 512, 128) == 0
+    assert qoq.packed_weight_bytes(512, 200, 128) == 0
+    assert L.qoq_protective_range() == 119
+    assert L.qoq_version() >= 1
+    for s in (0, 1, 2, 3, 99):
+        assert qoq.status_str(s)
+
+
+def test_plan_is_host_only(L):
+    for M in (1, 16, 17, 64, 100, 256, 1024, 4096):
+        p = qoq.gemm_plan(M, 6144, 4096, 128)
+        assert p["tok_tile"] in (16, 32, 64, 128, 256)
+        assert p["tok_tile"] >= min(M, 256) or M > 256
+        assert 1 <= p["splits"] <= 8
+        assert p["ctas"] == 48 * -(-M // p["tok_tile"]) * p["splits"]
+    with pytest.raises(qoq.QoQError):
+        qoq.gemm_plan(0, 6144, 4096, 128)
+    with pytest.raises(qoq.QoQError):
+        qoq.gemm_plan(1, 6000, 4096, 128)
+
+
+FAKE = 0x10000          # 16-byte aligned fake device address (never dereferenced)
+P = ctypes.c_void_p
+
+
+def _gemm(L, X8=FAKE, sx=FAKE, packed=FAKE, s1=FAKE, M=16, N=512, K=512, G=128, Y=FAKE):
+    return L.qoq_w4a8_gemm(P(X8), P(sx), P(packed), P(s1), M, N, K, G, P(Y), None)
+
+
+def test_gemm_argument_validation(L):
+    assert _gemm(L, M=0) == qoq.QOQ_ERR_INVALID_ARG
+    assert _gemm(L, M=-3) == qoq.QOQ_ERR_INVALID_ARG
+    assert _gemm(L, N=100) == qoq.QOQ_ERR_INVALID_ARG
+    assert _gemm(L, K=192) == qoq.QOQ_ERR_INVALID_ARG          # K % 128
+    assert _gemm(L, G=32) == qoq.QOQ_ERR_UNSUPPORTED
+    assert _gemm(L, K=133248) == qoq.QOQ_ERR_UNSUPPORTED        # INT32 bound
+    assert _gemm(L, X8=None) == qoq.QOQ_ERR_INVALID_ARG
+    assert _gemm(L, Y=None) == qoq.QOQ_ERR_INVALID_ARG
+    assert _gemm(L, sx=None) == qoq.QOQ_ERR_INVALID_ARG
+    assert _gemm(L, X8=FAKE + 8) == qoq.QOQ_ERR_INVALID_ARG     # alignment
+    assert _gemm(L, Y=FAKE + 2) == qoq.QOQ_ERR_INVALID_ARG
+    cfg = L.qoq_w4a8_gemm_config
+    # both outputs / neither output
+    assert cfg(P(FAKE), P(FAKE), P(FAKE), P(FAKE), 16, 512, 512, 128, P(FAKE), P(FAKE), 0, 0,
+               None) == qoq.QOQ_ERR_INVALID_ARG
+    assert cfg(P(FAKE), P(FAKE), P(FAKE), P(FAKE), 16, 512, 512, 128, None, None, 0, 0,
+               None) == qoq.QOQ_ERR_INVALID_ARG
+    # bad tile / split requests
+    assert cfg(P(FAKE), None, P(FAKE), None, 16, 512, 512, 128, None, P(FAKE), 48, 0,
+               None) == qoq.QOQ_ERR_INVALID_ARG
+    assert cfg(P(FAKE), None, P(FAKE), None, 16, 512, 512, 128, None, P(FAKE), 16, 9,
+               None) == qoq.QOQ_ERR_INVALID_ARG
+    assert cfg(P(FAKE), None, P(FAKE), None, 16, 512, 512, 128, None, P(FAKE), 16, 5,
+               None) == qoq.QOQ_ERR_INVALID_ARG          # more splits than k-tiles
+
+
+def test_other_entry_validation(L):
+    assert L.qoq_quantize_act_per_token(None, 4, 512, P(FAKE), P(FAKE), None) == 1
+    assert L.qoq_quantize_act_per_token(P(FAKE), 0, 512, P(FAKE), P(FAKE), None) == 1
+    assert L.qoq_quantize_act_per_token(P(FAKE), 4, 12, P(FAKE), P(FAKE), None) == 1
+    assert L.qoq_quantize_weights(P(FAKE), 512, 512, 96, P(FAKE), P(FAKE), None) == 2
+    assert L.qoq_quantize_weights(P(FAKE), 500, 512, 128, P(FAKE), P(FAKE), None) == 1
+    assert L.qoq_quantize_weights(P(FAKE), 512, 512, 128, P(FAKE + 4), P(FAKE), None) == 1
+    assert L.qoq_pack_codes(None, P(FAKE), P(FAKE), 512, 512, 128, P(FAKE), None) == 1
+    assert L.qoq_unpack_weights(None, 512, 512, 128, None, None, None, None, None) == 1
+    assert L.qoq_device_error(None, 0) == 1
+
+
+def _has_gpu():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+@pytest.mark.skipif(_has_gpu(), reason="a GPU is present")
+def test_valid_call_without_gpu_reports_cuda_error(L):
+    # with no device the first CUDA call fails; nothing is launched
+    assert _gemm(L) == qoq.QOQ_ERR_CUDA
+    assert L.qoq_quantize_act_per_token(P(FAKE), 4, 512, P(FAKE), P(FAKE), None) == 3

@@ -1,0 +1,307 @@
+"""CUDA path vs the oracle, element by element, on the same seeded inputs.
+
+Bit-exact: INT8 activations and their FP16 scales, FP16 per-channel scales,
+UINT4 codes / INT8 group scales / UINT4 zeros, the dequantized INT8 weights
+and the INT32 accumulators.  FP16 outputs: within 1e-2 * max|Y| (and, as a
+sharper diagnostic, within one FP16 step of the oracle's binary64 epilogue of
+the same accumulator).  All calls go through the C ABI.
+"""
+import numpy as np
+import pytest
+
+import synthetic_inputs as si
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():   # pragma: no cover - CPU container
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+import w4a8_quantized_gemm_02_b200 as qoq  # noqa: E402
+
+DEV = torch.device("cuda:0")
+TOKS = (16, 32, 64, 128, 256)
+
+
+def to_dev(a: np.ndarray):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def host(t) -> np.ndarray:
+    return t.cpu().numpy()
+
+
+def fp16_step(y: np.ndarray) -> np.ndarray:
+    return np.spacing(np.abs(y).astype(np.float16)).astype(np.float64)
+
+
+def check_y(Y_gpu: np.ndarray, Y_ref: np.ndarray):
+    g = Y_gpu.astype(np.float64)
+    r = Y_ref.astype(np.float64)
+    assert np.isfinite(g).all()
+    tol = 1e-2 * np.abs(r).max()
+    assert np.abs(g - r).max() <= tol
+    assert (np.abs(g - r) <= fp16_step(r) + 1e-30).all()
+
+
+@pytest.fixture(scope="module")
+def tiny(oracle):
+    L = si.TINY
+    W = si.weights(L, seed=0)
+    X = si.activations(L, 16, seed=0)
+    ref_w = oracle.quantize_weights(W, L.group)
+    X8, sx, acc, Y = oracle.w4a8_forward(X, ref_w["dq"], ref_w["s1"])
+    return dict(W=W, X=X, w=ref_w, X8=X8, sx=sx, acc=acc, Y=Y)
+
+
+@pytest.fixture(autouse=True)
+def _no_device_errors():
+    qoq.device_error(clear=True)
+    yield
+    torch.cuda.synchronize()
+    assert qoq.device_error(clear=True) == 0
+
+
+# ---------------------------------------------------------------------------
+# activations
+# ---------------------------------------------------------------------------
+
+def _act_cases():
+    rng = np.random.default_rng(7)
+    L = si.TINY
+    yield si.activations(L, 16, seed=0)
+    yield si.activations(L, 1, seed=1)
+    yield si.activations(si.LLAMA3_8B_QKV, 37, seed=2)
+    x = si.random_fp16((5, 384), seed=3)
+    x[1] = 0                                            # all-zero row
+    x[2] = np.float16(2.0 ** -24) * (rng.integers(-1, 2, 384))   # subnormal row
+    x[3, ::7] = np.float16(65504.0)                     # max finite
+    yield x
+    # ties: values that are exactly (k + 0.5) * sx
+    t = np.zeros((2, 128), np.float16)
+    t[:, 0] = np.float16(127 / 32)
+    t[:, 1:] = (np.arange(1, 128) % 9 - 4 + 0.5).astype(np.float16) / np.float16(32)
+    yield t
+
+
+@pytest.mark.parametrize("case", range(5))
+def test_act_quant_bit_exact(oracle, case):
+    X = list(_act_cases())[case]
+    X8_ref, sx_ref = oracle.quant_act(X)
+    X8, sx = qoq.quantize_act_per_token(to_dev(X))
+    torch.cuda.synchronize()
+    assert np.array_equal(host(sx).view(np.uint16), sx_ref.view(np.uint16))
+    assert np.array_equal(host(X8), X8_ref)
+
+
+# ---------------------------------------------------------------------------
+# weights
+# ---------------------------------------------------------------------------
+
+def _check_weights(oracle, W, group):
+    ref = oracle.quantize_weights(W, group)
+    packed, s1 = qoq.quantize_weights(to_dev(W), group)
+    N, K = W.shape
+    q, s2, z, dq = qoq.unpack_weights(packed, N, K, group)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(s1).view(np.uint16), ref["s1"].view(np.uint16))
+    assert np.array_equal(host(s2), ref["s2"])
+    assert np.array_equal(host(z), ref["z"])
+    assert np.array_equal(host(q), ref["q"])
+    assert np.array_equal(host(dq), ref["dq"])
+    return packed, s1, ref
+
+
+@pytest.mark.parametrize("group", (128, 64))
+def test_weight_quant_bit_exact_tiny(oracle, tiny, group):
+    _check_weights(oracle, tiny["W"], group)
+
+
+def test_weight_quant_edge_rows(oracle):
+    W = si.random_fp16((256, 384), seed=9, lo=-2, hi=2)
+    W[0] = 0                                              # zero row -> s1 = 1
+    W[1] = np.float16(2.0 ** -24)                         # subnormal row
+    W[2, :128] = 0                                        # zero group
+    W[3] = np.abs(W[3])                                   # one-signed rows
+    W[4] = -np.abs(W[4])
+    W[5, ::3] = np.float16(65504.0)
+    W[6] = np.float16(0.5)                                # constant row
+    for g in (128, 64):
+        _check_weights(oracle, W, g)
+
+
+def test_weight_quant_bit_exact_llama_qkv(oracle):
+    W = si.weights(si.LLAMA3_8B_QKV, seed=0)
+    _check_weights(oracle, W, 128)
+
+
+def test_pack_codes_roundtrip():
+    for group in (128, 64):
+        ops = si.sweep_operands(1, 384, 512, group, seed=4)
+        packed = qoq.pack_codes(to_dev(ops.q), to_dev(ops.s2), to_dev(ops.z), group)
+        q, s2, z, dq = qoq.unpack_weights(packed, 384, 512, group)
+        torch.cuda.synchronize()
+        assert np.array_equal(host(q), ops.q)
+        assert np.array_equal(host(s2), ops.s2)
+        assert np.array_equal(host(z), ops.z)
+        ref = (ops.q.astype(np.int32) - np.repeat(ops.z, group, 1).astype(np.int32)) * \
+            np.repeat(ops.s2, group, 1).astype(np.int32)
+        assert np.array_equal(host(dq).astype(np.int32), ref)
+
+
+def test_packed_layout_matches_documented_format(oracle, tiny):
+    """Decode the packed bytes in Python from the format described in the
+    public header (independently of the library's unpacker)."""
+    W = tiny["W"]
+    N, K = W.shape
+    group = 128
+    packed, _ = qoq.quantize_weights(to_dev(W), group)
+    buf = host(packed)
+    blk = qoq.packed_block_bytes(group)
+    ref = tiny["w"]
+    gpt = 128 // group
+    for nt in range(N // 128):
+        for kt in range(K // 128):
+            b = buf[(nt * (K // 128) + kt) * blk:][:blk]
+            codes = b[:8192].reshape(4, 128, 16)
+            for r in range(0, 128, 37):
+                n = nt * 128 + r
+                for j in range(4):
+                    for w in range(4):
+                        word = codes[j, r, 4 * w:4 * w + 4]
+                        k0 = kt * 128 + 32 * j + 8 * w
+                        assert list(word & 15) == list(ref["q"][n, k0:k0 + 4])
+                        assert list(word >> 4) == list(ref["q"][n, k0 + 4:k0 + 8])
+                for gl in range(gpt):
+                    g = kt * gpt + gl
+                    assert np.int8(b[8192 + gl * 128 + r].view(np.int8)) == ref["s2"][n, g]
+                    zb = b[8192 + gpt * 128 + gl * 64 + r // 2]
+                    assert ((zb >> 4) if r & 1 else (zb & 15)) == ref["z"][n, g]
+
+
+# ---------------------------------------------------------------------------
+# GEMM: tiny workload, every token tile, several K splits, ragged M
+# ---------------------------------------------------------------------------
+
+@pytest.fixture(scope="module")
+def tiny_dev(tiny):
+    packed, s1 = qoq.quantize_weights(to_dev(tiny["W"]), 128)
+    return packed, s1
+
+
+@pytest.mark.parametrize("tok", TOKS)
+@pytest.mark.parametrize("splits", (1, 2, 3, 4))
+def test_gemm_i32_bit_exact_tiny(tiny, tiny_dev, tok, splits):
+    packed, s1 = tiny_dev
+    X8 = to_dev(tiny["X8"])
+    acc = qoq.w4a8_gemm_config(X8, None, packed, None, 512, 128, tok_tile=tok, splits=splits,
+                               int32_out=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(acc), tiny["acc"])
+
+
+@pytest.mark.parametrize("tok", TOKS)
+def test_gemm_fp16_tiny(tiny, tiny_dev, tok):
+    packed, s1 = tiny_dev
+    X8, sx = to_dev(tiny["X8"]), to_dev(tiny["sx"])
+    for splits in (1, 4):
+        Y = qoq.w4a8_gemm_config(X8, sx, packed, s1, 512, 128, tok_tile=tok, splits=splits)
+        torch.cuda.synchronize()
+        check_y(host(Y), tiny["Y"])
+
+
+def test_gemm_auto_plan_tiny_end_to_end(tiny, tiny_dev):
+    packed, s1 = tiny_dev
+    X8, sx = qoq.quantize_act_per_token(to_dev(tiny["X"]))
+    Y = qoq.w4a8_gemm(X8, sx, packed, s1, 512, 128)
+    acc = qoq.w4a8_gemm_i32(X8, packed, 512, 128)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(acc), tiny["acc"])
+    check_y(host(Y), tiny["Y"])
+
+
+@pytest.mark.parametrize("M", (1, 2, 3, 15, 17, 33, 63, 65, 100, 129, 255, 257, 300, 513))
+def test_gemm_ragged_m(oracle, M):
+    L = si.TINY
+    W = si.weights(L, seed=1)
+    X = si.activations(L, M, seed=M)
+    ref = oracle.quantize_weights(W, 128)
+    X8r, sxr, accr, Yr = oracle.w4a8_forward(X, ref["dq"], ref["s1"])
+    packed, s1 = qoq.quantize_weights(to_dev(W), 128)
+    X8, sx = qoq.quantize_act_per_token(to_dev(X))
+    Y = qoq.w4a8_gemm(X8, sx, packed, s1, 512, 128)
+    acc = qoq.w4a8_gemm_i32(X8, packed, 512, 128)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(acc), accr)
+    check_y(host(Y), Yr)
+
+
+@pytest.mark.parametrize("group", (64, 128))
+@pytest.mark.parametrize("M,N,K", [(16, 128, 128), (5, 256, 256), (40, 384, 1152),
+                                   (200, 256, 2048)])
+def test_gemm_shapes_random_codes(oracle, group, M, N, K):
+    ops = si.sweep_operands(M, N, K, group, seed=M + N + K)
+    dq_ref = oracle.dequant_w(ops.q, ops.s2, ops.z, group)
+    acc_ref = oracle.int_gemm(ops.X8, dq_ref)
+    Y_ref = oracle.epilogue(acc_ref, ops.sx, ops.s1)
+    packed = qoq.pack_codes(to_dev(ops.q), to_dev(ops.s2), to_dev(ops.z), group)
+    X8 = to_dev(ops.X8)
+    kt = K // 128
+    for tok in (16, 64, 256):
+        for splits in sorted({1, min(2, kt), min(kt, 8)}):
+            acc = qoq.w4a8_gemm_config(X8, None, packed, None, N, group, tok_tile=tok,
+                                       splits=splits, int32_out=True)
+            torch.cuda.synchronize()
+            assert np.array_equal(host(acc), acc_ref), (tok, splits)
+    Y = qoq.w4a8_gemm(X8, to_dev(ops.sx), packed, to_dev(ops.s1), N, group)
+    torch.cuda.synchronize()
+    check_y(host(Y), Y_ref)
+
+
+def test_gemm_extreme_values(oracle):
+    """Largest |dq| and |X8|: accumulators near the INT32 edge stay exact."""
+    N, K, group = 128, 8192, 128
+    q = np.zeros((N, K), np.uint8)
+    q[::2] = 15
+    z = np.zeros((N, K // group), np.uint8)
+    z[1::2] = 15
+    s2 = np.full((N, K // group), 8, np.int8)             # dq = +-120
+    X8 = np.full((3, K), 127, np.int8)
+    X8[1] = -127
+    X8[2, ::2] = -127
+    dq_ref = oracle.dequant_w(q, s2, z, group)
+    acc_ref = oracle.int_gemm(X8, dq_ref)
+    packed = qoq.pack_codes(to_dev(q), to_dev(s2), to_dev(z), group)
+    for tok, splits in ((16, 1), (16, 8), (256, 2)):
+        acc = qoq.w4a8_gemm_config(to_dev(X8), None, packed, None, N, group, tok_tile=tok,
+                                   splits=splits, int32_out=True)
+        torch.cuda.synchronize()
+        assert np.array_equal(host(acc), acc_ref)
+
+
+def test_gemm_one_hot_columns(oracle, tiny, tiny_dev):
+    """One-hot activation rows return single columns of dq: catches any
+    mistake in the shared-memory swizzle or the operand order."""
+    packed, _ = tiny_dev
+    K = 512
+    ks = np.arange(0, K, 5)[:48]
+    X8 = np.zeros((len(ks), K), np.int8)
+    X8[np.arange(len(ks)), ks] = 1
+    acc = qoq.w4a8_gemm_config(to_dev(X8), None, packed, None, 512, 128, tok_tile=64,
+                               splits=1, int32_out=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(acc), tiny["w"]["dq"][:, ks].T.astype(np.int32))
+
+
+def test_gemm_stream_and_repeat(tiny, tiny_dev):
+    """Back-to-back launches on a side stream give identical results."""
+    packed, s1 = tiny_dev
+    X8, sx = to_dev(tiny["X8"]), to_dev(tiny["sx"])
+    s = torch.cuda.Stream()
+    outs = []
+    with torch.cuda.stream(s):
+        for _ in range(5):
+            outs.append(qoq.w4a8_gemm(X8, sx, packed, s1, 512, 128, stream=s))
+    s.synchronize()
+    for Y in outs:
+        check_y(host(Y), tiny["Y"])

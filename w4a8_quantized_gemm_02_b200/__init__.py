@@ -1,0 +1,267 @@
+"""Python binding of ``libqoq.so``: the B200 (sm_100a) W4A8 GEMM with
+progressive group quantization (QoQ, "QServe: W4A8KV4 Quantization and System
+Co-design for Efficient LLM Serving", Methods 1) Algorithm: QoQ and
+2) System: QServe).
+
+This module only marshals arguments (torch tensors -> device pointers, the
+current CUDA stream) into the C ABI declared in ``include/qoq.h``; every step
+of the computation runs in the library's CUDA kernels.  There is no CPU
+fallback: if the library is not built, or a call fails, an exception is
+raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqoq.so")
+
+QOQ_OK = 0
+QOQ_ERR_INVALID_ARG = 1
+QOQ_ERR_UNSUPPORTED = 2
+QOQ_ERR_CUDA = 3
+
+# Every symbol the public header declares.
+EXPORTS = (
+    "qoq_status_str", "qoq_version", "qoq_protective_range",
+    "qoq_packed_block_bytes", "qoq_packed_weight_bytes",
+    "qoq_quantize_weights", "qoq_pack_codes", "qoq_unpack_weights",
+    "qoq_quantize_act_per_token", "qoq_w4a8_gemm", "qoq_w4a8_gemm_i32",
+    "qoq_w4a8_gemm_config", "qoq_gemm_plan", "qoq_device_error",
+)
+
+_lock = threading.Lock()
+_lib = None
+
+
+class QoQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_str(status)} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``libqoq.so`` (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with "
+                    "`python -m w4a8_quantized_gemm_02_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            P, I = ctypes.c_void_p, ctypes.c_int
+            sz = ctypes.c_size_t
+            L.qoq_status_str.restype = ctypes.c_char_p
+            L.qoq_status_str.argtypes = [I]
+            L.qoq_version.restype = I
+            L.qoq_version.argtypes = []
+            L.qoq_protective_range.restype = I
+            L.qoq_protective_range.argtypes = []
+            L.qoq_packed_block_bytes.restype = sz
+            L.qoq_packed_block_bytes.argtypes = [I]
+            L.qoq_packed_weight_bytes.restype = sz
+            L.qoq_packed_weight_bytes.argtypes = [I, I, I]
+            L.qoq_quantize_weights.restype = I
+            L.qoq_quantize_weights.argtypes = [P, I, I, I, P, P, P]
+            L.qoq_pack_codes.restype = I
+            L.qoq_pack_codes.argtypes = [P, P, P, I, I, I, P, P]
+            L.qoq_unpack_weights.restype = I
+            L.qoq_unpack_weights.argtypes = [P, I, I, I, P, P, P, P, P]
+            L.qoq_quantize_act_per_token.restype = I
+            L.qoq_quantize_act_per_token.argtypes = [P, I, I, P, P, P]
+            L.qoq_w4a8_gemm.restype = I
+            L.qoq_w4a8_gemm.argtypes = [P, P, P, P, I, I, I, I, P, P]
+            L.qoq_w4a8_gemm_i32.restype = I
+            L.qoq_w4a8_gemm_i32.argtypes = [P, P, I, I, I, I, P, P]
+            L.qoq_w4a8_gemm_config.restype = I
+            L.qoq_w4a8_gemm_config.argtypes = [P, P, P, P, I, I, I, I, P, P, I, I, P]
+            L.qoq_gemm_plan.restype = I
+            L.qoq_gemm_plan.argtypes = [I, I, I, I] + [ctypes.POINTER(I)] * 4
+            L.qoq_device_error.restype = I
+            L.qoq_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), I]
+            _lib = L
+    return _lib
+
+
+def status_str(status: int) -> str:
+    return lib().qoq_status_str(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != QOQ_OK:
+        raise QoQError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need_cuda(t, name, dtype=None, ndim=None):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims")
+
+
+# ---------------------------------------------------------------------------
+# sizes / plan
+# ---------------------------------------------------------------------------
+
+def packed_block_bytes(group: int = 128) -> int:
+    return int(lib().qoq_packed_block_bytes(group))
+
+
+def packed_weight_bytes(N: int, K: int, group: int = 128) -> int:
+    return int(lib().qoq_packed_weight_bytes(N, K, group))
+
+
+def gemm_plan(M: int, N: int, K: int, group: int = 128) -> dict:
+    vals = [ctypes.c_int() for _ in range(4)]
+    _check(lib().qoq_gemm_plan(M, N, K, group, *[ctypes.byref(v) for v in vals]),
+           "qoq_gemm_plan")
+    return dict(zip(("tok_tile", "splits", "ctas", "stages"), (v.value for v in vals)))
+
+
+def device_error(clear: bool = True) -> int:
+    v = ctypes.c_uint()
+    _check(lib().qoq_device_error(ctypes.byref(v), int(clear)), "qoq_device_error")
+    return int(v.value)
+
+
+# ---------------------------------------------------------------------------
+# offline weight quantization
+# ---------------------------------------------------------------------------
+
+def quantize_weights(W, group: int = 128, stream=None):
+    """W: (N, K) float16 CUDA tensor -> (packed uint8 tensor, s1 float16[N])."""
+    import torch
+    _need_cuda(W, "W", torch.float16, 2)
+    N, K = W.shape
+    nbytes = packed_weight_bytes(N, K, group)
+    if nbytes == 0:
+        raise QoQError(QOQ_ERR_INVALID_ARG, "qoq_packed_weight_bytes")
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    s1 = torch.empty(N, dtype=torch.float16, device=W.device)
+    _check(lib().qoq_quantize_weights(_ptr(W), N, K, group, _ptr(packed), _ptr(s1),
+                                      _stream(stream)), "qoq_quantize_weights")
+    return packed, s1
+
+
+def pack_codes(q, s2, z, group: int = 128, stream=None):
+    """Canonical codes (uint8 N x K, int8 N x K/G, uint8 N x K/G) -> packed."""
+    import torch
+    _need_cuda(q, "q", torch.uint8, 2)
+    _need_cuda(s2, "s2", torch.int8, 2)
+    _need_cuda(z, "z", torch.uint8, 2)
+    N, K = q.shape
+    nbytes = packed_weight_bytes(N, K, group)
+    if nbytes == 0:
+        raise QoQError(QOQ_ERR_INVALID_ARG, "qoq_packed_weight_bytes")
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    _check(lib().qoq_pack_codes(_ptr(q), _ptr(s2), _ptr(z), N, K, group, _ptr(packed),
+                                _stream(stream)), "qoq_pack_codes")
+    return packed
+
+
+def unpack_weights(packed, N: int, K: int, group: int = 128, stream=None):
+    """packed -> (q uint8 N x K, s2 int8, z uint8, dq int8 N x K)."""
+    import torch
+    _need_cuda(packed, "packed", torch.uint8)
+    dev = packed.device
+    q = torch.empty((N, K), dtype=torch.uint8, device=dev)
+    s2 = torch.empty((N, K // group), dtype=torch.int8, device=dev)
+    z = torch.empty((N, K // group), dtype=torch.uint8, device=dev)
+    dq = torch.empty((N, K), dtype=torch.int8, device=dev)
+    _check(lib().qoq_unpack_weights(_ptr(packed), N, K, group, _ptr(q), _ptr(s2), _ptr(z),
+                                    _ptr(dq), _stream(stream)), "qoq_unpack_weights")
+    return q, s2, z, dq
+
+
+# ---------------------------------------------------------------------------
+# online path
+# ---------------------------------------------------------------------------
+
+def quantize_act_per_token(X, out=None, stream=None):
+    """X: (M, K) float16 -> (X8 int8 (M, K), sx float16 (M,))."""
+    import torch
+    _need_cuda(X, "X", torch.float16, 2)
+    M, K = X.shape
+    if out is None:
+        X8 = torch.empty((M, K), dtype=torch.int8, device=X.device)
+        sx = torch.empty(M, dtype=torch.float16, device=X.device)
+    else:
+        X8, sx = out
+    _check(lib().qoq_quantize_act_per_token(_ptr(X), M, K, _ptr(X8), _ptr(sx),
+                                            _stream(stream)), "qoq_quantize_act_per_token")
+    return X8, sx
+
+
+def w4a8_gemm(X8, sx, packed, s1, N: int, group: int = 128, out=None, stream=None):
+    """Y = (X8 . dq^T) * sx[m] * s1[n] as float16 (M, N)."""
+    import torch
+    _need_cuda(X8, "X8", torch.int8, 2)
+    M, K = X8.shape
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=X8.device)
+    _check(lib().qoq_w4a8_gemm(_ptr(X8), _ptr(sx), _ptr(packed), _ptr(s1), M, N, K, group,
+                               _ptr(Y), _stream(stream)), "qoq_w4a8_gemm")
+    return Y
+
+
+def w4a8_gemm_i32(X8, packed, N: int, group: int = 128, out=None, stream=None):
+    """Raw INT32 accumulator acc = X8 . dq^T (M, N)."""
+    import torch
+    _need_cuda(X8, "X8", torch.int8, 2)
+    M, K = X8.shape
+    acc = out if out is not None else torch.empty((M, N), dtype=torch.int32, device=X8.device)
+    _check(lib().qoq_w4a8_gemm_i32(_ptr(X8), _ptr(packed), M, N, K, group, _ptr(acc),
+                                   _stream(stream)), "qoq_w4a8_gemm_i32")
+    return acc
+
+
+def w4a8_gemm_config(X8, sx, packed, s1, N: int, group: int = 128, *, tok_tile=0, splits=0,
+                     int32_out=False, out=None, stream=None):
+    """The GEMM with an explicit token tile / split count (0 = auto)."""
+    import torch
+    _need_cuda(X8, "X8", torch.int8, 2)
+    M, K = X8.shape
+    if int32_out:
+        acc = out if out is not None else torch.empty((M, N), dtype=torch.int32, device=X8.device)
+        Y = None
+    else:
+        Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=X8.device)
+        acc = None
+    _check(lib().qoq_w4a8_gemm_config(_ptr(X8), _ptr(sx), _ptr(packed), _ptr(s1), M, N, K, group,
+                                      _ptr(Y), _ptr(acc), tok_tile, splits, _stream(stream)),
+           "qoq_w4a8_gemm_config")
+    return acc if int32_out else Y
+
+
+class QoQLinear:
+    """A linear layer y = x W^T with W stored in the packed W4 format.
+
+    ``forward`` quantizes the activations per token and runs the W4A8 GEMM;
+    both steps are CUDA kernels of ``libqoq.so``."""
+
+    def __init__(self, W, group: int = 128):
+        self.N, self.K = W.shape
+        self.group = group
+        self.packed, self.s1 = quantize_weights(W, group)
+
+    def __call__(self, X, stream=None):
+        X8, sx = quantize_act_per_token(X, stream=stream)
+        return w4a8_gemm(X8, sx, self.packed, self.s1, self.N, self.group, stream=stream)

@@ -1,0 +1,531 @@
+// W4A8 GEMM for sm_100a: Y[m, n] = fp16((sum_k X8[m,k] * dq[n,k]) * sx[m] * s1[n]).
+//
+// Method: "QServe: W4A8KV4 Quantization and System Co-design for Efficient
+// LLM Serving" -- Methods, 1) Algorithm: QoQ (all GEMMs on INT8 tensor cores
+// after progressive group quantization) and 2) System: QServe (UINT4 -> INT8
+// with register-level parallelism, "subtraction after multiplication");
+// Background (per-group W4A4 dequantizes INT32 partial sums in its main loop,
+// this kernel scales once, after the whole K reduction).
+//
+// One CTA computes a 128-channel x TOK-token output tile over a range of
+// K (the weights are the MMA's M operand, the tokens its N operand, so a
+// single decode token still fills the 128-row tensor-core tile):
+//   warp 0      TMA producer: one bulk copy of the packed weight block and one
+//               tensor-map copy of the X8 tile (128-byte swizzle) per k-tile,
+//               into a ring of shared-memory stages;
+//   warp 1      owns tensor memory and issues tcgen05.mma.kind::i8 (M = 128,
+//               N = TOK, K = 32 per instruction, 4 per k-tile), INT32
+//               accumulators in tensor memory;
+//   warps 2..5  dequantize the UINT4 block into the INT8 operand tile (four
+//               byte lanes per 32-bit multiply-add, written in the 128-byte
+//               swizzle the MMA descriptor expects), then run the epilogue:
+//               tcgen05.ld of their 32-lane quarter, one FP32 scale per
+//               element, FP16 stores.
+// When K is split over several CTAs, they form a thread-block cluster and
+// the partial INT32 tiles are added exactly into the rank-0 CTA's shared
+// memory (red.shared::cluster) before its epilogue.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "qoq.h"
+#include "qoq_device.cuh"
+#include "qoq_internal.h"
+
+namespace qoq {
+
+__device__ unsigned int g_error_word = 0;
+
+namespace {
+
+constexpr int kThreads = 192;        // 6 warps
+constexpr int kRawStageBytes = 8576; // largest packed block (group 64), 16-byte multiple
+constexpr int kDqTileBytes = kTileN * kTileK;
+
+template <int TOK>
+struct Cfg {
+  static constexpr int kStages = (TOK <= 32) ? 6 : 4;
+  static constexpr int kDqStages = 2;
+  static constexpr int kXBytes = TOK * kTileK;
+  static constexpr int kOffDq = 0;
+  static constexpr int kOffX = kOffDq + kDqStages * kDqTileBytes;
+  static constexpr int kOffRaw = kOffX + kStages * kXBytes;
+  static constexpr int kOffBar = kOffRaw + kStages * kRawStageBytes;
+  static constexpr int kNumBars = 2 * kStages + 2 * kDqStages + 3;
+  static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + base alignment slack
+  static constexpr int kTmemCols = TOK < 32 ? 32 : TOK;
+  static constexpr int kRedBytes = kTileN * TOK * 4;
+  static_assert(kOffX % 1024 == 0 && kXBytes % 1024 == 0, "swizzled tiles need 1 KiB alignment");
+  static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
+  static_assert(kRedBytes <= kOffRaw, "split-K slot must fit in the dq and X rings");
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+};
+
+struct GemmArgs {
+  const uint8_t* packed;
+  const __half* sx;
+  const __half* s1;
+  __half* Y;
+  int32_t* acc;
+  int M, N, K, group;
+  int splits;
+  int blk_bytes;
+};
+
+// Bounded wait that ignores the abort flag: used only to drain work already
+// in flight before a CTA tears down.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(&g_error_word, kErrProducer);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int TOK>
+__global__ void __launch_bounds__(kThreads, 1)
+w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args) {
+  using C = Cfg<TOK>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t base = (raw_base + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_base);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int splits = args.splits;
+  const int nt = blockIdx.x / splits;
+  const int split = blockIdx.x - nt * splits;   // cluster rank when splits > 1
+  const int m0 = blockIdx.y * TOK;
+  const int kt_total = args.K / kTileK;
+  const int kt_begin = (split * kt_total) / splits;
+  const int num_kt = ((split + 1) * kt_total) / splits - kt_begin;
+
+  const uint32_t bar_full = base + C::kOffBar;
+  const uint32_t bar_empty = bar_full + 8 * C::kStages;
+  const uint32_t bar_dqfull = bar_empty + 8 * C::kStages;
+  const uint32_t bar_dqempty = bar_dqfull + 8 * C::kDqStages;
+  const uint32_t bar_acc = bar_dqempty + 8 * C::kDqStages;
+  const uint32_t bar_redgo = bar_acc + 8;
+  const uint32_t bar_redfull = bar_redgo + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    for (int d = 0; d < C::kDqStages; ++d) {
+      mbar_init(bar_dqfull + 8 * d, 4);
+      mbar_init(bar_dqempty + 8 * d, 1);
+    }
+    mbar_init(bar_acc, 1);
+    mbar_init(bar_redgo, 1);
+    mbar_init(bar_redfull, splits > 1 ? kTileN * (splits - 1) : 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+    prefetch_tensormap(&tmap_x);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  if (splits > 1) {
+    // every CTA of the cluster has initialised its barriers before any
+    // remote arrive can reach them
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+  }
+  const uint32_t tmem_d = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      const uint64_t policy = l2_policy_evict_first();
+      const uint8_t* src =
+          args.packed + (static_cast<size_t>(nt) * kt_total + kt_begin) * args.blk_bytes;
+      const uint32_t tx = static_cast<uint32_t>(args.blk_bytes + C::kXBytes);
+      int i = 0;
+      for (; i < num_kt; ++i) {
+        const int s = i % C::kStages;
+        if (i >= C::kStages &&
+            !mbar_wait(bar_empty + 8 * s, ((i / C::kStages) & 1) ^ 1, abort_flag, &g_error_word, kErrProducer))
+          break;
+        mbar_arrive_expect_tx(bar_full + 8 * s, tx);
+        bulk_load(base + C::kOffRaw + s * kRawStageBytes, src + static_cast<size_t>(i) * args.blk_bytes,
+                  static_cast<uint32_t>(args.blk_bytes), bar_full + 8 * s, policy);
+        tma_load_2d(base + C::kOffX + s * C::kXBytes, &tmap_x, (kt_begin + i) * kTileK, m0,
+                    bar_full + 8 * s);
+      }
+      if (i < num_kt) {
+        // aborted: the copies already issued must land before the CTA exits
+        for (int j = (i > C::kStages ? i - C::kStages : 0); j < i; ++j)
+          drain_wait(bar_full + 8 * (j % C::kStages), (j / C::kStages) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(kTileN, TOK);
+      for (int i = 0; i < num_kt; ++i) {
+        const int s = i % C::kStages, d = i % C::kDqStages;
+        if (!mbar_wait(bar_full + 8 * s, (i / C::kStages) & 1, abort_flag, &g_error_word, kErrMma)) break;
+        if (!mbar_wait(bar_dqfull + 8 * d, (i / C::kDqStages) & 1, abort_flag, &g_error_word, kErrMma)) break;
+        tc_fence_after_sync();
+        const uint32_t a_addr = base + C::kOffDq + d * kDqTileBytes;
+        const uint32_t b_addr = base + C::kOffX + s * C::kXBytes;
+#pragma unroll
+        for (int kk = 0; kk < kTileK / 32; ++kk) {
+          mma_i8_ss(tmem_d, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32),
+                    idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(bar_empty + 8 * s);     // X tile and raw block of stage s are free
+        mma_commit(bar_dqempty + 8 * d);   // dq tile of stage d is free
+      }
+      mma_commit(bar_acc);                 // accumulator complete (or aborted)
+      drain_wait(bar_acc, 0);              // no MMA in flight past this point
+    }
+  } else {
+    // ---------------------------------------------------------------- dequant + epilogue
+    const int q4 = warp & 3;               // tensor-memory lane quarter of this warp
+    const int r = q4 * 32 + lane;          // weight row (output channel) within the tile
+    const int gpt = kTileK / args.group;
+    bool ok = true;
+    for (int i = 0; i < num_kt; ++i) {
+      const int s = i % C::kStages, d = i % C::kDqStages;
+      if (!mbar_wait(bar_full + 8 * s, (i / C::kStages) & 1, abort_flag, &g_error_word, kErrDequant)) {
+        ok = false;
+        break;
+      }
+      if (i >= C::kDqStages &&
+          !mbar_wait(bar_dqempty + 8 * d, ((i / C::kDqStages) & 1) ^ 1, abort_flag, &g_error_word, kErrDequant)) {
+        ok = false;
+        break;
+      }
+      const uint8_t* blk = smem + C::kOffRaw + s * kRawStageBytes;
+      uint8_t* dq_row = smem + C::kOffDq + d * kDqTileBytes + r * kTileK;
+      uint32_t s2v[2], bias[2];
+#pragma unroll
+      for (int gl = 0; gl < 2; ++gl) {
+        if (gl < gpt) {
+          s2v[gl] = blk[kCodesBytes + gl * kTileN + r];
+          const uint32_t zb = blk[kCodesBytes + gpt * kTileN + gl * 64 + (r >> 1)];
+          const uint32_t zv = (r & 1) ? (zb >> 4) : (zb & 15u);
+          bias[gl] = dq_bias(zv, s2v[gl]);
+        } else {
+          s2v[gl] = s2v[0];
+          bias[gl] = bias[0];
+        }
+      }
+      const int sw = r & 7;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 w = *reinterpret_cast<const uint4*>(blk + (j * kTileN + r) * 16);
+        const int gl = (gpt == 2) ? (j >> 1) : 0;
+        const uint32_t sv = s2v[gl], bv = bias[gl];
+        const uint4 c0 = make_uint4(dq_lanes(lo_codes(w.x), sv, bv), dq_lanes(hi_codes(w.x), sv, bv),
+                                    dq_lanes(lo_codes(w.y), sv, bv), dq_lanes(hi_codes(w.y), sv, bv));
+        const uint4 c1 = make_uint4(dq_lanes(lo_codes(w.z), sv, bv), dq_lanes(hi_codes(w.z), sv, bv),
+                                    dq_lanes(lo_codes(w.w), sv, bv), dq_lanes(hi_codes(w.w), sv, bv));
+        *reinterpret_cast<uint4*>(dq_row + (((2 * j) ^ sw) << 4)) = c0;
+        *reinterpret_cast<uint4*>(dq_row + (((2 * j + 1) ^ sw) << 4)) = c1;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_dqfull + 8 * d);
+    }
+
+    // ------------------------------------------------------------ epilogue
+    const bool have = ok && mbar_wait(bar_acc, 0, abort_flag, &g_error_word, kErrEpilogue);
+    tc_fence_after_sync();
+    const bool go = __all_sync(0xffffffffu, have && (*abort_flag == 0u));
+    const uint32_t t_row = tmem_d + (static_cast<uint32_t>(q4 * 32) << 16);
+    const int n = nt * kTileN + r;
+    const int M = args.M, N = args.N;
+
+    auto store = [&](int c, int32_t v) {
+      const int m = m0 + c;
+      if (m < M) {
+        if (args.acc) {
+          args.acc[static_cast<size_t>(m) * N + n] = v;
+        } else {
+          const float scale = __fmul_rn(__half2float(args.sx[m]), __half2float(args.s1[n]));
+          args.Y[static_cast<size_t>(m) * N + n] =
+              __float2half_rn(__fmul_rn(static_cast<float>(v), scale));
+        }
+      }
+    };
+
+    if (splits == 1) {
+      if (go) {
+#pragma unroll 1
+        for (int c0 = 0; c0 < TOK; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(t_row + c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) store(c0 + j, static_cast<int32_t>(v[j]));
+        }
+      }
+    } else {
+      // exact INT32 split-K reduction into rank 0's shared memory, laid out
+      // [token column][row] so that a warp touches 32 consecutive words
+      const uint32_t slot = base;
+      if (split == 0) {
+        if (go) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < TOK; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(t_row + c0, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              *reinterpret_cast<uint32_t*>(smem + ((c0 + j) * kTileN + r) * 4) = v[j];
+          }
+        }
+        epi_bar();
+        if (warp == 2 && lane == 0) {
+          for (int p = 1; p < splits; ++p) mbar_arrive_cluster(map_to_rank(bar_redgo, p));
+        }
+        const bool got = mbar_wait<true>(bar_redfull, 0, abort_flag, &g_error_word, kErrCluster);
+        if (__all_sync(0xffffffffu, go && got && (*abort_flag == 0u))) {
+#pragma unroll 4
+          for (int c = 0; c < TOK; ++c)
+            store(c, *reinterpret_cast<const int32_t*>(smem + (c * kTileN + r) * 4));
+        }
+      } else {
+        const bool got = mbar_wait<true>(bar_redgo, 0, abort_flag, &g_error_word, kErrCluster);
+        const bool push = __all_sync(0xffffffffu, go && got);
+        const uint32_t dst = map_to_rank(slot, 0);
+        if (push) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < TOK; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(t_row + c0, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              red_add_cluster_s32(dst + ((c0 + j) * kTileN + r) * 4, static_cast<int32_t>(v[j]));
+          }
+        }
+        mbar_arrive_cluster(map_to_rank(bar_redfull, 0));
+      }
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_d, C::kTmemCols);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Host side
+// ----------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+struct Plan {
+  int tok, splits, m_tiles, n_tiles, stages;
+};
+
+int stages_for(int tok) { return tok <= 32 ? 6 : 4; }
+
+bool valid_tok(int t) { return t == 16 || t == 32 || t == 64 || t == 128 || t == 256; }
+
+Plan make_plan(int M, int N, int K, int tok_req, int splits_req) {
+  Plan p;
+  p.n_tiles = N / kTileN;
+  const int kt = K / kTileK;
+  if (tok_req) {
+    p.tok = tok_req;
+  } else {
+    p.tok = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+  }
+  p.m_tiles = (M + p.tok - 1) / p.tok;
+  p.stages = stages_for(p.tok);
+  if (splits_req) {
+    p.splits = splits_req;
+  } else {
+    const int occ = p.tok <= 64 ? 2 : 1;
+    const long slots = static_cast<long>(sm_count()) * occ;
+    const long tiles = static_cast<long>(p.n_tiles) * p.m_tiles;
+    p.splits = 1;
+    if (tiles < slots) {
+      double best = 0.0;
+      for (int s = 1; s <= 8 && s <= kt; ++s) {
+        if (s > 1 && kt / s < 2) break;
+        const long ctas = tiles * s;
+        const long waves = (ctas + slots - 1) / slots;
+        const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
+        if (eff > best + 1e-9) {
+          best = eff;
+          p.splits = s;
+        }
+      }
+    }
+  }
+  return p;
+}
+
+template <int TOK>
+int launch_tok(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cudaStream_t stream) {
+  using C = Cfg<TOK>;
+  static int configured_mask = 0;   // one bit per device id < 31
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QOQ_ERR_CUDA;
+  const int bit = dev < 31 ? (1 << dev) : 0;
+  if (!bit || !(__atomic_load_n(&configured_mask, __ATOMIC_ACQUIRE) & bit)) {
+    if (cudaFuncSetAttribute(w4a8_gemm_kernel<TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess)
+      return QOQ_ERR_CUDA;
+    if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_RELEASE);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.n_tiles * p.splits), static_cast<unsigned>(p.m_tiles), 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(p.splits);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, w4a8_gemm_kernel<TOK>, map, a) != cudaSuccess) return QOQ_ERR_CUDA;
+  return QOQ_OK;
+}
+
+int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* s1, int M, int N,
+              int K, int group, void* Y, int32_t* acc, int tok_req, int splits_req,
+              void* stream) {
+  if (!X8 || !packed) return QOQ_ERR_INVALID_ARG;
+  if ((Y == nullptr) == (acc == nullptr)) return QOQ_ERR_INVALID_ARG;
+  if (Y && (!sx || !s1)) return QOQ_ERR_INVALID_ARG;
+  if (M <= 0) return QOQ_ERR_INVALID_ARG;
+  if (int st = check_weight_shape(N, K, group)) return st;
+  if (!aligned16(X8) || !aligned16(packed) || (Y && !aligned16(Y)) || (acc && !aligned16(acc)) ||
+      (sx && !aligned16(sx)) || (s1 && !aligned16(s1)))
+    return QOQ_ERR_INVALID_ARG;
+  if (tok_req && !valid_tok(tok_req)) return QOQ_ERR_INVALID_ARG;
+  if (splits_req && (splits_req < 1 || splits_req > 8 || splits_req > K / kTileK))
+    return QOQ_ERR_INVALID_ARG;
+  if (int st = check_device()) return st;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return QOQ_ERR_CUDA;
+
+  const Plan p = make_plan(M, N, K, tok_req, splits_req);
+  if (p.m_tiles > 65535) return QOQ_ERR_UNSUPPORTED;
+
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileK), static_cast<cuuint32_t>(p.tok)};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(X8), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return QOQ_ERR_CUDA;
+
+  GemmArgs a;
+  a.packed = static_cast<const uint8_t*>(packed);
+  a.sx = static_cast<const __half*>(sx);
+  a.s1 = static_cast<const __half*>(s1);
+  a.Y = static_cast<__half*>(Y);
+  a.acc = acc;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.group = group;
+  a.splits = p.splits;
+  a.blk_bytes = static_cast<int>(block_bytes(group));
+
+  cudaStream_t s = as_stream(stream);
+  switch (p.tok) {
+    case 16: return launch_tok<16>(map, a, p, s);
+    case 32: return launch_tok<32>(map, a, p, s);
+    case 64: return launch_tok<64>(map, a, p, s);
+    case 128: return launch_tok<128>(map, a, p, s);
+    default: return launch_tok<256>(map, a, p, s);
+  }
+}
+
+}  // namespace
+}  // namespace qoq
+
+using namespace qoq;
+
+extern "C" int qoq_w4a8_gemm(const int8_t* X8, const void* sx, const void* packed, const void* s1,
+                             int M, int N, int K, int group, void* Y, void* stream) {
+  if (!Y) return QOQ_ERR_INVALID_ARG;
+  return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, nullptr, 0, 0, stream);
+}
+
+extern "C" int qoq_w4a8_gemm_i32(const int8_t* X8, const void* packed, int M, int N, int K,
+                                 int group, int32_t* acc, void* stream) {
+  if (!acc) return QOQ_ERR_INVALID_ARG;
+  return gemm_impl(X8, nullptr, packed, nullptr, M, N, K, group, nullptr, acc, 0, 0, stream);
+}
+
+extern "C" int qoq_w4a8_gemm_config(const int8_t* X8, const void* sx, const void* packed,
+                                    const void* s1, int M, int N, int K, int group, void* Y,
+                                    int32_t* acc, int tok_tile, int splits, void* stream) {
+  return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, acc, tok_tile, splits, stream);
+}
+
+extern "C" int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int* splits, int* ctas,
+                             int* stages) {
+  if (M <= 0) return QOQ_ERR_INVALID_ARG;
+  if (int st = check_weight_shape(N, K, group)) return st;
+  const Plan p = make_plan(M, N, K, 0, 0);
+  if (tok_tile) *tok_tile = p.tok;
+  if (splits) *splits = p.splits;
+  if (ctas) *ctas = p.n_tiles * p.m_tiles * p.splits;
+  if (stages) *stages = p.stages;
+  return QOQ_OK;
+}
+
+extern "C" int qoq_device_error(unsigned int* value, int clear) {
+  if (!value) return QOQ_ERR_INVALID_ARG;
+  if (int st = check_device()) return st;
+  if (cudaMemcpyFromSymbol(value, g_error_word, sizeof(unsigned int)) != cudaSuccess)
+    return QOQ_ERR_CUDA;
+  if (clear) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(unsigned int)) != cudaSuccess)
+      return QOQ_ERR_CUDA;
+  }
+  return QOQ_OK;
+}

@@ -1,0 +1,46 @@
+// Host-side helpers shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "qoq.h"
+
+namespace qoq {
+
+constexpr int kTileN = 128;       // output channels per weight block / MMA M
+constexpr int kTileK = 128;       // input channels per weight block (one swizzle row)
+constexpr int kCodesBytes = kTileN * kTileK / 2;   // 8192
+constexpr int kMaxK = 133120;     // 127 * 127 * K < 2^31
+constexpr int kProtectiveRange = 119;
+
+inline bool aligned16(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline size_t block_bytes(int group) {
+  if (group != 64 && group != 128) return 0;
+  const int gpt = kTileK / group;                  // groups per block row
+  return static_cast<size_t>(kCodesBytes) + static_cast<size_t>(gpt) * (128 + 64);
+}
+
+// Shape checks common to every weight entry point.
+inline int check_weight_shape(int N, int K, int group) {
+  if (group != 64 && group != 128) return QOQ_ERR_UNSUPPORTED;
+  if (N <= 0 || K <= 0) return QOQ_ERR_INVALID_ARG;
+  if (N % kTileN != 0 || K % kTileK != 0 || K % group != 0) return QOQ_ERR_INVALID_ARG;
+  if (K > kMaxK) return QOQ_ERR_UNSUPPORTED;
+  return QOQ_OK;
+}
+
+// The current device must be compute capability 10.0 (sm_100a code only).
+int check_device();
+// Number of SMs of the current device (cached per device; 148 if unknown).
+int sm_count();
+// cudaGetLastError -> status.
+int launch_status();
+
+}  // namespace qoq

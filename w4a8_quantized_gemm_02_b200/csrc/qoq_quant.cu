@@ -1,0 +1,337 @@
+// Quantization kernels: per-token INT8 activations (online), progressive
+// group quantization of the weights into the packed block format (offline),
+// packing of given codes and the debug unpacker.
+//
+// Method: "QServe: W4A8KV4 Quantization and System Co-design for Efficient
+// LLM Serving" -- Methods, 1) Algorithm: QoQ (progressive group quantization:
+// per-channel INT8 with FP16 scales, then UINT4 per group) and 2) System:
+// QServe (protective range; "subtraction after multiplication").
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "qoq.h"
+#include "qoq_device.cuh"
+#include "qoq_internal.h"
+
+namespace qoq {
+namespace {
+
+// fp16(amax / qmax) with the two guards of the format: 1.0 for an all-zero
+// row, the smallest positive FP16 value when the quotient rounds to zero.
+__device__ __forceinline__ __half scale_from_absmax(float amax, float qmax) {
+  if (amax == 0.0f) return __ushort_as_half(0x3c00);
+  __half s = __float2half_rn(__fdiv_rn(amax, qmax));
+  if ((__half_as_ushort(s) & 0x7fff) == 0) s = __ushort_as_half(0x0001);
+  return s;
+}
+
+// Exact round-half-even of a / b for b > 0.
+__device__ __forceinline__ int div_rne(int a, int b) {
+  int q = a / b;
+  int r = a - q * b;
+  int ar = r < 0 ? -r : r;
+  if (2 * ar > b || (2 * ar == b && (q & 1))) q += (a < 0) ? -1 : 1;
+  return q;
+}
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    v = (lane < static_cast<int>(blockDim.x >> 5)) ? red[lane] : 0.0f;
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (lane == 0) red[0] = v;
+  }
+  __syncthreads();
+  float r = red[0];
+  __syncthreads();
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// Per-token activation quantization: one CTA per row.
+// ---------------------------------------------------------------------------
+constexpr int kActThreads = 256;
+
+__global__ void __launch_bounds__(kActThreads)
+act_quant_kernel(const __half* __restrict__ X, int K, int8_t* __restrict__ X8,
+                 __half* __restrict__ sx) {
+  __shared__ float red[kActThreads / 32];
+  const int m = blockIdx.x;
+  const uint4* row = reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K);
+  const int nvec = K / 8;
+  float amax = 0.0f;
+  for (int i = threadIdx.x; i < nvec; i += kActThreads) {
+    uint4 v = __ldg(row + i);
+    const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 f = __half22float2(h[j]);
+      amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+  amax = block_max(amax, red);
+  const __half s = scale_from_absmax(amax, 127.0f);
+  if (threadIdx.x == 0) sx[m] = s;
+  const float sf = __half2float(s);
+  uint2* out = reinterpret_cast<uint2*>(X8 + static_cast<size_t>(m) * K);
+  for (int i = threadIdx.x; i < nvec; i += kActThreads) {
+    uint4 v = __ldg(row + i);
+    const __half2* h = reinterpret_cast<const __half2*>(&v);
+    uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 f = __half22float2(h[j]);
+      int a = __float2int_rn(__fdiv_rn(f.x, sf));
+      int b = __float2int_rn(__fdiv_rn(f.y, sf));
+      a = max(-127, min(127, a));
+      b = max(-127, min(127, b));
+      const uint32_t pair = (static_cast<uint32_t>(a) & 0xffu) |
+                            ((static_cast<uint32_t>(b) & 0xffu) << 8);
+      packed[j >> 1] |= pair << (16 * (j & 1));
+    }
+    out[i] = make_uint2(packed[0], packed[1]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Level 1 scale: one warp per output channel.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+row_scale_kernel(const __half* __restrict__ W, int N, int K, __half* __restrict__ s1) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= N) return;
+  const uint4* row = reinterpret_cast<const uint4*>(W + static_cast<size_t>(warp) * K);
+  float amax = 0.0f;
+  for (int i = lane; i < K / 8; i += 32) {
+    uint4 v = __ldg(row + i);
+    const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 f = __half22float2(h[j]);
+      amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (lane == 0) s1[warp] = scale_from_absmax(amax, static_cast<float>(kProtectiveRange));
+}
+
+// ---------------------------------------------------------------------------
+// Level 2 + pack: one CTA of 128 threads per (n-tile, k-tile) block; thread r
+// owns output channel n0 + r.  The FP16 tile is staged through shared memory
+// (rows padded by 16 bytes so that a thread per row reads without bank
+// conflicts).
+// ---------------------------------------------------------------------------
+constexpr int kPackRowBytes = kTileK * 2 + 16;   // 272
+
+__device__ __forceinline__ int level1_code(float w, float s1f) {
+  int v = __float2int_rn(__fdiv_rn(w, s1f));
+  return max(-kProtectiveRange, min(kProtectiveRange, v));
+}
+
+__global__ void __launch_bounds__(128)
+pack_weights_kernel(const __half* __restrict__ W, int K, int group,
+                    const __half* __restrict__ s1, uint8_t* __restrict__ packed,
+                    int blk_bytes) {
+  __shared__ __align__(16) uint8_t tile[kTileN * kPackRowBytes];
+  const int kt = blockIdx.x, nt = blockIdx.y;
+  const int n0 = nt * kTileN, k0 = kt * kTileK;
+  const int r = threadIdx.x;
+  // coalesced staging: 128 rows x 256 bytes = 2048 chunks of 16 bytes
+  for (int c = threadIdx.x; c < kTileN * 16; c += 128) {
+    const int row = c >> 4, col = c & 15;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(
+                              W + static_cast<size_t>(n0 + row) * K + k0) + col);
+    *reinterpret_cast<uint4*>(tile + row * kPackRowBytes + col * 16) = v;
+  }
+  __syncthreads();
+
+  const float s1f = __half2float(s1[n0 + r]);
+  const __half* my = reinterpret_cast<const __half*>(tile + r * kPackRowBytes);
+  const int gpt = kTileK / group;
+  uint8_t* blk = packed + static_cast<size_t>(nt * (K / kTileK) + kt) * blk_bytes;
+
+  int s2g[2] = {1, 1}, zg[2] = {0, 0};
+  for (int gl = 0; gl < gpt; ++gl) {
+    int mn = 0, mx = 0;
+    for (int i = 0; i < group; ++i) {
+      const int v = level1_code(__half2float(my[gl * group + i]), s1f);
+      mn = min(mn, v);
+      mx = max(mx, v);
+    }
+    const int s2 = max(1, (mx - mn + 14) / 15);
+    s2g[gl] = s2;
+    zg[gl] = div_rne(-mn, s2);
+  }
+
+  // codes: word w of chunk j covers k = 32j + 8w .. +7
+#pragma unroll 1
+  for (int j = 0; j < 4; ++j) {
+    uint32_t words[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int kb = 32 * j + 8 * w;
+      const int gl = kb / group;
+      uint32_t word = 0;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        const int v = level1_code(__half2float(my[kb + b]), s1f);
+        const int q = max(0, min(15, div_rne(v, s2g[gl]) + zg[gl]));
+        const int lane = b & 3, hi = b >> 2;
+        word |= static_cast<uint32_t>(q) << (8 * lane + 4 * hi);
+      }
+      words[w] = word;
+    }
+    *reinterpret_cast<uint4*>(blk + (j * kTileN + r) * 16) =
+        make_uint4(words[0], words[1], words[2], words[3]);
+  }
+  // metadata
+  for (int gl = 0; gl < gpt; ++gl) {
+    blk[kCodesBytes + gl * kTileN + r] = static_cast<uint8_t>(s2g[gl]);
+    const int zo = __shfl_xor_sync(0xffffffffu, zg[gl], 1);
+    if ((r & 1) == 0) {
+      blk[kCodesBytes + gpt * kTileN + gl * 64 + (r >> 1)] =
+          static_cast<uint8_t>((zg[gl] & 15) | ((zo & 15) << 4));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Pack given canonical codes (one CTA of 128 threads per block).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128)
+pack_codes_kernel(const uint8_t* __restrict__ q, const int8_t* __restrict__ s2,
+                  const uint8_t* __restrict__ z, int K, int group,
+                  uint8_t* __restrict__ packed, int blk_bytes) {
+  const int kt = blockIdx.x, nt = blockIdx.y, r = threadIdx.x;
+  const int n = nt * kTileN + r, k0 = kt * kTileK;
+  const int gpt = kTileK / group, ng = K / group;
+  uint8_t* blk = packed + static_cast<size_t>(nt * (K / kTileK) + kt) * blk_bytes;
+  const uint8_t* qrow = q + static_cast<size_t>(n) * K + k0;
+  for (int j = 0; j < 4; ++j) {
+    uint32_t words[4];
+    for (int w = 0; w < 4; ++w) {
+      uint32_t word = 0;
+      for (int b = 0; b < 8; ++b) {
+        const uint32_t c = qrow[32 * j + 8 * w + b] & 15u;
+        word |= c << (8 * (b & 3) + 4 * (b >> 2));
+      }
+      words[w] = word;
+    }
+    *reinterpret_cast<uint4*>(blk + (j * kTileN + r) * 16) =
+        make_uint4(words[0], words[1], words[2], words[3]);
+  }
+  for (int gl = 0; gl < gpt; ++gl) {
+    const int g = kt * gpt + gl;
+    blk[kCodesBytes + gl * kTileN + r] = static_cast<uint8_t>(s2[static_cast<size_t>(n) * ng + g]);
+    const int zv = z[static_cast<size_t>(n) * ng + g] & 15;
+    const int zo = __shfl_xor_sync(0xffffffffu, zv, 1);
+    if ((r & 1) == 0) {
+      blk[kCodesBytes + gpt * kTileN + gl * 64 + (r >> 1)] =
+          static_cast<uint8_t>(zv | (zo << 4));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Debug unpacker: canonical q / s2 / z and dq via the GEMM's byte-lane path.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128)
+unpack_kernel(const uint8_t* __restrict__ packed, int K, int group, uint8_t* __restrict__ q,
+              int8_t* __restrict__ s2o, uint8_t* __restrict__ zo, int8_t* __restrict__ dq,
+              int blk_bytes) {
+  const int kt = blockIdx.x, nt = blockIdx.y, r = threadIdx.x;
+  const int n = nt * kTileN + r, k0 = kt * kTileK;
+  const int gpt = kTileK / group, ng = K / group;
+  const uint8_t* blk = packed + static_cast<size_t>(nt * (K / kTileK) + kt) * blk_bytes;
+  uint32_t s2v[2], zv[2], bias[2];
+  for (int gl = 0; gl < gpt; ++gl) {
+    s2v[gl] = static_cast<uint32_t>(static_cast<int8_t>(blk[kCodesBytes + gl * kTileN + r]));
+    const uint32_t zb = blk[kCodesBytes + gpt * kTileN + gl * 64 + (r >> 1)];
+    zv[gl] = (r & 1) ? (zb >> 4) : (zb & 15u);
+    bias[gl] = dq_bias(zv[gl], s2v[gl]);
+    const int g = kt * gpt + gl;
+    if (s2o) s2o[static_cast<size_t>(n) * ng + g] = static_cast<int8_t>(s2v[gl]);
+    if (zo) zo[static_cast<size_t>(n) * ng + g] = static_cast<uint8_t>(zv[gl]);
+  }
+  for (int j = 0; j < 4; ++j) {
+    const uint4 v = *reinterpret_cast<const uint4*>(blk + (j * kTileN + r) * 16);
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+    for (int w = 0; w < 4; ++w) {
+      const int kb = 32 * j + 8 * w;
+      const int gl = kb / group;
+      const uint32_t lo = lo_codes(w4[w]), hi = hi_codes(w4[w]);
+      const size_t base = static_cast<size_t>(n) * K + k0 + kb;
+      if (q) {
+        *reinterpret_cast<uint32_t*>(q + base) = lo;
+        *reinterpret_cast<uint32_t*>(q + base + 4) = hi;
+      }
+      if (dq) {
+        *reinterpret_cast<uint32_t*>(dq + base) = dq_lanes(lo, s2v[gl], bias[gl]);
+        *reinterpret_cast<uint32_t*>(dq + base + 4) = dq_lanes(hi, s2v[gl], bias[gl]);
+      }
+    }
+  }
+}
+
+}  // namespace
+}  // namespace qoq
+
+using namespace qoq;
+
+extern "C" int qoq_quantize_act_per_token(const void* X, int M, int K, int8_t* X8, void* sx,
+                                          void* stream) {
+  if (!X || !X8 || !sx) return QOQ_ERR_INVALID_ARG;
+  if (M <= 0 || K <= 0 || K % 8 != 0) return QOQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(X8) || !aligned16(sx)) return QOQ_ERR_INVALID_ARG;
+  if (int st = check_device()) return st;
+  act_quant_kernel<<<M, kActThreads, 0, as_stream(stream)>>>(
+      static_cast<const __half*>(X), K, X8, static_cast<__half*>(sx));
+  return launch_status();
+}
+
+extern "C" int qoq_quantize_weights(const void* W, int N, int K, int group, void* packed,
+                                    void* s1, void* stream) {
+  if (!W || !packed || !s1) return QOQ_ERR_INVALID_ARG;
+  if (int st = check_weight_shape(N, K, group)) return st;
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(s1)) return QOQ_ERR_INVALID_ARG;
+  if (int st = check_device()) return st;
+  cudaStream_t s = as_stream(stream);
+  const __half* Wh = static_cast<const __half*>(W);
+  __half* s1h = static_cast<__half*>(s1);
+  row_scale_kernel<<<(N + 7) / 8, 256, 0, s>>>(Wh, N, K, s1h);
+  if (int st = launch_status()) return st;
+  dim3 grid(K / kTileK, N / kTileN);
+  pack_weights_kernel<<<grid, 128, 0, s>>>(Wh, K, group, s1h, static_cast<uint8_t*>(packed),
+                                           static_cast<int>(block_bytes(group)));
+  return launch_status();
+}
+
+extern "C" int qoq_pack_codes(const uint8_t* q, const int8_t* s2, const uint8_t* z, int N,
+                              int K, int group, void* packed, void* stream) {
+  if (!q || !s2 || !z || !packed) return QOQ_ERR_INVALID_ARG;
+  if (int st = check_weight_shape(N, K, group)) return st;
+  if (!aligned16(packed)) return QOQ_ERR_INVALID_ARG;
+  if (int st = check_device()) return st;
+  dim3 grid(K / kTileK, N / kTileN);
+  pack_codes_kernel<<<grid, 128, 0, as_stream(stream)>>>(
+      q, s2, z, K, group, static_cast<uint8_t*>(packed), static_cast<int>(block_bytes(group)));
+  return launch_status();
+}
+
+extern "C" int qoq_unpack_weights(const void* packed, int N, int K, int group, uint8_t* q,
+                                  int8_t* s2, uint8_t* z, int8_t* dq, void* stream) {
+  if (!packed) return QOQ_ERR_INVALID_ARG;
+  if (int st = check_weight_shape(N, K, group)) return st;
+  if (!aligned16(packed) || (q && !aligned16(q)) || (dq && !aligned16(dq)))
+    return QOQ_ERR_INVALID_ARG;
+  if (int st = check_device()) return st;
+  dim3 grid(K / kTileK, N / kTileN);
+  unpack_kernel<<<grid, 128, 0, as_stream(stream)>>>(static_cast<const uint8_t*>(packed), K,
+                                                     group, q, s2, z, dq,
+                                                     static_cast<int>(block_bytes(group)));
+  return launch_status();
+}
