@@ -185,6 +185,21 @@ QOQ_API int qoq_w4a8_gemm_config(const int8_t* X8, const void* sx, const void* p
                          void* Y, int32_t* acc, int tok_tile, int splits,
                          void* stream);
 
+/* The whole online path of one linear layer: per-token activation
+ * quantization of X followed by the W4A8 GEMM, Y = X . W^T in FP16.
+ *   X      : device, FP16 M x K row-major, read only.
+ *   packed, s1 : the quantized weight (qoq_quantize_weights), N x K.
+ *   X8, sx : device buffers of M x K int8 and M FP16 for the quantized
+ *            activations (written; owned by the caller, reusable between
+ *            calls on the same stream).
+ *   Y      : device, FP16 M x N row-major, written.
+ * Same results as qoq_quantize_act_per_token followed by qoq_w4a8_gemm; here
+ * the GEMM is launched as a programmatic dependent of the quantizer, so it
+ * starts streaming weights while the activations are still being quantized.
+ * Asynchronous on `stream`. */
+QOQ_API int qoq_w4a8_linear(const void* X, int M, int K, const void* packed, const void* s1,
+                            int N, int group, int8_t* X8, void* sx, void* Y, void* stream);
+
 /* The launch configuration qoq_w4a8_gemm picks for a shape: token tile,
  * K splits, CTAs in the grid and pipeline stages.  Host only, no CUDA call
  * beyond reading the SM count of the current device (148 if none). */

@@ -293,6 +293,26 @@ def test_gemm_one_hot_columns(oracle, tiny, tiny_dev):
     assert np.array_equal(host(acc), tiny["w"]["dq"][:, ks].T.astype(np.int32))
 
 
+@pytest.mark.parametrize("M", (1, 16, 17, 300))
+def test_linear_entry_matches_two_calls(oracle, tiny, tiny_dev, M):
+    """The fused entry (quantizer + GEMM launched as a programmatic dependent)
+    gives the oracle's results, also when the buffers are reused."""
+    packed, s1 = tiny_dev
+    L = si.TINY
+    X = si.activations(L, M, seed=M + 5)
+    X8r, sxr, accr, Yr = oracle.w4a8_forward(X, tiny["w"]["dq"], tiny["w"]["s1"])
+    Xd = to_dev(X)
+    X8 = torch.empty((M, L.K), dtype=torch.int8, device=DEV)
+    sx = torch.empty(M, dtype=torch.float16, device=DEV)
+    Y = torch.empty((M, L.N), dtype=torch.float16, device=DEV)
+    for _ in range(3):
+        qoq.w4a8_linear(Xd, packed, s1, L.N, 128, out=Y, scratch=(X8, sx))
+    torch.cuda.synchronize()
+    assert np.array_equal(host(X8), X8r)
+    assert np.array_equal(host(sx).view(np.uint16), sxr.view(np.uint16))
+    check_y(host(Y), Yr)
+
+
 def test_gemm_stream_and_repeat(tiny, tiny_dev):
     """Back-to-back launches on a side stream give identical results."""
     packed, s1 = tiny_dev

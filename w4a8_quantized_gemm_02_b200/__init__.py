@@ -29,7 +29,7 @@ EXPORTS = (
     "qoq_packed_block_bytes", "qoq_packed_weight_bytes",
     "qoq_quantize_weights", "qoq_pack_codes", "qoq_unpack_weights",
     "qoq_quantize_act_per_token", "qoq_w4a8_gemm", "qoq_w4a8_gemm_i32",
-    "qoq_w4a8_gemm_config", "qoq_gemm_plan", "qoq_device_error",
+    "qoq_w4a8_gemm_config", "qoq_w4a8_linear", "qoq_gemm_plan", "qoq_device_error",
 )
 
 _lock = threading.Lock()
@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
             L.qoq_w4a8_gemm_i32.argtypes = [P, P, I, I, I, I, P, P]
             L.qoq_w4a8_gemm_config.restype = I
             L.qoq_w4a8_gemm_config.argtypes = [P, P, P, P, I, I, I, I, P, P, I, I, P]
+            L.qoq_w4a8_linear.restype = I
+            L.qoq_w4a8_linear.argtypes = [P, I, I, P, P, I, I, P, P, P, P]
             L.qoq_gemm_plan.restype = I
             L.qoq_gemm_plan.argtypes = [I, I, I, I] + [ctypes.POINTER(I)] * 4
             L.qoq_device_error.restype = I
@@ -251,10 +253,27 @@ def w4a8_gemm_config(X8, sx, packed, s1, N: int, group: int = 128, *, tok_tile=0
     return acc if int32_out else Y
 
 
+def w4a8_linear(X, packed, s1, N: int, group: int = 128, out=None, scratch=None, stream=None):
+    """Y = X . W^T: per-token activation quantization + W4A8 GEMM in one call
+    (the GEMM overlaps the quantizer's tail).  ``scratch`` = (X8, sx)."""
+    import torch
+    _need_cuda(X, "X", torch.float16, 2)
+    M, K = X.shape
+    if scratch is None:
+        X8 = torch.empty((M, K), dtype=torch.int8, device=X.device)
+        sx = torch.empty(M, dtype=torch.float16, device=X.device)
+    else:
+        X8, sx = scratch
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=X.device)
+    _check(lib().qoq_w4a8_linear(_ptr(X), M, K, _ptr(packed), _ptr(s1), N, group, _ptr(X8),
+                                 _ptr(sx), _ptr(Y), _stream(stream)), "qoq_w4a8_linear")
+    return Y
+
+
 class QoQLinear:
     """A linear layer y = x W^T with W stored in the packed W4 format.
 
-    ``forward`` quantizes the activations per token and runs the W4A8 GEMM;
+    Calling it quantizes the activations per token and runs the W4A8 GEMM;
     both steps are CUDA kernels of ``libqoq.so``."""
 
     def __init__(self, W, group: int = 128):
@@ -262,6 +281,6 @@ class QoQLinear:
         self.group = group
         self.packed, self.s1 = quantize_weights(W, group)
 
-    def __call__(self, X, stream=None):
-        X8, sx = quantize_act_per_token(X, stream=stream)
-        return w4a8_gemm(X8, sx, self.packed, self.s1, self.N, self.group, stream=stream)
+    def __call__(self, X, out=None, scratch=None, stream=None):
+        return w4a8_linear(X, self.packed, self.s1, self.N, self.group, out=out,
+                           scratch=scratch, stream=stream)

@@ -42,26 +42,37 @@ namespace {
 
 constexpr int kThreads = 192;        // 6 warps
 constexpr int kRawStageBytes = 8576; // largest packed block (group 64), 16-byte multiple
-constexpr int kDqTileBytes = kTileN * kTileK;
+constexpr int kSmemPerSm = 233472;   // 228 KiB of shared memory per SM
 
 template <int TOK>
 struct Cfg {
-  static constexpr int kStages = (TOK <= 32) ? 6 : 4;
-  static constexpr int kDqStages = 2;
+  static constexpr int kStages = TOK <= 32 ? 8 : (TOK <= 64 ? 6 : 4);
+  static constexpr int kDqStages = 4;
   static constexpr int kXBytes = TOK * kTileK;
-  static constexpr int kOffDq = 0;
-  static constexpr int kOffX = kOffDq + kDqStages * kDqTileBytes;
+  static constexpr int kOffX = 0;
   static constexpr int kOffRaw = kOffX + kStages * kXBytes;
-  static constexpr int kOffBar = kOffRaw + kStages * kRawStageBytes;
-  static constexpr int kNumBars = 2 * kStages + 2 * kDqStages + 3;
+  static constexpr int kOffSx = kOffRaw + kStages * kRawStageBytes;
+  static constexpr int kOffBar = kOffSx + ((TOK * 4 + 15) / 16) * 16;
+  static constexpr int kNumBars = 2 * kStages + 2 * kDqStages + 1;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + base alignment slack
-  static constexpr int kTmemCols = TOK < 32 ? 32 : TOK;
-  static constexpr int kRedBytes = kTileN * TOK * 4;
-  static_assert(kOffX % 1024 == 0 && kXBytes % 1024 == 0, "swizzled tiles need 1 KiB alignment");
+  static constexpr int kSmemUsed = kOffMisc + 16 + 1024;   // + base alignment slack
+  // tensor memory: A operand stages at columns 32 d, the accumulator after them
+  static constexpr int kTmemA = 0;
+  static constexpr int kTmemD = 32 * kDqStages;
+  static constexpr int kTmemCols = (kTmemD + TOK <= 256) ? 256 : 512;
+  // Never more CTAs on an SM than tensor memory holds: request enough shared
+  // memory that one more CTA cannot fit (a CTA blocked in tcgen05.alloc next
+  // to a cluster peer would otherwise wait for it forever).
+  static constexpr int kCtasPerSm = 512 / kTmemCols;
+  static constexpr int kSmemFloor = kSmemPerSm / (kCtasPerSm + 1);
+  static constexpr int kSmemBytes = kSmemUsed > kSmemFloor ? kSmemUsed : kSmemFloor;
+  // epilogue slot: the INT32 tile as [token column][row], in the X ring
+  static constexpr int kSlotBytes = kTileN * TOK * 4;
+  static_assert(kOffRaw % 1024 == 0 && kXBytes % 1024 == 0, "swizzled tiles need 1 KiB alignment");
   static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
-  static_assert(kRedBytes <= kOffRaw, "split-K slot must fit in the dq and X rings");
+  static_assert(kSlotBytes <= kStages * kXBytes, "epilogue slot must fit in the X ring");
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+  static_assert(kTmemD + TOK <= kTmemCols, "tensor memory");
 };
 
 struct GemmArgs {
@@ -87,7 +98,9 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ uint4 add4(uint4 a, uint4 b) {
+  return make_uint4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
 
 template <int TOK>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -113,10 +126,9 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   const uint32_t bar_dqfull = bar_empty + 8 * C::kStages;
   const uint32_t bar_dqempty = bar_dqfull + 8 * C::kDqStages;
   const uint32_t bar_acc = bar_dqempty + 8 * C::kDqStages;
-  const uint32_t bar_redgo = bar_acc + 8;
-  const uint32_t bar_redfull = bar_redgo + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc + 4);
+  float* sx_s = reinterpret_cast<float*>(smem + C::kOffSx);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -128,8 +140,6 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
       mbar_init(bar_dqempty + 8 * d, 1);
     }
     mbar_init(bar_acc, 1);
-    mbar_init(bar_redgo, 1);
-    mbar_init(bar_redfull, splits > 1 ? kTileN * (splits - 1) : 1);
     *abort_flag = 0u;
     fence_mbar_init();
     prefetch_tensormap(&tmap_x);
@@ -141,13 +151,9 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  if (splits > 1) {
-    // every CTA of the cluster has initialised its barriers before any
-    // remote arrive can reach them
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-  }
-  const uint32_t tmem_d = *tmem_slot;
+  if (splits > 1) cluster_sync_all();   // peers are running before any DSMEM access
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
@@ -156,11 +162,23 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
       const uint8_t* src =
           args.packed + (static_cast<size_t>(nt) * kt_total + kt_begin) * args.blk_bytes;
       const uint32_t tx = static_cast<uint32_t>(args.blk_bytes + C::kXBytes);
-      int i = 0;
+      const int pre = num_kt < C::kStages ? num_kt : C::kStages;
+      // the weight stream does not depend on the preceding grid: start it
+      // before waiting for the activations
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive_expect_tx(bar_full + 8 * i, tx);
+        bulk_load(base + C::kOffRaw + i * kRawStageBytes, src + static_cast<size_t>(i) * args.blk_bytes,
+                  static_cast<uint32_t>(args.blk_bytes), bar_full + 8 * i, policy);
+      }
+      grid_dependency_wait();
+      for (int i = 0; i < pre; ++i)
+        tma_load_2d(base + C::kOffX + i * C::kXBytes, &tmap_x, (kt_begin + i) * kTileK, m0,
+                    bar_full + 8 * i);
+      int i = pre;
       for (; i < num_kt; ++i) {
         const int s = i % C::kStages;
-        if (i >= C::kStages &&
-            !mbar_wait(bar_empty + 8 * s, ((i / C::kStages) & 1) ^ 1, abort_flag, &g_error_word, kErrProducer))
+        if (!mbar_wait(bar_empty + 8 * s, ((i / C::kStages) & 1) ^ 1, abort_flag, &g_error_word,
+                       kErrProducer))
           break;
         mbar_arrive_expect_tx(bar_full + 8 * s, tx);
         bulk_load(base + C::kOffRaw + s * kRawStageBytes, src + static_cast<size_t>(i) * args.blk_bytes,
@@ -178,43 +196,50 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_i8(kTileN, TOK);
+      const uint32_t d_tmem = tmem + C::kTmemD;
       for (int i = 0; i < num_kt; ++i) {
         const int s = i % C::kStages, d = i % C::kDqStages;
-        if (!mbar_wait(bar_full + 8 * s, (i / C::kStages) & 1, abort_flag, &g_error_word, kErrMma)) break;
-        if (!mbar_wait(bar_dqfull + 8 * d, (i / C::kDqStages) & 1, abort_flag, &g_error_word, kErrMma)) break;
+        if (!mbar_wait(bar_full + 8 * s, (i / C::kStages) & 1, abort_flag, &g_error_word, kErrMma))
+          break;
+        if (!mbar_wait(bar_dqfull + 8 * d, (i / C::kDqStages) & 1, abort_flag, &g_error_word,
+                       kErrMma))
+          break;
         tc_fence_after_sync();
-        const uint32_t a_addr = base + C::kOffDq + d * kDqTileBytes;
+        const uint32_t a_tmem = tmem + C::kTmemA + 32 * d;
         const uint32_t b_addr = base + C::kOffX + s * C::kXBytes;
 #pragma unroll
         for (int kk = 0; kk < kTileK / 32; ++kk) {
-          mma_i8_ss(tmem_d, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32),
-                    idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          // K = 32 bytes per instruction: 8 tensor-memory columns of A, 32
+          // bytes along the swizzled rows of B
+          mma_i8_ts(d_tmem, a_tmem + 8 * kk, smem_desc_sw128(b_addr + kk * 32), idesc,
+                    (i > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(bar_empty + 8 * s);     // X tile and raw block of stage s are free
-        mma_commit(bar_dqempty + 8 * d);   // dq tile of stage d is free
+        mma_commit(bar_dqempty + 8 * d);   // A stage d is free
       }
       mma_commit(bar_acc);                 // accumulator complete (or aborted)
       drain_wait(bar_acc, 0);              // no MMA in flight past this point
     }
   } else {
-    // ---------------------------------------------------------------- dequant + epilogue
+    // ---------------------------------------------------------------- dequantizer
     const int q4 = warp & 3;               // tensor-memory lane quarter of this warp
     const int r = q4 * 32 + lane;          // weight row (output channel) within the tile
+    const uint32_t row_tmem = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int gpt = kTileK / args.group;
-    bool ok = true;
     for (int i = 0; i < num_kt; ++i) {
       const int s = i % C::kStages, d = i % C::kDqStages;
-      if (!mbar_wait(bar_full + 8 * s, (i / C::kStages) & 1, abort_flag, &g_error_word, kErrDequant)) {
+      if (!mbar_wait(bar_full + 8 * s, (i / C::kStages) & 1, abort_flag, &g_error_word,
+                     kErrDequant)) {
         ok = false;
         break;
       }
       if (i >= C::kDqStages &&
-          !mbar_wait(bar_dqempty + 8 * d, ((i / C::kDqStages) & 1) ^ 1, abort_flag, &g_error_word, kErrDequant)) {
+          !mbar_wait(bar_dqempty + 8 * d, ((i / C::kDqStages) & 1) ^ 1, abort_flag, &g_error_word,
+                     kErrDequant)) {
         ok = false;
         break;
       }
       const uint8_t* blk = smem + C::kOffRaw + s * kRawStageBytes;
-      uint8_t* dq_row = smem + C::kOffDq + d * kDqTileBytes + r * kTileK;
       uint32_t s2v[2], bias[2];
 #pragma unroll
       for (int gl = 0; gl < 2; ++gl) {
@@ -228,101 +253,112 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
           bias[gl] = bias[0];
         }
       }
-      const int sw = r & 7;
+      uint32_t out[32];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const uint4 w = *reinterpret_cast<const uint4*>(blk + (j * kTileN + r) * 16);
         const int gl = (gpt == 2) ? (j >> 1) : 0;
         const uint32_t sv = s2v[gl], bv = bias[gl];
-        const uint4 c0 = make_uint4(dq_lanes(lo_codes(w.x), sv, bv), dq_lanes(hi_codes(w.x), sv, bv),
-                                    dq_lanes(lo_codes(w.y), sv, bv), dq_lanes(hi_codes(w.y), sv, bv));
-        const uint4 c1 = make_uint4(dq_lanes(lo_codes(w.z), sv, bv), dq_lanes(hi_codes(w.z), sv, bv),
-                                    dq_lanes(lo_codes(w.w), sv, bv), dq_lanes(hi_codes(w.w), sv, bv));
-        *reinterpret_cast<uint4*>(dq_row + (((2 * j) ^ sw) << 4)) = c0;
-        *reinterpret_cast<uint4*>(dq_row + (((2 * j + 1) ^ sw) << 4)) = c1;
+        out[8 * j + 0] = dq_lanes(lo_codes(w.x), sv, bv);
+        out[8 * j + 1] = dq_lanes(hi_codes(w.x), sv, bv);
+        out[8 * j + 2] = dq_lanes(lo_codes(w.y), sv, bv);
+        out[8 * j + 3] = dq_lanes(hi_codes(w.y), sv, bv);
+        out[8 * j + 4] = dq_lanes(lo_codes(w.z), sv, bv);
+        out[8 * j + 5] = dq_lanes(hi_codes(w.z), sv, bv);
+        out[8 * j + 6] = dq_lanes(lo_codes(w.w), sv, bv);
+        out[8 * j + 7] = dq_lanes(hi_codes(w.w), sv, bv);
       }
-      fence_proxy_async_smem();
+      // one 128-byte row of the INT8 A operand: column c holds K bytes 4c..4c+3
+      tmem_st_32x32b_x32(row_tmem + C::kTmemA + 32 * d, out);
+      tmem_st_wait();
+      tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_dqfull + 8 * d);
     }
+  }
 
-    // ------------------------------------------------------------ epilogue
+  // ------------------------------------------------------------------ epilogue
+  // 1) accumulator -> this CTA's slot [token column][row] (INT32)
+  uint32_t* slot = reinterpret_cast<uint32_t*>(smem + C::kOffX);
+  const bool epi = warp >= 2;
+  if (epi) {
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
     const bool have = ok && mbar_wait(bar_acc, 0, abort_flag, &g_error_word, kErrEpilogue);
     tc_fence_after_sync();
-    const bool go = __all_sync(0xffffffffu, have && (*abort_flag == 0u));
-    const uint32_t t_row = tmem_d + (static_cast<uint32_t>(q4 * 32) << 16);
-    const int n = nt * kTileN + r;
-    const int M = args.M, N = args.N;
-
-    auto store = [&](int c, int32_t v) {
-      const int m = m0 + c;
-      if (m < M) {
-        if (args.acc) {
-          args.acc[static_cast<size_t>(m) * N + n] = v;
-        } else {
-          const float scale = __fmul_rn(__half2float(args.sx[m]), __half2float(args.s1[n]));
-          args.Y[static_cast<size_t>(m) * N + n] =
-              __float2half_rn(__fmul_rn(static_cast<float>(v), scale));
-        }
+    if (__all_sync(0xffffffffu, have && (*abort_flag == 0u))) {
+      const uint32_t t_row = tmem + C::kTmemD + (static_cast<uint32_t>(q4 * 32) << 16);
+#pragma unroll 1
+      for (int c0 = 0; c0 < TOK; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(t_row + c0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) slot[(c0 + j) * kTileN + r] = v[j];
       }
-    };
-
-    if (splits == 1) {
-      if (go) {
-#pragma unroll 1
-        for (int c0 = 0; c0 < TOK; c0 += 16) {
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(t_row + c0, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) store(c0 + j, static_cast<int32_t>(v[j]));
-        }
-      }
-    } else {
-      // exact INT32 split-K reduction into rank 0's shared memory, laid out
-      // [token column][row] so that a warp touches 32 consecutive words
-      const uint32_t slot = base;
-      if (split == 0) {
-        if (go) {
-#pragma unroll 1
-          for (int c0 = 0; c0 < TOK; c0 += 16) {
-            uint32_t v[16];
-            tmem_ld_32x32b_x16(t_row + c0, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              *reinterpret_cast<uint32_t*>(smem + ((c0 + j) * kTileN + r) * 4) = v[j];
-          }
-        }
-        epi_bar();
-        if (warp == 2 && lane == 0) {
-          for (int p = 1; p < splits; ++p) mbar_arrive_cluster(map_to_rank(bar_redgo, p));
-        }
-        const bool got = mbar_wait<true>(bar_redfull, 0, abort_flag, &g_error_word, kErrCluster);
-        if (__all_sync(0xffffffffu, go && got && (*abort_flag == 0u))) {
-#pragma unroll 4
-          for (int c = 0; c < TOK; ++c)
-            store(c, *reinterpret_cast<const int32_t*>(smem + (c * kTileN + r) * 4));
-        }
-      } else {
-        const bool got = mbar_wait<true>(bar_redgo, 0, abort_flag, &g_error_word, kErrCluster);
-        const bool push = __all_sync(0xffffffffu, go && got);
-        const uint32_t dst = map_to_rank(slot, 0);
-        if (push) {
-#pragma unroll 1
-          for (int c0 = 0; c0 < TOK; c0 += 16) {
-            uint32_t v[16];
-            tmem_ld_32x32b_x16(t_row + c0, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              red_add_cluster_s32(dst + ((c0 + j) * kTileN + r) * 4, static_cast<int32_t>(v[j]));
-          }
-        }
-        mbar_arrive_cluster(map_to_rank(bar_redfull, 0));
+    }
+    if (args.Y) {
+      grid_dependency_wait();   // sx comes from the preceding grid under PDL
+      for (int c = threadIdx.x - 64; c < TOK; c += 128) {
+        const int m = m0 + c;
+        sx_s[c] = m < args.M ? __half2float(args.sx[m]) : 0.0f;
       }
     }
   }
+  __syncwarp();
+  if (splits > 1) {
+    cluster_sync_all();
+  } else {
+    __syncthreads();
+  }
+
+  // 2) sum the partial tiles of all K splits (DSMEM) and store: each rank owns
+  //    the token columns c = rank (mod splits); a thread owns 4 consecutive rows
+  if (epi && *abort_flag == 0u) {
+    const int we = warp - 2;
+    const int rq = 4 * lane;
+    const int n = nt * kTileN + rq;
+    const int M = args.M, N = args.N;
+    float s1q[4] = {0.f, 0.f, 0.f, 0.f};
+    if (args.Y) {
+      const uint2 sv = *reinterpret_cast<const uint2*>(args.s1 + n);
+      const __half2* h = reinterpret_cast<const __half2*>(&sv);
+      const float2 a = __half22float2(h[0]), b = __half22float2(h[1]);
+      s1q[0] = a.x;
+      s1q[1] = a.y;
+      s1q[2] = b.x;
+      s1q[3] = b.y;
+    }
+    const uint32_t slot_addr = base + C::kOffX;
+    for (int c = split + splits * we; c < TOK; c += 4 * splits) {
+      const int m = m0 + c;
+      if (m >= M) break;
+      const int e = c * kTileN + rq;
+      uint4 v = *reinterpret_cast<const uint4*>(slot + e);
+      for (int q = 0; q < splits; ++q) {
+        if (q == split) continue;
+        v = add4(v, ld_cluster_v4(map_to_rank(slot_addr + 4u * e, q)));
+      }
+      const size_t o = static_cast<size_t>(m) * N + n;
+      if (args.acc) {
+        *reinterpret_cast<uint4*>(args.acc + o) = v;
+      } else {
+        const float sxf = sx_s[c];
+        const __half2 y01 = __floats2half2_rn(
+            __fmul_rn(static_cast<float>(static_cast<int32_t>(v.x)), __fmul_rn(sxf, s1q[0])),
+            __fmul_rn(static_cast<float>(static_cast<int32_t>(v.y)), __fmul_rn(sxf, s1q[1])));
+        const __half2 y23 = __floats2half2_rn(
+            __fmul_rn(static_cast<float>(static_cast<int32_t>(v.z)), __fmul_rn(sxf, s1q[2])),
+            __fmul_rn(static_cast<float>(static_cast<int32_t>(v.w)), __fmul_rn(sxf, s1q[3])));
+        uint2 pk;
+        pk.x = *reinterpret_cast<const uint32_t*>(&y01);
+        pk.y = *reinterpret_cast<const uint32_t*>(&y23);
+        *reinterpret_cast<uint2*>(args.Y + o) = pk;
+      }
+    }
+  }
+  __syncwarp();
+  if (splits > 1) cluster_sync_all();   // peers keep their slots until every rank has read them
 
   // ------------------------------------------------------------------ teardown
   tc_fence_before_sync();
@@ -330,7 +366,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   if (warp == 1) {
     __syncwarp();
     tc_fence_after_sync();
-    tmem_dealloc(tmem_d, C::kTmemCols);
+    tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
@@ -360,7 +396,7 @@ struct Plan {
   int tok, splits, m_tiles, n_tiles, stages;
 };
 
-int stages_for(int tok) { return tok <= 32 ? 6 : 4; }
+int stages_for(int tok) { return tok <= 32 ? 8 : (tok <= 64 ? 6 : 4); }
 
 bool valid_tok(int t) { return t == 16 || t == 32 || t == 64 || t == 128 || t == 256; }
 
@@ -378,7 +414,7 @@ Plan make_plan(int M, int N, int K, int tok_req, int splits_req) {
   if (splits_req) {
     p.splits = splits_req;
   } else {
-    const int occ = p.tok <= 64 ? 2 : 1;
+    const int occ = p.tok <= 128 ? 2 : 1;
     const long slots = static_cast<long>(sm_count()) * occ;
     const long tiles = static_cast<long>(p.n_tiles) * p.m_tiles;
     p.splits = 1;
@@ -400,7 +436,8 @@ Plan make_plan(int M, int N, int K, int tok_req, int splits_req) {
 }
 
 template <int TOK>
-int launch_tok(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cudaStream_t stream) {
+int launch_tok(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cudaStream_t stream,
+               bool pdl) {
   using C = Cfg<TOK>;
   static int configured_mask = 0;   // one bit per device id < 31
   int dev = 0;
@@ -417,20 +454,24 @@ int launch_tok(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cudaStr
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(p.splits);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   if (cudaLaunchKernelEx(&cfg, w4a8_gemm_kernel<TOK>, map, a) != cudaSuccess) return QOQ_ERR_CUDA;
   return QOQ_OK;
 }
 
+}  // namespace
+
 int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* s1, int M, int N,
               int K, int group, void* Y, int32_t* acc, int tok_req, int splits_req,
-              void* stream) {
+              void* stream, bool pdl) {
   if (!X8 || !packed) return QOQ_ERR_INVALID_ARG;
   if ((Y == nullptr) == (acc == nullptr)) return QOQ_ERR_INVALID_ARG;
   if (Y && (!sx || !s1)) return QOQ_ERR_INVALID_ARG;
@@ -474,15 +515,14 @@ int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* 
 
   cudaStream_t s = as_stream(stream);
   switch (p.tok) {
-    case 16: return launch_tok<16>(map, a, p, s);
-    case 32: return launch_tok<32>(map, a, p, s);
-    case 64: return launch_tok<64>(map, a, p, s);
-    case 128: return launch_tok<128>(map, a, p, s);
-    default: return launch_tok<256>(map, a, p, s);
+    case 16: return launch_tok<16>(map, a, p, s, pdl);
+    case 32: return launch_tok<32>(map, a, p, s, pdl);
+    case 64: return launch_tok<64>(map, a, p, s, pdl);
+    case 128: return launch_tok<128>(map, a, p, s, pdl);
+    default: return launch_tok<256>(map, a, p, s, pdl);
   }
 }
 
-}  // namespace
 }  // namespace qoq
 
 using namespace qoq;
@@ -490,19 +530,34 @@ using namespace qoq;
 extern "C" int qoq_w4a8_gemm(const int8_t* X8, const void* sx, const void* packed, const void* s1,
                              int M, int N, int K, int group, void* Y, void* stream) {
   if (!Y) return QOQ_ERR_INVALID_ARG;
-  return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, nullptr, 0, 0, stream);
+  return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, nullptr, 0, 0, stream, false);
 }
 
 extern "C" int qoq_w4a8_gemm_i32(const int8_t* X8, const void* packed, int M, int N, int K,
                                  int group, int32_t* acc, void* stream) {
   if (!acc) return QOQ_ERR_INVALID_ARG;
-  return gemm_impl(X8, nullptr, packed, nullptr, M, N, K, group, nullptr, acc, 0, 0, stream);
+  return gemm_impl(X8, nullptr, packed, nullptr, M, N, K, group, nullptr, acc, 0, 0, stream, false);
 }
 
 extern "C" int qoq_w4a8_gemm_config(const int8_t* X8, const void* sx, const void* packed,
                                     const void* s1, int M, int N, int K, int group, void* Y,
                                     int32_t* acc, int tok_tile, int splits, void* stream) {
-  return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, acc, tok_tile, splits, stream);
+  return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, acc, tok_tile, splits, stream, false);
+}
+
+extern "C" int qoq_w4a8_linear(const void* X, int M, int K, const void* packed, const void* s1,
+                               int N, int group, int8_t* X8, void* sx, void* Y, void* stream) {
+  if (!X || !X8 || !sx || !Y || !packed || !s1) return QOQ_ERR_INVALID_ARG;
+  if (M <= 0) return QOQ_ERR_INVALID_ARG;
+  if (int st = check_weight_shape(N, K, group)) return st;
+  if (!aligned16(X) || !aligned16(X8) || !aligned16(sx) || !aligned16(Y) || !aligned16(packed) ||
+      !aligned16(s1))
+    return QOQ_ERR_INVALID_ARG;
+  if (int st = check_device()) return st;
+  if (int st = launch_act_quant(X, M, K, X8, sx, stream)) return st;
+  // both kernels are this library's: the GEMM reads nothing the quantizer
+  // writes before its grid-dependency wait, so it may overlap its tail
+  return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, nullptr, 0, 0, stream, true);
 }
 
 extern "C" int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int* splits, int* ctas,

@@ -51,48 +51,78 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 }
 
 // ---------------------------------------------------------------------------
-// Per-token activation quantization: one CTA per row.
+// Per-token activation quantization: one CTA per row.  A row of up to
+// kActThreads * 8 * kActMaxVec values stays in registers between the
+// abs-max reduction and the quantization (one pass over X); longer rows are
+// read twice.
 // ---------------------------------------------------------------------------
 constexpr int kActThreads = 256;
+constexpr int kActMaxVec = 16;
+
+__device__ __forceinline__ uint2 quantize8(uint4 v, float sf) {
+  const __half2* h = reinterpret_cast<const __half2*>(&v);
+  uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __half22float2(h[j]);
+    int a = __float2int_rn(__fdiv_rn(f.x, sf));
+    int b = __float2int_rn(__fdiv_rn(f.y, sf));
+    a = max(-127, min(127, a));
+    b = max(-127, min(127, b));
+    const uint32_t pair = (static_cast<uint32_t>(a) & 0xffu) |
+                          ((static_cast<uint32_t>(b) & 0xffu) << 8);
+    packed[j >> 1] |= pair << (16 * (j & 1));
+  }
+  return make_uint2(packed[0], packed[1]);
+}
+
+__device__ __forceinline__ float absmax8(uint4 v, float amax) {
+  const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __half22float2(h[j]);
+    amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+  }
+  return amax;
+}
 
 __global__ void __launch_bounds__(kActThreads)
 act_quant_kernel(const __half* __restrict__ X, int K, int8_t* __restrict__ X8,
                  __half* __restrict__ sx) {
+  // the GEMM that consumes X8 may start its weight prologue right away
+  grid_launch_dependents();
   __shared__ float red[kActThreads / 32];
   const int m = blockIdx.x;
   const uint4* row = reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K);
+  uint2* out = reinterpret_cast<uint2*>(X8 + static_cast<size_t>(m) * K);
   const int nvec = K / 8;
+  const bool in_regs = nvec <= kActThreads * kActMaxVec;
+  uint4 v[kActMaxVec];
   float amax = 0.0f;
-  for (int i = threadIdx.x; i < nvec; i += kActThreads) {
-    uint4 v = __ldg(row + i);
-    const __half2* h = reinterpret_cast<const __half2*>(&v);
+  if (in_regs) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float2 f = __half22float2(h[j]);
-      amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+    for (int u = 0; u < kActMaxVec; ++u) {
+      const int i = threadIdx.x + u * kActThreads;
+      if (i < nvec) {
+        v[u] = __ldg(row + i);
+        amax = absmax8(v[u], amax);
+      }
     }
+  } else {
+    for (int i = threadIdx.x; i < nvec; i += kActThreads) amax = absmax8(__ldg(row + i), amax);
   }
   amax = block_max(amax, red);
   const __half s = scale_from_absmax(amax, 127.0f);
   if (threadIdx.x == 0) sx[m] = s;
   const float sf = __half2float(s);
-  uint2* out = reinterpret_cast<uint2*>(X8 + static_cast<size_t>(m) * K);
-  for (int i = threadIdx.x; i < nvec; i += kActThreads) {
-    uint4 v = __ldg(row + i);
-    const __half2* h = reinterpret_cast<const __half2*>(&v);
-    uint32_t packed[2] = {0u, 0u};
+  if (in_regs) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float2 f = __half22float2(h[j]);
-      int a = __float2int_rn(__fdiv_rn(f.x, sf));
-      int b = __float2int_rn(__fdiv_rn(f.y, sf));
-      a = max(-127, min(127, a));
-      b = max(-127, min(127, b));
-      const uint32_t pair = (static_cast<uint32_t>(a) & 0xffu) |
-                            ((static_cast<uint32_t>(b) & 0xffu) << 8);
-      packed[j >> 1] |= pair << (16 * (j & 1));
+    for (int u = 0; u < kActMaxVec; ++u) {
+      const int i = threadIdx.x + u * kActThreads;
+      if (i < nvec) out[i] = quantize8(v[u], sf);
     }
-    out[i] = make_uint2(packed[0], packed[1]);
+  } else {
+    for (int i = threadIdx.x; i < nvec; i += kActThreads) out[i] = quantize8(__ldg(row + i), sf);
   }
 }
 
@@ -282,15 +312,21 @@ unpack_kernel(const uint8_t* __restrict__ packed, int K, int group, uint8_t* __r
 
 using namespace qoq;
 
+namespace qoq {
+int launch_act_quant(const void* X, int M, int K, int8_t* X8, void* sx, void* stream) {
+  act_quant_kernel<<<M, kActThreads, 0, as_stream(stream)>>>(
+      static_cast<const __half*>(X), K, X8, static_cast<__half*>(sx));
+  return launch_status();
+}
+}  // namespace qoq
+
 extern "C" int qoq_quantize_act_per_token(const void* X, int M, int K, int8_t* X8, void* sx,
                                           void* stream) {
   if (!X || !X8 || !sx) return QOQ_ERR_INVALID_ARG;
   if (M <= 0 || K <= 0 || K % 8 != 0) return QOQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(X8) || !aligned16(sx)) return QOQ_ERR_INVALID_ARG;
   if (int st = check_device()) return st;
-  act_quant_kernel<<<M, kActThreads, 0, as_stream(stream)>>>(
-      static_cast<const __half*>(X), K, X8, static_cast<__half*>(sx));
-  return launch_status();
+  return launch_act_quant(X, M, K, X8, sx, stream);
 }
 
 extern "C" int qoq_quantize_weights(const void* W, int N, int K, int group, void* packed,
