@@ -18,7 +18,8 @@
  * Conventions for every entry point:
  *  - Pointers named as device pointers must point to device memory of the
  *    current CUDA device; the caller owns all memory.  The library allocates
- *    no device memory; the only state it keeps between calls is the
+ *    no device memory (the GEMM's split-K workspace is the caller's); the
+ *    only state it keeps between calls is the
  *    device error word (qoq_device_error) and host-side caches of device
  *    attributes and of the driver's tensor-map entry point.
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
@@ -157,33 +158,53 @@ QOQ_API int qoq_quantize_act_per_token(const void* X, int M, int K, int8_t* X8,
  *   packed : device, packed weights (qoq_quantize_weights / qoq_pack_codes).
  *   s1     : device, FP16[N].
  *   Y      : device, FP16 M x N row-major, written (rows >= M untouched).
+ *   ws, ws_bytes : device workspace for splitting K over several CTAs, at
+ *            least qoq_gemm_workspace_bytes(M, N, K, group) bytes (0 for
+ *            shapes that are not split).  Owned by the caller; it may hold
+ *            anything before the first call and can be reused by later calls
+ *            on the same stream, whatever their shape.  Calls that can run at
+ *            the same time (different streams) need different workspaces.
+ *            With ws == NULL or too small the call still runs, without
+ *            splitting K (slower for small M).
  * The UINT4 codes are dequantized to INT8 inside the main loop
  * (dq = q*s2 - z*s2, four byte lanes per 32-bit operation), multiplied on the
  * INT8 tensor cores (tcgen05, INT32 accumulators in tensor memory), and the
  * FP16 scaling runs once in the epilogue: Y = fp16_rn(float(acc) *
- * (float(sx[m]) * float(s1[n]))).  The tile shape and the number of K splits
- * are chosen per (M, N, K); split partials are summed exactly in INT32 across
- * a thread-block cluster before the epilogue.  Sources: Methods, 1) and 2);
- * Background.  Asynchronous on `stream`.
+ * (float(sx[m]) * float(s1[n]))).  The token tile and the number of K splits
+ * are chosen per (M, N, K); split partials are added exactly in INT32 by the
+ * last CTA of each output tile before its epilogue.  Sources: Methods, 1) and
+ * 2); Background.  Asynchronous on `stream`.
  * ---------------------------------------------------------------------- */
 QOQ_API int qoq_w4a8_gemm(const int8_t* X8, const void* sx, const void* packed,
-                  const void* s1, int M, int N, int K, int group, void* Y,
-                  void* stream);
+                          const void* s1, int M, int N, int K, int group, void* Y,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes qoq_w4a8_gemm, qoq_w4a8_gemm_i32 and qoq_w4a8_linear use
+ * for this shape (0 if K is not split, or if the shape is invalid). */
+QOQ_API size_t qoq_gemm_workspace_bytes(int M, int N, int K, int group);
+
+/* Workspace bytes for an explicit configuration of qoq_w4a8_gemm_config
+ * (tok_tile / splits as there, 0 = auto). */
+QOQ_API size_t qoq_gemm_workspace_bytes_config(int M, int N, int K, int group,
+                                               int tok_tile, int splits);
 
 /* Debug: the same main loop, storing the raw INT32 accumulator
  * acc[m, n] = sum_k X8[m,k] * dq[n,k] (device, int32 M x N row-major). */
 QOQ_API int qoq_w4a8_gemm_i32(const int8_t* X8, const void* packed, int M, int N,
-                      int K, int group, int32_t* acc, void* stream);
+                              int K, int group, int32_t* acc, void* ws,
+                              size_t ws_bytes, void* stream);
 
 /* The same GEMM with an explicit launch configuration (tuning and tests).
  *   tok_tile : token tile (MMA N): 16, 32, 64, 128 or 256, or 0 for auto;
  *   splits   : K splits per output tile, 1..8 (at most K/128), or 0 for auto.
  * Exactly one of Y (FP16 output, needs sx and s1) and acc (INT32 output) is
- * non-NULL.  Asynchronous on `stream`. */
+ * non-NULL.  An explicit split count needs its workspace
+ * (qoq_gemm_workspace_bytes_config), else QOQ_ERR_INVALID_ARG.
+ * Asynchronous on `stream`. */
 QOQ_API int qoq_w4a8_gemm_config(const int8_t* X8, const void* sx, const void* packed,
-                         const void* s1, int M, int N, int K, int group,
-                         void* Y, int32_t* acc, int tok_tile, int splits,
-                         void* stream);
+                                 const void* s1, int M, int N, int K, int group,
+                                 void* Y, int32_t* acc, int tok_tile, int splits,
+                                 void* ws, size_t ws_bytes, void* stream);
 
 /* The whole online path of one linear layer: per-token activation
  * quantization of X followed by the W4A8 GEMM, Y = X . W^T in FP16.
@@ -193,12 +214,14 @@ QOQ_API int qoq_w4a8_gemm_config(const int8_t* X8, const void* sx, const void* p
  *            activations (written; owned by the caller, reusable between
  *            calls on the same stream).
  *   Y      : device, FP16 M x N row-major, written.
+ *   ws, ws_bytes : as for qoq_w4a8_gemm.
  * Same results as qoq_quantize_act_per_token followed by qoq_w4a8_gemm; here
  * the GEMM is launched as a programmatic dependent of the quantizer, so it
  * starts streaming weights while the activations are still being quantized.
  * Asynchronous on `stream`. */
 QOQ_API int qoq_w4a8_linear(const void* X, int M, int K, const void* packed, const void* s1,
-                            int N, int group, int8_t* X8, void* sx, void* Y, void* stream);
+                            int N, int group, int8_t* X8, void* sx, void* Y, void* ws,
+                            size_t ws_bytes, void* stream);
 
 /* The launch configuration qoq_w4a8_gemm picks for a shape: token tile,
  * K splits, CTAs in the grid and pipeline stages.  Host only, no CUDA call
@@ -212,7 +235,7 @@ QOQ_API int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int* sp
  * instead of hanging.  Synchronous (device-wide): reads the word of the
  * current device and, if `clear` is non-zero, resets it to 0.
  * Bits: 1 = producer wait, 2 = MMA wait, 4 = dequantizer wait,
- *       8 = epilogue wait, 16 = cluster reduction.
+ *       8 = epilogue wait, 16 = split-K arrival counter.
  * ---------------------------------------------------------------------- */
 QOQ_API int qoq_device_error(unsigned int* value, int clear);
 

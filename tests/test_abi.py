@@ -53,7 +53,7 @@ def test_plan_is_host_only(L):
     for M in (1, 16, 17, 64, 100, 256, 1024, 4096):
         p = qoq.gemm_plan(M, 6144, 4096, 128)
         assert p["tok_tile"] in (16, 32, 64, 128, 256)
-        assert p["tok_tile"] >= min(M, 256) or M > 256
+        assert p["tok_tile"] >= min(M, 128)
         assert 1 <= p["splits"] <= 8
         assert p["ctas"] == 48 * -(-M // p["tok_tile"]) * p["splits"]
     with pytest.raises(qoq.QoQError):
@@ -66,8 +66,9 @@ FAKE = 0x10000          # 16-byte aligned fake device address (never dereference
 P = ctypes.c_void_p
 
 
-def _gemm(L, X8=FAKE, sx=FAKE, packed=FAKE, s1=FAKE, M=16, N=512, K=512, G=128, Y=FAKE):
-    return L.qoq_w4a8_gemm(P(X8), P(sx), P(packed), P(s1), M, N, K, G, P(Y), None)
+def _gemm(L, X8=FAKE, sx=FAKE, packed=FAKE, s1=FAKE, M=16, N=512, K=512, G=128, Y=FAKE,
+          ws=None, wsb=0):
+    return L.qoq_w4a8_gemm(P(X8), P(sx), P(packed), P(s1), M, N, K, G, P(Y), P(ws), wsb, None)
 
 
 def test_gemm_argument_validation(L):
@@ -82,19 +83,22 @@ def test_gemm_argument_validation(L):
     assert _gemm(L, sx=None) == qoq.QOQ_ERR_INVALID_ARG
     assert _gemm(L, X8=FAKE + 8) == qoq.QOQ_ERR_INVALID_ARG     # alignment
     assert _gemm(L, Y=FAKE + 2) == qoq.QOQ_ERR_INVALID_ARG
+    assert _gemm(L, ws=FAKE + 4, wsb=1 << 20) == qoq.QOQ_ERR_INVALID_ARG
     cfg = L.qoq_w4a8_gemm_config
-    # both outputs / neither output
-    assert cfg(P(FAKE), P(FAKE), P(FAKE), P(FAKE), 16, 512, 512, 128, P(FAKE), P(FAKE), 0, 0,
-               None) == qoq.QOQ_ERR_INVALID_ARG
-    assert cfg(P(FAKE), P(FAKE), P(FAKE), P(FAKE), 16, 512, 512, 128, None, None, 0, 0,
-               None) == qoq.QOQ_ERR_INVALID_ARG
-    # bad tile / split requests
-    assert cfg(P(FAKE), None, P(FAKE), None, 16, 512, 512, 128, None, P(FAKE), 48, 0,
-               None) == qoq.QOQ_ERR_INVALID_ARG
-    assert cfg(P(FAKE), None, P(FAKE), None, 16, 512, 512, 128, None, P(FAKE), 16, 9,
-               None) == qoq.QOQ_ERR_INVALID_ARG
-    assert cfg(P(FAKE), None, P(FAKE), None, 16, 512, 512, 128, None, P(FAKE), 16, 5,
-               None) == qoq.QOQ_ERR_INVALID_ARG          # more splits than k-tiles
+
+    def c(Y, acc, tok, sp, ws=None, wsb=0):
+        return cfg(P(FAKE), P(FAKE), P(FAKE), P(FAKE), 16, 512, 512, 128, P(Y), P(acc), tok, sp,
+                   P(ws), wsb, None)
+    assert c(FAKE, FAKE, 0, 0) == qoq.QOQ_ERR_INVALID_ARG      # both outputs
+    assert c(None, None, 0, 0) == qoq.QOQ_ERR_INVALID_ARG      # neither output
+    assert c(None, FAKE, 48, 0) == qoq.QOQ_ERR_INVALID_ARG     # bad token tile
+    assert c(None, FAKE, 16, 9) == qoq.QOQ_ERR_INVALID_ARG     # too many splits
+    assert c(None, FAKE, 16, 5) == qoq.QOQ_ERR_INVALID_ARG     # more splits than k-tiles
+    # an explicit split needs its workspace
+    need = qoq.gemm_workspace_bytes(16, 512, 512, 128, 16, 2)
+    assert need > 0
+    assert c(None, FAKE, 16, 2) == qoq.QOQ_ERR_INVALID_ARG
+    assert c(None, FAKE, 16, 2, FAKE, need - 16) == qoq.QOQ_ERR_INVALID_ARG
 
 
 def test_other_entry_validation(L):
@@ -107,6 +111,22 @@ def test_other_entry_validation(L):
     assert L.qoq_pack_codes(None, P(FAKE), P(FAKE), 512, 512, 128, P(FAKE), None) == 1
     assert L.qoq_unpack_weights(None, 512, 512, 128, None, None, None, None, None) == 1
     assert L.qoq_device_error(None, 0) == 1
+    assert L.qoq_w4a8_linear(None, 4, 512, P(FAKE), P(FAKE), 512, 128, P(FAKE), P(FAKE),
+                             P(FAKE), None, 0, None) == 1
+    assert L.qoq_w4a8_linear(P(FAKE), 4, 512, P(FAKE), P(FAKE), 500, 128, P(FAKE), P(FAKE),
+                             P(FAKE), None, 0, None) == 1
+
+
+def test_workspace_sizes(L):
+    assert qoq.gemm_workspace_bytes(16, 512, 512, 128, 16, 1) == 0
+    # partials [m_tiles][splits][tok][N] int32 + counters, 256-byte rounded
+    assert qoq.gemm_workspace_bytes(16, 512, 512, 128, 16, 2) == 2 * 16 * 512 * 4 + 256
+    assert qoq.gemm_workspace_bytes(40, 512, 512, 128, 16, 4) == \
+        3 * 4 * 16 * 512 * 4 + 256
+    assert qoq.gemm_workspace_bytes(0, 512, 512, 128) == 0
+    p = qoq.gemm_plan(1, 6144, 4096, 128)
+    ws = qoq.gemm_workspace_bytes(1, 6144, 4096, 128)
+    assert (ws > 0) == (p["splits"] > 1)
 
 
 def _has_gpu():

@@ -30,6 +30,7 @@ EXPORTS = (
     "qoq_quantize_weights", "qoq_pack_codes", "qoq_unpack_weights",
     "qoq_quantize_act_per_token", "qoq_w4a8_gemm", "qoq_w4a8_gemm_i32",
     "qoq_w4a8_gemm_config", "qoq_w4a8_linear", "qoq_gemm_plan", "qoq_device_error",
+    "qoq_gemm_workspace_bytes", "qoq_gemm_workspace_bytes_config",
 )
 
 _lock = threading.Lock()
@@ -73,13 +74,17 @@ def lib() -> ctypes.CDLL:
             L.qoq_quantize_act_per_token.restype = I
             L.qoq_quantize_act_per_token.argtypes = [P, I, I, P, P, P]
             L.qoq_w4a8_gemm.restype = I
-            L.qoq_w4a8_gemm.argtypes = [P, P, P, P, I, I, I, I, P, P]
+            L.qoq_w4a8_gemm.argtypes = [P, P, P, P, I, I, I, I, P, P, sz, P]
             L.qoq_w4a8_gemm_i32.restype = I
-            L.qoq_w4a8_gemm_i32.argtypes = [P, P, I, I, I, I, P, P]
+            L.qoq_w4a8_gemm_i32.argtypes = [P, P, I, I, I, I, P, P, sz, P]
             L.qoq_w4a8_gemm_config.restype = I
-            L.qoq_w4a8_gemm_config.argtypes = [P, P, P, P, I, I, I, I, P, P, I, I, P]
+            L.qoq_w4a8_gemm_config.argtypes = [P, P, P, P, I, I, I, I, P, P, I, I, P, sz, P]
             L.qoq_w4a8_linear.restype = I
-            L.qoq_w4a8_linear.argtypes = [P, I, I, P, P, I, I, P, P, P, P]
+            L.qoq_w4a8_linear.argtypes = [P, I, I, P, P, I, I, P, P, P, P, sz, P]
+            L.qoq_gemm_workspace_bytes.restype = sz
+            L.qoq_gemm_workspace_bytes.argtypes = [I, I, I, I]
+            L.qoq_gemm_workspace_bytes_config.restype = sz
+            L.qoq_gemm_workspace_bytes_config.argtypes = [I, I, I, I, I, I]
             L.qoq_gemm_plan.restype = I
             L.qoq_gemm_plan.argtypes = [I, I, I, I] + [ctypes.POINTER(I)] * 4
             L.qoq_device_error.restype = I
@@ -137,6 +142,37 @@ def gemm_plan(M: int, N: int, K: int, group: int = 128) -> dict:
     _check(lib().qoq_gemm_plan(M, N, K, group, *[ctypes.byref(v) for v in vals]),
            "qoq_gemm_plan")
     return dict(zip(("tok_tile", "splits", "ctas", "stages"), (v.value for v in vals)))
+
+
+def gemm_workspace_bytes(M: int, N: int, K: int, group: int = 128, tok_tile: int = 0,
+                         splits: int = 0) -> int:
+    if tok_tile or splits:
+        return int(lib().qoq_gemm_workspace_bytes_config(M, N, K, group, tok_tile, splits))
+    return int(lib().qoq_gemm_workspace_bytes(M, N, K, group))
+
+
+_ws_cache = {}
+
+
+def workspace(nbytes: int, device):
+    """A reusable device workspace of at least `nbytes` bytes for this device
+    (one buffer per device, grown on demand; calls that share it must be
+    ordered on one stream)."""
+    import torch
+    if nbytes <= 0:
+        return None
+    key = torch.device(device).index
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        _ws_cache[key] = buf
+    return buf
+
+
+def _ws_args(ws):
+    if ws is None:
+        return None, 0
+    return ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size()
 
 
 def device_error(clear: bool = True) -> int:
@@ -213,30 +249,43 @@ def quantize_act_per_token(X, out=None, stream=None):
     return X8, sx
 
 
-def w4a8_gemm(X8, sx, packed, s1, N: int, group: int = 128, out=None, stream=None):
-    """Y = (X8 . dq^T) * sx[m] * s1[n] as float16 (M, N)."""
+_AUTO = object()
+
+
+def _auto_ws(ws, M, N, K, group, device, tok_tile=0, splits=0):
+    if ws is _AUTO:
+        return workspace(gemm_workspace_bytes(M, N, K, group, tok_tile, splits), device)
+    return ws
+
+
+def w4a8_gemm(X8, sx, packed, s1, N: int, group: int = 128, out=None, ws=_AUTO, stream=None):
+    """Y = (X8 . dq^T) * sx[m] * s1[n] as float16 (M, N).  `ws`: a uint8
+    device tensor for the split-K workspace (default: a cached one; None:
+    do not split K)."""
     import torch
     _need_cuda(X8, "X8", torch.int8, 2)
     M, K = X8.shape
     Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=X8.device)
+    w, wb = _ws_args(_auto_ws(ws, M, N, K, group, X8.device))
     _check(lib().qoq_w4a8_gemm(_ptr(X8), _ptr(sx), _ptr(packed), _ptr(s1), M, N, K, group,
-                               _ptr(Y), _stream(stream)), "qoq_w4a8_gemm")
+                               _ptr(Y), w, wb, _stream(stream)), "qoq_w4a8_gemm")
     return Y
 
 
-def w4a8_gemm_i32(X8, packed, N: int, group: int = 128, out=None, stream=None):
+def w4a8_gemm_i32(X8, packed, N: int, group: int = 128, out=None, ws=_AUTO, stream=None):
     """Raw INT32 accumulator acc = X8 . dq^T (M, N)."""
     import torch
     _need_cuda(X8, "X8", torch.int8, 2)
     M, K = X8.shape
     acc = out if out is not None else torch.empty((M, N), dtype=torch.int32, device=X8.device)
-    _check(lib().qoq_w4a8_gemm_i32(_ptr(X8), _ptr(packed), M, N, K, group, _ptr(acc),
+    w, wb = _ws_args(_auto_ws(ws, M, N, K, group, X8.device))
+    _check(lib().qoq_w4a8_gemm_i32(_ptr(X8), _ptr(packed), M, N, K, group, _ptr(acc), w, wb,
                                    _stream(stream)), "qoq_w4a8_gemm_i32")
     return acc
 
 
 def w4a8_gemm_config(X8, sx, packed, s1, N: int, group: int = 128, *, tok_tile=0, splits=0,
-                     int32_out=False, out=None, stream=None):
+                     int32_out=False, out=None, ws=_AUTO, stream=None):
     """The GEMM with an explicit token tile / split count (0 = auto)."""
     import torch
     _need_cuda(X8, "X8", torch.int8, 2)
@@ -247,13 +296,15 @@ def w4a8_gemm_config(X8, sx, packed, s1, N: int, group: int = 128, *, tok_tile=0
     else:
         Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=X8.device)
         acc = None
+    w, wb = _ws_args(_auto_ws(ws, M, N, K, group, X8.device, tok_tile, splits))
     _check(lib().qoq_w4a8_gemm_config(_ptr(X8), _ptr(sx), _ptr(packed), _ptr(s1), M, N, K, group,
-                                      _ptr(Y), _ptr(acc), tok_tile, splits, _stream(stream)),
-           "qoq_w4a8_gemm_config")
+                                      _ptr(Y), _ptr(acc), tok_tile, splits, w, wb,
+                                      _stream(stream)), "qoq_w4a8_gemm_config")
     return acc if int32_out else Y
 
 
-def w4a8_linear(X, packed, s1, N: int, group: int = 128, out=None, scratch=None, stream=None):
+def w4a8_linear(X, packed, s1, N: int, group: int = 128, out=None, scratch=None, ws=_AUTO,
+                stream=None):
     """Y = X . W^T: per-token activation quantization + W4A8 GEMM in one call
     (the GEMM overlaps the quantizer's tail).  ``scratch`` = (X8, sx)."""
     import torch
@@ -265,8 +316,9 @@ def w4a8_linear(X, packed, s1, N: int, group: int = 128, out=None, scratch=None,
     else:
         X8, sx = scratch
     Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=X.device)
+    w, wb = _ws_args(_auto_ws(ws, M, N, K, group, X.device))
     _check(lib().qoq_w4a8_linear(_ptr(X), M, K, _ptr(packed), _ptr(s1), N, group, _ptr(X8),
-                                 _ptr(sx), _ptr(Y), _stream(stream)), "qoq_w4a8_linear")
+                                 _ptr(sx), _ptr(Y), w, wb, _stream(stream)), "qoq_w4a8_linear")
     return Y
 
 

@@ -1,7 +1,7 @@
 // Device-side building blocks for the sm_100a W4A8 kernels: inline-PTX
 // wrappers for mbarriers (with bounded waits), bulk / tensor TMA copies,
-// tcgen05 tensor-memory allocation, MMA, commit and loads, cluster
-// distributed shared memory, and the byte-lane dequantization arithmetic.
+// tcgen05 tensor-memory allocation, MMA, commit, loads and stores,
+// programmatic dependent launch, and the byte-lane dequantization arithmetic.
 #pragma once
 
 #include <cuda.h>
@@ -16,7 +16,7 @@ enum : uint32_t {
   kErrMma = 2u,
   kErrDequant = 4u,
   kErrEpilogue = 8u,
-  kErrCluster = 16u,
+  kErrCounter = 16u,
 };
 
 // Every mbarrier wait gives up after this many nanoseconds of device time.
@@ -48,13 +48,6 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-// Arrive on a barrier that may live in another CTA of the cluster
-// (`bar` is a shared::cluster address), with cluster-scope release.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar)
-               : "memory");
-}
-
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
                "r"(bytes)
@@ -73,30 +66,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Wait for the phase of parity `parity` to complete.  Gives up (returns
 // false) when the CTA-wide abort flag is raised or after kWaitLimitNs, in
 // which case it raises the abort flag and records `err_bit` in `err_word`
 // (the library's device error word).  Never spins forever.
-template <bool kClusterScope = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile uint32_t* abort_flag,
                                           unsigned int* err_word, uint32_t err_bit) {
-  auto poll = [&]() {
-    return kClusterScope ? mbar_try_wait_cluster(bar, parity)
-                         : mbar_try_wait(bar, parity);
-  };
+  auto poll = [&]() { return mbar_try_wait(bar, parity); };
   if (poll()) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -278,35 +255,6 @@ __host__ __device__ constexpr uint32_t idesc_i8(int m, int n) {
          | (1u << 10)                               // B: signed 8-bit
          | (static_cast<uint32_t>(n >> 3) << 17)    // N / 8
          | (static_cast<uint32_t>(m >> 4) << 24);   // M / 16
-}
-
-// ----------------------------------------------------------------------------
-// Cluster helpers
-// ----------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
-
-__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t caddr) {
-  uint4 v;
-  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(caddr)
-               : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // ----------------------------------------------------------------------------

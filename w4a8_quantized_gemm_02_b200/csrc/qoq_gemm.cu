@@ -7,27 +7,29 @@
 // Background (per-group W4A4 dequantizes INT32 partial sums in its main loop,
 // this kernel scales once, after the whole K reduction).
 //
-// One CTA computes a 128-channel x TOK-token output tile over a range of
-// K (the weights are the MMA's M operand, the tokens its N operand, so a
-// single decode token still fills the 128-row tensor-core tile):
+// One CTA computes a 128-channel x TOK-token output tile over a range of K.
+// The weights are the MMA's M operand and the tokens its N operand, so a
+// single decode token still fills the 128-row tensor-core tile.
 //   warp 0      TMA producer: one bulk copy of the packed weight block and one
 //               tensor-map copy of the X8 tile (128-byte swizzle) per k-tile,
 //               into a ring of shared-memory stages;
 //   warp 1      owns tensor memory and issues tcgen05.mma.kind::i8 (M = 128,
-//               N = TOK, K = 32 per instruction, 4 per k-tile), INT32
-//               accumulators in tensor memory;
-//   warps 2..5  dequantize the UINT4 block into the INT8 operand tile (four
-//               byte lanes per 32-bit multiply-add, written in the 128-byte
-//               swizzle the MMA descriptor expects), then run the epilogue:
-//               tcgen05.ld of their 32-lane quarter, one FP32 scale per
-//               element, FP16 stores.
-// When K is split over several CTAs, they form a thread-block cluster and
-// the partial INT32 tiles are added exactly into the rank-0 CTA's shared
-// memory (red.shared::cluster) before its epilogue.
+//               N = TOK, K = 32 per instruction, 4 per k-tile) with the INT8
+//               weights read from tensor memory and X8 from shared memory,
+//               INT32 accumulators in tensor memory;
+//   warps 2..9  two dequantizing warpgroups taking alternate k-tiles: each
+//               thread turns one weight row of the UINT4 block into INT8 (four
+//               byte lanes per 32-bit multiply-add) and writes the 128-byte
+//               row into tensor memory with one tcgen05.st; afterwards the
+//               same warps run the epilogue.
+// When K is split over several CTAs, each writes its INT32 partial tile to the
+// caller's workspace and the last one to arrive (an epoch-tagged counter per
+// output tile) adds them up exactly and runs the epilogue.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "qoq.h"
@@ -40,9 +42,11 @@ __device__ unsigned int g_error_word = 0;
 
 namespace {
 
-constexpr int kThreads = 192;        // 6 warps
+constexpr int kThreads = 320;        // 10 warps
+constexpr int kEpiThreads = 256;     // warps 2..9
 constexpr int kRawStageBytes = 8576; // largest packed block (group 64), 16-byte multiple
 constexpr int kSmemPerSm = 233472;   // 228 KiB of shared memory per SM
+constexpr uint32_t kCasLimit = 1u << 20;
 
 template <int TOK>
 struct Cfg {
@@ -61,8 +65,7 @@ struct Cfg {
   static constexpr int kTmemD = 32 * kDqStages;
   static constexpr int kTmemCols = (kTmemD + TOK <= 256) ? 256 : 512;
   // Never more CTAs on an SM than tensor memory holds: request enough shared
-  // memory that one more CTA cannot fit (a CTA blocked in tcgen05.alloc next
-  // to a cluster peer would otherwise wait for it forever).
+  // memory that one more CTA cannot fit, so tcgen05.alloc never has to wait.
   static constexpr int kCtasPerSm = 512 / kTmemCols;
   static constexpr int kSmemFloor = kSmemPerSm / (kCtasPerSm + 1);
   static constexpr int kSmemBytes = kSmemUsed > kSmemFloor ? kSmemUsed : kSmemFloor;
@@ -81,9 +84,12 @@ struct GemmArgs {
   const __half* s1;
   __half* Y;
   int32_t* acc;
+  int32_t* ws_part;     // [m_tile][split][TOK][N] partial sums (splits > 1)
+  uint32_t* ws_count;   // [m_tile][n_tile] epoch-tagged arrival counters
   int M, N, K, group;
   int splits;
   int blk_bytes;
+  uint32_t epoch;       // 24-bit launch tag
 };
 
 // Bounded wait that ignores the abort flag: used only to drain work already
@@ -98,8 +104,37 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
+__device__ __forceinline__ void epi_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+}
+
 __device__ __forceinline__ uint4 add4(uint4 a, uint4 b) {
   return make_uint4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
+__device__ __forceinline__ uint4 ld_cg_v4(const int32_t* p) {
+  return __ldcg(reinterpret_cast<const uint4*>(p));
+}
+
+// Register this CTA's arrival at its output tile.  Returns true for the last
+// of `splits` arrivals of the launch tagged `epoch`.  The counter word is
+// (epoch << 8) | count; a word left by another launch (another epoch) starts a
+// new count, and the last arrival resets the count so that a replay of the
+// same launch (same epoch) starts from zero again.
+__device__ bool arrive_last(uint32_t* ctr, uint32_t epoch, int splits) {
+  uint32_t cur = *reinterpret_cast<volatile uint32_t*>(ctr);
+  for (uint32_t it = 0; it < kCasLimit; ++it) {
+    const uint32_t next = ((cur >> 8) == epoch) ? cur + 1u : ((epoch << 8) | 1u);
+    const uint32_t prev = atomicCAS(ctr, cur, next);
+    if (prev == cur) {
+      const bool last = static_cast<int>(next & 0xffu) == splits;
+      if (last) atomicExch(ctr, epoch << 8);
+      return last;
+    }
+    cur = prev;
+  }
+  atomicOr(&g_error_word, kErrCounter);
+  return false;
 }
 
 template <int TOK>
@@ -115,8 +150,9 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   const int lane = threadIdx.x & 31;
   const int splits = args.splits;
   const int nt = blockIdx.x / splits;
-  const int split = blockIdx.x - nt * splits;   // cluster rank when splits > 1
-  const int m0 = blockIdx.y * TOK;
+  const int split = blockIdx.x - nt * splits;
+  const int mt = blockIdx.y;
+  const int m0 = mt * TOK;
   const int kt_total = args.K / kTileK;
   const int kt_begin = (split * kt_total) / splits;
   const int num_kt = ((split + 1) * kt_total) / splits - kt_begin;
@@ -128,6 +164,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   const uint32_t bar_acc = bar_dqempty + 8 * C::kDqStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc + 4);
+  volatile uint32_t* last_flag = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc + 8);
   float* sx_s = reinterpret_cast<float*>(smem + C::kOffSx);
 
   if (threadIdx.x == 0) {
@@ -141,6 +178,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     }
     mbar_init(bar_acc, 1);
     *abort_flag = 0u;
+    *last_flag = 0u;
     fence_mbar_init();
     prefetch_tensormap(&tmap_x);
   }
@@ -151,7 +189,6 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  if (splits > 1) cluster_sync_all();   // peers are running before any DSMEM access
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
 
@@ -221,12 +258,13 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
       drain_wait(bar_acc, 0);              // no MMA in flight past this point
     }
   } else {
-    // ---------------------------------------------------------------- dequantizer
+    // ---------------------------------------------------------------- dequantizers
+    const int wg = (warp - 2) >> 2;        // warpgroup: even or odd k-tiles
     const int q4 = warp & 3;               // tensor-memory lane quarter of this warp
     const int r = q4 * 32 + lane;          // weight row (output channel) within the tile
     const uint32_t row_tmem = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int gpt = kTileK / args.group;
-    for (int i = 0; i < num_kt; ++i) {
+    for (int i = wg; i < num_kt; i += 2) {
       const int s = i % C::kStages, d = i % C::kDqStages;
       if (!mbar_wait(bar_full + 8 * s, (i / C::kStages) & 1, abort_flag, &g_error_word,
                      kErrDequant)) {
@@ -278,10 +316,12 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   }
 
   // ------------------------------------------------------------------ epilogue
-  // 1) accumulator -> this CTA's slot [token column][row] (INT32)
+  // 1) accumulator -> slot [token column][row] (INT32) in the X ring
   uint32_t* slot = reinterpret_cast<uint32_t*>(smem + C::kOffX);
   const bool epi = warp >= 2;
+  const int et = threadIdx.x - 64;         // epilogue thread 0..255
   if (epi) {
+    const int wg = (warp - 2) >> 2;
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const bool have = ok && mbar_wait(bar_acc, 0, abort_flag, &g_error_word, kErrEpilogue);
@@ -289,7 +329,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     if (__all_sync(0xffffffffu, have && (*abort_flag == 0u))) {
       const uint32_t t_row = tmem + C::kTmemD + (static_cast<uint32_t>(q4 * 32) << 16);
 #pragma unroll 1
-      for (int c0 = 0; c0 < TOK; c0 += 16) {
+      for (int c0 = 16 * wg; c0 < TOK; c0 += 32) {
         uint32_t v[16];
         tmem_ld_32x32b_x16(t_row + c0, v);
         tmem_ld_wait();
@@ -299,26 +339,39 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     }
     if (args.Y) {
       grid_dependency_wait();   // sx comes from the preceding grid under PDL
-      for (int c = threadIdx.x - 64; c < TOK; c += 128) {
+      for (int c = et; c < TOK; c += kEpiThreads) {
         const int m = m0 + c;
         sx_s[c] = m < args.M ? __half2float(args.sx[m]) : 0.0f;
       }
     }
-  }
-  __syncwarp();
-  if (splits > 1) {
-    cluster_sync_all();
-  } else {
-    __syncthreads();
+    epi_bar();
   }
 
-  // 2) sum the partial tiles of all K splits (DSMEM) and store: each rank owns
-  //    the token columns c = rank (mod splits); a thread owns 4 consecutive rows
-  if (epi && *abort_flag == 0u) {
-    const int we = warp - 2;
-    const int rq = 4 * lane;
-    const int n = nt * kTileN + rq;
-    const int M = args.M, N = args.N;
+  // 2) thread et owns rows 4*(et%32) .. +3 and token columns c = et/32 (mod 8)
+  const int M = args.M, N = args.N;
+  const int rq = 4 * (et & 31);
+  const int n = nt * kTileN + rq;
+  const int c_first = et >> 5;
+  int c_end = M - m0;
+  if (c_end > TOK) c_end = TOK;
+  if (epi && splits > 1) {
+    // publish this split's partial tile, then count the arrival
+    int32_t* part = args.ws_part + (static_cast<size_t>(mt * splits + split) * TOK) * N + n;
+    for (int c = c_first; c < c_end; c += 8) {
+      const uint4 v = *reinterpret_cast<const uint4*>(slot + c * kTileN + rq);
+      __stcg(reinterpret_cast<uint4*>(part + static_cast<size_t>(c) * N), v);
+    }
+    __threadfence();
+    epi_bar();
+    if (et == 0) {
+      const bool last = arrive_last(args.ws_count + mt * (N / kTileN) + nt, args.epoch, splits);
+      *last_flag = last ? 1u : 0u;
+    }
+    epi_bar();
+    __threadfence();
+  }
+  const bool writer = epi && (*abort_flag == 0u) && (splits == 1 || *last_flag != 0u);
+  if (writer) {
     float s1q[4] = {0.f, 0.f, 0.f, 0.f};
     if (args.Y) {
       const uint2 sv = *reinterpret_cast<const uint2*>(args.s1 + n);
@@ -329,17 +382,15 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
       s1q[2] = b.x;
       s1q[3] = b.y;
     }
-    const uint32_t slot_addr = base + C::kOffX;
-    for (int c = split + splits * we; c < TOK; c += 4 * splits) {
-      const int m = m0 + c;
-      if (m >= M) break;
-      const int e = c * kTileN + rq;
-      uint4 v = *reinterpret_cast<const uint4*>(slot + e);
+    const int32_t* parts = args.ws_part + (static_cast<size_t>(mt * splits) * TOK) * N + n;
+#pragma unroll 4
+    for (int c = c_first; c < c_end; c += 8) {
+      uint4 v = *reinterpret_cast<const uint4*>(slot + c * kTileN + rq);
       for (int q = 0; q < splits; ++q) {
         if (q == split) continue;
-        v = add4(v, ld_cluster_v4(map_to_rank(slot_addr + 4u * e, q)));
+        v = add4(v, ld_cg_v4(parts + (static_cast<size_t>(q) * TOK + c) * N));
       }
-      const size_t o = static_cast<size_t>(m) * N + n;
+      const size_t o = static_cast<size_t>(m0 + c) * N + n;
       if (args.acc) {
         *reinterpret_cast<uint4*>(args.acc + o) = v;
       } else {
@@ -357,8 +408,6 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
       }
     }
   }
-  __syncwarp();
-  if (splits > 1) cluster_sync_all();   // peers keep their slots until every rank has read them
 
   // ------------------------------------------------------------------ teardown
   tc_fence_before_sync();
@@ -392,6 +441,16 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+std::atomic<uint32_t> g_epoch{0};
+
+uint32_t next_epoch() {
+  uint32_t e;
+  do {
+    e = (g_epoch.fetch_add(1, std::memory_order_relaxed) + 1u) & 0xffffffu;
+  } while (e == 0);
+  return e;
+}
+
 struct Plan {
   int tok, splits, m_tiles, n_tiles, stages;
 };
@@ -400,39 +459,44 @@ int stages_for(int tok) { return tok <= 32 ? 8 : (tok <= 64 ? 6 : 4); }
 
 bool valid_tok(int t) { return t == 16 || t == 32 || t == 64 || t == 128 || t == 256; }
 
+int auto_tok(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
+
+int ctas_per_sm(int tok) { return tok <= 128 ? 2 : 1; }
+
+int auto_splits(int tiles, int kt, int tok) {
+  const long slots = static_cast<long>(sm_count()) * ctas_per_sm(tok);
+  int best_s = 1;
+  if (tiles >= slots) return 1;
+  double best = 0.0;
+  for (int s = 1; s <= 8 && s <= kt; ++s) {
+    if (s > 1 && kt / s < 4) break;
+    const long ctas = static_cast<long>(tiles) * s;
+    const long waves = (ctas + slots - 1) / slots;
+    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
+    if (eff > best + 1e-9) {
+      best = eff;
+      best_s = s;
+    }
+  }
+  return best_s;
+}
+
 Plan make_plan(int M, int N, int K, int tok_req, int splits_req) {
   Plan p;
   p.n_tiles = N / kTileN;
   const int kt = K / kTileK;
-  if (tok_req) {
-    p.tok = tok_req;
-  } else {
-    p.tok = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
-  }
+  p.tok = tok_req ? tok_req : auto_tok(M);
   p.m_tiles = (M + p.tok - 1) / p.tok;
   p.stages = stages_for(p.tok);
-  if (splits_req) {
-    p.splits = splits_req;
-  } else {
-    const int occ = p.tok <= 128 ? 2 : 1;
-    const long slots = static_cast<long>(sm_count()) * occ;
-    const long tiles = static_cast<long>(p.n_tiles) * p.m_tiles;
-    p.splits = 1;
-    if (tiles < slots) {
-      double best = 0.0;
-      for (int s = 1; s <= 8 && s <= kt; ++s) {
-        if (s > 1 && kt / s < 2) break;
-        const long ctas = tiles * s;
-        const long waves = (ctas + slots - 1) / slots;
-        const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
-        if (eff > best + 1e-9) {
-          best = eff;
-          p.splits = s;
-        }
-      }
-    }
-  }
+  p.splits = splits_req ? splits_req : auto_splits(p.n_tiles * p.m_tiles, kt, p.tok);
   return p;
+}
+
+size_t ws_bytes_for(const Plan& p, int N) {
+  if (p.splits <= 1) return 0;
+  const size_t part = static_cast<size_t>(p.m_tiles) * p.splits * p.tok * N * 4;
+  const size_t count = static_cast<size_t>(p.m_tiles) * p.n_tiles * 4;
+  return ((part + 255) / 256) * 256 + ((count + 255) / 256) * 256;
 }
 
 template <int TOK>
@@ -454,15 +518,11 @@ int launch_tok(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cudaStr
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(p.splits);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 2 : 1;
+  cfg.numAttrs = pdl ? 1 : 0;
   if (cudaLaunchKernelEx(&cfg, w4a8_gemm_kernel<TOK>, map, a) != cudaSuccess) return QOQ_ERR_CUDA;
   return QOQ_OK;
 }
@@ -470,25 +530,29 @@ int launch_tok(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cudaStr
 }  // namespace
 
 int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* s1, int M, int N,
-              int K, int group, void* Y, int32_t* acc, int tok_req, int splits_req,
-              void* stream, bool pdl) {
+              int K, int group, void* Y, int32_t* acc, int tok_req, int splits_req, void* ws,
+              size_t ws_bytes, void* stream, bool pdl) {
   if (!X8 || !packed) return QOQ_ERR_INVALID_ARG;
   if ((Y == nullptr) == (acc == nullptr)) return QOQ_ERR_INVALID_ARG;
   if (Y && (!sx || !s1)) return QOQ_ERR_INVALID_ARG;
   if (M <= 0) return QOQ_ERR_INVALID_ARG;
   if (int st = check_weight_shape(N, K, group)) return st;
   if (!aligned16(X8) || !aligned16(packed) || (Y && !aligned16(Y)) || (acc && !aligned16(acc)) ||
-      (sx && !aligned16(sx)) || (s1 && !aligned16(s1)))
+      (sx && !aligned16(sx)) || (s1 && !aligned16(s1)) || (ws && !aligned16(ws)))
     return QOQ_ERR_INVALID_ARG;
   if (tok_req && !valid_tok(tok_req)) return QOQ_ERR_INVALID_ARG;
   if (splits_req && (splits_req < 1 || splits_req > 8 || splits_req > K / kTileK))
     return QOQ_ERR_INVALID_ARG;
+
+  Plan p = make_plan(M, N, K, tok_req, splits_req);
+  if (p.m_tiles > 65535) return QOQ_ERR_UNSUPPORTED;
+  if (p.splits > 1 && (ws == nullptr || ws_bytes < ws_bytes_for(p, N))) {
+    if (splits_req) return QOQ_ERR_INVALID_ARG;   // explicit split needs its workspace
+    p.splits = 1;                                  // auto plan: do not split K
+  }
   if (int st = check_device()) return st;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return QOQ_ERR_CUDA;
-
-  const Plan p = make_plan(M, N, K, tok_req, splits_req);
-  if (p.m_tiles > 65535) return QOQ_ERR_UNSUPPORTED;
 
   CUtensorMap map;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
@@ -506,12 +570,20 @@ int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* 
   a.s1 = static_cast<const __half*>(s1);
   a.Y = static_cast<__half*>(Y);
   a.acc = acc;
+  a.ws_part = nullptr;
+  a.ws_count = nullptr;
+  if (p.splits > 1) {
+    const size_t part = static_cast<size_t>(p.m_tiles) * p.splits * p.tok * N * 4;
+    a.ws_part = static_cast<int32_t*>(ws);
+    a.ws_count = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + ((part + 255) / 256) * 256);
+  }
   a.M = M;
   a.N = N;
   a.K = K;
   a.group = group;
   a.splits = p.splits;
   a.blk_bytes = static_cast<int>(block_bytes(group));
+  a.epoch = next_epoch();
 
   cudaStream_t s = as_stream(stream);
   switch (p.tok) {
@@ -523,41 +595,66 @@ int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* 
   }
 }
 
+size_t gemm_ws_bytes(int M, int N, int K, int tok_req, int splits_req) {
+  return ws_bytes_for(make_plan(M, N, K, tok_req, splits_req), N);
+}
+
 }  // namespace qoq
 
 using namespace qoq;
 
+extern "C" size_t qoq_gemm_workspace_bytes(int M, int N, int K, int group) {
+  if (M <= 0 || check_weight_shape(N, K, group) != QOQ_OK) return 0;
+  return gemm_ws_bytes(M, N, K, 0, 0);
+}
+
+extern "C" size_t qoq_gemm_workspace_bytes_config(int M, int N, int K, int group, int tok_tile,
+                                                  int splits) {
+  if (M <= 0 || check_weight_shape(N, K, group) != QOQ_OK) return 0;
+  if (tok_tile && !valid_tok(tok_tile)) return 0;
+  if (splits < 0 || splits > 8 || splits > K / kTileK) return 0;
+  return gemm_ws_bytes(M, N, K, tok_tile, splits);
+}
+
 extern "C" int qoq_w4a8_gemm(const int8_t* X8, const void* sx, const void* packed, const void* s1,
-                             int M, int N, int K, int group, void* Y, void* stream) {
+                             int M, int N, int K, int group, void* Y, void* ws, size_t ws_bytes,
+                             void* stream) {
   if (!Y) return QOQ_ERR_INVALID_ARG;
-  return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, nullptr, 0, 0, stream, false);
+  return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, nullptr, 0, 0, ws, ws_bytes, stream,
+                   false);
 }
 
 extern "C" int qoq_w4a8_gemm_i32(const int8_t* X8, const void* packed, int M, int N, int K,
-                                 int group, int32_t* acc, void* stream) {
+                                 int group, int32_t* acc, void* ws, size_t ws_bytes,
+                                 void* stream) {
   if (!acc) return QOQ_ERR_INVALID_ARG;
-  return gemm_impl(X8, nullptr, packed, nullptr, M, N, K, group, nullptr, acc, 0, 0, stream, false);
+  return gemm_impl(X8, nullptr, packed, nullptr, M, N, K, group, nullptr, acc, 0, 0, ws, ws_bytes,
+                   stream, false);
 }
 
 extern "C" int qoq_w4a8_gemm_config(const int8_t* X8, const void* sx, const void* packed,
                                     const void* s1, int M, int N, int K, int group, void* Y,
-                                    int32_t* acc, int tok_tile, int splits, void* stream) {
-  return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, acc, tok_tile, splits, stream, false);
+                                    int32_t* acc, int tok_tile, int splits, void* ws,
+                                    size_t ws_bytes, void* stream) {
+  return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, acc, tok_tile, splits, ws, ws_bytes,
+                   stream, false);
 }
 
 extern "C" int qoq_w4a8_linear(const void* X, int M, int K, const void* packed, const void* s1,
-                               int N, int group, int8_t* X8, void* sx, void* Y, void* stream) {
+                               int N, int group, int8_t* X8, void* sx, void* Y, void* ws,
+                               size_t ws_bytes, void* stream) {
   if (!X || !X8 || !sx || !Y || !packed || !s1) return QOQ_ERR_INVALID_ARG;
   if (M <= 0) return QOQ_ERR_INVALID_ARG;
   if (int st = check_weight_shape(N, K, group)) return st;
   if (!aligned16(X) || !aligned16(X8) || !aligned16(sx) || !aligned16(Y) || !aligned16(packed) ||
-      !aligned16(s1))
+      !aligned16(s1) || (ws && !aligned16(ws)))
     return QOQ_ERR_INVALID_ARG;
   if (int st = check_device()) return st;
   if (int st = launch_act_quant(X, M, K, X8, sx, stream)) return st;
   // both kernels are this library's: the GEMM reads nothing the quantizer
   // writes before its grid-dependency wait, so it may overlap its tail
-  return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, nullptr, 0, 0, stream, true);
+  return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, nullptr, 0, 0, ws, ws_bytes, stream,
+                   true);
 }
 
 extern "C" int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int* splits, int* ctas,

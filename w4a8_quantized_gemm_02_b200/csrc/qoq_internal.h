@@ -47,8 +47,8 @@ int launch_status();
 // start while the preceding kernel on the stream is still running: it then
 // streams weights right away and waits for that grid before reading X8 / sx.
 int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* s1, int M, int N,
-              int K, int group, void* Y, int32_t* acc, int tok_req, int splits_req,
-              void* stream, bool pdl);
+              int K, int group, void* Y, int32_t* acc, int tok_req, int splits_req, void* ws,
+              size_t ws_bytes, void* stream, bool pdl);
 
 // Launch the per-token activation quantizer (no argument checks).
 int launch_act_quant(const void* X, int M, int K, int8_t* X8, void* sx, void* stream);
