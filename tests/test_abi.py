@@ -119,10 +119,10 @@ def test_other_entry_validation(L):
 
 def test_workspace_sizes(L):
     assert qoq.gemm_workspace_bytes(16, 512, 512, 128, 16, 1) == 0
-    # partials [m_tiles][splits][tok][N] int32 + counters, 256-byte rounded
-    assert qoq.gemm_workspace_bytes(16, 512, 512, 128, 16, 2) == 2 * 16 * 512 * 4 + 256
+    # 16 KiB of counters + partials [m_tiles][splits][tok][N] int32
+    assert qoq.gemm_workspace_bytes(16, 512, 512, 128, 16, 2) == 16384 + 2 * 16 * 512 * 4
     assert qoq.gemm_workspace_bytes(40, 512, 512, 128, 16, 4) == \
-        3 * 4 * 16 * 512 * 4 + 256
+        16384 + 3 * 4 * 16 * 512 * 4
     assert qoq.gemm_workspace_bytes(0, 512, 512, 128) == 0
     p = qoq.gemm_plan(1, 6144, 4096, 128)
     ws = qoq.gemm_workspace_bytes(1, 6144, 4096, 128)

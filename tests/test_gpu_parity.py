@@ -313,6 +313,37 @@ def test_linear_entry_matches_two_calls(oracle, tiny, tiny_dev, M):
     check_y(host(Y), Yr)
 
 
+def test_shared_workspace_across_shapes(oracle):
+    """One zero-initialized workspace reused by split-K launches of different
+    shapes, interleaved: every accumulator stays exact (a tile's arrival
+    counter never shares memory with another launch's partial sums)."""
+    ws = torch.zeros(32 << 20, dtype=torch.uint8, device=DEV)
+    cases = [(16, 512, 1024, 16, 4), (64, 384, 2048, 64, 8), (1, 256, 1024, 16, 8),
+             (40, 512, 1024, 32, 2), (200, 256, 2048, 128, 3)]
+    prepared = []
+    for i, (M, N, K, tok, sp) in enumerate(cases):
+        ops = si.sweep_operands(M, N, K, 128, seed=100 + i)
+        dq = oracle.dequant_w(ops.q, ops.s2, ops.z, 128)
+        acc_ref = oracle.int_gemm(ops.X8, dq)
+        y_ref = oracle.epilogue(acc_ref, ops.sx, ops.s1)
+        packed = qoq.pack_codes(to_dev(ops.q), to_dev(ops.s2), to_dev(ops.z), 128)
+        prepared.append((ops, packed, acc_ref, y_ref))
+    for rep in range(4):
+        order = list(range(len(cases)))[::(1 if rep % 2 == 0 else -1)]
+        for i in order:
+            M, N, K, tok, sp = cases[i]
+            ops, packed, acc_ref, y_ref = prepared[i]
+            assert qoq.gemm_workspace_bytes(M, N, K, 128, tok, sp) <= ws.numel()
+            X8 = to_dev(ops.X8)
+            acc = qoq.w4a8_gemm_config(X8, None, packed, None, N, 128, tok_tile=tok, splits=sp,
+                                       int32_out=True, ws=ws)
+            Y = qoq.w4a8_gemm_config(X8, to_dev(ops.sx), packed, to_dev(ops.s1), N, 128,
+                                     tok_tile=tok, splits=sp, ws=ws)
+            torch.cuda.synchronize()
+            assert np.array_equal(host(acc), acc_ref), (rep, cases[i])
+            check_y(host(Y), y_ref)
+
+
 def test_gemm_stream_and_repeat(tiny, tiny_dev):
     """Back-to-back launches on a side stream give identical results."""
     packed, s1 = tiny_dev

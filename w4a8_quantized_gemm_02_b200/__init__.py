@@ -155,16 +155,16 @@ _ws_cache = {}
 
 
 def workspace(nbytes: int, device):
-    """A reusable device workspace of at least `nbytes` bytes for this device
-    (one buffer per device, grown on demand; calls that share it must be
-    ordered on one stream)."""
+    """A reusable, zero-initialized device workspace of at least `nbytes`
+    bytes for this device (one buffer per device, grown on demand; calls that
+    share it must be ordered on one stream)."""
     import torch
     if nbytes <= 0:
         return None
     key = torch.device(device).index
     buf = _ws_cache.get(key)
     if buf is None or buf.numel() < nbytes:
-        buf = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
         _ws_cache[key] = buf
     return buf
 

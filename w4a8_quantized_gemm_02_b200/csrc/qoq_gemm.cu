@@ -47,6 +47,11 @@ constexpr int kEpiThreads = 256;     // warps 2..9
 constexpr int kRawStageBytes = 8576; // largest packed block (group 64), 16-byte multiple
 constexpr int kSmemPerSm = 233472;   // 228 KiB of shared memory per SM
 constexpr uint32_t kCasLimit = 1u << 20;
+// The workspace starts with a fixed region of arrival counters (one word per
+// output tile), so that counter words never share memory with the partial
+// sums of a launch of another shape.
+constexpr int kMaxCounterTiles = 4096;
+constexpr size_t kCounterBytes = kMaxCounterTiles * 4;
 
 template <int TOK>
 struct Cfg {
@@ -85,7 +90,7 @@ struct GemmArgs {
   __half* Y;
   int32_t* acc;
   int32_t* ws_part;     // [m_tile][split][TOK][N] partial sums (splits > 1)
-  uint32_t* ws_count;   // [m_tile][n_tile] epoch-tagged arrival counters
+  uint32_t* ws_count;   // [m_tile][n_tile] epoch-tagged arrival counters (fixed region)
   int M, N, K, group;
   int splits;
   int blk_bytes;
@@ -118,7 +123,8 @@ __device__ __forceinline__ uint4 ld_cg_v4(const int32_t* p) {
 
 // Register this CTA's arrival at its output tile.  Returns true for the last
 // of `splits` arrivals of the launch tagged `epoch`.  The counter word is
-// (epoch << 8) | count; a word left by another launch (another epoch) starts a
+// (epoch << 8) | count and only ever holds values written here (the region
+// starts zero-filled); a word left by another launch (another epoch) starts a
 // new count, and the last arrival resets the count so that a replay of the
 // same launch (same epoch) starts from zero again.
 __device__ bool arrive_last(uint32_t* ctr, uint32_t epoch, int splits) {
@@ -455,6 +461,10 @@ struct Plan {
   int tok, splits, m_tiles, n_tiles, stages;
 };
 
+bool splittable(const Plan& p) {
+  return static_cast<long>(p.m_tiles) * p.n_tiles <= kMaxCounterTiles;
+}
+
 int stages_for(int tok) { return tok <= 32 ? 8 : (tok <= 64 ? 6 : 4); }
 
 bool valid_tok(int t) { return t == 16 || t == 32 || t == 64 || t == 128 || t == 256; }
@@ -489,14 +499,14 @@ Plan make_plan(int M, int N, int K, int tok_req, int splits_req) {
   p.m_tiles = (M + p.tok - 1) / p.tok;
   p.stages = stages_for(p.tok);
   p.splits = splits_req ? splits_req : auto_splits(p.n_tiles * p.m_tiles, kt, p.tok);
+  if (!splits_req && !splittable(p)) p.splits = 1;
   return p;
 }
 
 size_t ws_bytes_for(const Plan& p, int N) {
   if (p.splits <= 1) return 0;
   const size_t part = static_cast<size_t>(p.m_tiles) * p.splits * p.tok * N * 4;
-  const size_t count = static_cast<size_t>(p.m_tiles) * p.n_tiles * 4;
-  return ((part + 255) / 256) * 256 + ((count + 255) / 256) * 256;
+  return kCounterBytes + part;
 }
 
 template <int TOK>
@@ -546,6 +556,10 @@ int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* 
 
   Plan p = make_plan(M, N, K, tok_req, splits_req);
   if (p.m_tiles > 65535) return QOQ_ERR_UNSUPPORTED;
+  if (p.splits > 1 && !splittable(p)) {
+    if (splits_req) return QOQ_ERR_UNSUPPORTED;
+    p.splits = 1;
+  }
   if (p.splits > 1 && (ws == nullptr || ws_bytes < ws_bytes_for(p, N))) {
     if (splits_req) return QOQ_ERR_INVALID_ARG;   // explicit split needs its workspace
     p.splits = 1;                                  // auto plan: do not split K
@@ -573,9 +587,8 @@ int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* 
   a.ws_part = nullptr;
   a.ws_count = nullptr;
   if (p.splits > 1) {
-    const size_t part = static_cast<size_t>(p.m_tiles) * p.splits * p.tok * N * 4;
-    a.ws_part = static_cast<int32_t*>(ws);
-    a.ws_count = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + ((part + 255) / 256) * 256);
+    a.ws_count = static_cast<uint32_t*>(ws);
+    a.ws_part = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kCounterBytes);
   }
   a.M = M;
   a.N = N;
@@ -596,7 +609,9 @@ int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* 
 }
 
 size_t gemm_ws_bytes(int M, int N, int K, int tok_req, int splits_req) {
-  return ws_bytes_for(make_plan(M, N, K, tok_req, splits_req), N);
+  const Plan p = make_plan(M, N, K, tok_req, splits_req);
+  if (!splittable(p)) return 0;
+  return ws_bytes_for(p, N);
 }
 
 }  // namespace qoq
