@@ -360,19 +360,6 @@ def run_ours(args):
                 qoq.w4a8_linear(xs[set_idx][j], weights[w], s1s[w], N, G, out=ys[j],
                                 scratch=(x8[j], sxb[j]), stream=stream)
 
-    def step_breakdown(set_idx, events):
-        """Every kernel between events: quantizer, GEMM, then the fused op."""
-        for j, M in enumerate(ms):
-            w = set_idx * len(ms) + j
-            events[3 * j].record(stream)
-            qoq.quantize_act_per_token(xs[set_idx][j], out=(x8[j], sxb[j]), stream=stream)
-            events[3 * j + 1].record(stream)
-            qoq.w4a8_gemm(x8[j], sxb[j], weights[w], s1s[w], N, G, out=ys[j], stream=stream)
-            events[3 * j + 2].record(stream)
-            qoq.w4a8_linear(xs[set_idx][j], weights[w], s1s[w], N, G, out=ys[j],
-                            scratch=(x8[j], sxb[j]), stream=stream)
-        events[3 * len(ms)].record(stream)
-
     # eager warm-up (first launches set kernel attributes), then capture
     with torch.cuda.stream(stream):
         for s_ in range(nsets):
@@ -393,14 +380,6 @@ def run_ours(args):
             step(g % nsets, evs)
         graphs.append(graph)
         graph_events.append(evs)
-    bgraphs, bevents = [], []
-    for g in range(nsets):
-        evs = [ev() for _ in range(3 * len(ms) + 1)]
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
-            step_breakdown(g, evs)
-        bgraphs.append(graph)
-        bevents.append(evs)
     torch.cuda.synchronize()
 
     # the captured step reproduces the eager one
@@ -449,20 +428,46 @@ def run_ours(args):
     dom_ms = [graph_events[(args.steps - 1 - g) % ngraphs][0].elapsed_time(
         graph_events[(args.steps - 1 - g) % ngraphs][1]) for g in range(n_used)]
 
-    # per-kernel breakdown (after the timed region, same rotation)
-    reps = 4
-    aq_ms = {M: [] for M in ms}
-    gemm_ms = {M: [] for M in ms}
-    lin_ms = {M: [] for M in ms}
-    for _ in range(reps):
-        for g in range(nsets):
-            bgraphs[g].replay()
-            torch.cuda.synchronize()
-            evs = bevents[g]
-            for j, M in enumerate(ms):
-                aq_ms[M].append(evs[3 * j].elapsed_time(evs[3 * j + 1]))
-                gemm_ms[M].append(evs[3 * j + 1].elapsed_time(evs[3 * j + 2]))
-                lin_ms[M].append(evs[3 * j + 2].elapsed_time(evs[3 * j + 3]))
+    # per-kernel breakdown (after the timed region): each kernel alone, R
+    # back-to-back launches in one graph over the rotated inputs
+    def per_launch_us(fn, reps=3):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            nlaunch = fn()
+        g.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        e1.synchronize()
+        del g
+        return e0.elapsed_time(e1) * 1e3 / (reps * nlaunch)
+
+    nw = len(weights)
+    aq_us, gemm_us, lin_us = {}, {}, {}
+    for j, M in enumerate(ms):
+        def aq():
+            for s_ in range(nsets):
+                qoq.quantize_act_per_token(xs[s_][j], out=(x8[j], sxb[j]), stream=stream)
+            return nsets
+
+        def gm():
+            for w in range(nw):
+                qoq.w4a8_gemm(x8[j], sxb[j], weights[w], s1s[w], N, G, out=ys[j], stream=stream)
+            return nw
+
+        def ln():
+            for w in range(nw):
+                qoq.w4a8_linear(xs[w % nsets][j], weights[w], s1s[w], N, G, out=ys[j],
+                                scratch=(x8[j], sxb[j]), stream=stream)
+            return nw
+        aq_us[M] = per_launch_us(aq)
+        gemm_us[M] = per_launch_us(gm)
+        lin_us[M] = per_launch_us(ln)
     assert qoq.device_error(clear=True) == 0
 
     peaks = load_peaks()
@@ -471,9 +476,9 @@ def run_ours(args):
     value = step_ops * args.steps * world / (elapsed_ms * 1e-3) / 1e12
     per_m = []
     for M in ms:
-        t = statistics.median(gemm_ms[M]) * 1e-3
-        ta = statistics.median(aq_ms[M]) * 1e-3
-        tl = statistics.median(lin_ms[M]) * 1e-3
+        t = gemm_us[M] * 1e-6
+        ta = aq_us[M] * 1e-6
+        tl = lin_us[M] * 1e-6
         plan = qoq.gemm_plan(M, N, K, G)
         per_m.append({
             "M": M, "gemm_us": t * 1e6, "act_quant_us": ta * 1e6, "linear_us": tl * 1e6,
@@ -524,6 +529,8 @@ def run_ours(args):
         "clocks": clocks,
         "gpu_launches": 2 * len(ms) * args.steps,
         "timed_region": "fused qoq_w4a8_linear per M (dominant M: quantizer + qoq_w4a8_gemm)",
+        "per_m_method": "each kernel alone: back-to-back launches in a CUDA graph over rotated "
+                        "inputs, device time / launches",
         "offline_pack_ms": pack_ms,
         "e2e": e2e,
     }
@@ -531,7 +538,7 @@ def run_ours(args):
         line["cpu_baseline"] = cpu_baseline(layer, args.cpu_budget_s)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graphs, bgraphs
+    del graphs
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

@@ -34,30 +34,15 @@ __device__ __forceinline__ int div_rne(int a, int b) {
   return q;
 }
 
-__device__ __forceinline__ float block_max(float v, float* red) {
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  if (warp == 0) {
-    v = (lane < static_cast<int>(blockDim.x >> 5)) ? red[lane] : 0.0f;
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    if (lane == 0) red[0] = v;
-  }
-  __syncthreads();
-  float r = red[0];
-  __syncthreads();
-  return r;
-}
-
 // ---------------------------------------------------------------------------
-// Per-token activation quantization: one CTA per row.  A row of up to
-// kActThreads * 8 * kActMaxVec values stays in registers between the
-// abs-max reduction and the quantization (one pass over X); longer rows are
-// read twice.
+// Per-token activation quantization: one warp per row, 8 rows per CTA.  The
+// first pass keeps many 16-byte loads in flight per lane and reduces the
+// abs-max with warp shuffles; the second pass re-reads the row (now in L2 /
+// L1) and writes the INT8 codes.  Rows of up to 32 * 8 * kActRegVec values
+// are kept in registers between the passes instead.
 // ---------------------------------------------------------------------------
-constexpr int kActThreads = 256;
-constexpr int kActMaxVec = 16;
+constexpr int kActWarps = 8;
+constexpr int kActRegVec = 16;
 
 __device__ __forceinline__ uint2 quantize8(uint4 v, float sf) {
   const __half2* h = reinterpret_cast<const __half2*>(&v);
@@ -86,43 +71,56 @@ __device__ __forceinline__ float absmax8(uint4 v, float amax) {
   return amax;
 }
 
-__global__ void __launch_bounds__(kActThreads)
-act_quant_kernel(const __half* __restrict__ X, int K, int8_t* __restrict__ X8,
+__global__ void __launch_bounds__(32 * kActWarps)
+act_quant_kernel(const __half* __restrict__ X, int M, int K, int8_t* __restrict__ X8,
                  __half* __restrict__ sx) {
   // the GEMM that consumes X8 may start its weight prologue right away
   grid_launch_dependents();
-  __shared__ float red[kActThreads / 32];
-  const int m = blockIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int m = blockIdx.x * kActWarps + (threadIdx.x >> 5);
+  if (m >= M) return;
   const uint4* row = reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K);
   uint2* out = reinterpret_cast<uint2*>(X8 + static_cast<size_t>(m) * K);
   const int nvec = K / 8;
-  const bool in_regs = nvec <= kActThreads * kActMaxVec;
-  uint4 v[kActMaxVec];
   float amax = 0.0f;
-  if (in_regs) {
+  if (nvec <= 32 * kActRegVec) {
+    uint4 v[kActRegVec];
 #pragma unroll
-    for (int u = 0; u < kActMaxVec; ++u) {
-      const int i = threadIdx.x + u * kActThreads;
-      if (i < nvec) {
-        v[u] = __ldg(row + i);
-        amax = absmax8(v[u], amax);
-      }
+    for (int u = 0; u < kActRegVec; ++u) {
+      const int i = lane + 32 * u;
+      if (i < nvec) v[u] = __ldg(row + i);
     }
-  } else {
-    for (int i = threadIdx.x; i < nvec; i += kActThreads) amax = absmax8(__ldg(row + i), amax);
-  }
-  amax = block_max(amax, red);
-  const __half s = scale_from_absmax(amax, 127.0f);
-  if (threadIdx.x == 0) sx[m] = s;
-  const float sf = __half2float(s);
-  if (in_regs) {
 #pragma unroll
-    for (int u = 0; u < kActMaxVec; ++u) {
-      const int i = threadIdx.x + u * kActThreads;
+    for (int u = 0; u < kActRegVec; ++u)
+      if (lane + 32 * u < nvec) amax = absmax8(v[u], amax);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const __half s = scale_from_absmax(amax, 127.0f);
+    if (lane == 0) sx[m] = s;
+    const float sf = __half2float(s);
+#pragma unroll
+    for (int u = 0; u < kActRegVec; ++u) {
+      const int i = lane + 32 * u;
       if (i < nvec) out[i] = quantize8(v[u], sf);
     }
   } else {
-    for (int i = threadIdx.x; i < nvec; i += kActThreads) out[i] = quantize8(__ldg(row + i), sf);
+    for (int i0 = 0; i0 < nvec; i0 += 32 * 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + lane + 32 * u;
+        if (i < nvec) v[u] = __ldg(row + i);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (i0 + lane + 32 * u < nvec) amax = absmax8(v[u], amax);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const __half s = scale_from_absmax(amax, 127.0f);
+    if (lane == 0) sx[m] = s;
+    const float sf = __half2float(s);
+    for (int i = lane; i < nvec; i += 32) out[i] = quantize8(__ldg(row + i), sf);
   }
 }
 
@@ -314,8 +312,8 @@ using namespace qoq;
 
 namespace qoq {
 int launch_act_quant(const void* X, int M, int K, int8_t* X8, void* sx, void* stream) {
-  act_quant_kernel<<<M, kActThreads, 0, as_stream(stream)>>>(
-      static_cast<const __half*>(X), K, X8, static_cast<__half*>(sx));
+  act_quant_kernel<<<(M + kActWarps - 1) / kActWarps, 32 * kActWarps, 0, as_stream(stream)>>>(
+      static_cast<const __half*>(X), M, K, X8, static_cast<__half*>(sx));
   return launch_status();
 }
 }  // namespace qoq
