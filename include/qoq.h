@@ -161,14 +161,15 @@ QOQ_API int qoq_quantize_act_per_token(const void* X, int M, int K, int8_t* X8,
  *   ws, ws_bytes : device workspace for splitting K over several CTAs, at
  *            least qoq_gemm_workspace_bytes(M, N, K, group) bytes (0 for
  *            shapes that are not split).  Owned by the caller, who fills it
- *            with zeros once before its first use (e.g. cudaMemset); from
- *            then on its contents are this library's, and it can be reused by
- *            later calls on the same stream whatever their shape.  Its first
- *            16 KiB hold one arrival counter per output tile, the rest the
- *            INT32 partial sums.  Calls that can run at the same time
- *            (different streams) need different workspaces.  With ws == NULL
- *            or too small the call still runs, without splitting K (slower
- *            for small M).
+ *            with zeros once before its first use (e.g. cudaMemset); every
+ *            call that completes leaves its first 16 KiB (one arrival counter
+ *            per output tile) at zero again, so it can be reused by later
+ *            calls on the same stream whatever their shape.  After a call
+ *            that reported a device error (qoq_device_error) it must be
+ *            zeroed again.  The rest holds INT32 partial sums.  Calls that
+ *            can run at the same time (different streams) need different
+ *            workspaces.  With ws == NULL or too small the call still runs,
+ *            without splitting K (slower for small M).
  * The UINT4 codes are dequantized to INT8 inside the main loop
  * (dq = q*s2 - z*s2, four byte lanes per 32-bit operation), multiplied on the
  * INT8 tensor cores (tcgen05, INT32 accumulators in tensor memory), and the

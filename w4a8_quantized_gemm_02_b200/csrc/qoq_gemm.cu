@@ -23,8 +23,8 @@
 //               row into tensor memory with one tcgen05.st; afterwards the
 //               same warps run the epilogue.
 // When K is split over several CTAs, each writes its INT32 partial tile to the
-// caller's workspace and the last one to arrive (an epoch-tagged counter per
-// output tile) adds them up exactly and runs the epilogue.
+// caller's workspace and the last one to arrive (an arrival counter per output
+// tile) adds them up exactly and runs the epilogue.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -46,7 +46,6 @@ constexpr int kThreads = 320;        // 10 warps
 constexpr int kEpiThreads = 256;     // warps 2..9
 constexpr int kRawStageBytes = 8576; // largest packed block (group 64), 16-byte multiple
 constexpr int kSmemPerSm = 233472;   // 228 KiB of shared memory per SM
-constexpr uint32_t kCasLimit = 1u << 20;
 // The workspace starts with a fixed region of arrival counters (one word per
 // output tile), so that counter words never share memory with the partial
 // sums of a launch of another shape.
@@ -90,11 +89,10 @@ struct GemmArgs {
   __half* Y;
   int32_t* acc;
   int32_t* ws_part;     // [m_tile][split][TOK][N] partial sums (splits > 1)
-  uint32_t* ws_count;   // [m_tile][n_tile] epoch-tagged arrival counters (fixed region)
+  uint32_t* ws_count;   // [m_tile][n_tile] arrival counters (fixed region, zero between launches)
   int M, N, K, group;
   int splits;
   int blk_bytes;
-  uint32_t epoch;       // 24-bit launch tag
 };
 
 // Bounded wait that ignores the abort flag: used only to drain work already
@@ -121,26 +119,17 @@ __device__ __forceinline__ uint4 ld_cg_v4(const int32_t* p) {
   return __ldcg(reinterpret_cast<const uint4*>(p));
 }
 
-// Register this CTA's arrival at its output tile.  Returns true for the last
-// of `splits` arrivals of the launch tagged `epoch`.  The counter word is
-// (epoch << 8) | count and only ever holds values written here (the region
-// starts zero-filled); a word left by another launch (another epoch) starts a
-// new count, and the last arrival resets the count so that a replay of the
-// same launch (same epoch) starts from zero again.
-__device__ bool arrive_last(uint32_t* ctr, uint32_t epoch, int splits) {
-  uint32_t cur = *reinterpret_cast<volatile uint32_t*>(ctr);
-  for (uint32_t it = 0; it < kCasLimit; ++it) {
-    const uint32_t next = ((cur >> 8) == epoch) ? cur + 1u : ((epoch << 8) | 1u);
-    const uint32_t prev = atomicCAS(ctr, cur, next);
-    if (prev == cur) {
-      const bool last = static_cast<int>(next & 0xffu) == splits;
-      if (last) atomicExch(ctr, epoch << 8);
-      return last;
-    }
-    cur = prev;
-  }
-  atomicOr(&g_error_word, kErrCounter);
-  return false;
+// Register this CTA's arrival at its output tile (one thread, after the
+// CTA's partial tile is written and a fence made it visible).  The counter
+// counts the arrivals of the current launch; the last of `splits` arrivals
+// resets it to zero, so the counter region returns to zero after every
+// launch that completes.
+__device__ __forceinline__ bool arrive_last(uint32_t* ctr, int splits) {
+  const uint32_t old = atomicAdd(ctr, 1u);
+  if (old >= static_cast<uint32_t>(splits)) atomicOr(&g_error_word, kErrCounter);
+  const bool last = old == static_cast<uint32_t>(splits - 1);
+  if (last) atomicExch(ctr, 0u);
+  return last;
 }
 
 template <int TOK>
@@ -353,64 +342,77 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     epi_bar();
   }
 
-  // 2) thread et owns rows 4*(et%32) .. +3 and token columns c = et/32 (mod 8)
+  // 2) thread et owns rows 8*(et%16) .. +7 and token columns c = et/16 (mod 16)
   const int M = args.M, N = args.N;
-  const int rq = 4 * (et & 31);
-  const int n = nt * kTileN + rq;
-  const int c_first = et >> 5;
+  const int r8 = 8 * (et & 15);
+  const int n = nt * kTileN + r8;
+  const int c_first = et >> 4;
   int c_end = M - m0;
   if (c_end > TOK) c_end = TOK;
   if (epi && splits > 1) {
-    // publish this split's partial tile, then count the arrival
+    // publish this split's partial tile, then count the arrival: the
+    // barrier orders every thread's stores before thread 0's fence, and the
+    // fence is cumulative (release); the last arrival fences again (acquire)
+    // before the barrier that releases the readers
     int32_t* part = args.ws_part + (static_cast<size_t>(mt * splits + split) * TOK) * N + n;
-    for (int c = c_first; c < c_end; c += 8) {
-      const uint4 v = *reinterpret_cast<const uint4*>(slot + c * kTileN + rq);
-      __stcg(reinterpret_cast<uint4*>(part + static_cast<size_t>(c) * N), v);
+    for (int c = c_first; c < c_end; c += 16) {
+      const uint4* sv = reinterpret_cast<const uint4*>(slot + c * kTileN + r8);
+      uint4* dst = reinterpret_cast<uint4*>(part + static_cast<size_t>(c) * N);
+      __stcg(dst, sv[0]);
+      __stcg(dst + 1, sv[1]);
     }
-    __threadfence();
     epi_bar();
     if (et == 0) {
-      const bool last = arrive_last(args.ws_count + mt * (N / kTileN) + nt, args.epoch, splits);
+      __threadfence();
+      const bool last = arrive_last(args.ws_count + mt * (N / kTileN) + nt, splits);
+      if (last) __threadfence();
       *last_flag = last ? 1u : 0u;
     }
     epi_bar();
-    __threadfence();
   }
   const bool writer = epi && (*abort_flag == 0u) && (splits == 1 || *last_flag != 0u);
   if (writer) {
-    float s1q[4] = {0.f, 0.f, 0.f, 0.f};
+    float s1o[8];
     if (args.Y) {
-      const uint2 sv = *reinterpret_cast<const uint2*>(args.s1 + n);
+      const uint4 sv = *reinterpret_cast<const uint4*>(args.s1 + n);
       const __half2* h = reinterpret_cast<const __half2*>(&sv);
-      const float2 a = __half22float2(h[0]), b = __half22float2(h[1]);
-      s1q[0] = a.x;
-      s1q[1] = a.y;
-      s1q[2] = b.x;
-      s1q[3] = b.y;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __half22float2(h[j]);
+        s1o[2 * j] = f.x;
+        s1o[2 * j + 1] = f.y;
+      }
     }
     const int32_t* parts = args.ws_part + (static_cast<size_t>(mt * splits) * TOK) * N + n;
-#pragma unroll 4
-    for (int c = c_first; c < c_end; c += 8) {
-      uint4 v = *reinterpret_cast<const uint4*>(slot + c * kTileN + rq);
+#pragma unroll 2
+    for (int c = c_first; c < c_end; c += 16) {
+      const uint4* sv = reinterpret_cast<const uint4*>(slot + c * kTileN + r8);
+      uint4 v0 = sv[0], v1 = sv[1];
       for (int q = 0; q < splits; ++q) {
         if (q == split) continue;
-        v = add4(v, ld_cg_v4(parts + (static_cast<size_t>(q) * TOK + c) * N));
+        const int32_t* p = parts + (static_cast<size_t>(q) * TOK + c) * N;
+        v0 = add4(v0, ld_cg_v4(p));
+        v1 = add4(v1, ld_cg_v4(p + 4));
       }
       const size_t o = static_cast<size_t>(m0 + c) * N + n;
       if (args.acc) {
-        *reinterpret_cast<uint4*>(args.acc + o) = v;
+        reinterpret_cast<uint4*>(args.acc + o)[0] = v0;
+        reinterpret_cast<uint4*>(args.acc + o)[1] = v1;
       } else {
         const float sxf = sx_s[c];
-        const __half2 y01 = __floats2half2_rn(
-            __fmul_rn(static_cast<float>(static_cast<int32_t>(v.x)), __fmul_rn(sxf, s1q[0])),
-            __fmul_rn(static_cast<float>(static_cast<int32_t>(v.y)), __fmul_rn(sxf, s1q[1])));
-        const __half2 y23 = __floats2half2_rn(
-            __fmul_rn(static_cast<float>(static_cast<int32_t>(v.z)), __fmul_rn(sxf, s1q[2])),
-            __fmul_rn(static_cast<float>(static_cast<int32_t>(v.w)), __fmul_rn(sxf, s1q[3])));
-        uint2 pk;
-        pk.x = *reinterpret_cast<const uint32_t*>(&y01);
-        pk.y = *reinterpret_cast<const uint32_t*>(&y23);
-        *reinterpret_cast<uint2*>(args.Y + o) = pk;
+        const int32_t a[8] = {static_cast<int32_t>(v0.x), static_cast<int32_t>(v0.y),
+                              static_cast<int32_t>(v0.z), static_cast<int32_t>(v0.w),
+                              static_cast<int32_t>(v1.x), static_cast<int32_t>(v1.y),
+                              static_cast<int32_t>(v1.z), static_cast<int32_t>(v1.w)};
+        uint32_t pk[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __half2 y = __floats2half2_rn(
+              __fmul_rn(static_cast<float>(a[2 * j]), __fmul_rn(sxf, s1o[2 * j])),
+              __fmul_rn(static_cast<float>(a[2 * j + 1]), __fmul_rn(sxf, s1o[2 * j + 1])));
+          pk[j] = *reinterpret_cast<const uint32_t*>(&y);
+        }
+        *reinterpret_cast<uint4*>(args.Y + o) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
     }
   }
@@ -445,16 +447,6 @@ EncodeTiledFn encode_fn() {
       fn = reinterpret_cast<EncodeTiledFn>(p);
   });
   return fn;
-}
-
-std::atomic<uint32_t> g_epoch{0};
-
-uint32_t next_epoch() {
-  uint32_t e;
-  do {
-    e = (g_epoch.fetch_add(1, std::memory_order_relaxed) + 1u) & 0xffffffu;
-  } while (e == 0);
-  return e;
 }
 
 struct Plan {
@@ -596,7 +588,6 @@ int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* 
   a.group = group;
   a.splits = p.splits;
   a.blk_bytes = static_cast<int>(block_bytes(group));
-  a.epoch = next_epoch();
 
   cudaStream_t s = as_stream(stream);
   switch (p.tok) {
