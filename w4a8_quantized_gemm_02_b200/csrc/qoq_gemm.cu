@@ -7,29 +7,33 @@
 // Background (per-group W4A4 dequantizes INT32 partial sums in its main loop,
 // this kernel scales once, after the whole K reduction).
 //
-// One CTA computes a 128-channel x TOK-token output tile over a range of K.
-// The weights are the MMA's M operand and the tokens its N operand, so a
-// single decode token still fills the 128-row tensor-core tile.
-//   warp 0      TMA producer: one bulk copy of the packed weight block and one
-//               tensor-map copy of the X8 tile (128-byte swizzle) per k-tile,
-//               into a ring of shared-memory stages;
-//   warp 1      owns tensor memory and issues tcgen05.mma.kind::i8 (M = 128,
-//               N = TOK, K = 32 per instruction, 4 per k-tile) with the INT8
-//               weights read from tensor memory and X8 from shared memory,
-//               INT32 accumulators in tensor memory;
-//   warps 2..9  two dequantizing warpgroups taking alternate k-tiles: each
-//               thread turns one weight row of the UINT4 block into INT8 (four
-//               byte lanes per 32-bit multiply-add) and writes the 128-byte
-//               row into tensor memory with one tcgen05.st; afterwards the
-//               same warps run the epilogue.
-// When K is split over several CTAs, each writes its INT32 partial tile to the
-// caller's workspace and the last one to arrive (an arrival counter per output
-// tile) adds them up exactly and runs the epilogue.
+// Persistent kernel, one CTA per SM.  A work unit is a 128-channel x
+// TOK-token output tile over a range of K (the weights are the MMA's M operand
+// and the tokens its N operand, so one decode token still fills the 128-row
+// tensor-core tile).  Units are ordered channel-tile major, token tile next,
+// K split innermost, so the CTAs running at the same time share weight blocks
+// through L2 and every weight byte comes from HBM about once.
+//   warp 0       TMA producer: per k-tile, one bulk copy of the packed weight
+//                block and one tensor-map copy of the X8 tile (128-byte
+//                swizzle) into a ring of shared-memory stages;
+//   warp 1       owns tensor memory and issues tcgen05.mma.kind::i8 (M = 128,
+//                N = TOK, K = 32 per instruction) with the INT8 weights read
+//                from tensor memory and X8 from shared memory, into one of two
+//                INT32 accumulators in tensor memory (double buffered);
+//   warps 2..13  three dequantizing warpgroups taking k-tiles in turn: each
+//                thread turns one weight row of the UINT4 block into INT8
+//                (four byte lanes per 32-bit multiply-add) and writes the
+//                128-byte row into a tensor-memory stage with one tcgen05.st;
+//   warps 14..17 epilogue: tcgen05.ld of a finished accumulator, one FP32
+//                scale per element, a transpose through shared memory and
+//                16-byte stores, overlapping the next unit's main loop.
+// When K is split, each unit writes its INT32 partial tile to the caller's
+// workspace and the last one to arrive (an arrival counter per output tile)
+// adds them up exactly and runs the scaling.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
-#include <atomic>
 #include <mutex>
 
 #include "qoq.h"
@@ -42,10 +46,16 @@ __device__ unsigned int g_error_word = 0;
 
 namespace {
 
-constexpr int kThreads = 320;        // 10 warps
-constexpr int kEpiThreads = 256;     // warps 2..9
-constexpr int kRawStageBytes = 8576; // largest packed block (group 64), 16-byte multiple
-constexpr int kSmemPerSm = 233472;   // 228 KiB of shared memory per SM
+constexpr int kDqGroups = 3;                     // dequantizing warpgroups
+constexpr int kWarpEpi0 = 2 + 4 * kDqGroups;     // first epilogue warp (14)
+constexpr int kWarps = kWarpEpi0 + 4;            // 18
+constexpr int kThreads = 32 * kWarps;            // 576
+constexpr int kRawStageBytes = 8576;             // largest packed block (group 64)
+constexpr int kDqStages = 6;                     // tensor-memory A stages
+constexpr int kTmemA = 0;                        // A stage d at column 32 d
+constexpr int kTmemD = 256;                      // accumulators from column 256
+constexpr int kTmemCols = 512;
+constexpr int kStageBytesEpi = 32 * 16 * 4;      // per epilogue warp: 16 columns x 32 rows
 // The workspace starts with a fixed region of arrival counters (one word per
 // output tile), so that counter words never share memory with the partial
 // sums of a launch of another shape.
@@ -54,32 +64,22 @@ constexpr size_t kCounterBytes = kMaxCounterTiles * 4;
 
 template <int TOK>
 struct Cfg {
-  static constexpr int kStages = TOK <= 32 ? 8 : (TOK <= 64 ? 6 : 4);
-  static constexpr int kDqStages = 4;
+  static constexpr int kStages = TOK <= 128 ? 8 : 4;
+  static constexpr int kAcc = TOK <= 128 ? 2 : 1;   // accumulator buffers
   static constexpr int kXBytes = TOK * kTileK;
   static constexpr int kOffX = 0;
   static constexpr int kOffRaw = kOffX + kStages * kXBytes;
-  static constexpr int kOffSx = kOffRaw + kStages * kRawStageBytes;
-  static constexpr int kOffBar = kOffSx + ((TOK * 4 + 15) / 16) * 16;
-  static constexpr int kNumBars = 2 * kStages + 2 * kDqStages + 1;
+  static constexpr int kOffEpi = kOffRaw + kStages * kRawStageBytes;
+  static constexpr int kOffSx = kOffEpi + 4 * kStageBytesEpi;          // 4 warps x TOK floats
+  static constexpr int kOffBar = kOffSx + 4 * TOK * 4;
+  static constexpr int kNumBars = 2 * kStages + 2 * kDqStages + 2 * kAcc + 3;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
-  static constexpr int kSmemUsed = kOffMisc + 16 + 1024;   // + base alignment slack
-  // tensor memory: A operand stages at columns 32 d, the accumulator after them
-  static constexpr int kTmemA = 0;
-  static constexpr int kTmemD = 32 * kDqStages;
-  static constexpr int kTmemCols = (kTmemD + TOK <= 256) ? 256 : 512;
-  // Never more CTAs on an SM than tensor memory holds: request enough shared
-  // memory that one more CTA cannot fit, so tcgen05.alloc never has to wait.
-  static constexpr int kCtasPerSm = 512 / kTmemCols;
-  static constexpr int kSmemFloor = kSmemPerSm / (kCtasPerSm + 1);
-  static constexpr int kSmemBytes = kSmemUsed > kSmemFloor ? kSmemUsed : kSmemFloor;
-  // epilogue slot: the INT32 tile as [token column][row], in the X ring
-  static constexpr int kSlotBytes = kTileN * TOK * 4;
+  static constexpr int kSmemBytes = kOffMisc + 32 + 1024;   // + base alignment slack
   static_assert(kOffRaw % 1024 == 0 && kXBytes % 1024 == 0, "swizzled tiles need 1 KiB alignment");
   static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
-  static_assert(kSlotBytes <= kStages * kXBytes, "epilogue slot must fit in the X ring");
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-  static_assert(kTmemD + TOK <= kTmemCols, "tensor memory");
+  static_assert(kTmemD + kAcc * TOK <= kTmemCols, "tensor memory");
+  static_assert(32 * kDqStages <= kTmemD, "tensor memory A stages");
 };
 
 struct GemmArgs {
@@ -89,11 +89,28 @@ struct GemmArgs {
   __half* Y;
   int32_t* acc;
   int32_t* ws_part;     // [m_tile][split][TOK][N] partial sums (splits > 1)
-  uint32_t* ws_count;   // [m_tile][n_tile] arrival counters (fixed region, zero between launches)
+  uint32_t* ws_count;   // [m_tile][n_tile] arrival counters (zero between launches)
   int M, N, K, group;
   int splits;
+  int m_tiles, n_tiles;
+  int units;            // n_tiles * m_tiles * splits
   int blk_bytes;
 };
+
+struct Unit {
+  int nt, mt, split, kt_begin, num_kt;
+};
+
+__device__ __forceinline__ Unit unit_of(const GemmArgs& a, int u, int kt_total) {
+  Unit w;
+  w.split = u % a.splits;
+  const int rest = u / a.splits;
+  w.mt = rest % a.m_tiles;
+  w.nt = rest / a.m_tiles;
+  w.kt_begin = (w.split * kt_total) / a.splits;
+  w.num_kt = ((w.split + 1) * kt_total) / a.splits - w.kt_begin;
+  return w;
+}
 
 // Bounded wait that ignores the abort flag: used only to drain work already
 // in flight before a CTA tears down.
@@ -107,23 +124,11 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
-__device__ __forceinline__ void epi_bar() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
-}
-
-__device__ __forceinline__ uint4 add4(uint4 a, uint4 b) {
-  return make_uint4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
-}
-
-__device__ __forceinline__ uint4 ld_cg_v4(const int32_t* p) {
-  return __ldcg(reinterpret_cast<const uint4*>(p));
-}
-
-// Register this CTA's arrival at its output tile (one thread, after the
-// CTA's partial tile is written and a fence made it visible).  The counter
-// counts the arrivals of the current launch; the last of `splits` arrivals
-// resets it to zero, so the counter region returns to zero after every
-// launch that completes.
+// Register this CTA's arrival at an output tile (one thread, after the
+// partial tile is written and a fence made it visible).  The counter counts
+// the arrivals of the current launch; the last of `splits` arrivals resets it
+// to zero, so the counter region returns to zero after every launch that
+// completes.
 __device__ __forceinline__ bool arrive_last(uint32_t* ctr, int splits) {
   const uint32_t old = atomicAdd(ctr, 1u);
   if (old >= static_cast<uint32_t>(splits)) atomicOr(&g_error_word, kErrCounter);
@@ -136,6 +141,7 @@ template <int TOK>
 __global__ void __launch_bounds__(kThreads, 1)
 w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args) {
   using C = Cfg<TOK>;
+  constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -143,277 +149,333 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int splits = args.splits;
-  const int nt = blockIdx.x / splits;
-  const int split = blockIdx.x - nt * splits;
-  const int mt = blockIdx.y;
-  const int m0 = mt * TOK;
   const int kt_total = args.K / kTileK;
-  const int kt_begin = (split * kt_total) / splits;
-  const int num_kt = ((split + 1) * kt_total) / splits - kt_begin;
 
   const uint32_t bar_full = base + C::kOffBar;
-  const uint32_t bar_empty = bar_full + 8 * C::kStages;
-  const uint32_t bar_dqfull = bar_empty + 8 * C::kStages;
-  const uint32_t bar_dqempty = bar_dqfull + 8 * C::kDqStages;
-  const uint32_t bar_acc = bar_dqempty + 8 * C::kDqStages;
+  const uint32_t bar_empty = bar_full + 8 * S;
+  const uint32_t bar_dqfull = bar_empty + 8 * S;
+  const uint32_t bar_dqempty = bar_dqfull + 8 * kDqStages;
+  const uint32_t bar_accfull = bar_dqempty + 8 * kDqStages;
+  const uint32_t bar_accempty = bar_accfull + 8 * C::kAcc;
+  const uint32_t bar_drain = bar_accempty + 8 * C::kAcc;
+  const uint32_t bar_epi_in = bar_drain + 8;    // four epilogue warps published a partial
+  const uint32_t bar_epi_go = bar_epi_in + 8;   // the arrival was counted
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc + 4);
   volatile uint32_t* last_flag = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc + 8);
-  float* sx_s = reinterpret_cast<float*>(smem + C::kOffSx);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
     }
-    for (int d = 0; d < C::kDqStages; ++d) {
+    for (int d = 0; d < kDqStages; ++d) {
       mbar_init(bar_dqfull + 8 * d, 4);
       mbar_init(bar_dqempty + 8 * d, 1);
     }
-    mbar_init(bar_acc, 1);
+    for (int b = 0; b < C::kAcc; ++b) {
+      mbar_init(bar_accfull + 8 * b, 1);
+      mbar_init(bar_accempty + 8 * b, 4);
+    }
+    mbar_init(bar_drain, 1);
+    mbar_init(bar_epi_in, 4);
+    mbar_init(bar_epi_go, 1);
     *abort_flag = 0u;
     *last_flag = 0u;
     fence_mbar_init();
     prefetch_tensormap(&tmap_x);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  bool ok = true;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       const uint64_t policy = l2_policy_evict_first();
-      const uint8_t* src =
-          args.packed + (static_cast<size_t>(nt) * kt_total + kt_begin) * args.blk_bytes;
       const uint32_t tx = static_cast<uint32_t>(args.blk_bytes + C::kXBytes);
-      const int pre = num_kt < C::kStages ? num_kt : C::kStages;
-      // the weight stream does not depend on the preceding grid: start it
-      // before waiting for the activations
-      for (int i = 0; i < pre; ++i) {
-        mbar_arrive_expect_tx(bar_full + 8 * i, tx);
-        bulk_load(base + C::kOffRaw + i * kRawStageBytes, src + static_cast<size_t>(i) * args.blk_bytes,
-                  static_cast<uint32_t>(args.blk_bytes), bar_full + 8 * i, policy);
+      uint32_t g = 0;              // running k-tile index of this CTA
+      bool aborted = false;
+      bool first = true;
+      for (int u = blockIdx.x; u < args.units && !aborted; u += gridDim.x) {
+        const Unit w = unit_of(args, u, kt_total);
+        const uint8_t* src =
+            args.packed + (static_cast<size_t>(w.nt) * kt_total + w.kt_begin) * args.blk_bytes;
+        const int m0 = w.mt * TOK;
+        int i = 0;
+        if (first) {
+          // the weight stream does not depend on the preceding grid: start it
+          // before waiting for the activations
+          first = false;
+          const int pre = w.num_kt < S ? w.num_kt : S;
+          for (int j = 0; j < pre; ++j) {
+            mbar_arrive_expect_tx(bar_full + 8 * j, tx);
+            bulk_load(base + C::kOffRaw + j * kRawStageBytes,
+                      src + static_cast<size_t>(j) * args.blk_bytes,
+                      static_cast<uint32_t>(args.blk_bytes), bar_full + 8 * j, policy);
+          }
+          grid_dependency_wait();
+          for (int j = 0; j < pre; ++j)
+            tma_load_2d(base + C::kOffX + j * C::kXBytes, &tmap_x, (w.kt_begin + j) * kTileK, m0,
+                        bar_full + 8 * j);
+          i = pre;
+          g = pre;
+        }
+        for (; i < w.num_kt; ++i, ++g) {
+          const int s = g % S;
+          if (g >= S && !mbar_wait(bar_empty + 8 * s, ((g / S) & 1) ^ 1, abort_flag, &g_error_word,
+                                   kErrProducer)) {
+            aborted = true;
+            break;
+          }
+          mbar_arrive_expect_tx(bar_full + 8 * s, tx);
+          bulk_load(base + C::kOffRaw + s * kRawStageBytes,
+                    src + static_cast<size_t>(i) * args.blk_bytes,
+                    static_cast<uint32_t>(args.blk_bytes), bar_full + 8 * s, policy);
+          tma_load_2d(base + C::kOffX + s * C::kXBytes, &tmap_x, (w.kt_begin + i) * kTileK, m0,
+                      bar_full + 8 * s);
+        }
       }
-      grid_dependency_wait();
-      for (int i = 0; i < pre; ++i)
-        tma_load_2d(base + C::kOffX + i * C::kXBytes, &tmap_x, (kt_begin + i) * kTileK, m0,
-                    bar_full + 8 * i);
-      int i = pre;
-      for (; i < num_kt; ++i) {
-        const int s = i % C::kStages;
-        if (!mbar_wait(bar_empty + 8 * s, ((i / C::kStages) & 1) ^ 1, abort_flag, &g_error_word,
-                       kErrProducer))
-          break;
-        mbar_arrive_expect_tx(bar_full + 8 * s, tx);
-        bulk_load(base + C::kOffRaw + s * kRawStageBytes, src + static_cast<size_t>(i) * args.blk_bytes,
-                  static_cast<uint32_t>(args.blk_bytes), bar_full + 8 * s, policy);
-        tma_load_2d(base + C::kOffX + s * C::kXBytes, &tmap_x, (kt_begin + i) * kTileK, m0,
-                    bar_full + 8 * s);
-      }
-      if (i < num_kt) {
-        // aborted: the copies already issued must land before the CTA exits
-        for (int j = (i > C::kStages ? i - C::kStages : 0); j < i; ++j)
-          drain_wait(bar_full + 8 * (j % C::kStages), (j / C::kStages) & 1);
+      if (aborted) {
+        // the copies already issued must land before the CTA exits
+        for (uint32_t j = (g > S ? g - S : 0); j < g; ++j)
+          drain_wait(bar_full + 8 * (j % S), (j / S) & 1);
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_i8(kTileN, TOK);
-      const uint32_t d_tmem = tmem + C::kTmemD;
-      for (int i = 0; i < num_kt; ++i) {
-        const int s = i % C::kStages, d = i % C::kDqStages;
-        if (!mbar_wait(bar_full + 8 * s, (i / C::kStages) & 1, abort_flag, &g_error_word, kErrMma))
-          break;
-        if (!mbar_wait(bar_dqfull + 8 * d, (i / C::kDqStages) & 1, abort_flag, &g_error_word,
+      uint32_t g = 0;
+      int lt = 0;
+      bool aborted = false;
+      for (int u = blockIdx.x; u < args.units && !aborted; u += gridDim.x, ++lt) {
+        const Unit w = unit_of(args, u, kt_total);
+        const int b = lt % C::kAcc;
+        if (lt >= C::kAcc &&
+            !mbar_wait(bar_accempty + 8 * b, ((lt / C::kAcc) & 1) ^ 1, abort_flag, &g_error_word,
                        kErrMma))
           break;
         tc_fence_after_sync();
-        const uint32_t a_tmem = tmem + C::kTmemA + 32 * d;
-        const uint32_t b_addr = base + C::kOffX + s * C::kXBytes;
+        const uint32_t d_tmem = tmem + kTmemD + b * TOK;
+        for (int i = 0; i < w.num_kt; ++i, ++g) {
+          const int s = g % S, d = g % kDqStages;
+          if (!mbar_wait(bar_full + 8 * s, (g / S) & 1, abort_flag, &g_error_word, kErrMma) ||
+              !mbar_wait(bar_dqfull + 8 * d, (g / kDqStages) & 1, abort_flag, &g_error_word,
+                         kErrMma)) {
+            aborted = true;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t a_tmem = tmem + kTmemA + 32 * d;
+          const uint32_t b_addr = base + C::kOffX + s * C::kXBytes;
 #pragma unroll
-        for (int kk = 0; kk < kTileK / 32; ++kk) {
-          // K = 32 bytes per instruction: 8 tensor-memory columns of A, 32
-          // bytes along the swizzled rows of B
-          mma_i8_ts(d_tmem, a_tmem + 8 * kk, smem_desc_sw128(b_addr + kk * 32), idesc,
-                    (i > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kTileK / 32; ++kk) {
+            // K = 32 bytes per instruction: 8 tensor-memory columns of A, 32
+            // bytes along the swizzled rows of B
+            mma_i8_ts(d_tmem, a_tmem + 8 * kk, smem_desc_sw128(b_addr + kk * 32), idesc,
+                      (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(bar_empty + 8 * s);     // X tile and raw block of stage s are free
+          mma_commit(bar_dqempty + 8 * d);   // A stage d is free
         }
-        mma_commit(bar_empty + 8 * s);     // X tile and raw block of stage s are free
-        mma_commit(bar_dqempty + 8 * d);   // A stage d is free
+        if (!aborted) mma_commit(bar_accfull + 8 * b);   // accumulator b is complete
       }
-      mma_commit(bar_acc);                 // accumulator complete (or aborted)
-      drain_wait(bar_acc, 0);              // no MMA in flight past this point
+      mma_commit(bar_drain);
+      drain_wait(bar_drain, 0);              // no MMA in flight past this point
     }
-  } else {
+  } else if (warp < kWarpEpi0) {
     // ---------------------------------------------------------------- dequantizers
-    const int wg = (warp - 2) >> 2;        // warpgroup: even or odd k-tiles
-    const int q4 = warp & 3;               // tensor-memory lane quarter of this warp
-    const int r = q4 * 32 + lane;          // weight row (output channel) within the tile
+    const int wg = (warp - 2) >> 2;         // 0 .. kDqGroups-1: takes k-tiles g = wg (mod 3)
+    const int q4 = warp & 3;                // tensor-memory lane quarter of this warp
+    const int r = q4 * 32 + lane;           // weight row (output channel) within the tile
     const uint32_t row_tmem = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int gpt = kTileK / args.group;
-    for (int i = wg; i < num_kt; i += 2) {
-      const int s = i % C::kStages, d = i % C::kDqStages;
-      if (!mbar_wait(bar_full + 8 * s, (i / C::kStages) & 1, abort_flag, &g_error_word,
-                     kErrDequant)) {
-        ok = false;
-        break;
-      }
-      if (i >= C::kDqStages &&
-          !mbar_wait(bar_dqempty + 8 * d, ((i / C::kDqStages) & 1) ^ 1, abort_flag, &g_error_word,
-                     kErrDequant)) {
-        ok = false;
-        break;
-      }
-      const uint8_t* blk = smem + C::kOffRaw + s * kRawStageBytes;
-      uint32_t s2v[2], bias[2];
-#pragma unroll
-      for (int gl = 0; gl < 2; ++gl) {
-        if (gl < gpt) {
-          s2v[gl] = blk[kCodesBytes + gl * kTileN + r];
-          const uint32_t zb = blk[kCodesBytes + gpt * kTileN + gl * 64 + (r >> 1)];
-          const uint32_t zv = (r & 1) ? (zb >> 4) : (zb & 15u);
-          bias[gl] = dq_bias(zv, s2v[gl]);
-        } else {
-          s2v[gl] = s2v[0];
-          bias[gl] = bias[0];
+    uint32_t g = 0;
+    bool aborted = false;
+    for (int u = blockIdx.x; u < args.units && !aborted; u += gridDim.x) {
+      const Unit w = unit_of(args, u, kt_total);
+      for (int i = 0; i < w.num_kt; ++i, ++g) {
+        if (static_cast<int>(g % kDqGroups) != wg) continue;
+        const int s = g % S, d = g % kDqStages;
+        if (!mbar_wait(bar_full + 8 * s, (g / S) & 1, abort_flag, &g_error_word, kErrDequant) ||
+            (g >= kDqStages &&
+             !mbar_wait(bar_dqempty + 8 * d, ((g / kDqStages) & 1) ^ 1, abort_flag, &g_error_word,
+                        kErrDequant))) {
+          aborted = true;
+          break;
         }
-      }
-      uint32_t out[32];
+        const uint8_t* blk = smem + C::kOffRaw + s * kRawStageBytes;
+        uint32_t s2v[2], bias[2];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint4 w = *reinterpret_cast<const uint4*>(blk + (j * kTileN + r) * 16);
-        const int gl = (gpt == 2) ? (j >> 1) : 0;
-        const uint32_t sv = s2v[gl], bv = bias[gl];
-        out[8 * j + 0] = dq_lanes(lo_codes(w.x), sv, bv);
-        out[8 * j + 1] = dq_lanes(hi_codes(w.x), sv, bv);
-        out[8 * j + 2] = dq_lanes(lo_codes(w.y), sv, bv);
-        out[8 * j + 3] = dq_lanes(hi_codes(w.y), sv, bv);
-        out[8 * j + 4] = dq_lanes(lo_codes(w.z), sv, bv);
-        out[8 * j + 5] = dq_lanes(hi_codes(w.z), sv, bv);
-        out[8 * j + 6] = dq_lanes(lo_codes(w.w), sv, bv);
-        out[8 * j + 7] = dq_lanes(hi_codes(w.w), sv, bv);
-      }
-      // one 128-byte row of the INT8 A operand: column c holds K bytes 4c..4c+3
-      tmem_st_32x32b_x32(row_tmem + C::kTmemA + 32 * d, out);
-      tmem_st_wait();
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_dqfull + 8 * d);
-    }
-  }
-
-  // ------------------------------------------------------------------ epilogue
-  // 1) accumulator -> slot [token column][row] (INT32) in the X ring
-  uint32_t* slot = reinterpret_cast<uint32_t*>(smem + C::kOffX);
-  const bool epi = warp >= 2;
-  const int et = threadIdx.x - 64;         // epilogue thread 0..255
-  if (epi) {
-    const int wg = (warp - 2) >> 2;
-    const int q4 = warp & 3;
-    const int r = q4 * 32 + lane;
-    const bool have = ok && mbar_wait(bar_acc, 0, abort_flag, &g_error_word, kErrEpilogue);
-    tc_fence_after_sync();
-    if (__all_sync(0xffffffffu, have && (*abort_flag == 0u))) {
-      const uint32_t t_row = tmem + C::kTmemD + (static_cast<uint32_t>(q4 * 32) << 16);
-#pragma unroll 1
-      for (int c0 = 16 * wg; c0 < TOK; c0 += 32) {
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(t_row + c0, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) slot[(c0 + j) * kTileN + r] = v[j];
-      }
-    }
-    if (args.Y) {
-      grid_dependency_wait();   // sx comes from the preceding grid under PDL
-      for (int c = et; c < TOK; c += kEpiThreads) {
-        const int m = m0 + c;
-        sx_s[c] = m < args.M ? __half2float(args.sx[m]) : 0.0f;
-      }
-    }
-    epi_bar();
-  }
-
-  // 2) thread et owns rows 8*(et%16) .. +7 and token columns c = et/16 (mod 16)
-  const int M = args.M, N = args.N;
-  const int r8 = 8 * (et & 15);
-  const int n = nt * kTileN + r8;
-  const int c_first = et >> 4;
-  int c_end = M - m0;
-  if (c_end > TOK) c_end = TOK;
-  if (epi && splits > 1) {
-    // publish this split's partial tile, then count the arrival: the
-    // barrier orders every thread's stores before thread 0's fence, and the
-    // fence is cumulative (release); the last arrival fences again (acquire)
-    // before the barrier that releases the readers
-    int32_t* part = args.ws_part + (static_cast<size_t>(mt * splits + split) * TOK) * N + n;
-    for (int c = c_first; c < c_end; c += 16) {
-      const uint4* sv = reinterpret_cast<const uint4*>(slot + c * kTileN + r8);
-      uint4* dst = reinterpret_cast<uint4*>(part + static_cast<size_t>(c) * N);
-      __stcg(dst, sv[0]);
-      __stcg(dst + 1, sv[1]);
-    }
-    epi_bar();
-    if (et == 0) {
-      __threadfence();
-      const bool last = arrive_last(args.ws_count + mt * (N / kTileN) + nt, splits);
-      if (last) __threadfence();
-      *last_flag = last ? 1u : 0u;
-    }
-    epi_bar();
-  }
-  const bool writer = epi && (*abort_flag == 0u) && (splits == 1 || *last_flag != 0u);
-  if (writer) {
-    float s1o[8];
-    if (args.Y) {
-      const uint4 sv = *reinterpret_cast<const uint4*>(args.s1 + n);
-      const __half2* h = reinterpret_cast<const __half2*>(&sv);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = __half22float2(h[j]);
-        s1o[2 * j] = f.x;
-        s1o[2 * j + 1] = f.y;
-      }
-    }
-    const int32_t* parts = args.ws_part + (static_cast<size_t>(mt * splits) * TOK) * N + n;
-#pragma unroll 2
-    for (int c = c_first; c < c_end; c += 16) {
-      const uint4* sv = reinterpret_cast<const uint4*>(slot + c * kTileN + r8);
-      uint4 v0 = sv[0], v1 = sv[1];
-      for (int q = 0; q < splits; ++q) {
-        if (q == split) continue;
-        const int32_t* p = parts + (static_cast<size_t>(q) * TOK + c) * N;
-        v0 = add4(v0, ld_cg_v4(p));
-        v1 = add4(v1, ld_cg_v4(p + 4));
-      }
-      const size_t o = static_cast<size_t>(m0 + c) * N + n;
-      if (args.acc) {
-        reinterpret_cast<uint4*>(args.acc + o)[0] = v0;
-        reinterpret_cast<uint4*>(args.acc + o)[1] = v1;
-      } else {
-        const float sxf = sx_s[c];
-        const int32_t a[8] = {static_cast<int32_t>(v0.x), static_cast<int32_t>(v0.y),
-                              static_cast<int32_t>(v0.z), static_cast<int32_t>(v0.w),
-                              static_cast<int32_t>(v1.x), static_cast<int32_t>(v1.y),
-                              static_cast<int32_t>(v1.z), static_cast<int32_t>(v1.w)};
-        uint32_t pk[4];
+        for (int gl = 0; gl < 2; ++gl) {
+          if (gl < gpt) {
+            s2v[gl] = blk[kCodesBytes + gl * kTileN + r];
+            const uint32_t zb = blk[kCodesBytes + gpt * kTileN + gl * 64 + (r >> 1)];
+            const uint32_t zv = (r & 1) ? (zb >> 4) : (zb & 15u);
+            bias[gl] = dq_bias(zv, s2v[gl]);
+          } else {
+            s2v[gl] = s2v[0];
+            bias[gl] = bias[0];
+          }
+        }
+        uint32_t out[32];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const __half2 y = __floats2half2_rn(
-              __fmul_rn(static_cast<float>(a[2 * j]), __fmul_rn(sxf, s1o[2 * j])),
-              __fmul_rn(static_cast<float>(a[2 * j + 1]), __fmul_rn(sxf, s1o[2 * j + 1])));
-          pk[j] = *reinterpret_cast<const uint32_t*>(&y);
+          const uint4 v = *reinterpret_cast<const uint4*>(blk + (j * kTileN + r) * 16);
+          const int gl = (gpt == 2) ? (j >> 1) : 0;
+          const uint32_t sv = s2v[gl], bv = bias[gl];
+          out[8 * j + 0] = dq_lanes(lo_codes(v.x), sv, bv);
+          out[8 * j + 1] = dq_lanes(hi_codes(v.x), sv, bv);
+          out[8 * j + 2] = dq_lanes(lo_codes(v.y), sv, bv);
+          out[8 * j + 3] = dq_lanes(hi_codes(v.y), sv, bv);
+          out[8 * j + 4] = dq_lanes(lo_codes(v.z), sv, bv);
+          out[8 * j + 5] = dq_lanes(hi_codes(v.z), sv, bv);
+          out[8 * j + 6] = dq_lanes(lo_codes(v.w), sv, bv);
+          out[8 * j + 7] = dq_lanes(hi_codes(v.w), sv, bv);
         }
-        *reinterpret_cast<uint4*>(args.Y + o) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        // one 128-byte row of the INT8 A operand: column c holds K bytes 4c..4c+3
+        tmem_st_32x32b_x32(row_tmem + kTmemA + 32 * d, out);
+        tmem_st_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_dqfull + 8 * d);
       }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q4 = warp & 3;                // tensor-memory lane quarter
+    const int ew = warp - kWarpEpi0;        // 0..3
+    const int r = q4 * 32 + lane;           // output channel within the tile
+    const int M = args.M, N = args.N;
+    uint8_t* stage = smem + C::kOffEpi + ew * kStageBytesEpi;   // [16 columns][32 rows] x 4 B
+    float* sx_w = reinterpret_cast<float*>(smem + C::kOffSx) + ew * TOK;
+    // transposed read of the staging buffer: lane reads column c = lane / 2,
+    // rows 16 * (lane & 1) .. +15 of this warp's 32-row slice
+    const int tc = lane >> 1, th = lane & 1;
+    grid_dependency_wait();                 // sx comes from the preceding grid under PDL
+    int lt = 0;
+    uint32_t ks = 0;                        // split units handled so far (barrier phases)
+    for (int u = blockIdx.x; u < args.units; u += gridDim.x, ++lt) {
+      const Unit w = unit_of(args, u, kt_total);
+      const int b = lt % C::kAcc;
+      const int m0 = w.mt * TOK;
+      const int nrow0 = w.nt * kTileN + q4 * 32;   // first channel of this warp's slice
+      const bool ok = mbar_wait(bar_accfull + 8 * b, (lt / C::kAcc) & 1, abort_flag,
+                                &g_error_word, kErrEpilogue);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after_sync();
+      const uint32_t t_acc = tmem + kTmemD + b * TOK + (static_cast<uint32_t>(q4 * 32) << 16);
+      int c_end = M - m0;
+      if (c_end > TOK) c_end = TOK;
+      float s1r = 0.0f;
+      if (args.Y) {
+        s1r = __half2float(args.s1[w.nt * kTileN + r]);
+        for (int c = lane; c < TOK; c += 32)
+          sx_w[c] = (m0 + c < M) ? __half2float(args.sx[m0 + c]) : 0.0f;
+        __syncwarp();
+      }
+      const int splits = args.splits;
+      bool write_out = true;
+      if (splits > 1) {
+        // publish this unit's partial tile (INT32, [token][channel]) ...
+        int32_t* part = args.ws_part + (static_cast<size_t>(w.mt * splits + w.split) * TOK) * N;
+        for (int c0 = 0; c0 < c_end; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(t_acc + c0, v);
+          tmem_ld_wait();
+          uint32_t* st = reinterpret_cast<uint32_t*>(stage);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) st[j * 32 + lane] = v[j];
+          __syncwarp();
+          if (c0 + tc < c_end) {
+            const uint4* src = reinterpret_cast<const uint4*>(st + tc * 32 + 16 * th);
+            uint4* dst = reinterpret_cast<uint4*>(part + static_cast<size_t>(c0 + tc) * N + nrow0 +
+                                                  16 * th);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) __stcg(dst + e, src[e]);
+          }
+          __syncwarp();
+        }
+        // ... then count the arrival: the mbarrier orders the four warps'
+        // stores before one thread's cumulative fence; the last arrival fences
+        // again before it releases the warps that read the other partials.
+        // The flag is rewritten only after all four warps arrive for the next
+        // split unit, i.e. after each of them has read it.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_epi_in);
+        bool got = true;
+        if (ew == 0 && lane == 0) {
+          got = mbar_wait(bar_epi_in, ks & 1u, abort_flag, &g_error_word, kErrEpilogue);
+          bool last = false;
+          if (got) {
+            __threadfence();
+            last = arrive_last(args.ws_count + w.mt * args.n_tiles + w.nt, splits);
+            if (last) __threadfence();
+          }
+          *last_flag = last ? 1u : 0u;
+          mbar_arrive(bar_epi_go);
+        }
+        got = mbar_wait(bar_epi_go, ks & 1u, abort_flag, &g_error_word, kErrEpilogue) && got;
+        ++ks;
+        write_out = __all_sync(0xffffffffu, got && *last_flag != 0u);
+      }
+      if (write_out && *abort_flag == 0u) {
+        const int32_t* parts = args.ws_part + (static_cast<size_t>(w.mt * splits) * TOK) * N;
+        for (int c0 = 0; c0 < c_end; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(t_acc + c0, v);
+          tmem_ld_wait();
+          if (splits > 1) {
+            for (int q = 0; q < splits; ++q) {
+              if (q == w.split) continue;
+              const int32_t* p = parts + (static_cast<size_t>(q) * TOK + c0) * N + nrow0 + lane;
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                if (c0 + j < c_end) v[j] += static_cast<uint32_t>(__ldcg(p + static_cast<size_t>(j) * N));
+            }
+          }
+          if (args.acc) {
+            uint32_t* st = reinterpret_cast<uint32_t*>(stage);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) st[j * 32 + lane] = v[j];
+            __syncwarp();
+            if (c0 + tc < c_end) {
+              const uint4* src = reinterpret_cast<const uint4*>(st + tc * 32 + 16 * th);
+              uint4* dst = reinterpret_cast<uint4*>(args.acc + static_cast<size_t>(m0 + c0 + tc) * N +
+                                                    nrow0 + 16 * th);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) dst[e] = src[e];
+            }
+          } else {
+            __half* st = reinterpret_cast<__half*>(stage);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float scale = __fmul_rn(sx_w[c0 + j], s1r);
+              st[j * 32 + lane] =
+                  __float2half_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(v[j])), scale));
+            }
+            __syncwarp();
+            if (c0 + tc < c_end) {
+              const uint4* src = reinterpret_cast<const uint4*>(st + tc * 32 + 16 * th);
+              uint4* dst = reinterpret_cast<uint4*>(args.Y + static_cast<size_t>(m0 + c0 + tc) * N +
+                                                    nrow0 + 16 * th);
+              dst[0] = src[0];
+              dst[1] = src[1];
+            }
+          }
+          __syncwarp();
+        }
+      }
+      // the accumulator may be overwritten by the unit after next
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_accempty + 8 * b);
     }
   }
 
@@ -423,7 +485,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   if (warp == 1) {
     __syncwarp();
     tc_fence_after_sync();
-    tmem_dealloc(tmem, C::kTmemCols);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -450,37 +512,45 @@ EncodeTiledFn encode_fn() {
 }
 
 struct Plan {
-  int tok, splits, m_tiles, n_tiles, stages;
+  int tok, splits, m_tiles, n_tiles, stages, units, grid;
 };
 
 bool splittable(const Plan& p) {
   return static_cast<long>(p.m_tiles) * p.n_tiles <= kMaxCounterTiles;
 }
 
-int stages_for(int tok) { return tok <= 32 ? 8 : (tok <= 64 ? 6 : 4); }
+int stages_for(int tok) { return tok <= 128 ? 8 : 4; }
 
 bool valid_tok(int t) { return t == 16 || t == 32 || t == 64 || t == 128 || t == 256; }
 
 int auto_tok(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
 
-int ctas_per_sm(int tok) { return tok <= 128 ? 2 : 1; }
-
-int auto_splits(int tiles, int kt, int tok) {
-  const long slots = static_cast<long>(sm_count()) * ctas_per_sm(tok);
+// Cost model for the number of K splits: units are spread over one CTA per
+// SM, a unit costs its k-tiles plus a fixed overhead (pipeline fill and
+// epilogue), a split unit a little more (partial tile out, final sum in).
+int auto_splits(int tiles, int kt) {
+  const long sms = sm_count();
   int best_s = 1;
-  if (tiles >= slots) return 1;
-  double best = 0.0;
+  double best = 1e30;
   for (int s = 1; s <= 8 && s <= kt; ++s) {
-    if (s > 1 && kt / s < 4) break;
-    const long ctas = static_cast<long>(tiles) * s;
-    const long waves = (ctas + slots - 1) / slots;
-    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
-    if (eff > best + 1e-9) {
-      best = eff;
+    if (s > 1 && kt / s < 2) break;
+    if (static_cast<long>(tiles) * s > 4L * sms && s > 1) break;
+    const long units = static_cast<long>(tiles) * s;
+    const long rounds = (units + sms - 1) / sms;
+    const double cost =
+        static_cast<double>(rounds) * (static_cast<double>(kt) / s + 3.0 + (s > 1 ? 2.0 : 0.0));
+    if (cost < best - 1e-9) {
+      best = cost;
       best_s = s;
     }
   }
   return best_s;
+}
+
+void finish_plan(Plan& p) {
+  p.units = p.n_tiles * p.m_tiles * p.splits;
+  const int sms = sm_count();
+  p.grid = p.units < sms ? p.units : sms;
 }
 
 Plan make_plan(int M, int N, int K, int tok_req, int splits_req) {
@@ -490,8 +560,9 @@ Plan make_plan(int M, int N, int K, int tok_req, int splits_req) {
   p.tok = tok_req ? tok_req : auto_tok(M);
   p.m_tiles = (M + p.tok - 1) / p.tok;
   p.stages = stages_for(p.tok);
-  p.splits = splits_req ? splits_req : auto_splits(p.n_tiles * p.m_tiles, kt, p.tok);
+  p.splits = splits_req ? splits_req : auto_splits(p.n_tiles * p.m_tiles, kt);
   if (!splits_req && !splittable(p)) p.splits = 1;
+  finish_plan(p);
   return p;
 }
 
@@ -516,7 +587,7 @@ int launch_tok(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cudaStr
     if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_RELEASE);
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(p.n_tiles * p.splits), static_cast<unsigned>(p.m_tiles), 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(p.grid), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
@@ -547,7 +618,7 @@ int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* 
     return QOQ_ERR_INVALID_ARG;
 
   Plan p = make_plan(M, N, K, tok_req, splits_req);
-  if (p.m_tiles > 65535) return QOQ_ERR_UNSUPPORTED;
+  if (static_cast<long>(p.n_tiles) * p.m_tiles * p.splits > 0x7fffffffL) return QOQ_ERR_UNSUPPORTED;
   if (p.splits > 1 && !splittable(p)) {
     if (splits_req) return QOQ_ERR_UNSUPPORTED;
     p.splits = 1;
@@ -556,6 +627,7 @@ int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* 
     if (splits_req) return QOQ_ERR_INVALID_ARG;   // explicit split needs its workspace
     p.splits = 1;                                  // auto plan: do not split K
   }
+  finish_plan(p);
   if (int st = check_device()) return st;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return QOQ_ERR_CUDA;
@@ -587,6 +659,9 @@ int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* 
   a.K = K;
   a.group = group;
   a.splits = p.splits;
+  a.m_tiles = p.m_tiles;
+  a.n_tiles = p.n_tiles;
+  a.units = p.units;
   a.blk_bytes = static_cast<int>(block_bytes(group));
 
   cudaStream_t s = as_stream(stream);
@@ -670,7 +745,7 @@ extern "C" int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int*
   const Plan p = make_plan(M, N, K, 0, 0);
   if (tok_tile) *tok_tile = p.tok;
   if (splits) *splits = p.splits;
-  if (ctas) *ctas = p.n_tiles * p.m_tiles * p.splits;
+  if (ctas) *ctas = p.grid;
   if (stages) *stages = p.stages;
   return QOQ_OK;
 }
