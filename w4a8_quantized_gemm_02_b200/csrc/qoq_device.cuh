@@ -19,18 +19,17 @@ enum : uint32_t {
   kErrCounter = 16u,
 };
 
-// Every mbarrier wait gives up after this many nanoseconds of device time.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Every mbarrier wait gives up after this many SM clock cycles (about two
+// seconds at the B200's clocks, longer when the clock is lower).  The cycle
+// counter is read only after many unsuccessful polls, never on the fast path.
+constexpr long long kWaitLimitCycles = 4000000000LL;
+constexpr uint32_t kPollsBeforeTiming = 1024;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t global_timer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
+__device__ __forceinline__ long long sm_clock() { return clock64(); }
 
 // ----------------------------------------------------------------------------
 // mbarrier
@@ -67,20 +66,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for the phase of parity `parity` to complete.  Gives up (returns
-// false) when the CTA-wide abort flag is raised or after kWaitLimitNs, in
+// false) when the CTA-wide abort flag is raised or after kWaitLimitCycles, in
 // which case it raises the abort flag and records `err_bit` in `err_word`
 // (the library's device error word).  Never spins forever.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile uint32_t* abort_flag,
                                           unsigned int* err_word, uint32_t err_bit) {
-  auto poll = [&]() { return mbar_try_wait(bar, parity); };
-  if (poll()) return true;
-  const uint64_t t0 = global_timer_ns();
+  if (mbar_try_wait(bar, parity)) return true;
+  long long t0 = 0;
   for (uint32_t it = 1;; ++it) {
-    if (poll()) return true;
-    if ((it & 63u) == 0) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it % kPollsBeforeTiming) == 0) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      const long long now = sm_clock();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitCycles) {
         *abort_flag = 1u;
         atomicOr(err_word, err_bit);
         return false;

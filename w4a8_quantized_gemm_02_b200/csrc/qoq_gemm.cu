@@ -115,11 +115,16 @@ __device__ __forceinline__ Unit unit_of(const GemmArgs& a, int u, int kt_total) 
 // Bounded wait that ignores the abort flag: used only to drain work already
 // in flight before a CTA tears down.
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
-      atomicOr(&g_error_word, kErrProducer);
-      return;
+  long long t0 = 0;
+  for (uint32_t it = 1; !mbar_try_wait(bar, parity); ++it) {
+    if ((it % kPollsBeforeTiming) == 0) {
+      const long long now = sm_clock();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitCycles) {
+        atomicOr(&g_error_word, kErrProducer);
+        return;
+      }
     }
   }
 }
