@@ -65,7 +65,13 @@ constexpr size_t kCounterBytes = kMaxCounterTiles * 4;
 template <int TOK>
 struct Cfg {
   static constexpr int kStages = TOK <= 128 ? 8 : 4;
-  static constexpr int kAcc = TOK <= 128 ? 2 : 1;   // accumulator buffers
+  // Consecutive MMAs into one accumulator wait for each other, so the K steps
+  // of a tile alternate between kChains independent accumulators (added up in
+  // the epilogue); kAcc sets of them let the epilogue of one unit overlap the
+  // main loop of the next.  Tensor memory: 192 columns of A stages plus
+  // kAcc * kChains * TOK columns of accumulators.
+  static constexpr int kChains = TOK <= 128 ? 2 : 1;
+  static constexpr int kAcc = TOK <= 64 ? 2 : 1;   // accumulator sets
   static constexpr int kXBytes = TOK * kTileK;
   static constexpr int kOffX = 0;
   static constexpr int kOffRaw = kOffX + kStages * kXBytes;
@@ -78,7 +84,7 @@ struct Cfg {
   static_assert(kOffRaw % 1024 == 0 && kXBytes % 1024 == 0, "swizzled tiles need 1 KiB alignment");
   static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-  static_assert(kTmemD + kAcc * TOK <= kTmemCols, "tensor memory");
+  static_assert(kTmemD + kAcc * kChains * TOK <= kTmemCols, "tensor memory");
   static_assert(32 * kDqStages <= kTmemD, "tensor memory A stages");
 };
 
@@ -140,6 +146,22 @@ __device__ __forceinline__ bool arrive_last(uint32_t* ctr, int splits) {
   const bool last = old == static_cast<uint32_t>(splits - 1);
   if (last) atomicExch(ctr, 0u);
   return last;
+}
+
+// 16 accumulator columns of this warp's 32 lanes, summed over the chains
+// (exact INT32 additions).
+template <int CHAINS, int TOK>
+__device__ __forceinline__ void load_acc(uint32_t taddr, uint32_t (&v)[16]) {
+  tmem_ld_32x32b_x16(taddr, v);
+  if (CHAINS > 1) {
+    uint32_t w[16];
+    tmem_ld_32x32b_x16(taddr + TOK, w);
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] += w[j];
+  } else {
+    tmem_ld_wait();
+  }
 }
 
 template <int TOK>
@@ -267,7 +289,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
                        kErrMma))
           break;
         tc_fence_after_sync();
-        const uint32_t d_tmem = tmem + kTmemD + b * TOK;
+        const uint32_t d_tmem = tmem + kTmemD + b * C::kChains * TOK;
         for (int i = 0; i < w.num_kt; ++i, ++g) {
           const int s = g % S, d = g % kDqStages;
           if (!mbar_wait(bar_full + 8 * s, (g / S) & 1, abort_flag, &g_error_word, kErrMma) ||
@@ -283,8 +305,9 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
           for (int kk = 0; kk < kTileK / 32; ++kk) {
             // K = 32 bytes per instruction: 8 tensor-memory columns of A, 32
             // bytes along the swizzled rows of B
-            mma_i8_ts(d_tmem, a_tmem + 8 * kk, smem_desc_sw128(b_addr + kk * 32), idesc,
-                      (i > 0 || kk > 0) ? 1u : 0u);
+            const int ch = kk % C::kChains;
+            mma_i8_ts(d_tmem + ch * TOK, a_tmem + 8 * kk, smem_desc_sw128(b_addr + kk * 32), idesc,
+                      (i > 0 || kk >= C::kChains) ? 1u : 0u);
           }
           mma_commit(bar_empty + 8 * s);     // X tile and raw block of stage s are free
           mma_commit(bar_dqempty + 8 * d);   // A stage d is free
@@ -375,7 +398,8 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
                                 &g_error_word, kErrEpilogue);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after_sync();
-      const uint32_t t_acc = tmem + kTmemD + b * TOK + (static_cast<uint32_t>(q4 * 32) << 16);
+      const uint32_t t_acc =
+          tmem + kTmemD + b * C::kChains * TOK + (static_cast<uint32_t>(q4 * 32) << 16);
       int c_end = M - m0;
       if (c_end > TOK) c_end = TOK;
       float s1r = 0.0f;
@@ -392,8 +416,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
         int32_t* part = args.ws_part + (static_cast<size_t>(w.mt * splits + w.split) * TOK) * N;
         for (int c0 = 0; c0 < c_end; c0 += 16) {
           uint32_t v[16];
-          tmem_ld_32x32b_x16(t_acc + c0, v);
-          tmem_ld_wait();
+          load_acc<C::kChains, TOK>(t_acc + c0, v);
           uint32_t* st = reinterpret_cast<uint32_t*>(stage);
 #pragma unroll
           for (int j = 0; j < 16; ++j) st[j * 32 + lane] = v[j];
@@ -434,8 +457,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
         const int32_t* parts = args.ws_part + (static_cast<size_t>(w.mt * splits) * TOK) * N;
         for (int c0 = 0; c0 < c_end; c0 += 16) {
           uint32_t v[16];
-          tmem_ld_32x32b_x16(t_acc + c0, v);
-          tmem_ld_wait();
+          load_acc<C::kChains, TOK>(t_acc + c0, v);
           if (splits > 1) {
             for (int q = 0; q < splits; ++q) {
               if (q == w.split) continue;
