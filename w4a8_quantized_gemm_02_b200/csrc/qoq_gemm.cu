@@ -223,23 +223,24 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      const uint64_t policy = l2_policy_evict_first();
-      const uint32_t tx = static_cast<uint32_t>(args.blk_bytes + C::kXBytes);
-      uint32_t g = 0;              // running k-tile index of this CTA
-      bool aborted = false;
-      bool first = true;
-      for (int u = blockIdx.x; u < args.units && !aborted; u += gridDim.x) {
-        const Unit w = unit_of(args, u, kt_total);
-        const uint8_t* src =
-            args.packed + (static_cast<size_t>(w.nt) * kt_total + w.kt_begin) * args.blk_bytes;
-        const int m0 = w.mt * TOK;
-        int i = 0;
-        if (first) {
-          // the weight stream does not depend on the preceding grid: start it
-          // before waiting for the activations
-          first = false;
-          const int pre = w.num_kt < S ? w.num_kt : S;
+    // The whole warp runs the loop and waits; one elected lane issues copies.
+    const uint64_t policy = l2_policy_evict_first();
+    const uint32_t tx = static_cast<uint32_t>(args.blk_bytes + C::kXBytes);
+    uint32_t g = 0;              // running k-tile index of this CTA
+    bool aborted = false;
+    bool first = true;
+    for (int u = blockIdx.x; u < args.units && !aborted; u += gridDim.x) {
+      const Unit w = unit_of(args, u, kt_total);
+      const uint8_t* src =
+          args.packed + (static_cast<size_t>(w.nt) * kt_total + w.kt_begin) * args.blk_bytes;
+      const int m0 = w.mt * TOK;
+      int i = 0;
+      if (first) {
+        // the weight stream does not depend on the preceding grid: start it
+        // before waiting for the activations
+        first = false;
+        const int pre = w.num_kt < S ? w.num_kt : S;
+        if (elect_one()) {
           for (int j = 0; j < pre; ++j) {
             mbar_arrive_expect_tx(bar_full + 8 * j, tx);
             bulk_load(base + C::kOffRaw + j * kRawStageBytes,
@@ -250,16 +251,20 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
           for (int j = 0; j < pre; ++j)
             tma_load_2d(base + C::kOffX + j * C::kXBytes, &tmap_x, (w.kt_begin + j) * kTileK, m0,
                         bar_full + 8 * j);
-          i = pre;
-          g = pre;
         }
-        for (; i < w.num_kt; ++i, ++g) {
-          const int s = g % S;
-          if (g >= S && !mbar_wait(bar_empty + 8 * s, ((g / S) & 1) ^ 1, abort_flag, &g_error_word,
-                                   kErrProducer)) {
-            aborted = true;
-            break;
-          }
+        __syncwarp();
+        i = pre;
+        g = pre;
+      }
+      for (; i < w.num_kt; ++i, ++g) {
+        const int s = g % S;
+        if (g >= S && !__all_sync(0xffffffffu, mbar_wait(bar_empty + 8 * s, ((g / S) & 1) ^ 1,
+                                                         abort_flag, &g_error_word,
+                                                         kErrProducer))) {
+          aborted = true;
+          break;
+        }
+        if (elect_one()) {
           mbar_arrive_expect_tx(bar_full + 8 * s, tx);
           bulk_load(base + C::kOffRaw + s * kRawStageBytes,
                     src + static_cast<size_t>(i) * args.blk_bytes,
@@ -267,38 +272,42 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
           tma_load_2d(base + C::kOffX + s * C::kXBytes, &tmap_x, (w.kt_begin + i) * kTileK, m0,
                       bar_full + 8 * s);
         }
+        __syncwarp();
       }
-      if (aborted) {
-        // the copies already issued must land before the CTA exits
-        for (uint32_t j = (g > S ? g - S : 0); j < g; ++j)
-          drain_wait(bar_full + 8 * (j % S), (j / S) & 1);
-      }
+    }
+    if (aborted) {
+      // the copies already issued must land before the CTA exits
+      for (uint32_t j = (g > S ? g - S : 0); j < g; ++j)
+        drain_wait(bar_full + 8 * (j % S), (j / S) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(kTileN, TOK);
-      uint32_t g = 0;
-      int lt = 0;
-      bool aborted = false;
-      for (int u = blockIdx.x; u < args.units && !aborted; u += gridDim.x, ++lt) {
-        const Unit w = unit_of(args, u, kt_total);
-        const int b = lt % C::kAcc;
-        if (lt >= C::kAcc &&
-            !mbar_wait(bar_accempty + 8 * b, ((lt / C::kAcc) & 1) ^ 1, abort_flag, &g_error_word,
-                       kErrMma))
+    // The whole warp runs the loop and waits; one elected lane issues each
+    // tcgen05.mma / tcgen05.commit.
+    constexpr uint32_t idesc = idesc_i8(kTileN, TOK);
+    uint32_t g = 0;
+    int lt = 0;
+    bool aborted = false;
+    for (int u = blockIdx.x; u < args.units && !aborted; u += gridDim.x, ++lt) {
+      const Unit w = unit_of(args, u, kt_total);
+      const int b = lt % C::kAcc;
+      if (lt >= C::kAcc &&
+          !__all_sync(0xffffffffu, mbar_wait(bar_accempty + 8 * b, ((lt / C::kAcc) & 1) ^ 1,
+                                             abort_flag, &g_error_word, kErrMma)))
+        break;
+      tc_fence_after_sync();
+      const uint32_t d_tmem = tmem + kTmemD + b * C::kChains * TOK;
+      for (int i = 0; i < w.num_kt; ++i, ++g) {
+        const int s = g % S, d = g % kDqStages;
+        const bool ready =
+            mbar_wait(bar_full + 8 * s, (g / S) & 1, abort_flag, &g_error_word, kErrMma) &&
+            mbar_wait(bar_dqfull + 8 * d, (g / kDqStages) & 1, abort_flag, &g_error_word, kErrMma);
+        if (!__all_sync(0xffffffffu, ready)) {
+          aborted = true;
           break;
+        }
         tc_fence_after_sync();
-        const uint32_t d_tmem = tmem + kTmemD + b * C::kChains * TOK;
-        for (int i = 0; i < w.num_kt; ++i, ++g) {
-          const int s = g % S, d = g % kDqStages;
-          if (!mbar_wait(bar_full + 8 * s, (g / S) & 1, abort_flag, &g_error_word, kErrMma) ||
-              !mbar_wait(bar_dqfull + 8 * d, (g / kDqStages) & 1, abort_flag, &g_error_word,
-                         kErrMma)) {
-            aborted = true;
-            break;
-          }
-          tc_fence_after_sync();
+        if (elect_one()) {
           const uint32_t a_tmem = tmem + kTmemA + 32 * d;
           const uint32_t b_addr = base + C::kOffX + s * C::kXBytes;
 #pragma unroll
@@ -312,11 +321,14 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
           mma_commit(bar_empty + 8 * s);     // X tile and raw block of stage s are free
           mma_commit(bar_dqempty + 8 * d);   // A stage d is free
         }
-        if (!aborted) mma_commit(bar_accfull + 8 * b);   // accumulator b is complete
+        __syncwarp();
       }
-      mma_commit(bar_drain);
-      drain_wait(bar_drain, 0);              // no MMA in flight past this point
+      if (!aborted && elect_one()) mma_commit(bar_accfull + 8 * b);   // accumulator b is complete
+      __syncwarp();
     }
+    if (elect_one()) mma_commit(bar_drain);
+    __syncwarp();
+    drain_wait(bar_drain, 0);                // no MMA in flight past this point
   } else if (warp < kWarpEpi0) {
     // ---------------------------------------------------------------- dequantizers
     const int wg = (warp - 2) >> 2;         // 0 .. kDqGroups-1: takes k-tiles g = wg (mod 3)
