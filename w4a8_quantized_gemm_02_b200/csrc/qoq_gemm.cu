@@ -19,7 +19,8 @@
 //   warp 1       owns tensor memory and issues tcgen05.mma.kind::i8 (M = 128,
 //                N = TOK, K = 32 per instruction) with the INT8 weights read
 //                from tensor memory and X8 from shared memory, into one of two
-//                INT32 accumulators in tensor memory (double buffered);
+//                INT32 accumulators in tensor memory (double buffered); one
+//                commit per k-tile releases the whole stage;
 //   warps 2..13  three dequantizing warpgroups taking k-tiles in turn: each
 //                thread turns one weight row of the UINT4 block into INT8
 //                (four byte lanes per 32-bit multiply-add) and writes the
@@ -51,8 +52,7 @@ constexpr int kWarpEpi0 = 2 + 4 * kDqGroups;     // first epilogue warp (14)
 constexpr int kWarps = kWarpEpi0 + 4;            // 18
 constexpr int kThreads = 32 * kWarps;            // 576
 constexpr int kRawStageBytes = 8576;             // largest packed block (group 64)
-constexpr int kDqStages = 6;                     // tensor-memory A stages
-constexpr int kTmemA = 0;                        // A stage d at column 32 d
+constexpr int kTmemA = 0;                        // A operand of stage s at column 32 s
 constexpr int kTmemD = 256;                      // accumulators from column 256
 constexpr int kTmemCols = 512;
 constexpr int kStageBytesEpi = 32 * 16 * 4;      // per epilogue warp: 16 columns x 32 rows
@@ -64,28 +64,26 @@ constexpr size_t kCounterBytes = kMaxCounterTiles * 4;
 
 template <int TOK>
 struct Cfg {
+  // One ring of kStages stages: stage s holds the X8 tile and the packed
+  // weight block in shared memory and the dequantized INT8 weights in tensor
+  // memory columns 32 s .. 32 s + 31.  kAcc accumulators of TOK columns let
+  // the epilogue of one unit overlap the main loop of the next.
   static constexpr int kStages = TOK <= 128 ? 8 : 4;
-  // Consecutive MMAs into one accumulator wait for each other, so the K steps
-  // of a tile alternate between kChains independent accumulators (added up in
-  // the epilogue); kAcc sets of them let the epilogue of one unit overlap the
-  // main loop of the next.  Tensor memory: 192 columns of A stages plus
-  // kAcc * kChains * TOK columns of accumulators.
-  static constexpr int kChains = TOK <= 128 ? 2 : 1;
-  static constexpr int kAcc = TOK <= 64 ? 2 : 1;   // accumulator sets
+  static constexpr int kAcc = TOK <= 128 ? 2 : 1;
   static constexpr int kXBytes = TOK * kTileK;
   static constexpr int kOffX = 0;
   static constexpr int kOffRaw = kOffX + kStages * kXBytes;
   static constexpr int kOffEpi = kOffRaw + kStages * kRawStageBytes;
   static constexpr int kOffSx = kOffEpi + 4 * kStageBytesEpi;          // 4 warps x TOK floats
   static constexpr int kOffBar = kOffSx + 4 * TOK * 4;
-  static constexpr int kNumBars = 2 * kStages + 2 * kDqStages + 2 * kAcc + 3;
+  static constexpr int kNumBars = 3 * kStages + 2 * kAcc + 3;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 32 + 1024;   // + base alignment slack
   static_assert(kOffRaw % 1024 == 0 && kXBytes % 1024 == 0, "swizzled tiles need 1 KiB alignment");
   static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-  static_assert(kTmemD + kAcc * kChains * TOK <= kTmemCols, "tensor memory");
-  static_assert(32 * kDqStages <= kTmemD, "tensor memory A stages");
+  static_assert(kTmemD + kAcc * TOK <= kTmemCols, "tensor memory");
+  static_assert(kTmemA + 32 * kStages <= kTmemD, "tensor memory A stages");
 };
 
 struct GemmArgs {
@@ -148,22 +146,6 @@ __device__ __forceinline__ bool arrive_last(uint32_t* ctr, int splits) {
   return last;
 }
 
-// 16 accumulator columns of this warp's 32 lanes, summed over the chains
-// (exact INT32 additions).
-template <int CHAINS, int TOK>
-__device__ __forceinline__ void load_acc(uint32_t taddr, uint32_t (&v)[16]) {
-  tmem_ld_32x32b_x16(taddr, v);
-  if (CHAINS > 1) {
-    uint32_t w[16];
-    tmem_ld_32x32b_x16(taddr + TOK, w);
-    tmem_ld_wait();
-#pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] += w[j];
-  } else {
-    tmem_ld_wait();
-  }
-}
-
 template <int TOK>
 __global__ void __launch_bounds__(kThreads, 1)
 w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args) {
@@ -178,11 +160,13 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   const int lane = threadIdx.x & 31;
   const int kt_total = args.K / kTileK;
 
+  // full[s]: X tile and weight block landed; dqfull[s]: A operand written
+  // (implies full); empty[s]: the MMAs of the stage completed (the producer
+  // may refill it, which in turn frees its A columns for the dequantizers)
   const uint32_t bar_full = base + C::kOffBar;
   const uint32_t bar_empty = bar_full + 8 * S;
   const uint32_t bar_dqfull = bar_empty + 8 * S;
-  const uint32_t bar_dqempty = bar_dqfull + 8 * kDqStages;
-  const uint32_t bar_accfull = bar_dqempty + 8 * kDqStages;
+  const uint32_t bar_accfull = bar_dqfull + 8 * S;
   const uint32_t bar_accempty = bar_accfull + 8 * C::kAcc;
   const uint32_t bar_drain = bar_accempty + 8 * C::kAcc;
   const uint32_t bar_epi_in = bar_drain + 8;    // four epilogue warps published a partial
@@ -195,10 +179,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     for (int s = 0; s < S; ++s) {
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
-    }
-    for (int d = 0; d < kDqStages; ++d) {
-      mbar_init(bar_dqfull + 8 * d, 4);
-      mbar_init(bar_dqempty + 8 * d, 1);
+      mbar_init(bar_dqfull + 8 * s, 4);
     }
     for (int b = 0; b < C::kAcc; ++b) {
       mbar_init(bar_accfull + 8 * b, 1);
@@ -296,30 +277,26 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
                                              abort_flag, &g_error_word, kErrMma)))
         break;
       tc_fence_after_sync();
-      const uint32_t d_tmem = tmem + kTmemD + b * C::kChains * TOK;
+      const uint32_t d_tmem = tmem + kTmemD + b * TOK;
       for (int i = 0; i < w.num_kt; ++i, ++g) {
-        const int s = g % S, d = g % kDqStages;
-        const bool ready =
-            mbar_wait(bar_full + 8 * s, (g / S) & 1, abort_flag, &g_error_word, kErrMma) &&
-            mbar_wait(bar_dqfull + 8 * d, (g / kDqStages) & 1, abort_flag, &g_error_word, kErrMma);
-        if (!__all_sync(0xffffffffu, ready)) {
+        const int s = g % S;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_dqfull + 8 * s, (g / S) & 1, abort_flag,
+                                               &g_error_word, kErrMma))) {
           aborted = true;
           break;
         }
         tc_fence_after_sync();
         if (elect_one()) {
-          const uint32_t a_tmem = tmem + kTmemA + 32 * d;
+          const uint32_t a_tmem = tmem + kTmemA + 32 * s;
           const uint32_t b_addr = base + C::kOffX + s * C::kXBytes;
 #pragma unroll
           for (int kk = 0; kk < kTileK / 32; ++kk) {
             // K = 32 bytes per instruction: 8 tensor-memory columns of A, 32
             // bytes along the swizzled rows of B
-            const int ch = kk % C::kChains;
-            mma_i8_ts(d_tmem + ch * TOK, a_tmem + 8 * kk, smem_desc_sw128(b_addr + kk * 32), idesc,
-                      (i > 0 || kk >= C::kChains) ? 1u : 0u);
+            mma_i8_ts(d_tmem, a_tmem + 8 * kk, smem_desc_sw128(b_addr + kk * 32), idesc,
+                      (i > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(bar_empty + 8 * s);     // X tile and raw block of stage s are free
-          mma_commit(bar_dqempty + 8 * d);   // A stage d is free
+          mma_commit(bar_empty + 8 * s);     // stage s is free once these MMAs complete
         }
         __syncwarp();
       }
@@ -342,11 +319,10 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
       const Unit w = unit_of(args, u, kt_total);
       for (int i = 0; i < w.num_kt; ++i, ++g) {
         if (static_cast<int>(g % kDqGroups) != wg) continue;
-        const int s = g % S, d = g % kDqStages;
-        if (!mbar_wait(bar_full + 8 * s, (g / S) & 1, abort_flag, &g_error_word, kErrDequant) ||
-            (g >= kDqStages &&
-             !mbar_wait(bar_dqempty + 8 * d, ((g / kDqStages) & 1) ^ 1, abort_flag, &g_error_word,
-                        kErrDequant))) {
+        const int s = g % S;
+        // the stage was refilled only after the MMAs that read its A columns
+        // completed, so landing data also means the A columns are free
+        if (!mbar_wait(bar_full + 8 * s, (g / S) & 1, abort_flag, &g_error_word, kErrDequant)) {
           aborted = true;
           break;
         }
@@ -380,11 +356,11 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
           out[8 * j + 7] = dq_lanes(hi_codes(v.w), sv, bv);
         }
         // one 128-byte row of the INT8 A operand: column c holds K bytes 4c..4c+3
-        tmem_st_32x32b_x32(row_tmem + kTmemA + 32 * d, out);
+        tmem_st_32x32b_x32(row_tmem + kTmemA + 32 * s, out);
         tmem_st_wait();
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_dqfull + 8 * d);
+        if (lane == 0) mbar_arrive(bar_dqfull + 8 * s);
       }
     }
   } else {
@@ -410,8 +386,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
                                 &g_error_word, kErrEpilogue);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after_sync();
-      const uint32_t t_acc =
-          tmem + kTmemD + b * C::kChains * TOK + (static_cast<uint32_t>(q4 * 32) << 16);
+      const uint32_t t_acc = tmem + kTmemD + b * TOK + (static_cast<uint32_t>(q4 * 32) << 16);
       int c_end = M - m0;
       if (c_end > TOK) c_end = TOK;
       float s1r = 0.0f;
@@ -428,7 +403,8 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
         int32_t* part = args.ws_part + (static_cast<size_t>(w.mt * splits + w.split) * TOK) * N;
         for (int c0 = 0; c0 < c_end; c0 += 16) {
           uint32_t v[16];
-          load_acc<C::kChains, TOK>(t_acc + c0, v);
+          tmem_ld_32x32b_x16(t_acc + c0, v);
+          tmem_ld_wait();
           uint32_t* st = reinterpret_cast<uint32_t*>(stage);
 #pragma unroll
           for (int j = 0; j < 16; ++j) st[j * 32 + lane] = v[j];
@@ -469,7 +445,8 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
         const int32_t* parts = args.ws_part + (static_cast<size_t>(w.mt * splits) * TOK) * N;
         for (int c0 = 0; c0 < c_end; c0 += 16) {
           uint32_t v[16];
-          load_acc<C::kChains, TOK>(t_acc + c0, v);
+          tmem_ld_32x32b_x16(t_acc + c0, v);
+          tmem_ld_wait();
           if (splits > 1) {
             for (int q = 0; q < splits; ++q) {
               if (q == w.split) continue;
