@@ -544,7 +544,10 @@ int auto_tok(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
 // Cost model for the number of K splits: units are spread over one CTA per
 // SM, a unit costs its k-tiles plus a fixed overhead (pipeline fill and
 // epilogue), a split unit a little more (partial tile out, final sum in).
-int auto_splits(int tiles, int kt) {
+// Only small token tiles are split: for 64 tokens and more the partial tiles
+// cost more than the parallelism gains.
+int auto_splits(int tiles, int kt, int tok) {
+  if (tok > 32) return 1;
   const long sms = sm_count();
   int best_s = 1;
   double best = 1e30;
@@ -576,7 +579,7 @@ Plan make_plan(int M, int N, int K, int tok_req, int splits_req) {
   p.tok = tok_req ? tok_req : auto_tok(M);
   p.m_tiles = (M + p.tok - 1) / p.tok;
   p.stages = stages_for(p.tok);
-  p.splits = splits_req ? splits_req : auto_splits(p.n_tiles * p.m_tiles, kt);
+  p.splits = splits_req ? splits_req : auto_splits(p.n_tiles * p.m_tiles, kt, p.tok);
   if (!splits_req && !splittable(p)) p.splits = 1;
   finish_plan(p);
   return p;
