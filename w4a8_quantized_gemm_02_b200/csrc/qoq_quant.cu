@@ -35,25 +35,39 @@ __device__ __forceinline__ int div_rne(int a, int b) {
 }
 
 // ---------------------------------------------------------------------------
-// Per-token activation quantization: one warp per row, 8 rows per CTA.  The
-// first pass keeps many 16-byte loads in flight per lane and reduces the
-// abs-max with warp shuffles; the second pass re-reads the row (now in L2 /
-// L1) and writes the INT8 codes.  Rows of up to 32 * 8 * kActRegVec values
-// are kept in registers between the passes instead.
+// Per-token activation quantization.
+//
+// The code of a value is rne(x / sx) clamped to [-127, 127].  Instead of an
+// IEEE division per element, the quotient is rounded through the reciprocal
+// of the row's scale and then corrected with the exact remainder
+// e = x - q * sx (a single fused multiply-add, exact because q * sx and x are
+// short FP16-derived numbers): |e| > sx/2 moves q one step towards e, and
+// |e| == sx/2 is a tie that goes to the even neighbour.  This yields the
+// round-half-even of the exact quotient x / sx.  For FP16 x and sx that equals
+// rounding the binary32 quotient (the binary32 result can only sit on a
+// half-integer if the exact quotient does), so the codes match an IEEE
+// binary32 division bit for bit.
 // ---------------------------------------------------------------------------
 constexpr int kActWarps = 8;
 constexpr int kActRegVec = 16;
 
-__device__ __forceinline__ uint2 quantize8(uint4 v, float sf) {
+__device__ __forceinline__ int quant_code(float x, float sf, float rcp, float half_sf) {
+  float q = rintf(__fmul_rn(x, rcp));
+  const float e = __fmaf_rn(-q, sf, x);
+  const float ae = fabsf(e);
+  if (ae > half_sf || (ae == half_sf && fmodf(q, 2.0f) != 0.0f)) q += copysignf(1.0f, e);
+  const int v = static_cast<int>(q);
+  return max(-127, min(127, v));
+}
+
+__device__ __forceinline__ uint2 quantize8(uint4 v, float sf, float rcp, float half_sf) {
   const __half2* h = reinterpret_cast<const __half2*>(&v);
   uint32_t packed[2] = {0u, 0u};
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const float2 f = __half22float2(h[j]);
-    int a = __float2int_rn(__fdiv_rn(f.x, sf));
-    int b = __float2int_rn(__fdiv_rn(f.y, sf));
-    a = max(-127, min(127, a));
-    b = max(-127, min(127, b));
+    const int a = quant_code(f.x, sf, rcp, half_sf);
+    const int b = quant_code(f.y, sf, rcp, half_sf);
     const uint32_t pair = (static_cast<uint32_t>(a) & 0xffu) |
                           ((static_cast<uint32_t>(b) & 0xffu) << 8);
     packed[j >> 1] |= pair << (16 * (j & 1));
@@ -71,56 +85,74 @@ __device__ __forceinline__ float absmax8(uint4 v, float amax) {
   return amax;
 }
 
+// WARPS_PER_ROW warps share a row (1 for many rows, 8 when rows are few);
+// kActWarps / WARPS_PER_ROW rows per CTA.
+template <int WARPS_PER_ROW>
 __global__ void __launch_bounds__(32 * kActWarps)
 act_quant_kernel(const __half* __restrict__ X, int M, int K, int8_t* __restrict__ X8,
                  __half* __restrict__ sx) {
   // the GEMM that consumes X8 may start its weight prologue right away
   grid_launch_dependents();
+  __shared__ float red[kActWarps];
+  const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m = blockIdx.x * kActWarps + (threadIdx.x >> 5);
-  if (m >= M) return;
-  const uint4* row = reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K);
-  uint2* out = reinterpret_cast<uint2*>(X8 + static_cast<size_t>(m) * K);
-  const int nvec = K / 8;
+  constexpr int kRows = kActWarps / WARPS_PER_ROW;
+  const int m = blockIdx.x * kRows + warp / WARPS_PER_ROW;
+  const int t = (warp % WARPS_PER_ROW) * 32 + lane;   // thread index within the row
+  constexpr int kT = 32 * WARPS_PER_ROW;               // threads per row
+  const bool active = m < M;
+  const uint4* row = reinterpret_cast<const uint4*>(X + static_cast<size_t>(active ? m : 0) * K);
+  uint2* out = reinterpret_cast<uint2*>(X8 + static_cast<size_t>(active ? m : 0) * K);
+  const int nvec = active ? K / 8 : 0;
+  const bool in_regs = K / 8 <= kT * kActRegVec;
+  uint4 v[kActRegVec];
   float amax = 0.0f;
-  if (nvec <= 32 * kActRegVec) {
-    uint4 v[kActRegVec];
+  if (in_regs) {
 #pragma unroll
     for (int u = 0; u < kActRegVec; ++u) {
-      const int i = lane + 32 * u;
+      const int i = t + kT * u;
       if (i < nvec) v[u] = __ldg(row + i);
     }
 #pragma unroll
     for (int u = 0; u < kActRegVec; ++u)
-      if (lane + 32 * u < nvec) amax = absmax8(v[u], amax);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const __half s = scale_from_absmax(amax, 127.0f);
-    if (lane == 0) sx[m] = s;
-    const float sf = __half2float(s);
-#pragma unroll
-    for (int u = 0; u < kActRegVec; ++u) {
-      const int i = lane + 32 * u;
-      if (i < nvec) out[i] = quantize8(v[u], sf);
-    }
+      if (t + kT * u < nvec) amax = absmax8(v[u], amax);
   } else {
-    for (int i0 = 0; i0 < nvec; i0 += 32 * 8) {
-      uint4 v[8];
+    for (int i0 = 0; i0 < nvec; i0 += kT * 8) {
+      uint4 w[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int i = i0 + lane + 32 * u;
-        if (i < nvec) v[u] = __ldg(row + i);
+        const int i = i0 + t + kT * u;
+        if (i < nvec) w[u] = __ldg(row + i);
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u)
-        if (i0 + lane + 32 * u < nvec) amax = absmax8(v[u], amax);
+        if (i0 + t + kT * u < nvec) amax = absmax8(w[u], amax);
     }
+  }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const __half s = scale_from_absmax(amax, 127.0f);
-    if (lane == 0) sx[m] = s;
-    const float sf = __half2float(s);
-    for (int i = lane; i < nvec; i += 32) out[i] = quantize8(__ldg(row + i), sf);
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (WARPS_PER_ROW > 1) {
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    amax = 0.0f;
+#pragma unroll
+    for (int w = 0; w < WARPS_PER_ROW; ++w)
+      amax = fmaxf(amax, red[(warp / WARPS_PER_ROW) * WARPS_PER_ROW + w]);
+  }
+  if (!active) return;
+  const __half s = scale_from_absmax(amax, 127.0f);
+  if (t == 0) sx[m] = s;
+  const float sf = __half2float(s);
+  const float rcp = __frcp_rn(sf);
+  const float half_sf = 0.5f * sf;
+  if (in_regs) {
+#pragma unroll
+    for (int u = 0; u < kActRegVec; ++u) {
+      const int i = t + kT * u;
+      if (i < nvec) out[i] = quantize8(v[u], sf, rcp, half_sf);
+    }
+  } else {
+    for (int i = t; i < nvec; i += kT) out[i] = quantize8(__ldg(row + i), sf, rcp, half_sf);
   }
 }
 
@@ -312,8 +344,15 @@ using namespace qoq;
 
 namespace qoq {
 int launch_act_quant(const void* X, int M, int K, int8_t* X8, void* sx, void* stream) {
-  act_quant_kernel<<<(M + kActWarps - 1) / kActWarps, 32 * kActWarps, 0, as_stream(stream)>>>(
-      static_cast<const __half*>(X), M, K, X8, static_cast<__half*>(sx));
+  const __half* Xh = static_cast<const __half*>(X);
+  __half* sxh = static_cast<__half*>(sx);
+  if (M <= 2 * sm_count()) {
+    // few rows: a whole CTA per row keeps many loads in flight per row
+    act_quant_kernel<kActWarps><<<M, 32 * kActWarps, 0, as_stream(stream)>>>(Xh, M, K, X8, sxh);
+  } else {
+    act_quant_kernel<1><<<(M + kActWarps - 1) / kActWarps, 32 * kActWarps, 0,
+                          as_stream(stream)>>>(Xh, M, K, X8, sxh);
+  }
   return launch_status();
 }
 }  // namespace qoq
