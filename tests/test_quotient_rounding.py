@@ -5,8 +5,10 @@ binary32 division (what the oracle does):
 
 1. for FP16 x and FP16 sx > 0, rounding the binary32 quotient to the nearest
    integer (ties to even) equals rounding the exact quotient;
-2. the remainder-corrected procedure, replayed here with numpy binary32
-   operations, returns the round-half-even of the exact quotient.
+2. the procedure (rounding x * rcp(sx) with the 1.5 * 2^23 offset in one
+   fused multiply-add, then correcting with the exact remainder), replayed
+   here with numpy binary32 operations, returns the round-half-even of the
+   exact quotient.
 """
 import numpy as np
 
@@ -29,15 +31,19 @@ def test_binary32_quotient_rounds_like_exact_quotient():
 
 def _remainder_rounding(x, s):
     """The kernel's steps with binary32 arithmetic."""
+    magic = np.float64(12582912.0)                 # 1.5 * 2^23
     s = np.float32(s)
     rcp = np.float32(1.0) / s                      # correctly rounded reciprocal
-    q = np.rint((x * rcp).astype(np.float32))      # binary32 product, then rint
+    # fma(x, rcp, magic): x * rcp + magic is exact in binary64 here, one rounding
+    t = (x.astype(np.float64) * np.float64(rcp) + magic).astype(np.float32)
+    q = t.astype(np.float64) - magic               # exact integer
     # fma(-q, s, x): exact in binary64 and representable in binary32 here
-    e = (x.astype(np.float64) - q.astype(np.float64) * np.float64(s))
+    e = (x.astype(np.float64) - q * np.float64(s))
     assert np.array_equal(e.astype(np.float32).astype(np.float64), e)
     ae = np.abs(e)
     half = np.float64(s) / 2
-    move = (ae > half) | ((ae == half) & (np.fmod(q, 2) != 0))
+    odd = (t.view(np.uint32) & 1) != 0             # parity of t is the parity of q
+    move = (ae > half) | ((ae == half) & odd)
     return q + np.where(move, np.sign(e), 0)
 
 

@@ -37,76 +37,96 @@ __device__ __forceinline__ int div_rne(int a, int b) {
 // ---------------------------------------------------------------------------
 // Per-token activation quantization.
 //
-// The code of a value is rne(x / sx) clamped to [-127, 127].  Instead of an
-// IEEE division per element, the quotient is rounded through the reciprocal
-// of the row's scale and then corrected with the exact remainder
-// e = x - q * sx (a single fused multiply-add, exact because q * sx and x are
-// short FP16-derived numbers): |e| > sx/2 moves q one step towards e, and
-// |e| == sx/2 is a tie that goes to the even neighbour.  This yields the
-// round-half-even of the exact quotient x / sx.  For FP16 x and sx that equals
-// rounding the binary32 quotient (the binary32 result can only sit on a
-// half-integer if the exact quotient does), so the codes match an IEEE
-// binary32 division bit for bit.
+// The code of a value is rne(x / sx) clamped to [-127, 127], computed without
+// a division:
+//  1. t = fma(x, rcp(sx), 1.5 * 2^23) rounds x * rcp to an integer q0 in one
+//     step: t holds 1.5 * 2^23 + q0, so its low byte is q0 as a two's
+//     complement INT8 and t - 1.5 * 2^23 is q0 exactly.
+//  2. e = x - q0 * sx is exact (one fused multiply-add: q0 * sx and x are short
+//     FP16-derived numbers).  q0 is within 0.5 + 2^-17 of x / sx, so it is the
+//     nearest integer unless |e| >= sx / 2.  That is rare (a quotient within
+//     2^-17 of a half-integer), and only then does a lane take the fix-up:
+//     |e| > sx / 2 moves q0 one step towards e, |e| == sx / 2 is a tie that
+//     goes to the even neighbour.
+// The result is the round-half-even of the exact quotient x / sx.  For FP16 x
+// and sx that equals rounding the binary32 quotient (the binary32 result can
+// only sit on a half-integer if the exact quotient does), so the codes match
+// an IEEE binary32 division bit for bit.
+// When sx is a normal FP16 number, |x| / sx <= 127 / (1 - 2^-11) < 127.5 and
+// no code can leave [-127, 127]; only rows whose scale is subnormal clamp.
 // ---------------------------------------------------------------------------
-constexpr int kActWarps = 8;
 constexpr int kActRegVec = 16;
+constexpr float kRoundMagic = 12582912.0f;   // 1.5 * 2^23
 
-__device__ __forceinline__ int quant_code(float x, float sf, float rcp, float half_sf) {
-  float q = rintf(__fmul_rn(x, rcp));
-  const float e = __fmaf_rn(-q, sf, x);
-  const float ae = fabsf(e);
-  if (ae > half_sf || (ae == half_sf && fmodf(q, 2.0f) != 0.0f)) q += copysignf(1.0f, e);
-  const int v = static_cast<int>(q);
-  return max(-127, min(127, v));
-}
-
+template <bool kClamp>
 __device__ __forceinline__ uint2 quantize8(uint4 v, float sf, float rcp, float half_sf) {
   const __half2* h = reinterpret_cast<const __half2*>(&v);
-  uint32_t packed[2] = {0u, 0u};
+  float x[8], t[8];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const float2 f = __half22float2(h[j]);
-    const int a = quant_code(f.x, sf, rcp, half_sf);
-    const int b = quant_code(f.y, sf, rcp, half_sf);
-    const uint32_t pair = (static_cast<uint32_t>(a) & 0xffu) |
-                          ((static_cast<uint32_t>(b) & 0xffu) << 8);
-    packed[j >> 1] |= pair << (16 * (j & 1));
+    x[2 * j] = f.x;
+    x[2 * j + 1] = f.y;
   }
-  return make_uint2(packed[0], packed[1]);
+  bool near_half = false;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    t[j] = __fmaf_rn(x[j], rcp, kRoundMagic);
+    const float e = __fmaf_rn(-(t[j] - kRoundMagic), sf, x[j]);
+    near_half |= fabsf(e) >= half_sf;
+  }
+  if (near_half) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float e = __fmaf_rn(-(t[j] - kRoundMagic), sf, x[j]);
+      const float ae = fabsf(e);
+      const bool odd = __float_as_uint(t[j]) & 1u;   // the offset 1.5 * 2^23 is even
+      if (ae > half_sf || (ae == half_sf && odd)) t[j] += e > 0.0f ? 1.0f : -1.0f;
+    }
+  }
+  if (kClamp) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) t[j] = fminf(fmaxf(t[j], kRoundMagic - 127.0f), kRoundMagic + 127.0f);
+  }
+  uint32_t b[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) b[j] = __float_as_uint(t[j]);
+  const uint32_t w0 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040),
+                                  0x5410);
+  const uint32_t w1 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040),
+                                  0x5410);
+  return make_uint2(w0, w1);
 }
 
-__device__ __forceinline__ float absmax8(uint4 v, float amax) {
+__device__ __forceinline__ __half2 absmax8(uint4 v, __half2 amax) {
   const __half2* h = reinterpret_cast<const __half2*>(&v);
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float2 f = __half22float2(h[j]);
-    amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
-  }
+  for (int j = 0; j < 4; ++j) amax = __hmax2(amax, __habs2(h[j]));
   return amax;
 }
 
-// WARPS_PER_ROW warps share a row (1 for many rows, 8 when rows are few);
-// kActWarps / WARPS_PER_ROW rows per CTA.
-template <int WARPS_PER_ROW>
-__global__ void __launch_bounds__(32 * kActWarps)
+// kWarps warps per CTA, kWarpsPerRow of them share a row: 1 for many rows
+// (a warp per row), kWarps when rows are few (a CTA per row).
+template <int kWarps, int kWarpsPerRow>
+__global__ void __launch_bounds__(32 * kWarps)
 act_quant_kernel(const __half* __restrict__ X, int M, int K, int8_t* __restrict__ X8,
                  __half* __restrict__ sx) {
   // the GEMM that consumes X8 may start its weight prologue right away
   grid_launch_dependents();
-  __shared__ float red[kActWarps];
+  __shared__ float red[kWarps];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  constexpr int kRows = kActWarps / WARPS_PER_ROW;
-  const int m = blockIdx.x * kRows + warp / WARPS_PER_ROW;
-  const int t = (warp % WARPS_PER_ROW) * 32 + lane;   // thread index within the row
-  constexpr int kT = 32 * WARPS_PER_ROW;               // threads per row
+  constexpr int kRows = kWarps / kWarpsPerRow;
+  const int m = blockIdx.x * kRows + warp / kWarpsPerRow;
+  const int t = (warp % kWarpsPerRow) * 32 + lane;   // thread index within the row
+  constexpr int kT = 32 * kWarpsPerRow;              // threads per row
   const bool active = m < M;
   const uint4* row = reinterpret_cast<const uint4*>(X + static_cast<size_t>(active ? m : 0) * K);
   uint2* out = reinterpret_cast<uint2*>(X8 + static_cast<size_t>(active ? m : 0) * K);
   const int nvec = active ? K / 8 : 0;
   const bool in_regs = K / 8 <= kT * kActRegVec;
   uint4 v[kActRegVec];
-  float amax = 0.0f;
+  __half2 hmax = __float2half2_rn(0.0f);
   if (in_regs) {
 #pragma unroll
     for (int u = 0; u < kActRegVec; ++u) {
@@ -115,7 +135,7 @@ act_quant_kernel(const __half* __restrict__ X, int M, int K, int8_t* __restrict_
     }
 #pragma unroll
     for (int u = 0; u < kActRegVec; ++u)
-      if (t + kT * u < nvec) amax = absmax8(v[u], amax);
+      if (t + kT * u < nvec) hmax = absmax8(v[u], hmax);
   } else {
     for (int i0 = 0; i0 < nvec; i0 += kT * 8) {
       uint4 w[8];
@@ -126,18 +146,19 @@ act_quant_kernel(const __half* __restrict__ X, int M, int K, int8_t* __restrict_
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u)
-        if (i0 + t + kT * u < nvec) amax = absmax8(w[u], amax);
+        if (i0 + t + kT * u < nvec) hmax = absmax8(w[u], hmax);
     }
   }
+  float amax = fmaxf(__low2float(hmax), __high2float(hmax));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  if (WARPS_PER_ROW > 1) {
+  if (kWarpsPerRow > 1) {
     if (lane == 0) red[warp] = amax;
     __syncthreads();
     amax = 0.0f;
 #pragma unroll
-    for (int w = 0; w < WARPS_PER_ROW; ++w)
-      amax = fmaxf(amax, red[(warp / WARPS_PER_ROW) * WARPS_PER_ROW + w]);
+    for (int w = 0; w < kWarpsPerRow; ++w)
+      amax = fmaxf(amax, red[(warp / kWarpsPerRow) * kWarpsPerRow + w]);
   }
   if (!active) return;
   const __half s = scale_from_absmax(amax, 127.0f);
@@ -145,14 +166,27 @@ act_quant_kernel(const __half* __restrict__ X, int M, int K, int8_t* __restrict_
   const float sf = __half2float(s);
   const float rcp = __frcp_rn(sf);
   const float half_sf = 0.5f * sf;
+  const bool clamp = sf < 6.103515625e-05f;   // subnormal FP16 scale (below 2^-14)
   if (in_regs) {
+    if (!clamp) {
 #pragma unroll
-    for (int u = 0; u < kActRegVec; ++u) {
-      const int i = t + kT * u;
-      if (i < nvec) out[i] = quantize8(v[u], sf, rcp, half_sf);
+      for (int u = 0; u < kActRegVec; ++u) {
+        const int i = t + kT * u;
+        if (i < nvec) out[i] = quantize8<false>(v[u], sf, rcp, half_sf);
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < kActRegVec; ++u) {
+        const int i = t + kT * u;
+        if (i < nvec) out[i] = quantize8<true>(v[u], sf, rcp, half_sf);
+      }
     }
   } else {
-    for (int i = t; i < nvec; i += kT) out[i] = quantize8(__ldg(row + i), sf, rcp, half_sf);
+    if (!clamp) {
+      for (int i = t; i < nvec; i += kT) out[i] = quantize8<false>(__ldg(row + i), sf, rcp, half_sf);
+    } else {
+      for (int i = t; i < nvec; i += kT) out[i] = quantize8<true>(__ldg(row + i), sf, rcp, half_sf);
+    }
   }
 }
 
@@ -348,10 +382,9 @@ int launch_act_quant(const void* X, int M, int K, int8_t* X8, void* sx, void* st
   __half* sxh = static_cast<__half*>(sx);
   if (M <= 2 * sm_count()) {
     // few rows: a whole CTA per row keeps many loads in flight per row
-    act_quant_kernel<kActWarps><<<M, 32 * kActWarps, 0, as_stream(stream)>>>(Xh, M, K, X8, sxh);
+    act_quant_kernel<8, 8><<<M, 256, 0, as_stream(stream)>>>(Xh, M, K, X8, sxh);
   } else {
-    act_quant_kernel<1><<<(M + kActWarps - 1) / kActWarps, 32 * kActWarps, 0,
-                          as_stream(stream)>>>(Xh, M, K, X8, sxh);
+    act_quant_kernel<4, 1><<<(M + 3) / 4, 128, 0, as_stream(stream)>>>(Xh, M, K, X8, sxh);
   }
   return launch_status();
 }
