@@ -20,8 +20,9 @@
  *    current CUDA device; the caller owns all memory.  The library allocates
  *    no device memory (the GEMM's split-K workspace is the caller's); the
  *    only state it keeps between calls is the
- *    device error word (qoq_device_error) and host-side caches of device
- *    attributes and of the driver's tensor-map entry point.
+ *    device error word (qoq_device_error), the fixed scratch array of
+ *    qoq_w4a8_gemm_static_ws, and host-side caches of device attributes, of
+ *    the driver's tensor-map entry point and of that array's address.
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
  *    compute entry point only enqueues work on `stream` and returns without
  *    synchronizing, except the ones marked "synchronous".
@@ -182,6 +183,40 @@ QOQ_API int qoq_quantize_act_per_token(const void* X, int M, int K, int8_t* X8,
 QOQ_API int qoq_w4a8_gemm(const int8_t* X8, const void* sx, const void* packed,
                           const void* s1, int M, int N, int K, int group, void* Y,
                           void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * qoq_w4a8_gemm without a caller workspace, for callers that cannot allocate
+ * device memory (for instance code that runs inside an allocator's own
+ * callbacks, or a runtime that reserved all device memory up front and hands
+ * out no scratch).  The method described in the pages has no counterpart to
+ * this entry point; it exists only for such callers.
+ *
+ * Arguments and results are those of qoq_w4a8_gemm, with the same automatic
+ * launch plan.  The K-split scratch is a fixed array of QOQ_STATIC_WS_BYTES
+ * (16 MiB) in this library's device memory, one per device; the library
+ * allocates nothing.
+ *   - The first call on each device (with that device current) looks up the
+ *     array's device address once; make that first call before any stream
+ *     capture begins on that device.
+ *   - A shape whose plan needs more scratch than the array holds
+ *     (qoq_gemm_workspace_bytes(M, N, K, group) > QOQ_STATIC_WS_BYTES) is
+ *     rejected with QOQ_ERR_UNSUPPORTED and nothing is launched; use
+ *     qoq_w4a8_gemm with a workspace for it.  The automatic plan splits K
+ *     only for token tiles of at most 32 and keeps at most 4 units per SM,
+ *     so it needs at most 16 KiB + 4 * SMs * 32 * 128 * 4 bytes (about
+ *     9.7 MB with 148 SMs): on such a GPU no valid shape is rejected.
+ *   - Every call on a device uses the same array, and it keeps the last
+ *     call's contents.  Each call that splits K clears the array's arrival
+ *     counters on `stream` before its GEMM, so nothing from an earlier call
+ *     (even one that failed) leaks into it.  Calls that may overlap in time
+ *     (different streams, or several host threads) race on the array and give
+ *     wrong results: order them on one stream or with events.
+ * Asynchronous on `stream`.
+ * ---------------------------------------------------------------------- */
+#define QOQ_STATIC_WS_BYTES ((size_t)16 << 20)
+QOQ_API int qoq_w4a8_gemm_static_ws(const int8_t* X8, const void* sx, const void* packed,
+                                    const void* s1, int M, int N, int K, int group,
+                                    void* Y, void* stream);
 
 /* Workspace bytes qoq_w4a8_gemm, qoq_w4a8_gemm_i32 and qoq_w4a8_linear use
  * for this shape (0 if K is not split, or if the shape is invalid). */

@@ -31,6 +31,7 @@ EXPORTS = (
     "qoq_quantize_act_per_token", "qoq_w4a8_gemm", "qoq_w4a8_gemm_i32",
     "qoq_w4a8_gemm_config", "qoq_w4a8_linear", "qoq_gemm_plan", "qoq_device_error",
     "qoq_gemm_workspace_bytes", "qoq_gemm_workspace_bytes_config",
+    "qoq_w4a8_gemm_static_ws",
 )
 
 _lock = threading.Lock()
@@ -75,6 +76,8 @@ def lib() -> ctypes.CDLL:
             L.qoq_quantize_act_per_token.argtypes = [P, I, I, P, P, P]
             L.qoq_w4a8_gemm.restype = I
             L.qoq_w4a8_gemm.argtypes = [P, P, P, P, I, I, I, I, P, P, sz, P]
+            L.qoq_w4a8_gemm_static_ws.restype = I
+            L.qoq_w4a8_gemm_static_ws.argtypes = [P, P, P, P, I, I, I, I, P, P]
             L.qoq_w4a8_gemm_i32.restype = I
             L.qoq_w4a8_gemm_i32.argtypes = [P, P, I, I, I, I, P, P, sz, P]
             L.qoq_w4a8_gemm_config.restype = I
@@ -269,6 +272,21 @@ def w4a8_gemm(X8, sx, packed, s1, N: int, group: int = 128, out=None, ws=_AUTO, 
     w, wb = _ws_args(_auto_ws(ws, M, N, K, group, X8.device))
     _check(lib().qoq_w4a8_gemm(_ptr(X8), _ptr(sx), _ptr(packed), _ptr(s1), M, N, K, group,
                                _ptr(Y), w, wb, _stream(stream)), "qoq_w4a8_gemm")
+    return Y
+
+
+def w4a8_gemm_static_ws(X8, sx, packed, s1, N: int, group: int = 128, out=None, stream=None):
+    """The same GEMM without a workspace argument: the library uses its own
+    fixed device array (shared by every call on the device, so calls must not
+    overlap in time).  Raises QoQError (unsupported) for shapes needing more
+    split-K scratch than that array holds."""
+    import torch
+    _need_cuda(X8, "X8", torch.int8, 2)
+    M, K = X8.shape
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=X8.device)
+    _check(lib().qoq_w4a8_gemm_static_ws(_ptr(X8), _ptr(sx), _ptr(packed), _ptr(s1), M, N, K,
+                                         group, _ptr(Y), _stream(stream)),
+           "qoq_w4a8_gemm_static_ws")
     return Y
 
 

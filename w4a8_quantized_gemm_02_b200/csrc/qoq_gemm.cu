@@ -724,6 +724,65 @@ extern "C" int qoq_w4a8_gemm(const int8_t* X8, const void* sx, const void* packe
                    false);
 }
 
+// ---------------------------------------------------------------------------
+// qoq_w4a8_gemm_static_ws: the same GEMM for callers that may not allocate
+// device memory at all (e.g. code running inside a caching allocator's own
+// hooks, or a runtime whose memory is fully reserved up front).  The K-split
+// workspace is a fixed array in this module's device memory instead of a
+// caller buffer: every call on a device shares it.
+// ---------------------------------------------------------------------------
+namespace qoq {
+namespace {
+
+constexpr size_t kStaticWsBytes = QOQ_STATIC_WS_BYTES;
+static_assert(kStaticWsBytes > kCounterBytes, "static workspace smaller than its counter region");
+
+static __device__ __align__(256) uint8_t g_static_ws[kStaticWsBytes];
+
+constexpr int kMaxStaticWsDevices = 64;
+std::mutex g_static_ws_mutex;
+void* g_static_ws_ptr[kMaxStaticWsDevices] = {};
+
+// Device address of g_static_ws on the current device, looked up once per
+// device (the first call on a device loads this module there if needed).
+int static_ws_ptr(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QOQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxStaticWsDevices) return QOQ_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+  if (!g_static_ws_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || p == nullptr) return QOQ_ERR_CUDA;
+    g_static_ws_ptr[dev] = p;
+  }
+  *out = g_static_ws_ptr[dev];
+  return QOQ_OK;
+}
+
+}  // namespace
+}  // namespace qoq
+
+extern "C" int qoq_w4a8_gemm_static_ws(const int8_t* X8, const void* sx, const void* packed,
+                                       const void* s1, int M, int N, int K, int group, void* Y,
+                                       void* stream) {
+  if (!X8 || !sx || !packed || !s1 || !Y) return QOQ_ERR_INVALID_ARG;
+  if (M <= 0) return QOQ_ERR_INVALID_ARG;
+  if (int st = check_weight_shape(N, K, group)) return st;
+  const size_t need = gemm_ws_bytes(M, N, K, 0, 0);
+  if (need > kStaticWsBytes) return QOQ_ERR_UNSUPPORTED;   // larger than the fixed array
+  if (int st = check_device()) return st;
+  void* ws = nullptr;
+  if (int st = static_ws_ptr(&ws)) return st;
+  if (need > 0) {
+    // the arrival counters must start at zero; a completed call leaves them
+    // so, but the array keeps whatever an interrupted earlier call left
+    if (cudaMemsetAsync(ws, 0, kCounterBytes, as_stream(stream)) != cudaSuccess)
+      return QOQ_ERR_CUDA;
+  }
+  return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, nullptr, 0, 0, ws, kStaticWsBytes,
+                   stream, false);
+}
+
 extern "C" int qoq_w4a8_gemm_i32(const int8_t* X8, const void* packed, int M, int N, int K,
                                  int group, int32_t* acc, void* ws, size_t ws_bytes,
                                  void* stream) {
