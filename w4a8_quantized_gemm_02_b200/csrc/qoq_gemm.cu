@@ -52,8 +52,7 @@ constexpr int kWarpEpi0 = 2 + 4 * kDqGroups;     // first epilogue warp (14)
 constexpr int kWarps = kWarpEpi0 + 4;            // 18
 constexpr int kThreads = 32 * kWarps;            // 576
 constexpr int kRawStageBytes = 8576;             // largest packed block (group 64)
-constexpr int kTmemA = 0;                        // A operand of stage s at column 32 s
-constexpr int kTmemD = 256;                      // accumulators from column 256
+constexpr int kTmemA = 0;                        // A operands of the stages from column 0
 constexpr int kTmemCols = 512;
 constexpr int kStageBytesEpi = 32 * 16 * 4;      // per epilogue warp: 16 columns x 32 rows
 // The workspace starts with a fixed region of arrival counters (one word per
@@ -64,16 +63,25 @@ constexpr size_t kCounterBytes = kMaxCounterTiles * 4;
 
 template <int TOK>
 struct Cfg {
-  // One ring of kStages stages: stage s holds the X8 tile and the packed
-  // weight block in shared memory and the dequantized INT8 weights in tensor
-  // memory columns 32 s .. 32 s + 31.  kAcc accumulators of TOK columns let
-  // the epilogue of one unit overlap the main loop of the next.
-  static constexpr int kStages = TOK <= 128 ? 8 : 4;
+  // One ring of kStages stages.  A stage covers kNB consecutive k-tiles of
+  // 128 (the last stage of a unit may cover fewer): their X8 tiles and packed
+  // weight blocks in shared memory, and the dequantized INT8 weights in tensor
+  // memory columns kACols s .. kACols s + kACols - 1.  Two k-tiles per stage
+  // halve the per-stage work of the single-warp producer and MMA loops, whose
+  // wait / issue / commit sequence costs about as much as the MMAs of one
+  // 128 x 128 x 128 k-tile.  kAcc accumulators of TOK columns let the
+  // epilogue of one unit overlap the main loop of the next.
+  static constexpr int kNB = TOK <= 128 ? 2 : 1;
+  static constexpr int kXBytes = TOK * kTileK;                // one 128-byte-wide X8 tile
+  static constexpr int kStageX = kNB * kXBytes;
+  static constexpr int kStageRaw = kNB * kRawStageBytes;
+  static constexpr int kStages = TOK <= 32 ? 7 : TOK == 64 ? 6 : 4;
   static constexpr int kAcc = TOK <= 128 ? 2 : 1;
-  static constexpr int kXBytes = TOK * kTileK;
+  static constexpr int kACols = 32 * kNB;                     // tensor-memory columns of A per stage
+  static constexpr int kTmemD = ((kStages * kACols + TOK - 1) / TOK) * TOK;   // accumulators
   static constexpr int kOffX = 0;
-  static constexpr int kOffRaw = kOffX + kStages * kXBytes;
-  static constexpr int kOffEpi = kOffRaw + kStages * kRawStageBytes;
+  static constexpr int kOffRaw = kOffX + kStages * kStageX;
+  static constexpr int kOffEpi = kOffRaw + kStages * kStageRaw;
   static constexpr int kOffSx = kOffEpi + 4 * kStageBytesEpi;          // 4 warps x TOK floats
   static constexpr int kOffBar = kOffSx + 4 * TOK * 4;
   static constexpr int kNumBars = 3 * kStages + 2 * kAcc + 3;
@@ -83,7 +91,8 @@ struct Cfg {
   static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
   static_assert(kTmemD + kAcc * TOK <= kTmemCols, "tensor memory");
-  static_assert(kTmemA + 32 * kStages <= kTmemD, "tensor memory A stages");
+  static_assert(kTmemA + kACols * kStages <= kTmemD, "tensor memory A stages");
+  static_assert(kStageRaw % 16 == 0, "bulk copies need 16-byte alignment");
 };
 
 struct GemmArgs {
@@ -206,8 +215,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     // ---------------------------------------------------------------- producer
     // The whole warp runs the loop and waits; one elected lane issues copies.
     const uint64_t policy = l2_policy_evict_first();
-    const uint32_t tx = static_cast<uint32_t>(args.blk_bytes + C::kXBytes);
-    uint32_t g = 0;              // running k-tile index of this CTA
+    uint32_t g = 0;              // running stage index of this CTA
     bool aborted = false;
     bool first = true;
     for (int u = blockIdx.x; u < args.units && !aborted; u += gridDim.x) {
@@ -215,29 +223,35 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
       const uint8_t* src =
           args.packed + (static_cast<size_t>(w.nt) * kt_total + w.kt_begin) * args.blk_bytes;
       const int m0 = w.mt * TOK;
+      const int nsteps = (w.num_kt + C::kNB - 1) / C::kNB;
       int i = 0;
       if (first) {
         // the weight stream does not depend on the preceding grid: start it
         // before waiting for the activations
         first = false;
-        const int pre = w.num_kt < S ? w.num_kt : S;
+        const int pre = nsteps < S ? nsteps : S;
         if (elect_one()) {
           for (int j = 0; j < pre; ++j) {
-            mbar_arrive_expect_tx(bar_full + 8 * j, tx);
-            bulk_load(base + C::kOffRaw + j * kRawStageBytes,
-                      src + static_cast<size_t>(j) * args.blk_bytes,
-                      static_cast<uint32_t>(args.blk_bytes), bar_full + 8 * j, policy);
+            const int nb = min(C::kNB, w.num_kt - j * C::kNB);
+            mbar_arrive_expect_tx(bar_full + 8 * j,
+                                  static_cast<uint32_t>(nb * (args.blk_bytes + C::kXBytes)));
+            bulk_load(base + C::kOffRaw + j * C::kStageRaw,
+                      src + static_cast<size_t>(j * C::kNB) * args.blk_bytes,
+                      static_cast<uint32_t>(nb * args.blk_bytes), bar_full + 8 * j, policy);
           }
           grid_dependency_wait();
-          for (int j = 0; j < pre; ++j)
-            tma_load_2d(base + C::kOffX + j * C::kXBytes, &tmap_x, (w.kt_begin + j) * kTileK, m0,
-                        bar_full + 8 * j);
+          for (int j = 0; j < pre; ++j) {
+            const int nb = min(C::kNB, w.num_kt - j * C::kNB);
+            for (int q = 0; q < nb; ++q)
+              tma_load_2d(base + C::kOffX + j * C::kStageX + q * C::kXBytes, &tmap_x,
+                          (w.kt_begin + j * C::kNB + q) * kTileK, m0, bar_full + 8 * j);
+          }
         }
         __syncwarp();
         i = pre;
         g = pre;
       }
-      for (; i < w.num_kt; ++i, ++g) {
+      for (; i < nsteps; ++i, ++g) {
         const int s = g % S;
         if (g >= S && !__all_sync(0xffffffffu, mbar_wait(bar_empty + 8 * s, ((g / S) & 1) ^ 1,
                                                          abort_flag, &g_error_word,
@@ -246,12 +260,15 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
           break;
         }
         if (elect_one()) {
-          mbar_arrive_expect_tx(bar_full + 8 * s, tx);
-          bulk_load(base + C::kOffRaw + s * kRawStageBytes,
-                    src + static_cast<size_t>(i) * args.blk_bytes,
-                    static_cast<uint32_t>(args.blk_bytes), bar_full + 8 * s, policy);
-          tma_load_2d(base + C::kOffX + s * C::kXBytes, &tmap_x, (w.kt_begin + i) * kTileK, m0,
-                      bar_full + 8 * s);
+          const int nb = min(C::kNB, w.num_kt - i * C::kNB);
+          mbar_arrive_expect_tx(bar_full + 8 * s,
+                                static_cast<uint32_t>(nb * (args.blk_bytes + C::kXBytes)));
+          bulk_load(base + C::kOffRaw + s * C::kStageRaw,
+                    src + static_cast<size_t>(i * C::kNB) * args.blk_bytes,
+                    static_cast<uint32_t>(nb * args.blk_bytes), bar_full + 8 * s, policy);
+          for (int q = 0; q < nb; ++q)
+            tma_load_2d(base + C::kOffX + s * C::kStageX + q * C::kXBytes, &tmap_x,
+                        (w.kt_begin + i * C::kNB + q) * kTileK, m0, bar_full + 8 * s);
         }
         __syncwarp();
       }
@@ -277,8 +294,9 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
                                              abort_flag, &g_error_word, kErrMma)))
         break;
       tc_fence_after_sync();
-      const uint32_t d_tmem = tmem + kTmemD + b * TOK;
-      for (int i = 0; i < w.num_kt; ++i, ++g) {
+      const uint32_t d_tmem = tmem + C::kTmemD + b * TOK;
+      const int nsteps = (w.num_kt + C::kNB - 1) / C::kNB;
+      for (int i = 0; i < nsteps; ++i, ++g) {
         const int s = g % S;
         if (!__all_sync(0xffffffffu, mbar_wait(bar_dqfull + 8 * s, (g / S) & 1, abort_flag,
                                                &g_error_word, kErrMma))) {
@@ -287,14 +305,21 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
         }
         tc_fence_after_sync();
         if (elect_one()) {
-          const uint32_t a_tmem = tmem + kTmemA + 32 * s;
-          const uint32_t b_addr = base + C::kOffX + s * C::kXBytes;
+          const int nb = min(C::kNB, w.num_kt - i * C::kNB);
+          const uint32_t a_tmem = tmem + kTmemA + C::kACols * s;
+          const uint32_t b_addr = base + C::kOffX + s * C::kStageX;
 #pragma unroll
-          for (int kk = 0; kk < kTileK / 32; ++kk) {
-            // K = 32 bytes per instruction: 8 tensor-memory columns of A, 32
-            // bytes along the swizzled rows of B
-            mma_i8_ts(d_tmem, a_tmem + 8 * kk, smem_desc_sw128(b_addr + kk * 32), idesc,
-                      (i > 0 || kk > 0) ? 1u : 0u);
+          for (int q = 0; q < C::kNB; ++q) {
+            if (q < nb) {
+#pragma unroll
+              for (int kk = 0; kk < kTileK / 32; ++kk) {
+                // K = 32 bytes per instruction: 8 tensor-memory columns of A,
+                // 32 bytes along the swizzled rows of B
+                mma_i8_ts(d_tmem, a_tmem + 32 * q + 8 * kk,
+                          smem_desc_sw128(b_addr + q * C::kXBytes + kk * 32), idesc,
+                          (i > 0 || q > 0 || kk > 0) ? 1u : 0u);
+              }
+            }
           }
           mma_commit(bar_empty + 8 * s);     // stage s is free once these MMAs complete
         }
@@ -308,7 +333,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     drain_wait(bar_drain, 0);                // no MMA in flight past this point
   } else if (warp < kWarpEpi0) {
     // ---------------------------------------------------------------- dequantizers
-    const int wg = (warp - 2) >> 2;         // 0 .. kDqGroups-1: takes k-tiles g = wg (mod 3)
+    const int wg = (warp - 2) >> 2;         // 0 .. kDqGroups-1: takes stages g = wg (mod 3)
     const int q4 = warp & 3;                // tensor-memory lane quarter of this warp
     const int r = q4 * 32 + lane;           // weight row (output channel) within the tile
     const uint32_t row_tmem = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
@@ -317,7 +342,8 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     bool aborted = false;
     for (int u = blockIdx.x; u < args.units && !aborted; u += gridDim.x) {
       const Unit w = unit_of(args, u, kt_total);
-      for (int i = 0; i < w.num_kt; ++i, ++g) {
+      const int nsteps = (w.num_kt + C::kNB - 1) / C::kNB;
+      for (int i = 0; i < nsteps; ++i, ++g) {
         if (static_cast<int>(g % kDqGroups) != wg) continue;
         const int s = g % S;
         // the stage was refilled only after the MMAs that read its A columns
@@ -326,37 +352,44 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
           aborted = true;
           break;
         }
-        const uint8_t* blk = smem + C::kOffRaw + s * kRawStageBytes;
-        uint32_t s2v[2], bias[2];
+        const int nb = min(C::kNB, w.num_kt - i * C::kNB);
 #pragma unroll
-        for (int gl = 0; gl < 2; ++gl) {
-          if (gl < gpt) {
-            s2v[gl] = blk[kCodesBytes + gl * kTileN + r];
-            const uint32_t zb = blk[kCodesBytes + gpt * kTileN + gl * 64 + (r >> 1)];
-            const uint32_t zv = (r & 1) ? (zb >> 4) : (zb & 15u);
-            bias[gl] = dq_bias(zv, s2v[gl]);
-          } else {
-            s2v[gl] = s2v[0];
-            bias[gl] = bias[0];
+        for (int q = 0; q < C::kNB; ++q) {
+          if (q >= nb) break;
+          const uint8_t* blk = smem + C::kOffRaw + s * C::kStageRaw + q * args.blk_bytes;
+          uint32_t s2v[2], bias[2];
+#pragma unroll
+          for (int gl = 0; gl < 2; ++gl) {
+            if (gl < gpt) {
+              s2v[gl] = blk[kCodesBytes + gl * kTileN + r];
+              const uint32_t zb = blk[kCodesBytes + gpt * kTileN + gl * 64 + (r >> 1)];
+              const uint32_t zv = (r & 1) ? (zb >> 4) : (zb & 15u);
+              bias[gl] = dq_bias(zv, s2v[gl]);
+            } else {
+              s2v[gl] = s2v[0];
+              bias[gl] = bias[0];
+            }
           }
-        }
-        uint32_t out[32];
+          uint32_t out[32];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint4 v = *reinterpret_cast<const uint4*>(blk + (j * kTileN + r) * 16);
-          const int gl = (gpt == 2) ? (j >> 1) : 0;
-          const uint32_t sv = s2v[gl], bv = bias[gl];
-          out[8 * j + 0] = dq_lanes(lo_codes(v.x), sv, bv);
-          out[8 * j + 1] = dq_lanes(hi_codes(v.x), sv, bv);
-          out[8 * j + 2] = dq_lanes(lo_codes(v.y), sv, bv);
-          out[8 * j + 3] = dq_lanes(hi_codes(v.y), sv, bv);
-          out[8 * j + 4] = dq_lanes(lo_codes(v.z), sv, bv);
-          out[8 * j + 5] = dq_lanes(hi_codes(v.z), sv, bv);
-          out[8 * j + 6] = dq_lanes(lo_codes(v.w), sv, bv);
-          out[8 * j + 7] = dq_lanes(hi_codes(v.w), sv, bv);
+          for (int j = 0; j < 4; ++j) {
+            const uint4 v = *reinterpret_cast<const uint4*>(blk + (j * kTileN + r) * 16);
+            const int gl = (gpt == 2) ? (j >> 1) : 0;
+            const uint32_t sv = s2v[gl], bv = bias[gl];
+            out[8 * j + 0] = dq_lanes(lo_codes(v.x), sv, bv);
+            out[8 * j + 1] = dq_lanes(hi_codes(v.x), sv, bv);
+            out[8 * j + 2] = dq_lanes(lo_codes(v.y), sv, bv);
+            out[8 * j + 3] = dq_lanes(hi_codes(v.y), sv, bv);
+            out[8 * j + 4] = dq_lanes(lo_codes(v.z), sv, bv);
+            out[8 * j + 5] = dq_lanes(hi_codes(v.z), sv, bv);
+            out[8 * j + 6] = dq_lanes(lo_codes(v.w), sv, bv);
+            out[8 * j + 7] = dq_lanes(hi_codes(v.w), sv, bv);
+          }
+          // one 128-byte row of the INT8 A operand per k-tile: column c holds
+          // K bytes 4c..4c+3 (the source registers are read at issue; one
+          // wait below covers both stores)
+          tmem_st_32x32b_x32(row_tmem + kTmemA + C::kACols * s + 32 * q, out);
         }
-        // one 128-byte row of the INT8 A operand: column c holds K bytes 4c..4c+3
-        tmem_st_32x32b_x32(row_tmem + kTmemA + 32 * s, out);
         tmem_st_wait();
         tc_fence_before_sync();
         __syncwarp();
@@ -382,13 +415,10 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
       const int b = lt % C::kAcc;
       const int m0 = w.mt * TOK;
       const int nrow0 = w.nt * kTileN + q4 * 32;   // first channel of this warp's slice
-      const bool ok = mbar_wait(bar_accfull + 8 * b, (lt / C::kAcc) & 1, abort_flag,
-                                &g_error_word, kErrEpilogue);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after_sync();
-      const uint32_t t_acc = tmem + kTmemD + b * TOK + (static_cast<uint32_t>(q4 * 32) << 16);
       int c_end = M - m0;
       if (c_end > TOK) c_end = TOK;
+      // the scales do not depend on the accumulator: fetch them while the
+      // main loop of this unit is still running
       float s1r = 0.0f;
       if (args.Y) {
         s1r = __half2float(args.s1[w.nt * kTileN + r]);
@@ -396,6 +426,11 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
           sx_w[c] = (m0 + c < M) ? __half2float(args.sx[m0 + c]) : 0.0f;
         __syncwarp();
       }
+      const bool ok = mbar_wait(bar_accfull + 8 * b, (lt / C::kAcc) & 1, abort_flag,
+                                &g_error_word, kErrEpilogue);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after_sync();
+      const uint32_t t_acc = tmem + C::kTmemD + b * TOK + (static_cast<uint32_t>(q4 * 32) << 16);
       const int splits = args.splits;
       bool write_out = true;
       if (splits > 1) {
@@ -535,7 +570,7 @@ bool splittable(const Plan& p) {
   return static_cast<long>(p.m_tiles) * p.n_tiles <= kMaxCounterTiles;
 }
 
-int stages_for(int tok) { return tok <= 128 ? 8 : 4; }
+int stages_for(int tok) { return tok <= 32 ? 7 : tok == 64 ? 6 : 4; }
 
 bool valid_tok(int t) { return t == 16 || t == 32 || t == 64 || t == 128 || t == 256; }
 
