@@ -23,7 +23,6 @@ enum : uint32_t {
 // seconds at the B200's clocks, longer when the clock is lower).  The cycle
 // counter is read only after many unsuccessful polls, never on the fast path.
 constexpr long long kWaitLimitCycles = 4000000000LL;
-constexpr uint32_t kPollsBeforeTiming = 1024;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -76,27 +75,42 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// One test that may suspend the thread until the phase completes or about
+// `hint_ns` nanoseconds pass, whichever is first: a waiting warp then sleeps
+// instead of taking issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr uint32_t kSuspendHintNs = 1000000;   // 1 ms per suspended test
+
 // Wait for the phase of parity `parity` to complete.  Gives up (returns
 // false) when the CTA-wide abort flag is raised or after kWaitLimitCycles, in
 // which case it raises the abort flag and records `err_bit` in `err_word`
-// (the library's device error word).  Never spins forever.
+// (the library's device error word).  Never spins forever: each test after
+// the first suspends the thread for at most kSuspendHintNs, and the abort flag
+// and the clock are checked after every one.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile uint32_t* abort_flag,
                                           unsigned int* err_word, uint32_t err_bit) {
   if (mbar_try_wait(bar, parity)) return true;
-  long long t0 = 0;
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it % kPollsBeforeTiming) == 0) {
-      if (*abort_flag) return false;
-      const long long now = sm_clock();
-      if (t0 == 0) {
-        t0 = now;
-      } else if (now - t0 > kWaitLimitCycles) {
-        *abort_flag = 1u;
-        atomicOr(err_word, err_bit);
-        return false;
-      }
+  const long long t0 = sm_clock();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) return true;
+    if (*abort_flag) return false;
+    if (sm_clock() - t0 > kWaitLimitCycles) {
+      *abort_flag = 1u;
+      atomicOr(err_word, err_bit);
+      return false;
     }
   }
 }

@@ -12,19 +12,25 @@
 // and the tokens its N operand, so one decode token still fills the 128-row
 // tensor-core tile).  Units are ordered channel-tile major, token tile next,
 // K split innermost, so the CTAs running at the same time share weight blocks
-// through L2 and every weight byte comes from HBM about once.
-//   warp 0       TMA producer: per k-tile, one bulk copy of the packed weight
-//                block and one tensor-map copy of the X8 tile (128-byte
-//                swizzle) into a ring of shared-memory stages;
+// through L2 and every weight byte comes from HBM about once.  A pipeline
+// stage covers two k-tiles of 128 (one for TOK = 256).
+//   warp 0       X producer: tensor-map copies of the X8 tiles (128-byte
+//                swizzle) into the X ring, refilled when the stage's MMAs
+//                completed;
+//   warp 18      W producer: one bulk copy of the stage's packed weight
+//                blocks into the weight ring, refilled as soon as the
+//                dequantizers hold the blocks in registers, so the weight
+//                stream runs ahead of the MMAs;
 //   warp 1       owns tensor memory and issues tcgen05.mma.kind::i8 (M = 128,
 //                N = TOK, K = 32 per instruction) with the INT8 weights read
 //                from tensor memory and X8 from shared memory, into one of two
 //                INT32 accumulators in tensor memory (double buffered); one
-//                commit per k-tile releases the whole stage;
-//   warps 2..13  three dequantizing warpgroups taking k-tiles in turn: each
-//                thread turns one weight row of the UINT4 block into INT8
-//                (four byte lanes per 32-bit multiply-add) and writes the
-//                128-byte row into a tensor-memory stage with one tcgen05.st;
+//                commit per stage frees its X8 tiles and A columns;
+//   warps 2..13  three dequantizing warpgroups taking stages in turn: each
+//                thread turns one weight row of the UINT4 blocks into INT8
+//                (four byte lanes per 32-bit multiply-add) and writes one
+//                128-byte row per k-tile into the stage's tensor-memory
+//                columns with tcgen05.st;
 //   warps 14..17 epilogue: tcgen05.ld of a finished accumulator, one FP32
 //                scale per element, a transpose through shared memory and
 //                16-byte stores, overlapping the next unit's main loop.
@@ -49,8 +55,9 @@ namespace {
 
 constexpr int kDqGroups = 3;                     // dequantizing warpgroups
 constexpr int kWarpEpi0 = 2 + 4 * kDqGroups;     // first epilogue warp (14)
-constexpr int kWarps = kWarpEpi0 + 4;            // 18
-constexpr int kThreads = 32 * kWarps;            // 576
+constexpr int kWarpW = kWarpEpi0 + 4;            // weight producer warp (18)
+constexpr int kWarps = kWarpW + 1;               // 19
+constexpr int kThreads = 32 * kWarps;            // 608
 constexpr int kRawStageBytes = 8576;             // largest packed block (group 64)
 constexpr int kTmemA = 0;                        // A operands of the stages from column 0
 constexpr int kTmemCols = 512;
@@ -84,7 +91,7 @@ struct Cfg {
   static constexpr int kOffEpi = kOffRaw + kStages * kStageRaw;
   static constexpr int kOffSx = kOffEpi + 4 * kStageBytesEpi;          // 4 warps x TOK floats
   static constexpr int kOffBar = kOffSx + 4 * TOK * 4;
-  static constexpr int kNumBars = 3 * kStages + 2 * kAcc + 3;
+  static constexpr int kNumBars = 5 * kStages + 2 * kAcc + 3;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 32 + 1024;   // + base alignment slack
   static_assert(kOffRaw % 1024 == 0 && kXBytes % 1024 == 0, "swizzled tiles need 1 KiB alignment");
@@ -128,16 +135,12 @@ __device__ __forceinline__ Unit unit_of(const GemmArgs& a, int u, int kt_total) 
 // Bounded wait that ignores the abort flag: used only to drain work already
 // in flight before a CTA tears down.
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
-  long long t0 = 0;
-  for (uint32_t it = 1; !mbar_try_wait(bar, parity); ++it) {
-    if ((it % kPollsBeforeTiming) == 0) {
-      const long long now = sm_clock();
-      if (t0 == 0) {
-        t0 = now;
-      } else if (now - t0 > kWaitLimitCycles) {
-        atomicOr(&g_error_word, kErrProducer);
-        return;
-      }
+  if (mbar_try_wait(bar, parity)) return;
+  const long long t0 = sm_clock();
+  while (!mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) {
+    if (sm_clock() - t0 > kWaitLimitCycles) {
+      atomicOr(&g_error_word, kErrProducer);
+      return;
     }
   }
 }
@@ -169,12 +172,21 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   const int lane = threadIdx.x & 31;
   const int kt_total = args.K / kTileK;
 
-  // full[s]: X tile and weight block landed; dqfull[s]: A operand written
-  // (implies full); empty[s]: the MMAs of the stage completed (the producer
-  // may refill it, which in turn frees its A columns for the dequantizers)
-  const uint32_t bar_full = base + C::kOffBar;
-  const uint32_t bar_empty = bar_full + 8 * S;
-  const uint32_t bar_dqfull = bar_empty + 8 * S;
+  // Two rings of S slots, both indexed by the running stage g (slot g % S):
+  //   X ring     xfull[s]: the X8 tiles of stage g landed (X producer);
+  //              empty[s]: the MMAs of stage g completed, which frees both the
+  //              X8 tiles and the tensor-memory A columns of slot s;
+  //   weight ring wfull[s]: the packed blocks of stage g landed (W producer);
+  //              wempty[s]: the dequantizers copied them into registers.
+  // dqfull[s]: A operand of stage g written and its X8 tiles landed (the MMA
+  // warp waits on this one barrier).  The weight ring is released as soon as
+  // the blocks are in registers, so the weight stream runs ahead of the MMAs
+  // and the weight copy overlaps the previous stages' dequantization.
+  const uint32_t bar_xfull = base + C::kOffBar;
+  const uint32_t bar_empty = bar_xfull + 8 * S;
+  const uint32_t bar_wfull = bar_empty + 8 * S;
+  const uint32_t bar_wempty = bar_wfull + 8 * S;
+  const uint32_t bar_dqfull = bar_wempty + 8 * S;
   const uint32_t bar_accfull = bar_dqfull + 8 * S;
   const uint32_t bar_accempty = bar_accfull + 8 * C::kAcc;
   const uint32_t bar_drain = bar_accempty + 8 * C::kAcc;
@@ -186,8 +198,10 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_xfull + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
+      mbar_init(bar_wfull + 8 * s, 1);
+      mbar_init(bar_wempty + 8 * s, 4);
       mbar_init(bar_dqfull + 8 * s, 4);
     }
     for (int b = 0; b < C::kAcc; ++b) {
@@ -212,46 +226,16 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- producer
+    // -------------------------------------------------------------- X producer
     // The whole warp runs the loop and waits; one elected lane issues copies.
-    const uint64_t policy = l2_policy_evict_first();
     uint32_t g = 0;              // running stage index of this CTA
     bool aborted = false;
-    bool first = true;
+    grid_dependency_wait();      // X8 comes from the preceding grid under PDL
     for (int u = blockIdx.x; u < args.units && !aborted; u += gridDim.x) {
       const Unit w = unit_of(args, u, kt_total);
-      const uint8_t* src =
-          args.packed + (static_cast<size_t>(w.nt) * kt_total + w.kt_begin) * args.blk_bytes;
       const int m0 = w.mt * TOK;
       const int nsteps = (w.num_kt + C::kNB - 1) / C::kNB;
-      int i = 0;
-      if (first) {
-        // the weight stream does not depend on the preceding grid: start it
-        // before waiting for the activations
-        first = false;
-        const int pre = nsteps < S ? nsteps : S;
-        if (elect_one()) {
-          for (int j = 0; j < pre; ++j) {
-            const int nb = min(C::kNB, w.num_kt - j * C::kNB);
-            mbar_arrive_expect_tx(bar_full + 8 * j,
-                                  static_cast<uint32_t>(nb * (args.blk_bytes + C::kXBytes)));
-            bulk_load(base + C::kOffRaw + j * C::kStageRaw,
-                      src + static_cast<size_t>(j * C::kNB) * args.blk_bytes,
-                      static_cast<uint32_t>(nb * args.blk_bytes), bar_full + 8 * j, policy);
-          }
-          grid_dependency_wait();
-          for (int j = 0; j < pre; ++j) {
-            const int nb = min(C::kNB, w.num_kt - j * C::kNB);
-            for (int q = 0; q < nb; ++q)
-              tma_load_2d(base + C::kOffX + j * C::kStageX + q * C::kXBytes, &tmap_x,
-                          (w.kt_begin + j * C::kNB + q) * kTileK, m0, bar_full + 8 * j);
-          }
-        }
-        __syncwarp();
-        i = pre;
-        g = pre;
-      }
-      for (; i < nsteps; ++i, ++g) {
+      for (int i = 0; i < nsteps; ++i, ++g) {
         const int s = g % S;
         if (g >= S && !__all_sync(0xffffffffu, mbar_wait(bar_empty + 8 * s, ((g / S) & 1) ^ 1,
                                                          abort_flag, &g_error_word,
@@ -261,14 +245,10 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
         }
         if (elect_one()) {
           const int nb = min(C::kNB, w.num_kt - i * C::kNB);
-          mbar_arrive_expect_tx(bar_full + 8 * s,
-                                static_cast<uint32_t>(nb * (args.blk_bytes + C::kXBytes)));
-          bulk_load(base + C::kOffRaw + s * C::kStageRaw,
-                    src + static_cast<size_t>(i * C::kNB) * args.blk_bytes,
-                    static_cast<uint32_t>(nb * args.blk_bytes), bar_full + 8 * s, policy);
+          mbar_arrive_expect_tx(bar_xfull + 8 * s, static_cast<uint32_t>(nb * C::kXBytes));
           for (int q = 0; q < nb; ++q)
             tma_load_2d(base + C::kOffX + s * C::kStageX + q * C::kXBytes, &tmap_x,
-                        (w.kt_begin + i * C::kNB + q) * kTileK, m0, bar_full + 8 * s);
+                        (w.kt_begin + i * C::kNB + q) * kTileK, m0, bar_xfull + 8 * s);
         }
         __syncwarp();
       }
@@ -276,7 +256,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     if (aborted) {
       // the copies already issued must land before the CTA exits
       for (uint32_t j = (g > S ? g - S : 0); j < g; ++j)
-        drain_wait(bar_full + 8 * (j % S), (j / S) & 1);
+        drain_wait(bar_xfull + 8 * (j % S), (j / S) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -346,57 +326,83 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
       for (int i = 0; i < nsteps; ++i, ++g) {
         if (static_cast<int>(g % kDqGroups) != wg) continue;
         const int s = g % S;
-        // the stage was refilled only after the MMAs that read its A columns
-        // completed, so landing data also means the A columns are free
-        if (!mbar_wait(bar_full + 8 * s, (g / S) & 1, abort_flag, &g_error_word, kErrDequant)) {
+        const uint32_t ph = (g / S) & 1;
+        if (!mbar_wait(bar_wfull + 8 * s, ph, abort_flag, &g_error_word, kErrDequant)) {
           aborted = true;
           break;
         }
         const int nb = min(C::kNB, w.num_kt - i * C::kNB);
+        // this row of every block of the stage, into registers
+        uint4 v[C::kNB][4];
+        uint32_t s2v[C::kNB][2], bias[C::kNB][2];
 #pragma unroll
         for (int q = 0; q < C::kNB; ++q) {
-          if (q >= nb) break;
-          const uint8_t* blk = smem + C::kOffRaw + s * C::kStageRaw + q * args.blk_bytes;
-          uint32_t s2v[2], bias[2];
+          if (q < nb) {
+            const uint8_t* blk = smem + C::kOffRaw + s * C::kStageRaw + q * args.blk_bytes;
 #pragma unroll
-          for (int gl = 0; gl < 2; ++gl) {
-            if (gl < gpt) {
-              s2v[gl] = blk[kCodesBytes + gl * kTileN + r];
-              const uint32_t zb = blk[kCodesBytes + gpt * kTileN + gl * 64 + (r >> 1)];
-              const uint32_t zv = (r & 1) ? (zb >> 4) : (zb & 15u);
-              bias[gl] = dq_bias(zv, s2v[gl]);
-            } else {
-              s2v[gl] = s2v[0];
-              bias[gl] = bias[0];
+            for (int gl = 0; gl < 2; ++gl) {
+              if (gl < gpt) {
+                s2v[q][gl] = blk[kCodesBytes + gl * kTileN + r];
+                const uint32_t zb = blk[kCodesBytes + gpt * kTileN + gl * 64 + (r >> 1)];
+                const uint32_t zv = (r & 1) ? (zb >> 4) : (zb & 15u);
+                bias[q][gl] = dq_bias(zv, s2v[q][gl]);
+              } else {
+                s2v[q][gl] = s2v[q][0];
+                bias[q][gl] = bias[q][0];
+              }
             }
-          }
-          uint32_t out[32];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint4 v = *reinterpret_cast<const uint4*>(blk + (j * kTileN + r) * 16);
-            const int gl = (gpt == 2) ? (j >> 1) : 0;
-            const uint32_t sv = s2v[gl], bv = bias[gl];
-            out[8 * j + 0] = dq_lanes(lo_codes(v.x), sv, bv);
-            out[8 * j + 1] = dq_lanes(hi_codes(v.x), sv, bv);
-            out[8 * j + 2] = dq_lanes(lo_codes(v.y), sv, bv);
-            out[8 * j + 3] = dq_lanes(hi_codes(v.y), sv, bv);
-            out[8 * j + 4] = dq_lanes(lo_codes(v.z), sv, bv);
-            out[8 * j + 5] = dq_lanes(hi_codes(v.z), sv, bv);
-            out[8 * j + 6] = dq_lanes(lo_codes(v.w), sv, bv);
-            out[8 * j + 7] = dq_lanes(hi_codes(v.w), sv, bv);
+            for (int j = 0; j < 4; ++j)
+              v[q][j] = *reinterpret_cast<const uint4*>(blk + (j * kTileN + r) * 16);
           }
-          // one 128-byte row of the INT8 A operand per k-tile: column c holds
-          // K bytes 4c..4c+3 (the source registers are read at issue; one
-          // wait below covers both stores)
-          tmem_st_32x32b_x32(row_tmem + kTmemA + C::kACols * s + 32 * q, out);
+        }
+        // the weight slot may be refilled once every lane has read it (the
+        // arrive releases this warp's reads, ordered by the warp barrier)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_wempty + 8 * s);
+        // the A columns of slot s are free once the MMAs of stage g - S completed
+        if (g >= S && !mbar_wait(bar_empty + 8 * s, ph ^ 1, abort_flag, &g_error_word,
+                                 kErrDequant)) {
+          aborted = true;
+          break;
+        }
+        tc_fence_after_sync();
+#pragma unroll
+        for (int q = 0; q < C::kNB; ++q) {
+          if (q < nb) {
+            uint32_t out[32];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int gl = (gpt == 2) ? (j >> 1) : 0;
+              const uint32_t sv = s2v[q][gl], bv = bias[q][gl];
+              out[8 * j + 0] = dq_lanes(lo_codes(v[q][j].x), sv, bv);
+              out[8 * j + 1] = dq_lanes(hi_codes(v[q][j].x), sv, bv);
+              out[8 * j + 2] = dq_lanes(lo_codes(v[q][j].y), sv, bv);
+              out[8 * j + 3] = dq_lanes(hi_codes(v[q][j].y), sv, bv);
+              out[8 * j + 4] = dq_lanes(lo_codes(v[q][j].z), sv, bv);
+              out[8 * j + 5] = dq_lanes(hi_codes(v[q][j].z), sv, bv);
+              out[8 * j + 6] = dq_lanes(lo_codes(v[q][j].w), sv, bv);
+              out[8 * j + 7] = dq_lanes(hi_codes(v[q][j].w), sv, bv);
+            }
+            // one 128-byte row of the INT8 A operand per k-tile: column c
+            // holds K bytes 4c..4c+3 (the source registers are read at issue;
+            // one wait below covers both stores)
+            tmem_st_32x32b_x32(row_tmem + kTmemA + C::kACols * s + 32 * q, out);
+          }
         }
         tmem_st_wait();
+        // the MMAs of the stage also read its X8 tiles: the MMA warp waits on
+        // dqfull alone
+        if (!mbar_wait(bar_xfull + 8 * s, ph, abort_flag, &g_error_word, kErrDequant)) {
+          aborted = true;
+          break;
+        }
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_dqfull + 8 * s);
       }
     }
-  } else {
+  } else if (warp < kWarpW) {
     // ---------------------------------------------------------------- epilogue
     const int q4 = warp & 3;                // tensor-memory lane quarter
     const int ew = warp - kWarpEpi0;        // 0..3
@@ -527,6 +533,40 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_accempty + 8 * b);
+    }
+  } else {
+    // -------------------------------------------------------------- W producer
+    // Packed weight blocks: independent of the preceding grid, so this warp
+    // starts at once under PDL.
+    const uint64_t policy = l2_policy_evict_first();
+    uint32_t g = 0;
+    bool aborted = false;
+    for (int u = blockIdx.x; u < args.units && !aborted; u += gridDim.x) {
+      const Unit w = unit_of(args, u, kt_total);
+      const uint8_t* src =
+          args.packed + (static_cast<size_t>(w.nt) * kt_total + w.kt_begin) * args.blk_bytes;
+      const int nsteps = (w.num_kt + C::kNB - 1) / C::kNB;
+      for (int i = 0; i < nsteps; ++i, ++g) {
+        const int s = g % S;
+        if (g >= S && !__all_sync(0xffffffffu, mbar_wait(bar_wempty + 8 * s, ((g / S) & 1) ^ 1,
+                                                         abort_flag, &g_error_word,
+                                                         kErrProducer))) {
+          aborted = true;
+          break;
+        }
+        if (elect_one()) {
+          const int nb = min(C::kNB, w.num_kt - i * C::kNB);
+          mbar_arrive_expect_tx(bar_wfull + 8 * s, static_cast<uint32_t>(nb * args.blk_bytes));
+          bulk_load(base + C::kOffRaw + s * C::kStageRaw,
+                    src + static_cast<size_t>(i * C::kNB) * args.blk_bytes,
+                    static_cast<uint32_t>(nb * args.blk_bytes), bar_wfull + 8 * s, policy);
+        }
+        __syncwarp();
+      }
+    }
+    if (aborted) {
+      for (uint32_t j = (g > S ? g - S : 0); j < g; ++j)
+        drain_wait(bar_wfull + 8 * (j % S), (j / S) & 1);
     }
   }
 
