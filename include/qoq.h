@@ -163,8 +163,10 @@ QOQ_API int qoq_quantize_act_per_token(const void* X, int M, int K, int8_t* X8,
  *            least qoq_gemm_workspace_bytes(M, N, K, group) bytes (0 for
  *            shapes that are not split).  Owned by the caller, who fills it
  *            with zeros once before its first use (e.g. cudaMemset); every
- *            call that completes leaves its first 16 KiB (one arrival counter
- *            per output tile) at zero again, so it can be reused by later
+ *            call that completes leaves its first 16 KiB (arrival counters,
+ *            one per 32-channel slice of an output tile; K is split only when
+ *            there are at most 1024 output tiles) at zero again, so it can be
+ *            reused by later
  *            calls on the same stream whatever their shape.  After a call
  *            that reported a device error (qoq_device_error) it must be
  *            zeroed again.  The rest holds INT32 partial sums.  Calls that

@@ -20,7 +20,7 @@ if not torch.cuda.is_available():   # pragma: no cover - CPU container
 import w4a8_quantized_gemm_02_b200 as qoq  # noqa: E402
 
 DEV = torch.device("cuda:0")
-TOKS = (16, 32, 64, 128, 256)
+TOKS = (16, 32, 64, 128, 176, 192, 256)
 
 
 def to_dev(a: np.ndarray):
@@ -236,6 +236,26 @@ def test_gemm_ragged_m(oracle, M):
     check_y(host(Y), Yr)
 
 
+@pytest.mark.parametrize("tok", (176, 192))
+def test_gemm_wide_tiles_persistent(oracle, tok):
+    """Wide token tiles with more output tiles than CTAs, so every CTA runs
+    several units and both accumulators take turns; ragged last token tile."""
+    M, N, K, group = 1100, 3840, 512, 128
+    ops = si.sweep_operands(M, N, K, group, seed=tok)
+    acc_ref = oracle.int_gemm(ops.X8, oracle.dequant_w(ops.q, ops.s2, ops.z, group))
+    packed = qoq.pack_codes(to_dev(ops.q), to_dev(ops.s2), to_dev(ops.z), group)
+    X8 = to_dev(ops.X8)
+    qoq.device_error(clear=True)
+    acc = qoq.w4a8_gemm_config(X8, None, packed, None, N, group, tok_tile=tok, splits=1,
+                               int32_out=True)
+    Y = qoq.w4a8_gemm_config(X8, to_dev(ops.sx), packed, to_dev(ops.s1), N, group,
+                             tok_tile=tok, splits=1)
+    torch.cuda.synchronize()
+    assert qoq.device_error() == 0
+    assert np.array_equal(host(acc), acc_ref)
+    check_y(host(Y), oracle.epilogue(acc_ref, ops.sx, ops.s1))
+
+
 @pytest.mark.parametrize("group", (64, 128))
 @pytest.mark.parametrize("M,N,K", [(16, 128, 128), (5, 256, 256), (40, 384, 1152),
                                    (200, 256, 2048)])
@@ -247,7 +267,7 @@ def test_gemm_shapes_random_codes(oracle, group, M, N, K):
     packed = qoq.pack_codes(to_dev(ops.q), to_dev(ops.s2), to_dev(ops.z), group)
     X8 = to_dev(ops.X8)
     kt = K // 128
-    for tok in (16, 64, 256):
+    for tok in (16, 64, 176, 256):
         for splits in sorted({1, min(2, kt), min(kt, 8)}):
             acc = qoq.w4a8_gemm_config(X8, None, packed, None, N, group, tok_tile=tok,
                                        splits=splits, int32_out=True)

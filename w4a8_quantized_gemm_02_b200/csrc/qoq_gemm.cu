@@ -59,14 +59,16 @@ constexpr int kWarpW = kWarpEpi0 + 4;            // weight producer warp (18)
 constexpr int kWarps = kWarpW + 1;               // 19
 constexpr int kThreads = 32 * kWarps;            // 608
 constexpr int kRawStageBytes = 8576;             // largest packed block (group 64)
-constexpr int kTmemA = 0;                        // A operands of the stages from column 0
 constexpr int kTmemCols = 512;
 constexpr int kStageBytesEpi = 32 * 16 * 4;      // per epilogue warp: 16 columns x 32 rows
 // The workspace starts with a fixed region of arrival counters (one word per
 // output tile), so that counter words never share memory with the partial
 // sums of a launch of another shape.
-constexpr int kMaxCounterTiles = 4096;
-constexpr size_t kCounterBytes = kMaxCounterTiles * 4;
+// Each epilogue warp counts the arrivals at its own 32-channel slice of an
+// output tile, so a tile has four counters.
+constexpr int kSlicesPerTile = 4;
+constexpr int kMaxCounterTiles = 1024;
+constexpr size_t kCounterBytes = kMaxCounterTiles * kSlicesPerTile * 4;
 
 template <int TOK>
 struct Cfg {
@@ -82,23 +84,33 @@ struct Cfg {
   static constexpr int kXBytes = TOK * kTileK;                // one 128-byte-wide X8 tile
   static constexpr int kStageX = kNB * kXBytes;
   static constexpr int kStageRaw = kNB * kRawStageBytes;
-  static constexpr int kStages = TOK <= 32 ? 7 : TOK == 64 ? 6 : 4;
-  static constexpr int kAcc = TOK <= 128 ? 2 : 1;
+  static constexpr int kStages = TOK <= 32 ? 7 : TOK == 64 ? 6 : TOK == 176 ? 5 : 4;
+  static constexpr int kAcc = TOK <= 192 ? 2 : 1;
   static constexpr int kACols = 32 * kNB;                     // tensor-memory columns of A per stage
-  static constexpr int kTmemD = ((kStages * kACols + TOK - 1) / TOK) * TOK;   // accumulators
+  // Tensor-memory columns: up to 128 tokens the A slots come first and the
+  // accumulators after them (at a multiple of TOK); for the wide token tiles
+  // of 176 and 192 the two accumulators come first (at columns 0 and TOK)
+  // and the A slots after them, at a multiple of 32.
+  static constexpr bool kAccFirst = TOK == 176 || TOK == 192;
+  static constexpr int kTmemA = kAccFirst ? kAcc * TOK : 0;
+  static constexpr int kTmemD =
+      kAccFirst ? 0 : ((kStages * kACols + TOK - 1) / TOK) * TOK;   // accumulators
   static constexpr int kOffX = 0;
   static constexpr int kOffRaw = kOffX + kStages * kStageX;
   static constexpr int kOffEpi = kOffRaw + kStages * kStageRaw;
   static constexpr int kOffSx = kOffEpi + 4 * kStageBytesEpi;          // 4 warps x TOK floats
   static constexpr int kOffBar = kOffSx + 4 * TOK * 4;
-  static constexpr int kNumBars = 5 * kStages + 2 * kAcc + 3;
+  static constexpr int kNumBars = 5 * kStages + 2 * kAcc + 1;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 32 + 1024;   // + base alignment slack
   static_assert(kOffRaw % 1024 == 0 && kXBytes % 1024 == 0, "swizzled tiles need 1 KiB alignment");
   static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
   static_assert(kTmemD + kAcc * TOK <= kTmemCols, "tensor memory");
-  static_assert(kTmemA + kACols * kStages <= kTmemD, "tensor memory A stages");
+  static_assert(kAccFirst ? kTmemA + kACols * kStages <= kTmemCols
+                          : kTmemA + kACols * kStages <= kTmemD,
+                "tensor memory A stages");
+  static_assert(kTmemA % 32 == 0 && kTmemD % TOK == 0, "tensor memory alignment");
   static_assert(kStageRaw % 16 == 0, "bulk copies need 16-byte alignment");
 };
 
@@ -190,11 +202,8 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   const uint32_t bar_accfull = bar_dqfull + 8 * S;
   const uint32_t bar_accempty = bar_accfull + 8 * C::kAcc;
   const uint32_t bar_drain = bar_accempty + 8 * C::kAcc;
-  const uint32_t bar_epi_in = bar_drain + 8;    // four epilogue warps published a partial
-  const uint32_t bar_epi_go = bar_epi_in + 8;   // the arrival was counted
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc + 4);
-  volatile uint32_t* last_flag = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc + 8);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -209,10 +218,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
       mbar_init(bar_accempty + 8 * b, 4);
     }
     mbar_init(bar_drain, 1);
-    mbar_init(bar_epi_in, 4);
-    mbar_init(bar_epi_go, 1);
     *abort_flag = 0u;
-    *last_flag = 0u;
     fence_mbar_init();
     prefetch_tensormap(&tmap_x);
   }
@@ -286,7 +292,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
         tc_fence_after_sync();
         if (elect_one()) {
           const int nb = min(C::kNB, w.num_kt - i * C::kNB);
-          const uint32_t a_tmem = tmem + kTmemA + C::kACols * s;
+          const uint32_t a_tmem = tmem + C::kTmemA + C::kACols * s;
           const uint32_t b_addr = base + C::kOffX + s * C::kStageX;
 #pragma unroll
           for (int q = 0; q < C::kNB; ++q) {
@@ -387,7 +393,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
             // one 128-byte row of the INT8 A operand per k-tile: column c
             // holds K bytes 4c..4c+3 (the source registers are read at issue;
             // one wait below covers both stores)
-            tmem_st_32x32b_x32(row_tmem + kTmemA + C::kACols * s + 32 * q, out);
+            tmem_st_32x32b_x32(row_tmem + C::kTmemA + C::kACols * s + 32 * q, out);
           }
         }
         tmem_st_wait();
@@ -415,7 +421,6 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     const int tc = lane >> 1, th = lane & 1;
     grid_dependency_wait();                 // sx comes from the preceding grid under PDL
     int lt = 0;
-    uint32_t ks = 0;                        // split units handled so far (barrier phases)
     for (int u = blockIdx.x; u < args.units; u += gridDim.x, ++lt) {
       const Unit w = unit_of(args, u, kt_total);
       const int b = lt % C::kAcc;
@@ -459,28 +464,20 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
           }
           __syncwarp();
         }
-        // ... then count the arrival: the mbarrier orders the four warps'
-        // stores before one thread's cumulative fence; the last arrival fences
-        // again before it releases the warps that read the other partials.
-        // The flag is rewritten only after all four warps arrive for the next
-        // split unit, i.e. after each of them has read it.
+        // ... then count this warp's arrival at its slice.  The warp barrier
+        // orders the lanes' stores before lane 0's cumulative fence and
+        // atomic; the last arrival fences again, and the second warp barrier
+        // orders its lanes' reads of the other partials after that fence.
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_epi_in);
-        bool got = true;
-        if (ew == 0 && lane == 0) {
-          got = mbar_wait(bar_epi_in, ks & 1u, abort_flag, &g_error_word, kErrEpilogue);
-          bool last = false;
-          if (got) {
-            __threadfence();
-            last = arrive_last(args.ws_count + w.mt * args.n_tiles + w.nt, splits);
-            if (last) __threadfence();
-          }
-          *last_flag = last ? 1u : 0u;
-          mbar_arrive(bar_epi_go);
+        bool last = false;
+        if (lane == 0) {
+          __threadfence();
+          last = arrive_last(
+              args.ws_count + (w.mt * args.n_tiles + w.nt) * kSlicesPerTile + q4, splits);
+          if (last) __threadfence();
         }
-        got = mbar_wait(bar_epi_go, ks & 1u, abort_flag, &g_error_word, kErrEpilogue) && got;
-        ++ks;
-        write_out = __all_sync(0xffffffffu, got && *last_flag != 0u);
+        __syncwarp();
+        write_out = __shfl_sync(0xffffffffu, last ? 1 : 0, 0) != 0;
       }
       if (write_out && *abort_flag == 0u) {
         const int32_t* parts = args.ws_part + (static_cast<size_t>(w.mt * splits) * TOK) * N;
@@ -607,14 +604,41 @@ struct Plan {
 };
 
 bool splittable(const Plan& p) {
-  return static_cast<long>(p.m_tiles) * p.n_tiles <= kMaxCounterTiles;
+  return static_cast<long>(p.m_tiles) * p.n_tiles <= kMaxCounterTiles;   // one counter per slice
 }
 
-int stages_for(int tok) { return tok <= 32 ? 7 : tok == 64 ? 6 : 4; }
+int stages_for(int tok) { return tok <= 32 ? 7 : tok == 64 ? 6 : tok == 176 ? 5 : 4; }
 
-bool valid_tok(int t) { return t == 16 || t == 32 || t == 64 || t == 128 || t == 256; }
+bool valid_tok(int t) {
+  return t == 16 || t == 32 || t == 64 || t == 128 || t == 176 || t == 192 || t == 256;
+}
 
-int auto_tok(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
+// Token tile for a shape.  Up to 64 tokens the smallest tile that holds M.
+// Beyond that the choice is between 128 (two k-tiles per pipeline stage) and
+// the wide tiles 176 / 192 (one k-tile per stage, so more control work per
+// K but fewer output tiles): the cost of a shape is the number of rounds of
+// units over the SMs times the time a unit takes per k-tile, measured on B200
+// with every SM busy as about 272, 393 and 445 ns for 128, 176 and 192 tokens.
+int auto_tok(int M, int n_tiles) {
+  if (M <= 16) return 16;
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  const long sms = sm_count();
+  const int cand[3] = {128, 176, 192};
+  const double per_kt[3] = {272.0, 393.0, 445.0};
+  int best = 128;
+  double best_cost = 1e30;
+  for (int i = 0; i < 3; ++i) {
+    const long units = static_cast<long>((M + cand[i] - 1) / cand[i]) * n_tiles;
+    const long rounds = (units + sms - 1) / sms;
+    const double cost = static_cast<double>(rounds) * per_kt[i];
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = cand[i];
+    }
+  }
+  return best;
+}
 
 // Cost model for the number of K splits: units are spread over one CTA per
 // SM, a unit costs its k-tiles plus a fixed overhead (pipeline fill and
@@ -651,7 +675,7 @@ Plan make_plan(int M, int N, int K, int tok_req, int splits_req) {
   Plan p;
   p.n_tiles = N / kTileN;
   const int kt = K / kTileK;
-  p.tok = tok_req ? tok_req : auto_tok(M);
+  p.tok = tok_req ? tok_req : auto_tok(M, p.n_tiles);
   p.m_tiles = (M + p.tok - 1) / p.tok;
   p.stages = stages_for(p.tok);
   p.splits = splits_req ? splits_req : auto_splits(p.n_tiles * p.m_tiles, kt, p.tok);
@@ -764,6 +788,8 @@ int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* 
     case 32: return launch_tok<32>(map, a, p, s, pdl);
     case 64: return launch_tok<64>(map, a, p, s, pdl);
     case 128: return launch_tok<128>(map, a, p, s, pdl);
+    case 176: return launch_tok<176>(map, a, p, s, pdl);
+    case 192: return launch_tok<192>(map, a, p, s, pdl);
     default: return launch_tok<256>(map, a, p, s, pdl);
   }
 }
