@@ -333,6 +333,18 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
         if (static_cast<int>(g % kDqGroups) != wg) continue;
         const int s = g % S;
         const uint32_t ph = (g / S) & 1;
+        // A parity wait is only exact while the barrier has completed the
+        // phase before the awaited one.  This warpgroup last used slot s
+        // several stages ago, so it first waits for the A columns of slot s
+        // (the MMAs of stage g - S completed, in order): those MMAs read the
+        // dequantized weights of stage g - S, so the weight slot's previous
+        // phase has completed before its parity is tested below.
+        if (g >= S && !mbar_wait(bar_empty + 8 * s, ph ^ 1, abort_flag, &g_error_word,
+                                 kErrDequant)) {
+          aborted = true;
+          break;
+        }
+        tc_fence_after_sync();
         if (!mbar_wait(bar_wfull + 8 * s, ph, abort_flag, &g_error_word, kErrDequant)) {
           aborted = true;
           break;
@@ -366,13 +378,6 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
         // arrive releases this warp's reads, ordered by the warp barrier)
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_wempty + 8 * s);
-        // the A columns of slot s are free once the MMAs of stage g - S completed
-        if (g >= S && !mbar_wait(bar_empty + 8 * s, ph ^ 1, abort_flag, &g_error_word,
-                                 kErrDequant)) {
-          aborted = true;
-          break;
-        }
-        tc_fence_after_sync();
 #pragma unroll
         for (int q = 0; q < C::kNB; ++q) {
           if (q < nb) {
@@ -928,6 +933,22 @@ extern "C" int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int*
   if (stages) *stages = p.stages;
   return QOQ_OK;
 }
+
+namespace qoq {
+unsigned int* error_word_ptr() {
+  static std::mutex mu;
+  static unsigned int* ptr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+    ptr[dev] = static_cast<unsigned int*>(p);
+  }
+  return ptr[dev];
+}
+}  // namespace qoq
 
 extern "C" int qoq_device_error(unsigned int* value, int clear) {
   if (!value) return QOQ_ERR_INVALID_ARG;
