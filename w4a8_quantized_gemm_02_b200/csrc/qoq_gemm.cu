@@ -934,22 +934,6 @@ extern "C" int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int*
   return QOQ_OK;
 }
 
-namespace qoq {
-unsigned int* error_word_ptr() {
-  static std::mutex mu;
-  static unsigned int* ptr[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
-    ptr[dev] = static_cast<unsigned int*>(p);
-  }
-  return ptr[dev];
-}
-}  // namespace qoq
-
 extern "C" int qoq_device_error(unsigned int* value, int clear) {
   if (!value) return QOQ_ERR_INVALID_ARG;
   if (int st = check_device()) return st;

@@ -55,7 +55,6 @@ __device__ __forceinline__ int div_rne(int a, int b) {
 // When sx is a normal FP16 number, |x| / sx <= 127 / (1 - 2^-11) < 127.5 and
 // no code can leave [-127, 127]; only rows whose scale is subnormal clamp.
 // ---------------------------------------------------------------------------
-constexpr int kActRegVec = 16;
 constexpr float kRoundMagic = 12582912.0f;   // 1.5 * 2^23
 
 template <bool kClamp>
@@ -105,9 +104,12 @@ __device__ __forceinline__ __half2 absmax8(uint4 v, __half2 amax) {
   return amax;
 }
 
-// kWarps warps per CTA, kWarpsPerRow of them share a row: 1 for many rows
-// (a warp per row), kWarps when rows are few (a CTA per row).
-template <int kWarps, int kWarpsPerRow>
+// kWarps warps per CTA, kWarpsPerRow of them share a row (1: a warp per row;
+// kWarps: a CTA per row).  Each thread keeps up to kRegVec 16-byte vectors of
+// its row in registers (one pass over global memory); longer rows are read
+// twice.  Few vectors per thread keep the register count low, so that many
+// CTAs share an SM and many loads are in flight.
+template <int kWarps, int kWarpsPerRow, int kRegVec>
 __global__ void __launch_bounds__(32 * kWarps)
 act_quant_kernel(const __half* __restrict__ X, int M, int K, int8_t* __restrict__ X8,
                  __half* __restrict__ sx) {
@@ -124,17 +126,17 @@ act_quant_kernel(const __half* __restrict__ X, int M, int K, int8_t* __restrict_
   const uint4* row = reinterpret_cast<const uint4*>(X + static_cast<size_t>(active ? m : 0) * K);
   uint2* out = reinterpret_cast<uint2*>(X8 + static_cast<size_t>(active ? m : 0) * K);
   const int nvec = active ? K / 8 : 0;
-  const bool in_regs = K / 8 <= kT * kActRegVec;
-  uint4 v[kActRegVec];
+  const bool in_regs = K / 8 <= kT * kRegVec;
+  uint4 v[kRegVec];
   __half2 hmax = __float2half2_rn(0.0f);
   if (in_regs) {
 #pragma unroll
-    for (int u = 0; u < kActRegVec; ++u) {
+    for (int u = 0; u < kRegVec; ++u) {
       const int i = t + kT * u;
       if (i < nvec) v[u] = __ldg(row + i);
     }
 #pragma unroll
-    for (int u = 0; u < kActRegVec; ++u)
+    for (int u = 0; u < kRegVec; ++u)
       if (t + kT * u < nvec) hmax = absmax8(v[u], hmax);
   } else {
     for (int i0 = 0; i0 < nvec; i0 += kT * 8) {
@@ -170,13 +172,13 @@ act_quant_kernel(const __half* __restrict__ X, int M, int K, int8_t* __restrict_
   if (in_regs) {
     if (!clamp) {
 #pragma unroll
-      for (int u = 0; u < kActRegVec; ++u) {
+      for (int u = 0; u < kRegVec; ++u) {
         const int i = t + kT * u;
         if (i < nvec) out[i] = quantize8<false>(v[u], sf, rcp, half_sf);
       }
     } else {
 #pragma unroll
-      for (int u = 0; u < kActRegVec; ++u) {
+      for (int u = 0; u < kRegVec; ++u) {
         const int i = t + kT * u;
         if (i < nvec) out[i] = quantize8<true>(v[u], sf, rcp, half_sf);
       }
@@ -380,11 +382,20 @@ namespace qoq {
 int launch_act_quant(const void* X, int M, int K, int8_t* X8, void* sx, void* stream) {
   const __half* Xh = static_cast<const __half*>(X);
   __half* sxh = static_cast<__half*>(sx);
+  cudaStream_t st = as_stream(stream);
+  const int nvec = K / 8;
   if (M <= 2 * sm_count()) {
-    // few rows: a whole CTA per row keeps many loads in flight per row
-    act_quant_kernel<8, 8><<<M, 256, 0, as_stream(stream)>>>(Xh, M, K, X8, sxh);
+    // few rows: 8 warps per row keep many loads in flight per row
+    act_quant_kernel<8, 8, 16><<<M, 256, 0, st>>>(Xh, M, K, X8, sxh);
+  } else if (nvec <= 128 * 4) {
+    // many rows: a CTA of 4 warps per row holding 4 vectors per thread
+    act_quant_kernel<4, 4, 4><<<M, 128, 0, st>>>(Xh, M, K, X8, sxh);
+  } else if (nvec <= 256 * 4) {
+    act_quant_kernel<8, 8, 4><<<M, 256, 0, st>>>(Xh, M, K, X8, sxh);
+  } else if (nvec <= 256 * 8) {
+    act_quant_kernel<8, 8, 8><<<M, 256, 0, st>>>(Xh, M, K, X8, sxh);
   } else {
-    act_quant_kernel<4, 1><<<(M + 3) / 4, 128, 0, as_stream(stream)>>>(Xh, M, K, X8, sxh);
+    act_quant_kernel<8, 8, 16><<<M, 256, 0, st>>>(Xh, M, K, X8, sxh);
   }
   return launch_status();
 }
