@@ -34,9 +34,10 @@
 //   warps 14..17 epilogue: tcgen05.ld of a finished accumulator, one FP32
 //                scale per element, a transpose through shared memory and
 //                16-byte stores, overlapping the next unit's main loop.
-// When K is split, each unit writes its INT32 partial tile to the caller's
-// workspace and the last one to arrive (an arrival counter per output tile)
-// adds them up exactly and runs the scaling.
+// When K is split, each epilogue warp writes its 32-channel slice of the INT32
+// partial tile to the caller's workspace, and the last warp to arrive at a
+// slice (an arrival counter per slice) adds the slices up exactly and runs
+// the scaling.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -61,11 +62,10 @@ constexpr int kThreads = 32 * kWarps;            // 608
 constexpr int kRawStageBytes = 8576;             // largest packed block (group 64)
 constexpr int kTmemCols = 512;
 constexpr int kStageBytesEpi = 32 * 16 * 4;      // per epilogue warp: 16 columns x 32 rows
-// The workspace starts with a fixed region of arrival counters (one word per
-// output tile), so that counter words never share memory with the partial
-// sums of a launch of another shape.
-// Each epilogue warp counts the arrivals at its own 32-channel slice of an
-// output tile, so a tile has four counters.
+// The workspace starts with a fixed region of arrival counters, so that
+// counter words never share memory with the partial sums of a launch of
+// another shape.  Each epilogue warp counts the arrivals at its own 32-channel
+// slice of an output tile, so a tile has four counters.
 constexpr int kSlicesPerTile = 4;
 constexpr int kMaxCounterTiles = 1024;
 constexpr size_t kCounterBytes = kMaxCounterTiles * kSlicesPerTile * 4;
@@ -127,20 +127,43 @@ struct GemmArgs {
   int m_tiles, n_tiles;
   int units;            // n_tiles * m_tiles * splits
   int blk_bytes;
+  float rcp_splits;     // 1 / splits and 1 / m_tiles, rounded (for small_div)
+  float rcp_mtiles;
 };
 
 struct Unit {
   int nt, mt, split, kt_begin, num_kt;
 };
 
+// n / d for 0 <= n < 2^22 and d >= 1 without an integer division: the
+// binary32 product n * rn(1/d), truncated, is within one of the quotient (its
+// relative error is below 2^-22), and the remainder check corrects it.
+__device__ __forceinline__ int small_div(int n, int d, float rcp_d) {
+  int q = static_cast<int>(__fmul_rz(static_cast<float>(n), rcp_d));
+  const int r = n - q * d;
+  if (r < 0) {
+    --q;
+  } else if (r >= d) {
+    ++q;
+  }
+  return q;
+}
+
 __device__ __forceinline__ Unit unit_of(const GemmArgs& a, int u, int kt_total) {
   Unit w;
-  w.split = u % a.splits;
-  const int rest = u / a.splits;
-  w.mt = rest % a.m_tiles;
-  w.nt = rest / a.m_tiles;
-  w.kt_begin = (w.split * kt_total) / a.splits;
-  w.num_kt = ((w.split + 1) * kt_total) / a.splits - w.kt_begin;
+  int rest = u;
+  if (a.splits == 1) {
+    w.split = 0;
+    w.kt_begin = 0;
+    w.num_kt = kt_total;
+  } else {
+    rest = small_div(u, a.splits, a.rcp_splits);
+    w.split = u - rest * a.splits;
+    w.kt_begin = small_div(w.split * kt_total, a.splits, a.rcp_splits);
+    w.num_kt = small_div((w.split + 1) * kt_total, a.splits, a.rcp_splits) - w.kt_begin;
+  }
+  w.nt = small_div(rest, a.m_tiles, a.rcp_mtiles);
+  w.mt = rest - w.nt * a.m_tiles;
   return w;
 }
 
@@ -205,22 +228,20 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc + 4);
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(bar_xfull + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, 1);
-      mbar_init(bar_wfull + 8 * s, 1);
-      mbar_init(bar_wempty + 8 * s, 4);
-      mbar_init(bar_dqfull + 8 * s, 4);
+  if (warp == 0) {
+    // the barriers are contiguous from bar_xfull: xfull, empty, wfull, wempty,
+    // dqfull (S each), accfull, accempty (kAcc each), drain; the lanes of
+    // warp 0 initialize them in parallel
+    for (int i = lane; i < C::kNumBars; i += 32) {
+      const bool four = (i >= 3 * S && i < 5 * S) ||
+                        (i >= 5 * S + C::kAcc && i < 5 * S + 2 * C::kAcc);
+      mbar_init(bar_xfull + 8 * i, four ? 4u : 1u);
     }
-    for (int b = 0; b < C::kAcc; ++b) {
-      mbar_init(bar_accfull + 8 * b, 1);
-      mbar_init(bar_accempty + 8 * b, 4);
+    if (lane == 0) {
+      *abort_flag = 0u;
+      prefetch_tensormap(&tmap_x);
     }
-    mbar_init(bar_drain, 1);
-    *abort_flag = 0u;
     fence_mbar_init();
-    prefetch_tensormap(&tmap_x);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -741,7 +762,8 @@ int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* 
     return QOQ_ERR_INVALID_ARG;
 
   Plan p = make_plan(M, N, K, tok_req, splits_req);
-  if (static_cast<long>(p.n_tiles) * p.m_tiles * p.splits > 0x7fffffffL) return QOQ_ERR_UNSUPPORTED;
+  // the kernel divides unit indices below 2^22 by multiplication (small_div)
+  if (static_cast<long>(p.n_tiles) * p.m_tiles * p.splits >= (1L << 22)) return QOQ_ERR_UNSUPPORTED;
   if (p.splits > 1 && !splittable(p)) {
     if (splits_req) return QOQ_ERR_UNSUPPORTED;
     p.splits = 1;
@@ -786,6 +808,8 @@ int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* 
   a.n_tiles = p.n_tiles;
   a.units = p.units;
   a.blk_bytes = static_cast<int>(block_bytes(group));
+  a.rcp_splits = 1.0f / static_cast<float>(p.splits);
+  a.rcp_mtiles = 1.0f / static_cast<float>(p.m_tiles);
 
   cudaStream_t s = as_stream(stream);
   switch (p.tok) {
