@@ -53,8 +53,10 @@ def test_plan_is_host_only(L):
     for M in (1, 16, 17, 64, 100, 256, 1024, 4096):
         p = qoq.gemm_plan(M, 6144, 4096, 128)
         assert p["tok_tile"] in (16, 32, 64, 128, 176, 192, 256)
-        assert p["tok_tile"] >= min(M, 128)
+        assert p["tok_tile"] >= min(M, 32)
         assert 1 <= p["splits"] <= 8
+        # K is split only while all units fit one round of CTAs
+        assert p["splits"] == 1 or 48 * -(-M // p["tok_tile"]) * p["splits"] <= 148
         # persistent grid: one CTA per SM at most (148 without a device)
         assert p["ctas"] == min(48 * -(-M // p["tok_tile"]) * p["splits"], 148)
     with pytest.raises(qoq.QoQError):

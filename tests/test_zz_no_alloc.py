@@ -41,7 +41,7 @@ def _close(y, y_ref):
 
 
 # (M, N, K): decode shapes that split K (largest scratch last) and one that does not
-SHAPES = [(1, 6144, 4096), (32, 6144, 4096), (256, 6144, 4096), (32, 24576, 8192)]
+SHAPES = [(1, 6144, 4096), (32, 6144, 4096), (256, 6144, 4096), (64, 4096, 14336)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES, ids=[f"M{m}_N{n}_K{k}" for m, n, k in SHAPES])
@@ -49,7 +49,7 @@ def test_static_ws_matches_workspace_entry(M, N, K):
     X8, sx, packed, s1 = _operands(M, N, K, seed=M + N + K)
     need = qoq.gemm_workspace_bytes(M, N, K, GROUP)
     assert need <= STATIC_WS_BYTES
-    if M <= 32:
+    if M != 256:
         assert qoq.gemm_plan(M, N, K, GROUP)["splits"] > 1   # the fixed array is used
     qoq.device_error(clear=True)
     y_ref = qoq.w4a8_gemm(X8, sx, packed, s1, N, GROUP)

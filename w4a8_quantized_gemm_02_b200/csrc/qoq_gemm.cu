@@ -180,13 +180,20 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
-// Register this CTA's arrival at an output tile (one thread, after the
-// partial tile is written and a fence made it visible).  The counter counts
-// the arrivals of the current launch; the last of `splits` arrivals resets it
-// to zero, so the counter region returns to zero after every launch that
-// completes.
+// Register one warp's arrival at its slice of an output tile (lane 0, after
+// the warp's partial slice is written and a warp barrier ordered the lanes'
+// stores before this thread).  The add has acquire-release semantics at GPU
+// scope: it releases those stores (cumulatively) to the last arrival and, for
+// the last arrival, acquires the stores of the others, in one round trip.
+// The counter counts the arrivals of the current launch; the last of `splits`
+// arrivals resets it to zero, so the counter region returns to zero after
+// every launch that completes.
 __device__ __forceinline__ bool arrive_last(uint32_t* ctr, int splits) {
-  const uint32_t old = atomicAdd(ctr, 1u);
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+               : "=r"(old)
+               : "l"(ctr)
+               : "memory");
   if (old >= static_cast<uint32_t>(splits)) atomicOr(&g_error_word, kErrCounter);
   const bool last = old == static_cast<uint32_t>(splits - 1);
   if (last) atomicExch(ctr, 0u);
@@ -491,16 +498,14 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
           __syncwarp();
         }
         // ... then count this warp's arrival at its slice.  The warp barrier
-        // orders the lanes' stores before lane 0's cumulative fence and
-        // atomic; the last arrival fences again, and the second warp barrier
-        // orders its lanes' reads of the other partials after that fence.
+        // orders the lanes' stores before lane 0's release, and the second
+        // warp barrier orders the lanes' reads of the other partials after
+        // the last arrival's acquire.
         __syncwarp();
         bool last = false;
         if (lane == 0) {
-          __threadfence();
           last = arrive_last(
               args.ws_count + (w.mt * args.n_tiles + w.nt) * kSlicesPerTile + q4, splits);
-          if (last) __threadfence();
         }
         __syncwarp();
         write_out = __shfl_sync(0xffffffffu, last ? 1 : 0, 0) != 0;
@@ -639,17 +644,21 @@ bool valid_tok(int t) {
   return t == 16 || t == 32 || t == 64 || t == 128 || t == 176 || t == 192 || t == 256;
 }
 
-// Token tile for a shape.  Up to 64 tokens the smallest tile that holds M.
+// Token tile for a shape.  Up to 32 tokens the smallest tile that holds M; up
+// to 64 two 32-token tiles when they fit one round of units, else one of 64.
 // Beyond that the choice is between 128 (two k-tiles per pipeline stage) and
 // the wide tiles 176 / 192 (one k-tile per stage, so more control work per
 // K but fewer output tiles): the cost of a shape is the number of rounds of
 // units over the SMs times the time a unit takes per k-tile, measured on B200
 // with every SM busy as about 272, 393 and 445 ns for 128, 176 and 192 tokens.
 int auto_tok(int M, int n_tiles) {
+  const long sms = sm_count();
   if (M <= 16) return 16;
   if (M <= 32) return 32;
-  if (M <= 64) return 64;
-  const long sms = sm_count();
+  if (M <= 64) {
+    // two 32-token tiles run on twice the SMs as long as they fit one round
+    return static_cast<long>((M + 31) / 32) * n_tiles <= sms ? 32 : 64;
+  }
   const int cand[3] = {128, 176, 192};
   const double per_kt[3] = {272.0, 393.0, 445.0};
   int best = 128;
@@ -669,8 +678,8 @@ int auto_tok(int M, int n_tiles) {
 // Cost model for the number of K splits: units are spread over one CTA per
 // SM, a unit costs its k-tiles plus a fixed overhead (pipeline fill and
 // epilogue), a split unit a little more (partial tile out, final sum in).
-// Only small token tiles are split: for 64 tokens and more the partial tiles
-// cost more than the parallelism gains.
+// Only small token tiles are split, and only while all units fit one round:
+// otherwise the partial tiles cost more than the parallelism gains.
 int auto_splits(int tiles, int kt, int tok) {
   if (tok > 32) return 1;
   const long sms = sm_count();
@@ -678,7 +687,7 @@ int auto_splits(int tiles, int kt, int tok) {
   double best = 1e30;
   for (int s = 1; s <= 8 && s <= kt; ++s) {
     if (s > 1 && kt / s < 2) break;
-    if (static_cast<long>(tiles) * s > 4L * sms && s > 1) break;
+    if (static_cast<long>(tiles) * s > sms && s > 1) break;   // one round of units
     const long units = static_cast<long>(tiles) * s;
     const long rounds = (units + sms - 1) / sms;
     const double cost =
