@@ -17,7 +17,7 @@
 //   warp 0       X producer: tensor-map copies of the X8 tiles (128-byte
 //                swizzle) into the X ring, refilled when the stage's MMAs
 //                completed;
-//   warp 18      W producer: one bulk copy of the stage's packed weight
+//   last warp    W producer: one bulk copy of the stage's packed weight
 //                blocks into the weight ring, refilled as soon as the
 //                dequantizers hold the blocks in registers, so the weight
 //                stream runs ahead of the MMAs;
@@ -26,12 +26,13 @@
 //                from tensor memory and X8 from shared memory, into one of two
 //                INT32 accumulators in tensor memory (double buffered); one
 //                commit per stage frees its X8 tiles and A columns;
-//   warps 2..13  three dequantizing warpgroups taking stages in turn: each
+//   warps 2..     three or four dequantizing warpgroups (four for token
+//                tiles up to 64) taking stages in turn: each
 //                thread turns one weight row of the UINT4 blocks into INT8
 //                (four byte lanes per 32-bit multiply-add) and writes one
 //                128-byte row per k-tile into the stage's tensor-memory
 //                columns with tcgen05.st;
-//   warps 14..17 epilogue: tcgen05.ld of a finished accumulator, one FP32
+//   next 4 warps epilogue: tcgen05.ld of a finished accumulator, one FP32
 //                scale per element, a transpose through shared memory and
 //                16-byte stores, overlapping the next unit's main loop.
 // When K is split, each epilogue warp writes its 32-channel slice of the INT32
@@ -54,11 +55,6 @@ __device__ unsigned int g_error_word = 0;
 
 namespace {
 
-constexpr int kDqGroups = 3;                     // dequantizing warpgroups
-constexpr int kWarpEpi0 = 2 + 4 * kDqGroups;     // first epilogue warp (14)
-constexpr int kWarpW = kWarpEpi0 + 4;            // weight producer warp (18)
-constexpr int kWarps = kWarpW + 1;               // 19
-constexpr int kThreads = 32 * kWarps;            // 608
 constexpr int kRawStageBytes = 8576;             // largest packed block (group 64)
 constexpr int kTmemCols = 512;
 constexpr int kStageBytesEpi = 32 * 16 * 4;      // per epilogue warp: 16 columns x 32 rows
@@ -80,6 +76,15 @@ struct Cfg {
   // wait / issue / commit sequence costs about as much as the MMAs of one
   // 128 x 128 x 128 k-tile.  kAcc accumulators of TOK columns let the
   // epilogue of one unit overlap the main loop of the next.
+  // Warp layout: producers and MMA (warps 0, 1), kDqGroups dequantizing
+  // warpgroups, four epilogue warps, the weight producer last.  Small token
+  // tiles (decode) are limited by how fast one CTA dequantizes its share of
+  // the weights, so they get four warpgroups; from 128 tokens on the SM's
+  // issue slots are the limit and three warpgroups run faster.
+  static constexpr int kDqGroups = TOK <= 64 ? 4 : 3;
+  static constexpr int kWarpEpi0 = 2 + 4 * kDqGroups;        // first epilogue warp
+  static constexpr int kWarpW = kWarpEpi0 + 4;               // weight producer warp
+  static constexpr int kThreads = 32 * (kWarpW + 1);
   static constexpr int kNB = TOK <= 128 ? 2 : 1;
   static constexpr int kXBytes = TOK * kTileK;                // one 128-byte-wide X8 tile
   static constexpr int kStageX = kNB * kXBytes;
@@ -200,8 +205,57 @@ __device__ __forceinline__ bool arrive_last(uint32_t* ctr, int splits) {
   return last;
 }
 
+// One weight row of one packed block in registers: its 64 code bytes and
+// the group scale / dequantization bias of its (one or two) groups.
+struct RowBlock {
+  uint4 v[4];
+  uint32_t s2v[2], bias[2];
+};
+
+__device__ __forceinline__ void load_row_block(const uint8_t* blk, int r, int gpt, RowBlock& rb) {
+#pragma unroll
+  for (int gl = 0; gl < 2; ++gl) {
+    if (gl < gpt) {
+      rb.s2v[gl] = blk[kCodesBytes + gl * kTileN + r];
+      const uint32_t zb = blk[kCodesBytes + gpt * kTileN + gl * 64 + (r >> 1)];
+      const uint32_t zv = (r & 1) ? (zb >> 4) : (zb & 15u);
+      rb.bias[gl] = dq_bias(zv, rb.s2v[gl]);
+    } else {
+      rb.s2v[gl] = rb.s2v[0];
+      rb.bias[gl] = rb.bias[0];
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) rb.v[j] = *reinterpret_cast<const uint4*>(blk + (j * kTileN + r) * 16);
+}
+
+// Four byte lanes per 32-bit op into INT8 and one 128-byte row into tensor
+// memory at `taddr`: column c holds K bytes 4c..4c+3.  The source registers
+// are read at issue; the caller waits for the stores once per stage.
+__device__ __forceinline__ void dequant_store_row_block(const RowBlock& rb, int gpt,
+                                                        uint32_t taddr) {
+  uint32_t out[32];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    // second group of the block (group 64) for the last two 32-byte chunks;
+    // a select rather than an index keeps the struct in registers
+    const bool g1 = gpt == 2 && j >= 2;
+    const uint32_t sv = g1 ? rb.s2v[1] : rb.s2v[0];
+    const uint32_t bv = g1 ? rb.bias[1] : rb.bias[0];
+    out[8 * j + 0] = dq_lanes(lo_codes(rb.v[j].x), sv, bv);
+    out[8 * j + 1] = dq_lanes(hi_codes(rb.v[j].x), sv, bv);
+    out[8 * j + 2] = dq_lanes(lo_codes(rb.v[j].y), sv, bv);
+    out[8 * j + 3] = dq_lanes(hi_codes(rb.v[j].y), sv, bv);
+    out[8 * j + 4] = dq_lanes(lo_codes(rb.v[j].z), sv, bv);
+    out[8 * j + 5] = dq_lanes(hi_codes(rb.v[j].z), sv, bv);
+    out[8 * j + 6] = dq_lanes(lo_codes(rb.v[j].w), sv, bv);
+    out[8 * j + 7] = dq_lanes(hi_codes(rb.v[j].w), sv, bv);
+  }
+  tmem_st_32x32b_x32(taddr, out);
+}
+
 template <int TOK>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<TOK>::kThreads, 1)
 w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args) {
   using C = Cfg<TOK>;
   constexpr int S = C::kStages;
@@ -345,28 +399,32 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     if (elect_one()) mma_commit(bar_drain);
     __syncwarp();
     drain_wait(bar_drain, 0);                // no MMA in flight past this point
-  } else if (warp < kWarpEpi0) {
+  } else if (warp < C::kWarpEpi0) {
     // ---------------------------------------------------------------- dequantizers
-    const int wg = (warp - 2) >> 2;         // 0 .. kDqGroups-1: takes stages g = wg (mod 3)
+    constexpr int kDqGroups = C::kDqGroups;
+    const int wg = (warp - 2) >> 2;         // 0 .. kDqGroups-1: takes stages g = wg (mod kDqGroups)
     const int q4 = warp & 3;                // tensor-memory lane quarter of this warp
     const int r = q4 * 32 + lane;           // weight row (output channel) within the tile
     const uint32_t row_tmem = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int gpt = kTileK / args.group;
-    uint32_t g = 0;
+    uint32_t g0 = 0;                        // running stage index of the unit's first stage
     bool aborted = false;
     for (int u = blockIdx.x; u < args.units && !aborted; u += gridDim.x) {
       const Unit w = unit_of(args, u, kt_total);
       const int nsteps = (w.num_kt + C::kNB - 1) / C::kNB;
-      for (int i = 0; i < nsteps; ++i, ++g) {
-        if (static_cast<int>(g % kDqGroups) != wg) continue;
+      // this warpgroup's first stage of the unit, then every kDqGroups-th
+      int i = static_cast<int>((static_cast<uint32_t>(wg) + kDqGroups - g0 % kDqGroups) %
+                               kDqGroups);
+      for (; i < nsteps; i += kDqGroups) {
+        const uint32_t g = g0 + i;
         const int s = g % S;
         const uint32_t ph = (g / S) & 1;
         // A parity wait is only exact while the barrier has completed the
-        // phase before the awaited one.  This warpgroup last used slot s
-        // several stages ago, so it first waits for the A columns of slot s
-        // (the MMAs of stage g - S completed, in order): those MMAs read the
-        // dequantized weights of stage g - S, so the weight slot's previous
-        // phase has completed before its parity is tested below.
+        // phase before the awaited one.  This warpgroup first waits for the
+        // A columns of slot s (the MMAs of stage g - S completed, in order):
+        // those MMAs read the dequantized weights of stage g - S, so the
+        // weight slot's previous phase has completed before its parity is
+        // tested below.
         if (g >= S && !mbar_wait(bar_empty + 8 * s, ph ^ 1, abort_flag, &g_error_word,
                                  kErrDequant)) {
           aborted = true;
@@ -378,55 +436,36 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
           break;
         }
         const int nb = min(C::kNB, w.num_kt - i * C::kNB);
-        // this row of every block of the stage, into registers
-        uint4 v[C::kNB][4];
-        uint32_t s2v[C::kNB][2], bias[C::kNB][2];
+        const uint8_t* stage_raw = smem + C::kOffRaw + s * C::kStageRaw;
+        const uint32_t a_cols = row_tmem + C::kTmemA + C::kACols * s;
+        if constexpr (C::kDqGroups == 3) {
+          // every block of the stage into registers first, so the weight slot
+          // is released as early as possible
+          RowBlock rb[C::kNB];
 #pragma unroll
-        for (int q = 0; q < C::kNB; ++q) {
-          if (q < nb) {
-            const uint8_t* blk = smem + C::kOffRaw + s * C::kStageRaw + q * args.blk_bytes;
+          for (int q = 0; q < C::kNB; ++q)
+            if (q < nb) load_row_block(stage_raw + q * args.blk_bytes, r, gpt, rb[q]);
+          // the weight slot may be refilled once every lane has read it (the
+          // arrive releases this warp's reads, ordered by the warp barrier)
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_wempty + 8 * s);
 #pragma unroll
-            for (int gl = 0; gl < 2; ++gl) {
-              if (gl < gpt) {
-                s2v[q][gl] = blk[kCodesBytes + gl * kTileN + r];
-                const uint32_t zb = blk[kCodesBytes + gpt * kTileN + gl * 64 + (r >> 1)];
-                const uint32_t zv = (r & 1) ? (zb >> 4) : (zb & 15u);
-                bias[q][gl] = dq_bias(zv, s2v[q][gl]);
-              } else {
-                s2v[q][gl] = s2v[q][0];
-                bias[q][gl] = bias[q][0];
+          for (int q = 0; q < C::kNB; ++q)
+            if (q < nb) dequant_store_row_block(rb[q], gpt, a_cols + 32 * q);
+        } else {
+          // four warpgroups leave fewer registers per thread: one block at a
+          // time, the weight slot released after the last block's loads
+#pragma unroll
+          for (int q = 0; q < C::kNB; ++q) {
+            if (q < nb) {
+              RowBlock rb;
+              load_row_block(stage_raw + q * args.blk_bytes, r, gpt, rb);
+              if (q == nb - 1) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_wempty + 8 * s);
               }
+              dequant_store_row_block(rb, gpt, a_cols + 32 * q);
             }
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              v[q][j] = *reinterpret_cast<const uint4*>(blk + (j * kTileN + r) * 16);
-          }
-        }
-        // the weight slot may be refilled once every lane has read it (the
-        // arrive releases this warp's reads, ordered by the warp barrier)
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_wempty + 8 * s);
-#pragma unroll
-        for (int q = 0; q < C::kNB; ++q) {
-          if (q < nb) {
-            uint32_t out[32];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int gl = (gpt == 2) ? (j >> 1) : 0;
-              const uint32_t sv = s2v[q][gl], bv = bias[q][gl];
-              out[8 * j + 0] = dq_lanes(lo_codes(v[q][j].x), sv, bv);
-              out[8 * j + 1] = dq_lanes(hi_codes(v[q][j].x), sv, bv);
-              out[8 * j + 2] = dq_lanes(lo_codes(v[q][j].y), sv, bv);
-              out[8 * j + 3] = dq_lanes(hi_codes(v[q][j].y), sv, bv);
-              out[8 * j + 4] = dq_lanes(lo_codes(v[q][j].z), sv, bv);
-              out[8 * j + 5] = dq_lanes(hi_codes(v[q][j].z), sv, bv);
-              out[8 * j + 6] = dq_lanes(lo_codes(v[q][j].w), sv, bv);
-              out[8 * j + 7] = dq_lanes(hi_codes(v[q][j].w), sv, bv);
-            }
-            // one 128-byte row of the INT8 A operand per k-tile: column c
-            // holds K bytes 4c..4c+3 (the source registers are read at issue;
-            // one wait below covers both stores)
-            tmem_st_32x32b_x32(row_tmem + C::kTmemA + C::kACols * s + 32 * q, out);
           }
         }
         tmem_st_wait();
@@ -440,11 +479,12 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_dqfull + 8 * s);
       }
+      g0 += static_cast<uint32_t>(nsteps);
     }
-  } else if (warp < kWarpW) {
+  } else if (warp < C::kWarpW) {
     // ---------------------------------------------------------------- epilogue
     const int q4 = warp & 3;                // tensor-memory lane quarter
-    const int ew = warp - kWarpEpi0;        // 0..3
+    const int ew = warp - C::kWarpEpi0;     // 0..3
     const int r = q4 * 32 + lane;           // output channel within the tile
     const int M = args.M, N = args.N;
     uint8_t* stage = smem + C::kOffEpi + ew * kStageBytesEpi;   // [16 columns][32 rows] x 4 B
@@ -741,7 +781,7 @@ int launch_tok(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cudaStr
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(p.grid), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
