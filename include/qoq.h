@@ -204,9 +204,9 @@ QOQ_API int qoq_w4a8_gemm(const int8_t* X8, const void* sx, const void* packed,
  *     (qoq_gemm_workspace_bytes(M, N, K, group) > QOQ_STATIC_WS_BYTES) is
  *     rejected with QOQ_ERR_UNSUPPORTED and nothing is launched; use
  *     qoq_w4a8_gemm with a workspace for it.  The automatic plan splits K
- *     only for token tiles of at most 32 and only while every unit gets its
- *     own SM, so it needs at most 16 KiB + SMs * 32 * 128 * 4 bytes (about
- *     2.4 MB with 148 SMs): on such a GPU no valid shape is rejected.
+ *     only for token tiles of at most 32 and into at most 4 units per SM,
+ *     so it needs at most 16 KiB + 4 * SMs * 32 * 128 * 4 bytes (about
+ *     9.7 MB with 148 SMs): on such a GPU no valid shape is rejected.
  *   - Every call on a device uses the same array, and it keeps the last
  *     call's contents.  Each call that splits K clears the array's arrival
  *     counters on `stream` before its GEMM, so nothing from an earlier call

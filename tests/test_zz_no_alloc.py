@@ -41,7 +41,7 @@ def _close(y, y_ref):
 
 
 # (M, N, K): decode shapes that split K (largest scratch last) and one that does not
-SHAPES = [(1, 6144, 4096), (32, 6144, 4096), (256, 6144, 4096), (64, 4096, 14336)]
+SHAPES = [(1, 6144, 4096), (16, 4096, 14336), (256, 6144, 4096), (16, 24576, 8192)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES, ids=[f"M{m}_N{n}_K{k}" for m, n, k in SHAPES])
@@ -64,11 +64,13 @@ def test_static_ws_matches_workspace_entry(M, N, K):
 def test_static_ws_back_to_back_shapes():
     """Consecutive calls with different shapes reuse the array's contents
     from the call before; each result must still agree."""
-    a = _operands(1, 6144, 4096, seed=7)
-    b = _operands(16, 6144, 4096, seed=8)
+    a = _operands(1, 6144, 4096, seed=7)      # K split 3 ways
+    b = _operands(16, 4096, 14336, seed=8)    # K split 4 ways
+    assert qoq.gemm_plan(1, 6144, 4096, GROUP)["splits"] > 1
+    assert qoq.gemm_plan(16, 4096, 14336, GROUP)["splits"] > 1
     qoq.device_error(clear=True)
-    refs = [qoq.w4a8_gemm(*a, 6144, GROUP), qoq.w4a8_gemm(*b, 6144, GROUP)]
-    outs = [qoq.w4a8_gemm_static_ws(*a, 6144, GROUP), qoq.w4a8_gemm_static_ws(*b, 6144, GROUP),
+    refs = [qoq.w4a8_gemm(*a, 6144, GROUP), qoq.w4a8_gemm(*b, 4096, GROUP)]
+    outs = [qoq.w4a8_gemm_static_ws(*a, 6144, GROUP), qoq.w4a8_gemm_static_ws(*b, 4096, GROUP),
             qoq.w4a8_gemm_static_ws(*a, 6144, GROUP)]
     torch.cuda.synchronize()
     assert qoq.device_error(clear=True) == 0

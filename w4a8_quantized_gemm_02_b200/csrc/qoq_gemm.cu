@@ -718,16 +718,19 @@ int auto_tok(int M, int n_tiles) {
 // Cost model for the number of K splits: units are spread over one CTA per
 // SM, a unit costs its k-tiles plus a fixed overhead (pipeline fill and
 // epilogue), a split unit a little more (partial tile out, final sum in).
-// Only small token tiles are split, and only while all units fit one round:
-// otherwise the partial tiles cost more than the parallelism gains.
-int auto_splits(int tiles, int kt, int tok) {
+// Only small token tiles are split.  The split tail (partial slices written,
+// the last arrival reads the others back) grows with the tokens in the tile:
+// on B200 a 16-token Llama QKV tile (32 k-tiles) ran fastest unsplit, while
+// single tokens, or 64+ k-tiles per unit, gained from splitting.
+int auto_splits(int tiles, int kt, int tok, int M) {
   if (tok > 32) return 1;
+  if ((M < tok ? M : tok) > 4 && kt < 64) return 1;
   const long sms = sm_count();
   int best_s = 1;
   double best = 1e30;
   for (int s = 1; s <= 8 && s <= kt; ++s) {
     if (s > 1 && kt / s < 2) break;
-    if (static_cast<long>(tiles) * s > sms && s > 1) break;   // one round of units
+    if (static_cast<long>(tiles) * s > 4L * sms && s > 1) break;
     const long units = static_cast<long>(tiles) * s;
     const long rounds = (units + sms - 1) / sms;
     const double cost =
@@ -753,7 +756,7 @@ Plan make_plan(int M, int N, int K, int tok_req, int splits_req) {
   p.tok = tok_req ? tok_req : auto_tok(M, p.n_tiles);
   p.m_tiles = (M + p.tok - 1) / p.tok;
   p.stages = stages_for(p.tok);
-  p.splits = splits_req ? splits_req : auto_splits(p.n_tiles * p.m_tiles, kt, p.tok);
+  p.splits = splits_req ? splits_req : auto_splits(p.n_tiles * p.m_tiles, kt, p.tok, M);
   if (!splits_req && !splittable(p)) p.splits = 1;
   finish_plan(p);
   return p;
