@@ -276,9 +276,19 @@ QOQ_API int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int* sp
  * instead of hanging.  Synchronous (device-wide): reads the word of the
  * current device and, if `clear` is non-zero, resets it to 0.
  * Bits: 1 = producer wait, 2 = MMA wait, 4 = dequantizer wait,
- *       8 = epilogue wait, 16 = split-K arrival counter.
+ *       8 = epilogue wait, 16 = split-K arrival counter,
+ *       64 = qoq_selftest_wait_timeout.
  * ---------------------------------------------------------------------- */
 QOQ_API int qoq_device_error(unsigned int* value, int clear);
+
+/* Self-test of the bounded waits: launches one warp that waits, with the
+ * same bounded mbarrier wait as every kernel of this library, on a barrier
+ * that nothing arrives at.  The wait gives up after its SM-clock limit
+ * (about 2 s at full clock), sets bit 64 in the device error word and the
+ * kernel returns; the CUDA context stays usable.  It makes a stuck wait
+ * observable without faulting or hanging the GPU.  Asynchronous on `stream`
+ * (the kernel runs for about two seconds). */
+QOQ_API int qoq_selftest_wait_timeout(void* stream);
 
 #ifdef __cplusplus
 }

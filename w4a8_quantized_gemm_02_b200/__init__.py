@@ -31,7 +31,7 @@ EXPORTS = (
     "qoq_quantize_act_per_token", "qoq_w4a8_gemm", "qoq_w4a8_gemm_i32",
     "qoq_w4a8_gemm_config", "qoq_w4a8_linear", "qoq_gemm_plan", "qoq_device_error",
     "qoq_gemm_workspace_bytes", "qoq_gemm_workspace_bytes_config",
-    "qoq_w4a8_gemm_static_ws",
+    "qoq_w4a8_gemm_static_ws", "qoq_selftest_wait_timeout",
 )
 
 _lock = threading.Lock()
@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
             L.qoq_quantize_act_per_token.argtypes = [P, I, I, P, P, P]
             L.qoq_w4a8_gemm.restype = I
             L.qoq_w4a8_gemm.argtypes = [P, P, P, P, I, I, I, I, P, P, sz, P]
+            L.qoq_selftest_wait_timeout.restype = I
+            L.qoq_selftest_wait_timeout.argtypes = [P]
             L.qoq_w4a8_gemm_static_ws.restype = I
             L.qoq_w4a8_gemm_static_ws.argtypes = [P, P, P, P, I, I, I, I, P, P]
             L.qoq_w4a8_gemm_i32.restype = I
@@ -176,6 +178,12 @@ def _ws_args(ws):
     if ws is None:
         return None, 0
     return ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size()
+
+
+def selftest_wait_timeout(stream=None):
+    """Launch the bounded-wait self-test kernel (about 2 s on the device);
+    afterwards device_error() has bit 64 set."""
+    _check(lib().qoq_selftest_wait_timeout(_stream(stream)), "qoq_selftest_wait_timeout")
 
 
 def device_error(clear: bool = True) -> int:

@@ -17,6 +17,7 @@ enum : uint32_t {
   kErrDequant = 4u,
   kErrEpilogue = 8u,
   kErrCounter = 16u,
+  kErrSelfTest = 64u,
 };
 
 // Every mbarrier wait gives up after this many SM clock cycles (about two

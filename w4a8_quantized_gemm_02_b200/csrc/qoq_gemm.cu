@@ -1010,6 +1010,32 @@ extern "C" int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int*
   return QOQ_OK;
 }
 
+namespace qoq {
+namespace {
+// One warp waits, with the library's bounded wait, on an mbarrier that
+// nothing ever arrives at: the wait gives up after its SM-clock limit (about
+// two seconds), records kErrSelfTest in the error word and the kernel returns.
+__global__ void __launch_bounds__(32, 1) wait_timeout_selftest_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t abort_word;
+  volatile uint32_t* abort_flag = &abort_word;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_word = 0u;
+    fence_mbar_init();
+  }
+  __syncwarp();
+  mbar_wait(smem_u32(&bar), 0, abort_flag, &g_error_word, kErrSelfTest);
+}
+}  // namespace
+}  // namespace qoq
+
+extern "C" int qoq_selftest_wait_timeout(void* stream) {
+  if (int st = check_device()) return st;
+  wait_timeout_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>();
+  return launch_status();
+}
+
 extern "C" int qoq_device_error(unsigned int* value, int clear) {
   if (!value) return QOQ_ERR_INVALID_ARG;
   if (int st = check_device()) return st;
