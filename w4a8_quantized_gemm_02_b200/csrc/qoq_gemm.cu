@@ -523,7 +523,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
         for (int c0 = 0; c0 < c_end; c0 += 16) {
           uint32_t v[16];
           tmem_ld_32x32b_x16(t_acc + c0, v);
-          tmem_ld_wait();
+          tmem_ld_wait(v);
           uint32_t* st = reinterpret_cast<uint32_t*>(stage);
 #pragma unroll
           for (int j = 0; j < 16; ++j) st[j * 32 + lane] = v[j];
@@ -552,10 +552,16 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
       }
       if (write_out && *abort_flag == 0u) {
         const int32_t* parts = args.ws_part + (static_cast<size_t>(w.mt * splits) * TOK) * N;
+        // software-pipelined over 16-column chunks: the next chunk's load
+        // from tensor memory is in flight while this chunk is scaled and
+        // stored
+        uint32_t v[16], vn[16];
+        tmem_ld_32x32b_x16(t_acc, vn);
         for (int c0 = 0; c0 < c_end; c0 += 16) {
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(t_acc + c0, v);
-          tmem_ld_wait();
+          tmem_ld_wait(vn);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = vn[j];
+          if (c0 + 16 < c_end) tmem_ld_32x32b_x16(t_acc + c0 + 16, vn);
           if (splits > 1) {
             for (int q = 0; q < splits; ++q) {
               if (q == w.split) continue;
