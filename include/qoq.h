@@ -259,7 +259,10 @@ QOQ_API int qoq_w4a8_gemm_config(const int8_t* X8, const void* sx, const void* p
  * Same results as qoq_quantize_act_per_token followed by qoq_w4a8_gemm; here
  * the GEMM is launched as a programmatic dependent of the quantizer, so it
  * starts streaming weights while the activations are still being quantized.
- * Asynchronous on `stream`. */
+ * For M <= 2 x SMs the quantizer is itself launched as a programmatic
+ * dependent of whatever kernel precedes it on `stream`: it may be scheduled
+ * while that kernel drains, but touches no memory before that kernel has
+ * completed.  Asynchronous on `stream`. */
 QOQ_API int qoq_w4a8_linear(const void* X, int M, int K, const void* packed, const void* s1,
                             int N, int group, int8_t* X8, void* sx, void* Y, void* ws,
                             size_t ws_bytes, void* stream);

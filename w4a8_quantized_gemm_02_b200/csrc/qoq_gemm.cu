@@ -513,6 +513,11 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
       const bool ok = mbar_wait(bar_accfull + 8 * b, (lt / C::kAcc) & 1, abort_flag,
                                 &g_error_word, kErrEpilogue);
       if (!__all_sync(0xffffffffu, ok)) break;
+      // At this CTA's last accumulator a kernel launched after this one as
+      // its programmatic dependent (the next layer's activation quantizer in
+      // qoq_w4a8_linear) may be scheduled: it waits for this grid to complete
+      // before touching memory, so only its launch overlaps this tail.
+      if (u + static_cast<int>(gridDim.x) >= args.units) grid_launch_dependents();
       tc_fence_after_sync();
       const uint32_t t_acc = tmem + C::kTmemD + b * TOK + (static_cast<uint32_t>(q4 * 32) << 16);
       const int splits = args.splits;
@@ -997,7 +1002,12 @@ extern "C" int qoq_w4a8_linear(const void* X, int M, int K, const void* packed, 
       !aligned16(s1) || (ws && !aligned16(ws)))
     return QOQ_ERR_INVALID_ARG;
   if (int st = check_device()) return st;
-  if (int st = launch_act_quant(X, M, K, X8, sx, stream)) return st;
+  // For few rows the quantizer may start while the preceding kernel on the
+  // stream drains (it waits for that grid before touching memory); this hides
+  // its launch latency.  For many rows that overlap measured slower on B200,
+  // so the quantizer is then an ordinary launch.
+  const bool aq_pdl = M <= 2 * sm_count();
+  if (int st = launch_act_quant(X, M, K, X8, sx, stream, aq_pdl)) return st;
   // both kernels are this library's: the GEMM reads nothing the quantizer
   // writes before its grid-dependency wait, so it may overlap its tail
   return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, nullptr, 0, 0, ws, ws_bytes, stream,

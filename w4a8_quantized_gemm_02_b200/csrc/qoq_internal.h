@@ -50,7 +50,9 @@ int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* 
               int K, int group, void* Y, int32_t* acc, int tok_req, int splits_req, void* ws,
               size_t ws_bytes, void* stream, bool pdl);
 
-// Launch the per-token activation quantizer (no argument checks).
-int launch_act_quant(const void* X, int M, int K, int8_t* X8, void* sx, void* stream);
+// Launch the per-token activation quantizer (no argument checks).  With
+// `pdl` it may start while the preceding kernel on the stream drains; it
+// waits for that grid before touching memory.
+int launch_act_quant(const void* X, int M, int K, int8_t* X8, void* sx, void* stream, bool pdl);
 
 }  // namespace qoq

@@ -113,6 +113,11 @@ template <int kWarps, int kWarpsPerRow, int kRegVec>
 __global__ void __launch_bounds__(32 * kWarps)
 act_quant_kernel(const __half* __restrict__ X, int M, int K, int8_t* __restrict__ X8,
                  __half* __restrict__ sx) {
+  // Launched as a programmatic dependent of the previous kernel on the stream
+  // (qoq_w4a8_linear), this CTA may start while that kernel drains: nothing
+  // is read or written before that grid has completed and its writes are
+  // visible.  Without the launch attribute the wait returns at once.
+  grid_dependency_wait();
   // the GEMM that consumes X8 may start its weight prologue right away
   grid_launch_dependents();
   __shared__ float red[kWarps];
@@ -379,25 +384,40 @@ unpack_kernel(const uint8_t* __restrict__ packed, int K, int group, uint8_t* __r
 using namespace qoq;
 
 namespace qoq {
-int launch_act_quant(const void* X, int M, int K, int8_t* X8, void* sx, void* stream) {
+template <int kWarps, int kWarpsPerRow, int kRegVec>
+int launch_aq(const __half* X, int M, int K, int8_t* X8, __half* sx, cudaStream_t st, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(M), 1, 1);
+  cfg.blockDim = dim3(32 * kWarps, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, act_quant_kernel<kWarps, kWarpsPerRow, kRegVec>, X, M, K, X8, sx) !=
+      cudaSuccess)
+    return QOQ_ERR_CUDA;
+  return QOQ_OK;
+}
+
+int launch_act_quant(const void* X, int M, int K, int8_t* X8, void* sx, void* stream, bool pdl) {
   const __half* Xh = static_cast<const __half*>(X);
   __half* sxh = static_cast<__half*>(sx);
   cudaStream_t st = as_stream(stream);
   const int nvec = K / 8;
+  // one row per CTA in every variant
   if (M <= 2 * sm_count()) {
     // few rows: 8 warps per row keep many loads in flight per row
-    act_quant_kernel<8, 8, 16><<<M, 256, 0, st>>>(Xh, M, K, X8, sxh);
-  } else if (nvec <= 128 * 4) {
-    // many rows: a CTA of 4 warps per row holding 4 vectors per thread
-    act_quant_kernel<4, 4, 4><<<M, 128, 0, st>>>(Xh, M, K, X8, sxh);
-  } else if (nvec <= 256 * 4) {
-    act_quant_kernel<8, 8, 4><<<M, 256, 0, st>>>(Xh, M, K, X8, sxh);
-  } else if (nvec <= 256 * 8) {
-    act_quant_kernel<8, 8, 8><<<M, 256, 0, st>>>(Xh, M, K, X8, sxh);
-  } else {
-    act_quant_kernel<8, 8, 16><<<M, 256, 0, st>>>(Xh, M, K, X8, sxh);
+    return launch_aq<8, 8, 16>(Xh, M, K, X8, sxh, st, pdl);
   }
-  return launch_status();
+  if (nvec <= 128 * 4) {
+    // many rows: a CTA of 4 warps per row holding 4 vectors per thread
+    return launch_aq<4, 4, 4>(Xh, M, K, X8, sxh, st, pdl);
+  }
+  if (nvec <= 256 * 4) return launch_aq<8, 8, 4>(Xh, M, K, X8, sxh, st, pdl);
+  if (nvec <= 256 * 8) return launch_aq<8, 8, 8>(Xh, M, K, X8, sxh, st, pdl);
+  return launch_aq<8, 8, 16>(Xh, M, K, X8, sxh, st, pdl);
 }
 }  // namespace qoq
 
@@ -407,7 +427,7 @@ extern "C" int qoq_quantize_act_per_token(const void* X, int M, int K, int8_t* X
   if (M <= 0 || K <= 0 || K % 8 != 0) return QOQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(X8) || !aligned16(sx)) return QOQ_ERR_INVALID_ARG;
   if (int st = check_device()) return st;
-  return launch_act_quant(X, M, K, X8, sx, stream);
+  return launch_act_quant(X, M, K, X8, sx, stream, false);
 }
 
 extern "C" int qoq_quantize_weights(const void* W, int N, int K, int group, void* packed,
