@@ -36,25 +36,39 @@ R1 = 119        # protective range of the first level (the largest that keeps dq
 QMAX_X = 127    # symmetric per-token activation range
 
 
+def compile_library(src: str, out: str) -> str:
+    """Compile one C source of the oracle into a shared library with gcc
+    (no fast-math, no FMA contraction)."""
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+           "-fno-fast-math", "-ffp-contract=off", "-o", tmp, src, "-lm"]
+    subprocess.check_call(cmd)
+    os.replace(tmp, out)
+    return out
+
+
 def build(force: bool = False) -> str:
-    """Compile the oracle with gcc (no fast-math, no FMA contraction)."""
+    """Compile ``qoq_oracle.c`` into ``_build/liboracle.so`` when stale."""
     os.makedirs(_BUILD, exist_ok=True)
     if (not force and os.path.exists(_LIB_PATH)
             and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
         return _LIB_PATH
-    tmp = _LIB_PATH + f".tmp{os.getpid()}"
-    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
-           "-fno-fast-math", "-ffp-contract=off", "-o", tmp, _SRC, "-lm"]
-    subprocess.check_call(cmd)
-    os.replace(tmp, _LIB_PATH)
-    return _LIB_PATH
+    return compile_library(_SRC, _LIB_PATH)
+
+
+def _library_path() -> str:
+    """The oracle library to load.  ``QOQ_ORACLE_LIB`` names another build of
+    the same source; the pin tests use it to check that deliberately broken
+    copies of the oracle fail them."""
+    override = os.environ.get("QOQ_ORACLE_LIB")
+    return override if override else build()
 
 
 def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
+            lib = ctypes.CDLL(_library_path())
             P = ctypes.c_void_p
             I = ctypes.c_int
             lib.orc_h2d.restype = ctypes.c_double

@@ -55,6 +55,10 @@ def test_fp16_roundtrip_all_patterns(oracle):
     assert np.array_equal(back[finite], bits[finite])
     back32 = oracle.f2h_array(vals.astype(np.float32))
     assert np.array_equal(back32[finite], bits[finite])
+    # a NaN encodes as a NaN: all-ones exponent and a non-zero fraction
+    for enc in (back[~finite], back32[~finite]):
+        assert enc.size == 2 * 1023
+        assert ((enc & 0x7c00) == 0x7c00).all() and ((enc & 0x03ff) != 0).all()
 
 
 def test_fp16_ties_go_to_even(oracle):
@@ -173,6 +177,29 @@ def test_level2_bruteforce_scale_is_minimal(level2_domain):
     assert np.array_equal(dq[lossless], W8[lossless])
 
 
+def test_level2_groups_are_independent(level2_domain, oracle):
+    # Rows of several groups: each group's (q, s2, z, dq) must be exactly
+    # what that group gives alone, in its own place along K, for G = 128 and
+    # for G = 64 (where each half of a 128-wide domain group is its own group).
+    W8, q, s2, z, dq = level2_domain
+    n = (W8.shape[0] // 4) * 4
+    rows = W8[:n].reshape(n // 4, 4 * 128)
+    qr, s2r, zr = oracle.quant_w_level2(rows, 128)
+    assert np.array_equal(qr, q[:n].reshape(n // 4, 512))
+    assert np.array_equal(s2r.astype(np.int32), s2[:n].reshape(n // 4, 4))
+    assert np.array_equal(zr.astype(np.int32), z[:n].reshape(n // 4, 4))
+    dqr = oracle.dequant_w(qr, s2r, zr, 128)
+    assert np.array_equal(dqr, dq[:n].reshape(n // 4, 512))
+    halves = W8[:n].reshape(2 * n, 64)
+    qh, s2h, zh = oracle.quant_w_level2(halves, 64)
+    q64, s264, z64 = oracle.quant_w_level2(rows, 64)
+    assert np.array_equal(q64, qh.reshape(n // 4, 512))
+    assert np.array_equal(s264, s2h.reshape(n // 4, 8))
+    assert np.array_equal(z64, zh.reshape(n // 4, 8))
+    assert np.array_equal(oracle.dequant_w(q64, s264, z64, 64),
+                          oracle.dequant_w(qh, s2h, zh, 64).reshape(n // 4, 512))
+
+
 def test_level2_full_range_reduces_to_grid(oracle):
     # every group spans exactly [-119, 119]: s2 = 16, z = 7 and the result is
     # the nearest multiple of 16 (ties to even multiple), clipped to 7 steps
@@ -234,6 +261,33 @@ def test_level1_tiny_scale_guard(oracle):
     assert W8[1, 3] == 1 and W8[0].tolist() == [0] * 8
 
 
+def test_level1_subnormal_scale_keeps_protective_range(oracle):
+    # Row maxima of k * 2^-24 for every k up to the first normal binary16
+    # values: there the FP16 scale fp16(amax / 119) can round down by far more
+    # than half a step, and only the clamp keeps the codes inside the
+    # protective range of +-119 (a code of 120 or more would push level-2 dq
+    # past INT8).
+    k = np.arange(1, 2048, dtype=np.float64)
+    W = np.zeros((k.size, 4), np.float16)
+    W[:, 0] = (k * 2.0 ** -24).astype(np.float16)
+    W[:, 1] = (-k * 2.0 ** -24).astype(np.float16)
+    W[:, 2] = (k * 2.0 ** -25).astype(np.float16)
+    assert np.array_equal(W[:, 0].astype(np.float64), k * 2.0 ** -24)
+    s1, W8 = oracle.quant_w_level1(W)
+    w8 = W8.astype(np.int32)
+    assert np.abs(w8).max() == 119
+    assert np.array_equal(w8[:, 1], -w8[:, 0])
+    # amax / 119 is below 18 quanta of 2^-24, so the FP16 scale is that many
+    # quanta rounded to nearest (never a tie: 119 is odd), or the smallest
+    # positive FP16 value where that rounds to 0
+    s = s1.astype(np.float64)
+    assert np.array_equal(s, np.maximum(1, np.round(k / 119)) * 2.0 ** -24)
+    # where rounding the scale cost more than half a code, the code saturates
+    ratio = k * 2.0 ** -24 / s
+    assert (w8[ratio >= 119.5, 0] == 119).all()
+    assert (ratio >= 119.5).any()
+
+
 # ---------------------------------------------------------------------------
 # Per-token activations
 # ---------------------------------------------------------------------------
@@ -259,6 +313,23 @@ def test_act_bounds(oracle):
     assert (err <= s[:, None] / 2 + slack[:, None] + 1e-12).all()
     X8n, sxn = oracle.quant_act(-X)
     assert np.array_equal(X8n, -X8) and np.array_equal(sxn, sx)
+
+
+def test_act_subnormal_scale_stays_symmetric(oracle):
+    # As for the weights: with a subnormal FP16 scale, X / sx can exceed 127
+    # by far; the codes must still stay in the symmetric range [-127, 127].
+    k = np.arange(1, 2048, dtype=np.float64)
+    X = np.zeros((k.size, 3), np.float16)
+    X[:, 0] = (-k * 2.0 ** -24).astype(np.float16)
+    X[:, 1] = (k * 2.0 ** -25).astype(np.float16)
+    X8, sx = oracle.quant_act(X)
+    x8 = X8.astype(np.int32)
+    assert x8.min() == -127 and x8.max() <= 127
+    X8n, sxn = oracle.quant_act(-X)
+    assert np.array_equal(X8n.astype(np.int32), -x8) and np.array_equal(sxn, sx)
+    ratio = k * 2.0 ** -24 / sx.astype(np.float64)
+    assert (x8[ratio >= 127.5, 0] == -127).all()
+    assert (ratio >= 127.5).any()
 
 
 # ---------------------------------------------------------------------------
@@ -308,6 +379,21 @@ def test_int_gemm_extreme_fits_int32(oracle):
     dq[1] = -121
     acc = oracle.int_gemm(X8, dq)
     assert acc.tolist() == [[-127 * 121 * K, 127 * 121 * K]]
+
+
+def test_int_gemm_reports_int32_overflow(oracle):
+    # 127 * 127 * K fits INT32 up to K = 133144 and not beyond: the bound on
+    # K that keeps the INT32 accumulator exact for any INT8 operands.
+    for K, fits in ((133144, True), (133145, False)):
+        X8 = np.full((1, K), 127, np.int8)
+        dq = np.full((2, K), 127, np.int8)
+        dq[1] = -127
+        if fits:
+            acc = oracle.int_gemm(X8, dq)
+            assert acc.tolist() == [[127 * 127 * K, -127 * 127 * K]]
+        else:
+            with pytest.raises(OverflowError):
+                oracle.int_gemm(X8, dq)
 
 
 def test_epilogue_matches_numpy(oracle):
