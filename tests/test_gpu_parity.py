@@ -82,9 +82,18 @@ def _act_cases():
     t[:, 0] = np.float16(127 / 32)
     t[:, 1:] = (np.arange(1, 128) % 9 - 4 + 0.5).astype(np.float16) / np.float16(32)
     yield t
+    # row maxima of k * 2^-24, k = 1 .. 2048: subnormal scales that round far
+    # from amax / 127, where only the clamp keeps codes in [-127, 127]
+    k = np.arange(1, 2049)
+    u = np.zeros((k.size, 128), np.float16)
+    u[:, 0] = (-k * 2.0 ** -24).astype(np.float16)
+    u[:, 1] = (k * 2.0 ** -25).astype(np.float16)
+    u[:, 2:] = (rng.integers(-1, 2, (k.size, 126)) * rng.integers(0, k[:, None] + 1, (k.size, 126))
+                * 2.0 ** -24).astype(np.float16)
+    yield u
 
 
-@pytest.mark.parametrize("case", range(5))
+@pytest.mark.parametrize("case", range(6))
 def test_act_quant_bit_exact(oracle, case):
     X = list(_act_cases())[case]
     X8_ref, sx_ref = oracle.quant_act(X)
@@ -126,6 +135,20 @@ def test_weight_quant_edge_rows(oracle):
     W[4] = -np.abs(W[4])
     W[5, ::3] = np.float16(65504.0)
     W[6] = np.float16(0.5)                                # constant row
+    for g in (128, 64):
+        _check_weights(oracle, W, g)
+
+
+def test_weight_quant_subnormal_scales(oracle):
+    # row maxima of k * 2^-24, k = 1 .. 2048: the FP16 scale rounds far from
+    # amax / 119 and the level-1 clamp decides the codes
+    rng = np.random.default_rng(11)
+    k = np.arange(1, 2049)
+    W = np.zeros((k.size, 256), np.float16)
+    W[:, 0] = (k * 2.0 ** -24).astype(np.float16)
+    W[:, 1] = (-k * 2.0 ** -24).astype(np.float16)
+    W[:, 2:] = (rng.integers(-k[:, None], k[:, None] + 1, (k.size, 254))
+                * 2.0 ** -24).astype(np.float16)
     for g in (128, 64):
         _check_weights(oracle, W, g)
 
