@@ -146,3 +146,31 @@ def test_valid_call_without_gpu_reports_cuda_error(L):
     # with no device the first CUDA call fails; nothing is launched
     assert _gemm(L) == qoq.QOQ_ERR_CUDA
     assert L.qoq_quantize_act_per_token(P(FAKE), 4, 512, P(FAKE), P(FAKE), None) == 3
+
+
+def test_binding_rejects_host_tensors(L):
+    """The binding refuses host (or otherwise unusable) tensors before any
+    call into the library, so no host pointer ever reaches a kernel."""
+    import torch
+    M, N, K = 4, 128, 128
+    X = torch.zeros((M, K), dtype=torch.float16)
+    X8 = torch.zeros((M, K), dtype=torch.int8)
+    sx = torch.ones(M, dtype=torch.float16)
+    s1 = torch.ones(N, dtype=torch.float16)
+    packed = torch.zeros(qoq.packed_weight_bytes(N, K, 128), dtype=torch.uint8)
+    calls = [
+        lambda: qoq.quantize_weights(torch.zeros((N, K), dtype=torch.float16)),
+        lambda: qoq.quantize_act_per_token(X),
+        lambda: qoq.w4a8_gemm(X8, sx, packed, s1, N),
+        lambda: qoq.w4a8_gemm_i32(X8, packed, N),
+        lambda: qoq.w4a8_gemm_static_ws(X8, sx, packed, s1, N),
+        lambda: qoq.w4a8_gemm_config(X8, sx, packed, s1, N, tok_tile=16, splits=1),
+        lambda: qoq.w4a8_linear(X, packed, s1, N),
+        lambda: qoq.unpack_weights(packed, N, K),
+        lambda: qoq.pack_codes(torch.zeros((N, K), dtype=torch.uint8),
+                               torch.ones((N, 1), dtype=torch.int8),
+                               torch.zeros((N, 1), dtype=torch.uint8)),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            call()

@@ -118,7 +118,10 @@ def _stream(stream=None):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _need_cuda(t, name, dtype=None, ndim=None):
+def _need_cuda(t, name, dtype=None, ndim=None, shape=None, device=None, min_bytes=None):
+    """Reject anything the library would read or write through a bad pointer:
+    a host tensor, another device's tensor, a strided view, the wrong dtype,
+    shape or size."""
     import torch
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
@@ -128,6 +131,51 @@ def _need_cuda(t, name, dtype=None, ndim=None):
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if ndim is not None and t.dim() != ndim:
         raise ValueError(f"{name} must have {ndim} dims")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if min_bytes is not None and t.numel() * t.element_size() < min_bytes:
+        raise ValueError(f"{name} holds {t.numel() * t.element_size()} bytes, "
+                         f"needs {min_bytes}")
+
+
+def _need_packed(packed, N, K, group, device):
+    import torch
+    nbytes = packed_weight_bytes(N, K, group)
+    if nbytes == 0:
+        raise QoQError(QOQ_ERR_INVALID_ARG, "qoq_packed_weight_bytes")
+    _need_cuda(packed, "packed", torch.uint8, device=device, min_bytes=nbytes)
+
+
+def _need_gemm_operands(X8, sx, packed, s1, N, group):
+    """X8 (M, K) int8 and, where given, sx (M,) fp16, s1 (N,) fp16 and the
+    packed weights of an N x K layer, all on X8's device.  Returns M, K."""
+    import torch
+    _need_cuda(X8, "X8", torch.int8, 2)
+    M, K = X8.shape
+    dev = X8.device
+    if sx is not None:
+        _need_cuda(sx, "sx", torch.float16, shape=(M,), device=dev)
+    if s1 is not None:
+        _need_cuda(s1, "s1", torch.float16, shape=(N,), device=dev)
+    _need_packed(packed, N, K, group, dev)
+    return M, K
+
+
+def _out(out, shape, dtype, device):
+    """The caller's output tensor after checking it, or a new one."""
+    import torch
+    if out is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    _need_cuda(out, "out", dtype, shape=shape, device=device)
+    return out
+
+
+def _need_ws(ws, device):
+    import torch
+    if ws is not None:
+        _need_cuda(ws, "ws", torch.uint8, device=device)
 
 
 # ---------------------------------------------------------------------------
@@ -159,18 +207,25 @@ def gemm_workspace_bytes(M: int, N: int, K: int, group: int = 128, tok_tile: int
 _ws_cache = {}
 
 
-def workspace(nbytes: int, device):
+def workspace(nbytes: int, device, stream=None):
     """A reusable, zero-initialized device workspace of at least `nbytes`
-    bytes for this device (one buffer per device, grown on demand; calls that
-    share it must be ordered on one stream)."""
+    bytes.  There is one buffer per (device, stream), grown on demand and
+    allocated and zeroed on that stream: the split-K counters in it assume
+    that the calls sharing it run one after another, which calls on one
+    stream do."""
     import torch
     if nbytes <= 0:
         return None
-    key = torch.device(device).index
-    buf = _ws_cache.get(key)
-    if buf is None or buf.numel() < nbytes:
-        buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
-        _ws_cache[key] = buf
+    device = torch.device(device)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    key = (device.index, stream.cuda_stream)
+    with _lock:
+        buf = _ws_cache.get(key)
+        if buf is None or buf.numel() < nbytes:
+            with torch.cuda.stream(stream):
+                buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+            _ws_cache[key] = buf
     return buf
 
 
@@ -215,9 +270,11 @@ def pack_codes(q, s2, z, group: int = 128, stream=None):
     """Canonical codes (uint8 N x K, int8 N x K/G, uint8 N x K/G) -> packed."""
     import torch
     _need_cuda(q, "q", torch.uint8, 2)
-    _need_cuda(s2, "s2", torch.int8, 2)
-    _need_cuda(z, "z", torch.uint8, 2)
     N, K = q.shape
+    if group <= 0 or K % group:
+        raise QoQError(QOQ_ERR_INVALID_ARG, "qoq_pack_codes")
+    _need_cuda(s2, "s2", torch.int8, shape=(N, K // group), device=q.device)
+    _need_cuda(z, "z", torch.uint8, shape=(N, K // group), device=q.device)
     nbytes = packed_weight_bytes(N, K, group)
     if nbytes == 0:
         raise QoQError(QOQ_ERR_INVALID_ARG, "qoq_packed_weight_bytes")
@@ -232,6 +289,7 @@ def unpack_weights(packed, N: int, K: int, group: int = 128, stream=None):
     import torch
     _need_cuda(packed, "packed", torch.uint8)
     dev = packed.device
+    _need_packed(packed, N, K, group, dev)
     q = torch.empty((N, K), dtype=torch.uint8, device=dev)
     s2 = torch.empty((N, K // group), dtype=torch.int8, device=dev)
     z = torch.empty((N, K // group), dtype=torch.uint8, device=dev)
@@ -255,6 +313,8 @@ def quantize_act_per_token(X, out=None, stream=None):
         sx = torch.empty(M, dtype=torch.float16, device=X.device)
     else:
         X8, sx = out
+        _need_cuda(X8, "X8", torch.int8, shape=(M, K), device=X.device)
+        _need_cuda(sx, "sx", torch.float16, shape=(M,), device=X.device)
     _check(lib().qoq_quantize_act_per_token(_ptr(X), M, K, _ptr(X8), _ptr(sx),
                                             _stream(stream)), "qoq_quantize_act_per_token")
     return X8, sx
@@ -263,9 +323,11 @@ def quantize_act_per_token(X, out=None, stream=None):
 _AUTO = object()
 
 
-def _auto_ws(ws, M, N, K, group, device, tok_tile=0, splits=0):
+def _auto_ws(ws, M, N, K, group, device, tok_tile=0, splits=0, stream=None):
     if ws is _AUTO:
-        return workspace(gemm_workspace_bytes(M, N, K, group, tok_tile, splits), device)
+        return workspace(gemm_workspace_bytes(M, N, K, group, tok_tile, splits), device,
+                         stream)
+    _need_ws(ws, device)
     return ws
 
 
@@ -274,10 +336,9 @@ def w4a8_gemm(X8, sx, packed, s1, N: int, group: int = 128, out=None, ws=_AUTO, 
     device tensor for the split-K workspace (default: a cached one; None:
     do not split K)."""
     import torch
-    _need_cuda(X8, "X8", torch.int8, 2)
-    M, K = X8.shape
-    Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=X8.device)
-    w, wb = _ws_args(_auto_ws(ws, M, N, K, group, X8.device))
+    M, K = _need_gemm_operands(X8, sx, packed, s1, N, group)
+    Y = _out(out, (M, N), torch.float16, X8.device)
+    w, wb = _ws_args(_auto_ws(ws, M, N, K, group, X8.device, stream=stream))
     _check(lib().qoq_w4a8_gemm(_ptr(X8), _ptr(sx), _ptr(packed), _ptr(s1), M, N, K, group,
                                _ptr(Y), w, wb, _stream(stream)), "qoq_w4a8_gemm")
     return Y
@@ -289,9 +350,8 @@ def w4a8_gemm_static_ws(X8, sx, packed, s1, N: int, group: int = 128, out=None, 
     overlap in time).  Raises QoQError (unsupported) for shapes needing more
     split-K scratch than that array holds."""
     import torch
-    _need_cuda(X8, "X8", torch.int8, 2)
-    M, K = X8.shape
-    Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=X8.device)
+    M, K = _need_gemm_operands(X8, sx, packed, s1, N, group)
+    Y = _out(out, (M, N), torch.float16, X8.device)
     _check(lib().qoq_w4a8_gemm_static_ws(_ptr(X8), _ptr(sx), _ptr(packed), _ptr(s1), M, N, K,
                                          group, _ptr(Y), _stream(stream)),
            "qoq_w4a8_gemm_static_ws")
@@ -301,10 +361,9 @@ def w4a8_gemm_static_ws(X8, sx, packed, s1, N: int, group: int = 128, out=None, 
 def w4a8_gemm_i32(X8, packed, N: int, group: int = 128, out=None, ws=_AUTO, stream=None):
     """Raw INT32 accumulator acc = X8 . dq^T (M, N)."""
     import torch
-    _need_cuda(X8, "X8", torch.int8, 2)
-    M, K = X8.shape
-    acc = out if out is not None else torch.empty((M, N), dtype=torch.int32, device=X8.device)
-    w, wb = _ws_args(_auto_ws(ws, M, N, K, group, X8.device))
+    M, K = _need_gemm_operands(X8, None, packed, None, N, group)
+    acc = _out(out, (M, N), torch.int32, X8.device)
+    w, wb = _ws_args(_auto_ws(ws, M, N, K, group, X8.device, stream=stream))
     _check(lib().qoq_w4a8_gemm_i32(_ptr(X8), _ptr(packed), M, N, K, group, _ptr(acc), w, wb,
                                    _stream(stream)), "qoq_w4a8_gemm_i32")
     return acc
@@ -314,15 +373,15 @@ def w4a8_gemm_config(X8, sx, packed, s1, N: int, group: int = 128, *, tok_tile=0
                      int32_out=False, out=None, ws=_AUTO, stream=None):
     """The GEMM with an explicit token tile / split count (0 = auto)."""
     import torch
-    _need_cuda(X8, "X8", torch.int8, 2)
-    M, K = X8.shape
     if int32_out:
-        acc = out if out is not None else torch.empty((M, N), dtype=torch.int32, device=X8.device)
+        M, K = _need_gemm_operands(X8, None, packed, None, N, group)
+        acc = _out(out, (M, N), torch.int32, X8.device)
         Y = None
     else:
-        Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=X8.device)
+        M, K = _need_gemm_operands(X8, sx, packed, s1, N, group)
+        Y = _out(out, (M, N), torch.float16, X8.device)
         acc = None
-    w, wb = _ws_args(_auto_ws(ws, M, N, K, group, X8.device, tok_tile, splits))
+    w, wb = _ws_args(_auto_ws(ws, M, N, K, group, X8.device, tok_tile, splits, stream))
     _check(lib().qoq_w4a8_gemm_config(_ptr(X8), _ptr(sx), _ptr(packed), _ptr(s1), M, N, K, group,
                                       _ptr(Y), _ptr(acc), tok_tile, splits, w, wb,
                                       _stream(stream)), "qoq_w4a8_gemm_config")
@@ -336,13 +395,18 @@ def w4a8_linear(X, packed, s1, N: int, group: int = 128, out=None, scratch=None,
     import torch
     _need_cuda(X, "X", torch.float16, 2)
     M, K = X.shape
+    dev = X.device
+    _need_cuda(s1, "s1", torch.float16, shape=(N,), device=dev)
+    _need_packed(packed, N, K, group, dev)
     if scratch is None:
-        X8 = torch.empty((M, K), dtype=torch.int8, device=X.device)
-        sx = torch.empty(M, dtype=torch.float16, device=X.device)
+        X8 = torch.empty((M, K), dtype=torch.int8, device=dev)
+        sx = torch.empty(M, dtype=torch.float16, device=dev)
     else:
         X8, sx = scratch
-    Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=X.device)
-    w, wb = _ws_args(_auto_ws(ws, M, N, K, group, X.device))
+        _need_cuda(X8, "X8", torch.int8, shape=(M, K), device=dev)
+        _need_cuda(sx, "sx", torch.float16, shape=(M,), device=dev)
+    Y = _out(out, (M, N), torch.float16, dev)
+    w, wb = _ws_args(_auto_ws(ws, M, N, K, group, dev, stream=stream))
     _check(lib().qoq_w4a8_linear(_ptr(X), M, K, _ptr(packed), _ptr(s1), N, group, _ptr(X8),
                                  _ptr(sx), _ptr(Y), w, wb, _stream(stream)), "qoq_w4a8_linear")
     return Y
