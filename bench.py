@@ -26,6 +26,7 @@ import datetime
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -584,14 +585,49 @@ def measure_e2e(qoq, torch, layer, packed, s1, dev, stream, world, steps):
             "d2h_bytes_per_step": sum(M * N * 2 for M in ms), "steps": steps}
 
 
+def _c_code_only(text):
+    """C/C++/CUDA source with its comments removed and every run of white
+    space made one blank: what the compiler sees, so that editing a comment
+    does not count as changing the kernel."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":                       # string or character literal
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return re.sub(r"\s+", " ", "".join(out)).strip()
+
+
+GEMM_SOURCES = ("w4a8_quantized_gemm_02_b200/csrc/qoq_gemm.cu",
+                "w4a8_quantized_gemm_02_b200/csrc/qoq_device.cuh",
+                "w4a8_quantized_gemm_02_b200/csrc/qoq_internal.h",
+                "include/qoq.h")
+
+
 def kernel_source_hash():
-    """Hash of the GEMM kernel's sources: ncu counters taken from another
+    """Hash of the code (comments aside) that builds the GEMM kernel, and of
+    the build script with its compiler flags: ncu counters taken from another
     version of the kernel are not reported."""
     import hashlib
     h = hashlib.sha256()
-    for name in ("qoq_gemm.cu", "qoq_device.cuh"):
-        with open(os.path.join(ROOT, "w4a8_quantized_gemm_02_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            h.update(_c_code_only(f.read()).encode())
+    with open(os.path.join(ROOT, "w4a8_quantized_gemm_02_b200", "build.py"), "rb") as f:
+        h.update(f.read())
     return h.hexdigest()[:16]
 
 

@@ -36,3 +36,16 @@ def test_reference_arm_json_line(monkeypatch):
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+def test_kernel_hash_ignores_comments_only():
+    """The DRAM-traffic figure is reported only for the kernel it was measured
+    on; the hash that decides this sees code, not comments or layout."""
+    src = ('// header "quoted" /* not a block */\n'
+           'const char* s = "a // b /* c */";  /* block\n comment */ int x = \'"\';\n'
+           'int   y  =  1; // trailing\n')
+    code = bench._c_code_only(src)
+    assert code == 'const char* s = "a // b /* c */"; int x = \'"\'; int y = 1;'
+    assert bench._c_code_only(src.replace("trailing", "other words")) == code
+    assert bench._c_code_only(src.replace("y  =  1", "y = 2")) != code
+
