@@ -13,7 +13,8 @@
 // tensor-core tile).  Units are ordered channel-tile major, token tile next,
 // K split innermost, so the CTAs running at the same time share weight blocks
 // through L2 and every weight byte comes from HBM about once.  A pipeline
-// stage covers two k-tiles of 128 (one for TOK = 256).
+// stage covers two k-tiles of 128 for token tiles up to 128, one for the
+// wider tiles (176, 192, 256).
 //   warp 0       X producer: tensor-map copies of the X8 tiles (128-byte
 //                swizzle) into the X ring, refilled when the stage's MMAs
 //                completed;
