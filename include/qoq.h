@@ -166,13 +166,12 @@ QOQ_API int qoq_quantize_act_per_token(const void* X, int M, int K, int8_t* X8,
  *            call that completes leaves its first 16 KiB (arrival counters,
  *            one per 32-channel slice of an output tile; K is split only when
  *            there are at most 1024 output tiles) at zero again, so it can be
- *            reused by later
- *            calls on the same stream whatever their shape.  After a call
- *            that reported a device error (qoq_device_error) it must be
- *            zeroed again.  The rest holds INT32 partial sums.  Calls that
- *            can run at the same time (different streams) need different
- *            workspaces.  With ws == NULL or too small the call still runs,
- *            without splitting K (slower for small M).
+ *            reused by later calls on the same stream whatever their shape.
+ *            After a call that reported a device error (qoq_device_error) it
+ *            must be zeroed again.  The rest holds INT32 partial sums.  Calls
+ *            that can run at the same time (different streams) need
+ *            different workspaces.  With ws == NULL or too small the call
+ *            still runs, without splitting K (slower for small M).
  * The UINT4 codes are dequantized to INT8 inside the main loop
  * (dq = q*s2 - z*s2, four byte lanes per 32-bit operation), multiplied on the
  * INT8 tensor cores (tcgen05, INT32 accumulators in tensor memory), and the
