@@ -195,31 +195,50 @@ def barrier(world: int):
 # ---------------------------------------------------------------------------
 
 def oracle_sample_plan(layer, budget_s: float, oracle, dq_full):
-    """Pick how many output channels of every M the oracle computes so that
-    one pass takes about `budget_s` seconds."""
+    """Choose the bounded sample of one step that the oracle computes in about
+    `budget_s` seconds: the first `rows[j]` token rows of every M (all rows
+    when the budget allows) and the first `n_cols` output channels.  Both
+    costs are measured here: the per-token quantization per element and the
+    integer GEMM per multiply-add."""
     K = layer.K
     cal_M, cal_N = 64, 64
     X = si.activations(layer, cal_M, seed=0)
+    t = time.perf_counter()
     X8, sx = oracle.quant_act(X)
+    t_elem = max(time.perf_counter() - t, 1e-6) / (cal_M * K)       # s per quantized element
     t = time.perf_counter()
     oracle.int_gemm(X8, dq_full[:cal_N])
-    dt = max(time.perf_counter() - t, 1e-4)
-    macs_per_s = cal_M * cal_N * K / dt
+    t_mac = max(time.perf_counter() - t, 1e-6) / (cal_M * cal_N * K)  # s per multiply-add
     total_rows = sum(layer.ms)
-    n_cols = int(budget_s * macs_per_s / (total_rows * K))
-    n_cols = max(8, min(layer.N, (n_cols // 8) * 8))
-    return n_cols
+    # all rows: spend what the quantization leaves on as many channels as fit
+    n_cols = int((budget_s - total_rows * K * t_elem) / (total_rows * K * t_mac))
+    if n_cols >= 64:
+        return list(layer.ms), max(8, min(layer.N, (n_cols // 8) * 8))
+    # else a fraction of the rows of every M, against 64 channels
+    n_cols = min(64, layer.N)
+    per_row = K * t_elem + n_cols * K * t_mac
+    frac = min(1.0, budget_s / (total_rows * per_row))
+    rows = [max(1, min(M, int(round(frac * M)))) for M in layer.ms]
+    return rows, n_cols
 
 
 def run_oracle_pass(layer, oracle, dq, s1, Xs, n_cols):
-    """One bounded pass: per M, full activation quantization, then the GEMM
-    and output scaling for the first n_cols output channels."""
+    """One bounded pass: per M, per-token quantization of the sampled rows of
+    X, then the GEMM and output scaling for the first n_cols channels."""
     ops = 0
     t = time.perf_counter()
-    for M, X in zip(layer.ms, Xs):
+    for X in Xs:
         oracle.w4a8_forward(X, dq[:n_cols], s1[:n_cols])
-        ops += gemm_ops(M, n_cols, layer.K)
+        ops += gemm_ops(X.shape[0], n_cols, layer.K)
     return ops, time.perf_counter() - t
+
+
+def _sample_text(layer, rows, n_cols):
+    full = list(rows) == list(layer.ms)
+    what = ("every row" if full else
+            "the first " + ", ".join(f"{r} of {M}" for r, M in zip(rows, layer.ms)) + " rows")
+    return (f"{layer.name}: M in {list(layer.ms)}, {what} through per-token quantization, "
+            f"INT32 GEMM and FP16 scaling for the first {n_cols} of {layer.N} output channels")
 
 
 def cpu_baseline(layer, budget_s: float):
@@ -227,14 +246,16 @@ def cpu_baseline(layer, budget_s: float):
     W = si.weights(layer, seed=0)
     ref = oracle.quantize_weights(W, layer.group)
     del W
-    n_cols = oracle_sample_plan(layer, budget_s, oracle, ref["dq"])
-    Xs = [si.activations(layer, M, seed=0) for M in layer.ms]
+    rows, n_cols = oracle_sample_plan(layer, budget_s, oracle, ref["dq"])
+    Xs = [si.activations(layer, M, seed=0)[:r] for M, r in zip(layer.ms, rows)]
     ops, dt = run_oracle_pass(layer, oracle, ref["dq"], ref["s1"], Xs, n_cols)
     return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": oracle.num_threads(),
-            "kind": "oracle",
-            "sample": (f"{layer.name}: every M in {list(layer.ms)}, full per-token "
-                       f"quantization of X, INT32 GEMM + FP16 scaling for the first "
-                       f"{n_cols} of {layer.N} output channels ({dt:.1f} s)")}
+            "kind": "oracle", "sample": f"{_sample_text(layer, rows, n_cols)} ({dt:.1f} s)"}
+
+
+# The reference arm's whole run (warm-up and timed steps) is held to about
+# this many seconds of host time, whatever --steps and --warmup are.
+REFERENCE_RUN_S = 150.0
 
 
 def run_reference(args):
@@ -247,9 +268,9 @@ def run_reference(args):
     ref = oracle.quantize_weights(W, layer.group)
     del W
     total = args.steps + args.warmup
-    per_step = max(0.05, min(args.cpu_budget_s, 150.0 / max(total, 1)))
-    n_cols = oracle_sample_plan(layer, per_step, oracle, ref["dq"])
-    Xs = [si.activations(layer, M, seed=0) for M in layer.ms]
+    per_step = max(0.01, min(args.cpu_budget_s, REFERENCE_RUN_S / max(total, 1)))
+    rows, n_cols = oracle_sample_plan(layer, per_step, oracle, ref["dq"])
+    Xs = [si.activations(layer, M, seed=0)[:r] for M, r in zip(layer.ms, rows)]
     for _ in range(args.warmup):
         run_oracle_pass(layer, oracle, ref["dq"], ref["s1"], Xs, n_cols)
     ops_total, t_total = 0, 0.0
@@ -258,9 +279,7 @@ def run_reference(args):
         ops_total += ops
         t_total += dt
     value = ops_total / t_total / 1e12
-    sample = (f"{layer.name}: per step every M in {list(layer.ms)}, full per-token "
-              f"quantization of X, INT32 GEMM + FP16 scaling for the first {n_cols} of "
-              f"{layer.N} output channels")
+    sample = "per step " + _sample_text(layer, rows, n_cols)
     line = {"metric": METRIC, "value": value, "unit": "TOPS", "impl": "reference",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * t_total / max(args.steps, 1), "higher_is_better": True,

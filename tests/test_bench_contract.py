@@ -49,3 +49,21 @@ def test_kernel_hash_ignores_comments_only():
     assert bench._c_code_only(src.replace("trailing", "other words")) == code
     assert bench._c_code_only(src.replace("y  =  1", "y = 2")) != code
 
+
+
+def test_reference_step_sample_is_bounded():
+    """With the default 2000 timed steps the reference arm has about 75 ms of
+    host time per step: its sample must shrink to that (rows of every M,
+    against 64 channels) instead of quantizing every row of X each step."""
+    import oracle
+    import synthetic_inputs as si
+    layer = si.LAYERS["llama3_8b_qkv"]
+    ref = oracle.quantize_weights(si.weights(layer, 0), layer.group)
+    budget = bench.REFERENCE_RUN_S / 2020
+    rows, n_cols = bench.oracle_sample_plan(layer, budget, oracle, ref["dq"])
+    assert n_cols == 64 and sum(rows) < sum(layer.ms) // 4
+    assert all(1 <= r <= M for r, M in zip(rows, layer.ms))
+    Xs = [si.activations(layer, M, seed=0)[:r] for M, r in zip(layer.ms, rows)]
+    ops, dt = bench.run_oracle_pass(layer, oracle, ref["dq"], ref["s1"], Xs, n_cols)
+    assert ops == sum(2 * r * n_cols * layer.K for r in rows)
+    assert dt < 5 * budget + 0.2
