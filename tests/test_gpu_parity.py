@@ -302,7 +302,8 @@ def test_gemm_shapes_random_codes(oracle, group, M, N, K):
 
 
 def test_gemm_extreme_values(oracle):
-    """Largest |dq| and |X8|: accumulators near the INT32 edge stay exact."""
+    """Large |dq| (120) and the largest |X8| (127) in every term, over K = 8192:
+    accumulators of about +-1.25e8 stay exact on every token tile and split."""
     N, K, group = 128, 8192, 128
     q = np.zeros((N, K), np.uint8)
     q[::2] = 15
