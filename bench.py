@@ -59,6 +59,10 @@ def parse_args(argv=None):
     p.add_argument("--profile-gemm", type=int, default=0, metavar="M",
                    help="only launch the GEMM for this M a few times (for ncu)")
     p.add_argument("--profile-launches", type=int, default=3)
+    p.add_argument("--no-layers", action="store_true",
+                   help="skip the per-M timing of the other layer workloads")
+    p.add_argument("--no-sweep", action="store_true",
+                   help="skip the K = N shape sweep")
     return p.parse_args(argv)
 
 
@@ -317,6 +321,185 @@ def run_profile(args, qoq, torch):
     return 0
 
 
+def graph_us_per_launch(torch, stream, fn, reps=3):
+    """Device time per launch of `fn`'s launches, captured back to back in one
+    CUDA graph and replayed `reps` times (after one untimed replay)."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        nlaunch = fn()
+    g.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    e1.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e3 / (reps * nlaunch)
+
+
+def copies_for(nbytes, l2, lo=4, hi=256):
+    """How many rotated copies of an input of `nbytes` make every launch read
+    memory that was last touched more than 3 L2 capacities earlier."""
+    return int(min(hi, max(lo, math.ceil(3 * l2 / max(nbytes, 1)) + 1)))
+
+
+def per_m_entry(M, N, K, G, t_us, peaks, int8_peak, plan, extra=None):
+    t = t_us * 1e-6
+    d = {"M": M, "gemm_us": t_us, "tops": gemm_ops(M, N, K) / t / 1e12,
+         "weight_gbs": weight_bytes(N, K, G) / t / 1e9,
+         "hbm_frac": algo_bytes(M, N, K, G) / t / 1e9 / peaks["hbm_gbs"],
+         "int8_frac": gemm_ops(M, N, K) / t / 1e12 / int8_peak,
+         "tok_tile": plan["tok_tile"], "splits": plan["splits"], "ctas": plan["ctas"]}
+    if extra:
+        d.update(extra)
+    return d
+
+
+def layer_per_m(qoq, torch, layer, dev, stream, l2, peaks, int8_peak, packed0=None, s1_0=None,
+                isolated=False):
+    """Each kernel of one layer alone, per M: the quantizer, the GEMM and the
+    fused linear, as back-to-back launches in a CUDA graph over rotated
+    inputs.  With `isolated`, also one GEMM launch at a time after an L2
+    flush (median of 5)."""
+    N, K, G = layer.N, layer.K, layer.group
+    if packed0 is None:
+        W = torch.from_numpy(si.weights(layer, seed=0)).to(dev)
+        packed0, s1_0 = qoq.quantize_weights(W, G, stream=stream)
+        stream.synchronize()
+        del W
+    nw = copies_for(packed0.numel(), l2, hi=64)
+    weights = [packed0] + [packed0.clone() for _ in range(nw - 1)]
+    s1s = [s1_0] + [s1_0.clone() for _ in range(nw - 1)]
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev) if isolated else None
+    out = []
+    for M in layer.ms:
+        nx = copies_for(M * K * 2, l2, lo=2, hi=nw)
+        xs = [torch.from_numpy(si.activations(layer, M, seed=s)).to(dev) for s in range(nx)]
+        x8 = torch.empty((M, K), dtype=torch.int8, device=dev)
+        sx = torch.empty(M, dtype=torch.float16, device=dev)
+        y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        with torch.cuda.stream(stream):
+            qoq.quantize_act_per_token(xs[0], out=(x8, sx), stream=stream)
+            qoq.w4a8_gemm(x8, sx, weights[0], s1s[0], N, G, out=y, stream=stream)
+        stream.synchronize()
+
+        def aq():
+            for x in xs:
+                qoq.quantize_act_per_token(x, out=(x8, sx), stream=stream)
+            return len(xs)
+
+        def gm():
+            for w in range(nw):
+                qoq.w4a8_gemm(x8, sx, weights[w], s1s[w], N, G, out=y, stream=stream)
+            return nw
+
+        def ln():
+            for w in range(nw):
+                qoq.w4a8_linear(xs[w % nx], weights[w], s1s[w], N, G, out=y, scratch=(x8, sx),
+                                stream=stream)
+            return nw
+        aq_us = graph_us_per_launch(torch, stream, aq)
+        gemm_us = graph_us_per_launch(torch, stream, gm)
+        lin_us = graph_us_per_launch(torch, stream, ln)
+        extra = {"act_quant_us": aq_us, "linear_us": lin_us,
+                 "linear_tops": gemm_ops(M, N, K) / lin_us / 1e6}
+        if isolated:
+            times = []
+            for i in range(5):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    flush.fill_(i)
+                    e0.record(stream)
+                    qoq.w4a8_gemm(x8, sx, weights[i % nw], s1s[i % nw], N, G, out=y,
+                                  stream=stream)
+                    e1.record(stream)
+                e1.synchronize()
+                times.append(e0.elapsed_time(e1) * 1e3)
+            extra["gemm_isolated_us"] = statistics.median(times)
+        out.append(per_m_entry(M, N, K, G, gemm_us, peaks, int8_peak,
+                               qoq.gemm_plan(M, N, K, G), extra))
+        del xs
+    del weights, s1s, flush
+    torch.cuda.synchronize()
+    return out
+
+
+def sweep_per_m(qoq, torch, dev, stream, l2, peaks, int8_peak):
+    """The pure-throughput shape sweep: K = N in {2048, 4096, 8192}, group 64
+    and 128, M = 1 .. 8192 in powers of two; random UINT4 codes, zeros and
+    group scales packed once per shape (host draws), INT8 activations drawn
+    on the device from a seeded generator; GEMM alone, back to back in a
+    CUDA graph over rotated weights."""
+    res = {}
+    gen = torch.Generator(device=dev)
+    for kn in si.SWEEP_KN:
+        for G in si.SWEEP_GROUPS:
+            N = K = kn
+            ops = si.sweep_operands(1, N, K, G, seed=kn + G)
+            packed0 = qoq.pack_codes(torch.from_numpy(ops.q).to(dev),
+                                     torch.from_numpy(ops.s2).to(dev),
+                                     torch.from_numpy(ops.z).to(dev), G, stream=stream)
+            s1_0 = torch.from_numpy(ops.s1).to(dev)
+            stream.synchronize()
+            nw = copies_for(packed0.numel(), l2, hi=128)
+            weights = [packed0] + [packed0.clone() for _ in range(nw - 1)]
+            row = {"M": [], "us": [], "tops": [], "hbm_frac": [], "int8_frac": [],
+                   "tok_tile": [], "splits": []}
+            for M in si.SWEEP_MS:
+                gen.manual_seed(M)
+                x8 = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev,
+                                   generator=gen)
+                sx = (torch.rand(M, device=dev, generator=gen) * 1e-3 + 0.5e-3).half()
+                y = torch.empty((M, N), dtype=torch.float16, device=dev)
+                with torch.cuda.stream(stream):
+                    qoq.w4a8_gemm(x8, sx, weights[0], s1_0, N, G, out=y, stream=stream)
+                stream.synchronize()
+
+                def gm():
+                    for w in range(nw):
+                        qoq.w4a8_gemm(x8, sx, weights[w], s1_0, N, G, out=y, stream=stream)
+                    return nw
+                us = graph_us_per_launch(torch, stream, gm)
+                e = per_m_entry(M, N, K, G, us, peaks, int8_peak, qoq.gemm_plan(M, N, K, G))
+                for k in ("M", "tops", "hbm_frac", "int8_frac", "tok_tile", "splits"):
+                    row[k].append(round(e[k], 4) if isinstance(e[k], float) else e[k])
+                row["us"].append(round(us, 3))
+                del x8, sx, y
+            res[f"K=N={kn},G={G}"] = row
+            del weights
+            torch.cuda.synchronize()
+    return res
+
+
+def cublas_int8_tops(torch, dev, n=8192, reps=10):
+    """Dense INT8 throughput of cuBLAS (torch._int_mm) at n^3, best of `reps`
+    single launches: a measured reference beside the nominal INT8 peak."""
+    try:
+        a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev)
+        b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev)
+        for _ in range(3):
+            torch._int_mm(a, b)
+        torch.cuda.synchronize()
+        best = 1e30
+        for _ in range(reps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._int_mm(a, b)
+            e1.record()
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        del a, b
+        return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+    except Exception:
+        return None
+
+
 def run_ours(args):
     import torch
     import w4a8_quantized_gemm_02_b200 as qoq
@@ -448,67 +631,31 @@ def run_ours(args):
     dom_ms = [graph_events[(args.steps - 1 - g) % ngraphs][0].elapsed_time(
         graph_events[(args.steps - 1 - g) % ngraphs][1]) for g in range(n_used)]
 
-    # per-kernel breakdown (after the timed region): each kernel alone, R
-    # back-to-back launches in one graph over the rotated inputs
-    def per_launch_us(fn, reps=3):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            nlaunch = fn()
-        g.replay()
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(reps):
-                g.replay()
-            e1.record(stream)
-        e1.synchronize()
-        del g
-        return e0.elapsed_time(e1) * 1e3 / (reps * nlaunch)
-
-    nw = len(weights)
-    aq_us, gemm_us, lin_us = {}, {}, {}
-    for j, M in enumerate(ms):
-        def aq():
-            for s_ in range(nsets):
-                qoq.quantize_act_per_token(xs[s_][j], out=(x8[j], sxb[j]), stream=stream)
-            return nsets
-
-        def gm():
-            for w in range(nw):
-                qoq.w4a8_gemm(x8[j], sxb[j], weights[w], s1s[w], N, G, out=ys[j], stream=stream)
-            return nw
-
-        def ln():
-            for w in range(nw):
-                qoq.w4a8_linear(xs[w % nsets][j], weights[w], s1s[w], N, G, out=ys[j],
-                                scratch=(x8[j], sxb[j]), stream=stream)
-            return nw
-        aq_us[M] = per_launch_us(aq)
-        gemm_us[M] = per_launch_us(gm)
-        lin_us[M] = per_launch_us(ln)
-    assert qoq.device_error(clear=True) == 0
-
     peaks = load_peaks()
     int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    int8_cublas = cublas_int8_tops(torch, dev)
+    if int8_cublas is not None and int8_cublas > int8_peak:
+        int8_peak = int8_cublas
     step_ops = sum(gemm_ops(M, N, K) for M in ms)
     value = step_ops * args.steps * world / (elapsed_ms * 1e-3) / 1e12
-    per_m = []
-    for M in ms:
-        t = gemm_us[M] * 1e-6
-        ta = aq_us[M] * 1e-6
-        tl = lin_us[M] * 1e-6
-        plan = qoq.gemm_plan(M, N, K, G)
-        per_m.append({
-            "M": M, "gemm_us": t * 1e6, "act_quant_us": ta * 1e6, "linear_us": tl * 1e6,
-            "tops": gemm_ops(M, N, K) / t / 1e12,
-            "weight_gbs": weight_bytes(N, K, G) / t / 1e9,
-            "hbm_frac": algo_bytes(M, N, K, G) / t / 1e9 / peaks["hbm_gbs"],
-            "int8_frac": gemm_ops(M, N, K) / t / 1e12 / int8_peak,
-            "linear_tops": gemm_ops(M, N, K) / tl / 1e12,
-            "tok_tile": plan["tok_tile"], "splits": plan["splits"], "ctas": plan["ctas"],
-        })
+    del graphs, graph_events, weights, s1s, xs
+    torch.cuda.synchronize()
+
+    # per-kernel breakdown (after the timed region): each kernel alone,
+    # back-to-back launches in a CUDA graph over rotated inputs
+    per_m = layer_per_m(qoq, torch, layer, dev, stream, l2, peaks, int8_peak, packed0, s1_0,
+                        isolated=True)
+    layers = {}
+    if not args.no_layers and world == 1:
+        for name, other in si.LAYERS.items():
+            if name in (layer.name, si.TINY.name):
+                continue
+            layers[name] = layer_per_m(qoq, torch, other, dev, stream, l2, peaks, int8_peak)
+    sweep = None
+    if not args.no_sweep and world == 1:
+        sweep = sweep_per_m(qoq, torch, dev, stream, l2, peaks, int8_peak)
+    assert qoq.device_error(clear=True) == 0
+
     td = statistics.mean(dom_ms) * 1e-3
     Md = m_dom
     hbm_frac_d = algo_bytes(Md, N, K, G) / td / 1e9 / peaks["hbm_gbs"]
@@ -520,11 +667,18 @@ def run_ours(args):
     else:
         roofline = {"bound": "hbm", "achieved": algo_bytes(Md, N, K, G) / td / 1e9,
                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": hbm_frac_d}
+    nominal = peaks["bf16_tflops"] * INT8_OVER_BF16
     roofline.update({"traffic": None, "kernel": f"w4a8_gemm M={Md}",
                      "launch_us": td * 1e6, "launches_averaged": n_used,
-                     "peak_source": (f"{peaks['source']} bf16 burst x {INT8_OVER_BF16:g} "
-                                     f"(nominal int8:bf16), of measured" if tensor_bound
-                                     else f"{peaks['source']} hbm copy, of measured")})
+                     "peak_source": (f"max({peaks['source']} bf16 burst x {INT8_OVER_BF16:g} "
+                                     f"(nominal int8:bf16) = {nominal:.0f}, cuBLAS int8 "
+                                     f"8192^3 measured in this run = "
+                                     f"{int8_cublas if int8_cublas else float('nan'):.0f}), "
+                                     f"of measured" if tensor_bound
+                                     else f"{peaks['source']} hbm copy, of measured"),
+                     "int8_cublas_tops": int8_cublas,
+                     "frac_of_cublas_int8": (gemm_ops(Md, N, K) / td / 1e12 / int8_cublas
+                                             if int8_cublas else None)})
     traffic = load_traffic(layer.name, Md)
     if traffic is not None:
         roofline["traffic"] = traffic
@@ -532,8 +686,8 @@ def run_ours(args):
     # end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = measure_e2e(qoq, torch, layer, packed0, s1_0, dev, stream, world,
-                          steps=max(3, min(20, args.steps // 100 + 3)))
+        e2e = measure_e2e(qoq, torch, layer, packed0, s1_0, dev, world,
+                          steps=max(20, min(100, args.steps // 20)))
 
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
@@ -546,11 +700,14 @@ def run_ours(args):
                           f"MiB, > 3x L2 {l2 / 2**20:.0f} MiB); one CUDA graph per step")},
         "roofline": roofline,
         "per_m": per_m,
+        "layers": layers,
+        "sweep": sweep,
         "clocks": clocks,
         "gpu_launches": 2 * len(ms) * args.steps,
         "timed_region": "fused qoq_w4a8_linear per M (dominant M: quantizer + qoq_w4a8_gemm)",
         "per_m_method": "each kernel alone: back-to-back launches in a CUDA graph over rotated "
-                        "inputs, device time / launches",
+                        "inputs, device time / launches; gemm_isolated_us: one launch between "
+                        "events after an L2 flush, median of 5",
         "offline_pack_ms": pack_ms,
         "e2e": e2e,
     }
@@ -558,50 +715,103 @@ def run_ours(args):
         line["cpu_baseline"] = cpu_baseline(layer, args.cpu_budget_s)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graphs
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
 
 
-def measure_e2e(qoq, torch, layer, packed, s1, dev, stream, world, steps):
+def measure_e2e(qoq, torch, layer, packed, s1, dev, world, steps):
     """The same step through the public API from pinned host memory: per M,
-    copy X host->device, quantize + GEMM, copy Y device->host."""
+    copy X host->device, quantize + GEMM (qoq_w4a8_linear), copy Y
+    device->host.  Three streams (copy in, compute, copy out) with events per
+    M and two device buffer sets, so the copies of one M overlap the compute
+    of its neighbours and PCIe carries both directions at once.  Returns the
+    throughput and the bytes moved per step, plus the measured link rates."""
     ms = list(layer.ms)
     N, K, G = layer.N, layer.K, layer.group
+    nb = 2
     hx = [torch.from_numpy(si.activations(layer, M, seed=7)).pin_memory() for M in ms]
-    hy = [torch.empty((M, N), dtype=torch.float16).pin_memory() for M in ms]
-    dx = [torch.empty((M, K), dtype=torch.float16, device=dev) for M in ms]
-    x8 = [torch.empty((M, K), dtype=torch.int8, device=dev) for M in ms]
-    sxb = [torch.empty(M, dtype=torch.float16, device=dev) for M in ms]
-    dy = [torch.empty((M, N), dtype=torch.float16, device=dev) for M in ms]
+    hy = [[torch.empty((M, N), dtype=torch.float16).pin_memory() for M in ms] for _ in range(nb)]
+    dx = [[torch.empty((M, K), dtype=torch.float16, device=dev) for M in ms] for _ in range(nb)]
+    x8 = [[torch.empty((M, K), dtype=torch.int8, device=dev) for M in ms] for _ in range(nb)]
+    sxb = [[torch.empty(M, dtype=torch.float16, device=dev) for M in ms] for _ in range(nb)]
+    dy = [[torch.empty((M, N), dtype=torch.float16, device=dev) for M in ms] for _ in range(nb)]
+    s_in = torch.cuda.Stream(device=dev)
+    s_comp = torch.cuda.Stream(device=dev)
+    s_out = torch.cuda.Stream(device=dev)
+    nm = len(ms)
+    # events of the last use of every buffer, per set and M
+    comp_done = [[None] * nm for _ in range(nb)]
+    out_done = [[None] * nm for _ in range(nb)]
 
-    def one():
-        for j in range(len(ms)):
-            dx[j].copy_(hx[j], non_blocking=True)
-            qoq.w4a8_linear(dx[j], packed, s1, N, G, out=dy[j], scratch=(x8[j], sxb[j]),
-                            stream=stream)
-            hy[j].copy_(dy[j], non_blocking=True)
+    def one(step):
+        b = step % nb
+        for j in range(nm):
+            with torch.cuda.stream(s_in):
+                if comp_done[b][j] is not None:
+                    s_in.wait_event(comp_done[b][j])       # dx[b][j] no longer read
+                dx[b][j].copy_(hx[j], non_blocking=True)
+                e_in = torch.cuda.Event()
+                e_in.record(s_in)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(e_in)
+                if out_done[b][j] is not None:
+                    s_comp.wait_event(out_done[b][j])      # dy[b][j] copied out
+                qoq.w4a8_linear(dx[b][j], packed, s1, N, G, out=dy[b][j],
+                                scratch=(x8[b][j], sxb[b][j]), stream=s_comp)
+                e_c = torch.cuda.Event()
+                e_c.record(s_comp)
+                comp_done[b][j] = e_c
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(e_c)
+                hy[b][j].copy_(dy[b][j], non_blocking=True)
+                e_o = torch.cuda.Event()
+                e_o.record(s_out)
+                out_done[b][j] = e_o
 
-    with torch.cuda.stream(stream):
-        one()
-    stream.synchronize()
+    one(0)
+    one(1)
+    torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        start.record(stream)
-        for _ in range(steps):
-            one()
-        end.record(stream)
+    start.record(s_in)
+    s_comp.wait_event(start)
+    s_out.wait_event(start)
+    for i in range(steps):
+        one(i)
+    e_last_c = torch.cuda.Event()
+    e_last_c.record(s_comp)
+    e_last_i = torch.cuda.Event()
+    e_last_i.record(s_in)
+    s_out.wait_event(e_last_c)
+    s_out.wait_event(e_last_i)
+    end.record(s_out)
     end.synchronize()
     ms_total = max_over_ranks(start.elapsed_time(end), world, dev)
     ops = sum(gemm_ops(M, N, K) for M in ms) * steps * world
+    h2d = sum(M * K * 2 for M in ms)
+    d2h = sum(M * N * 2 for M in ms)
+
+    def link_gbs(src, dst, s):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s):
+            dst.copy_(src, non_blocking=True)
+            e0.record(s)
+            for _ in range(5):
+                dst.copy_(src, non_blocking=True)
+            e1.record(s)
+        e1.synchronize()
+        return 5 * src.numel() * src.element_size() / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    big = max(range(nm), key=lambda j: ms[j])
     return {"value": ops / (ms_total * 1e-3) / 1e12, "unit": "TOPS",
-            "h2d_bytes_per_step": sum(M * K * 2 for M in ms),
-            "d2h_bytes_per_step": sum(M * N * 2 for M in ms), "steps": steps}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "method": "3 streams (H2D, compute, D2H), events per M, 2 buffer sets",
+            "link_h2d_gbs": link_gbs(hx[big], dx[0][big], s_in),
+            "link_d2h_gbs": link_gbs(dy[0][big], hy[0][big], s_out)}
 
 
 def _c_code_only(text):

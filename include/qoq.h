@@ -27,9 +27,9 @@
  *    compute entry point only enqueues work on `stream` and returns without
  *    synchronizing, except the ones marked "synchronous".
  *  - Arguments are validated before anything is launched.  A violated
- *    precondition returns QOQ_ERR_INVALID_ARG or QOQ_ERR_UNSUPPORTED and
- *    launches nothing.  A CUDA launch or driver error returns QOQ_ERR_CUDA.
- *    No exception or abort crosses the ABI.
+ *    precondition returns QOQ_ERR_INVALID_ARG, QOQ_ERR_UNSUPPORTED or
+ *    QOQ_ERR_WORKSPACE and launches nothing.  A CUDA launch or driver error
+ *    returns QOQ_ERR_CUDA.  No exception or abort crosses the ABI.
  *  - FP16 arrays hold IEEE binary16 values (`__half` / `torch.float16`).
  *    Inputs must be finite; this is not checked on the device.
  *  - Every device pointer must be 16-byte aligned.
@@ -60,6 +60,7 @@ enum {
   QOQ_ERR_INVALID_ARG = 1,  /* bad pointer, shape or alignment */
   QOQ_ERR_UNSUPPORTED = 2,  /* valid but not supported (device, group, size) */
   QOQ_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+  QOQ_ERR_WORKSPACE = 4,    /* the split-K workspace given is too small */
 };
 
 /* Human-readable text for a status code (static storage, never NULL). */
@@ -92,11 +93,14 @@ QOQ_API int qoq_protective_range(void);
  * ---------------------------------------------------------------------- */
 
 /* Bytes of one (128 x 128) block: 8192 + 192 for group 128, 8192 + 384 for
- * group 64.  Returns 0 for an unsupported group. */
+ * group 64.  Returns 0 for an unsupported group.  The block holds the
+ * level-2 result of Methods, 1) Algorithm: QoQ (UINT4 codes, INT8 group
+ * scales, UINT4 zeros per group of input channels). */
 QOQ_API size_t qoq_packed_block_bytes(int group);
 
 /* Bytes of the whole packed buffer for an N x K weight (0 if the shape is
- * invalid). */
+ * invalid): N*K/2 bytes of UINT4 codes plus 1.5 bytes per group (s2, z),
+ * the W4 storage of Methods, 1) Algorithm: QoQ. */
 QOQ_API size_t qoq_packed_weight_bytes(int N, int K, int group);
 
 /* ------------------------------------------------------------------------
@@ -132,6 +136,9 @@ QOQ_API int qoq_pack_codes(const uint8_t* q, const int8_t* s2, const uint8_t* z,
  * NULL to skip it.  q: uint8 N x K; s2: int8 N x (K/group);
  * z: uint8 N x (K/group); dq: int8 N x K with dq = q*s2 - z*s2, computed
  * with the same byte-lane arithmetic as the GEMM main loop.
+ * Source: Methods, 1) Algorithm: QoQ (the level-2 codes, scales and zeros)
+ * and 2) System: QServe (dequantization to INT8, the zero subtracted after
+ * the scale multiply).  q and dq must be 16-byte aligned.
  * Asynchronous on `stream`. */
 QOQ_API int qoq_unpack_weights(const void* packed, int N, int K, int group,
                        uint8_t* q, int8_t* s2, uint8_t* z, int8_t* dq,
@@ -170,8 +177,10 @@ QOQ_API int qoq_quantize_act_per_token(const void* X, int M, int K, int8_t* X8,
  *            After a call that reported a device error (qoq_device_error) it
  *            must be zeroed again.  The rest holds INT32 partial sums.  Calls
  *            that can run at the same time (different streams) need
- *            different workspaces.  With ws == NULL or too small the call
- *            still runs, without splitting K (slower for small M).
+ *            different workspaces.  ws == NULL (with any ws_bytes) is an
+ *            explicit request not to split K: the call runs unsplit (slower
+ *            for small M).  A non-NULL ws smaller than the plan needs
+ *            returns QOQ_ERR_WORKSPACE and launches nothing.
  * The UINT4 codes are dequantized to INT8 inside the main loop
  * (dq = q*s2 - z*s2, four byte lanes per 32-bit operation), multiplied on the
  * INT8 tensor cores (tcgen05, INT32 accumulators in tensor memory), and the
@@ -220,16 +229,26 @@ QOQ_API int qoq_w4a8_gemm_static_ws(const int8_t* X8, const void* sx, const void
                                     void* Y, void* stream);
 
 /* Workspace bytes qoq_w4a8_gemm, qoq_w4a8_gemm_i32 and qoq_w4a8_linear use
- * for this shape (0 if K is not split, or if the shape is invalid). */
+ * for this shape (0 if K is not split, or if the shape is invalid): 16 KiB
+ * of arrival counters plus the INT32 partial sums of the K splits.  Partial
+ * sums stay INT32 and are added exactly before the single FP16 scaling
+ * (Background: no dequantization of partial sums; Methods, 1) Algorithm:
+ * QoQ, INT32 accumulation on INT8 tensor cores). */
 QOQ_API size_t qoq_gemm_workspace_bytes(int M, int N, int K, int group);
 
 /* Workspace bytes for an explicit configuration of qoq_w4a8_gemm_config
- * (tok_tile / splits as there, 0 = auto). */
+ * (tok_tile / splits as there, 0 = auto).  Same layout and source as
+ * qoq_gemm_workspace_bytes. */
 QOQ_API size_t qoq_gemm_workspace_bytes_config(int M, int N, int K, int group,
                                                int tok_tile, int splits);
 
 /* Debug: the same main loop, storing the raw INT32 accumulator
- * acc[m, n] = sum_k X8[m,k] * dq[n,k] (device, int32 M x N row-major). */
+ * acc[m, n] = sum_k X8[m,k] * dq[n,k] (device, int32 M x N row-major,
+ * 16-byte aligned) instead of the scaled FP16 output.  This is the INT8 x
+ * INT8 -> INT32 product of Methods, 1) Algorithm: QoQ (every GEMM on INT8
+ * tensor cores) over the dequantized weights of 2) System: QServe, before
+ * the per-token x per-channel scaling.  ws / ws_bytes and the errors as for
+ * qoq_w4a8_gemm.  Asynchronous on `stream`. */
 QOQ_API int qoq_w4a8_gemm_i32(const int8_t* X8, const void* packed, int M, int N,
                               int K, int group, int32_t* acc, void* ws,
                               size_t ws_bytes, void* stream);
@@ -238,8 +257,9 @@ QOQ_API int qoq_w4a8_gemm_i32(const int8_t* X8, const void* packed, int M, int N
  *   tok_tile : token tile (MMA N): 16, 32, 64, 128 or 256, or 0 for auto;
  *   splits   : K splits per output tile, 1..8 (at most K/128), or 0 for auto.
  * Exactly one of Y (FP16 output, needs sx and s1) and acc (INT32 output) is
- * non-NULL.  An explicit split count needs its workspace
- * (qoq_gemm_workspace_bytes_config), else QOQ_ERR_INVALID_ARG.
+ * non-NULL.  An explicit split count > 1 needs its workspace
+ * (qoq_gemm_workspace_bytes_config), else QOQ_ERR_WORKSPACE (also for
+ * ws == NULL).
  * Asynchronous on `stream`. */
 QOQ_API int qoq_w4a8_gemm_config(const int8_t* X8, const void* sx, const void* packed,
                                  const void* s1, int M, int N, int K, int group,
@@ -268,7 +288,9 @@ QOQ_API int qoq_w4a8_linear(const void* X, int M, int K, const void* packed, con
 
 /* The launch configuration qoq_w4a8_gemm picks for a shape: token tile,
  * K splits, CTAs in the grid and pipeline stages.  Host only, no CUDA call
- * beyond reading the SM count of the current device (148 if none). */
+ * beyond reading the SM count of the current device (148 if none).  The
+ * pages fix no tiling; this reports the library's own choice for the GEMM of
+ * Methods, 1) Algorithm: QoQ. */
 QOQ_API int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int* splits,
                   int* ctas, int* stages);
 

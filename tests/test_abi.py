@@ -45,8 +45,9 @@ def test_sizes(L):
     assert qoq.packed_weight_bytes(512, 200, 128) == 0
     assert L.qoq_protective_range() == 119
     assert L.qoq_version() >= 1
-    for s in (0, 1, 2, 3, 99):
+    for s in (0, 1, 2, 3, 4, 99):
         assert qoq.status_str(s)
+    assert "workspace" in qoq.status_str(qoq.QOQ_ERR_WORKSPACE)
 
 
 def test_plan_is_host_only(L):
@@ -101,8 +102,50 @@ def test_gemm_argument_validation(L):
     # an explicit split needs its workspace
     need = qoq.gemm_workspace_bytes(16, 512, 512, 128, 16, 2)
     assert need > 0
-    assert c(None, FAKE, 16, 2) == qoq.QOQ_ERR_INVALID_ARG
-    assert c(None, FAKE, 16, 2, FAKE, need - 16) == qoq.QOQ_ERR_INVALID_ARG
+    assert c(None, FAKE, 16, 2) == qoq.QOQ_ERR_WORKSPACE
+    assert c(None, FAKE, 16, 2, FAKE, need - 16) == qoq.QOQ_ERR_WORKSPACE
+
+
+def test_auto_plan_workspace_status(L):
+    """The automatic plan splits K for a decode shape; a workspace that is
+    given but too small is refused before any CUDA call (on a machine without
+    a GPU every CUDA call fails, so QOQ_ERR_WORKSPACE here proves that no call
+    was made), while ws == NULL asks for an unsplit launch."""
+    M, N, K = 1, 6144, 4096
+    assert qoq.gemm_plan(M, N, K, 128)["splits"] > 1
+    need = qoq.gemm_workspace_bytes(M, N, K, 128)
+    assert _gemm(L, M=M, N=N, K=K, ws=FAKE, wsb=need - 16) == qoq.QOQ_ERR_WORKSPACE
+    assert _gemm(L, M=M, N=N, K=K, ws=FAKE, wsb=0) == qoq.QOQ_ERR_WORKSPACE
+    i32 = L.qoq_w4a8_gemm_i32(P(FAKE), P(FAKE), M, N, K, 128, P(FAKE), P(FAKE), need - 16, None)
+    assert i32 == qoq.QOQ_ERR_WORKSPACE
+    lin = L.qoq_w4a8_linear(P(FAKE), M, K, P(FAKE), P(FAKE), N, 128, P(FAKE), P(FAKE), P(FAKE),
+                            P(FAKE), need - 16, None)
+    assert lin == qoq.QOQ_ERR_WORKSPACE     # refused before the quantizer is launched
+    if not _has_gpu():
+        assert _gemm(L, M=M, N=N, K=K, ws=None, wsb=0) == qoq.QOQ_ERR_CUDA
+        assert _gemm(L, M=M, N=N, K=K, ws=FAKE, wsb=need) == qoq.QOQ_ERR_CUDA
+
+
+def _static(L, X8=FAKE, sx=FAKE, packed=FAKE, s1=FAKE, M=1, N=6144, K=4096, G=128, Y=FAKE):
+    return L.qoq_w4a8_gemm_static_ws(P(X8), P(sx), P(packed), P(s1), M, N, K, G, P(Y), None)
+
+
+def test_static_ws_validates_before_any_cuda_call(L):
+    """The no-allocation entry checks every pointer and size before it touches
+    CUDA (before looking up its array or clearing counters on the stream):
+    on a machine without a GPU a rejected call reports the argument error,
+    not a CUDA error."""
+    assert _static(L, X8=FAKE + 8) == qoq.QOQ_ERR_INVALID_ARG
+    assert _static(L, sx=FAKE + 2) == qoq.QOQ_ERR_INVALID_ARG
+    assert _static(L, packed=FAKE + 4) == qoq.QOQ_ERR_INVALID_ARG
+    assert _static(L, s1=FAKE + 2) == qoq.QOQ_ERR_INVALID_ARG
+    assert _static(L, Y=FAKE + 2) == qoq.QOQ_ERR_INVALID_ARG
+    assert _static(L, Y=None) == qoq.QOQ_ERR_INVALID_ARG
+    assert _static(L, M=0) == qoq.QOQ_ERR_INVALID_ARG
+    assert _static(L, N=100) == qoq.QOQ_ERR_INVALID_ARG
+    assert _static(L, G=32) == qoq.QOQ_ERR_UNSUPPORTED
+    if not _has_gpu():
+        assert _static(L) == qoq.QOQ_ERR_CUDA
 
 
 def test_other_entry_validation(L):

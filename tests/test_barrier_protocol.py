@@ -53,21 +53,31 @@ class Bar:
 
 
 class KernelModel:
-    def __init__(self, S, G, kAcc, unit_stages, seed, weights_first=False):
-        self.S, self.G, self.kAcc = S, G, kAcc
+    """One CTA of the kernel.  ``abort_prob`` > 0 lets a blocked wait give up
+    at random (the kernel's bounded wait running out): the role raises the
+    CTA's abort flag, and from then on every wait that is not already
+    satisfied gives up too, as the kernel's waits do when they see the flag.
+    The producers' final drains wait regardless of the flag."""
+
+    def __init__(self, S, G, kAcc, unit_stages, seed, weights_first=False, SW=None,
+                 abort_prob=0.0):
+        SW = S if SW is None else SW
+        self.S, self.SW, self.G, self.kAcc = S, SW, G, kAcc
         self.units = unit_stages
         self.rng = random.Random(seed)
         self.weights_first = weights_first
+        self.abort_prob = abort_prob
+        self.aborted = False
         self.xfull = [Bar(f"xfull{i}", 1) for i in range(S)]
         self.empty = [Bar(f"empty{i}", 1) for i in range(S)]
-        self.wfull = [Bar(f"wfull{i}", 1) for i in range(S)]
-        self.wempty = [Bar(f"wempty{i}", 4) for i in range(S)]
+        self.wfull = [Bar(f"wfull{i}", 1) for i in range(SW)]
+        self.wempty = [Bar(f"wempty{i}", 4) for i in range(SW)]
         self.dqfull = [Bar(f"dqfull{i}", 4) for i in range(S)]
         self.accfull = [Bar(f"accfull{i}", 1) for i in range(kAcc)]
         self.accempty = [Bar(f"accempty{i}", 4) for i in range(kAcc)]
         self.drain = Bar("drain", 1)
         self.xslot = [None] * S
-        self.wslot = [None] * S
+        self.wslot = [None] * SW
         self.aslot = [None] * S
         self.acc_unit = [None] * kAcc
         self.w_reads = {}
@@ -77,73 +87,100 @@ class KernelModel:
         self.mma_q = []
 
     # ------------------------------------------------------------------ roles
+    # A role yields ("wait", bar, phase) and receives True (the phase
+    # completed) or False (the wait gave up); ("drain", bar, phase) always
+    # returns once the phase completed.
     def x_producer(self):
         S, g = self.S, 0
+        ok = True
         for n in self.units:
             for _ in range(n):
                 s = g % S
                 if g >= S:
-                    yield ("wait", self.empty[s], g // S - 1)
+                    ok = yield ("wait", self.empty[s], g // S - 1)
+                    if not ok:
+                        break
                     assert self.mma_done >= g - S, "X slot refilled before its MMAs completed"
                 self.xslot[s] = ("inflight", g)
                 self.tma.append(("x", g))
                 g += 1
+            if not ok:
+                break
+        # every copy issued lands before the CTA exits
+        for j in range(max(0, g - S), g):
+            yield ("drain", self.xfull[j % S], j // S)
 
     def w_producer(self):
-        S, g = self.S, 0
+        SW, g = self.SW, 0
+        ok = True
         for n in self.units:
             for _ in range(n):
-                s = g % S
-                if g >= S:
-                    yield ("wait", self.wempty[s], g // S - 1)
-                    assert self.w_reads.get(g - S, 0) == 4, "weight slot refilled before read"
+                s = g % SW
+                if g >= SW:
+                    ok = yield ("wait", self.wempty[s], g // SW - 1)
+                    if not ok:
+                        break
+                    assert self.w_reads.get(g - SW, 0) == 4, "weight slot refilled before read"
                 self.wslot[s] = ("inflight", g)
                 self.tma.append(("w", g))
                 g += 1
+            if not ok:
+                break
+        for j in range(max(0, g - SW), g):
+            yield ("drain", self.wfull[j % SW], j // SW)
 
     def mma(self):
         S, kAcc, g = self.S, self.kAcc, 0
         for lt, n in enumerate(self.units):
             b = lt % kAcc
             if lt >= kAcc:
-                yield ("wait", self.accempty[b], lt // kAcc - 1)
+                if not (yield ("wait", self.accempty[b], lt // kAcc - 1)):
+                    break
                 assert self.epi_done.get(lt - kAcc) == 4, "accumulator reused early"
+            ok = True
             for _ in range(n):
                 s = g % S
-                yield ("wait", self.dqfull[s], g // S)
+                ok = yield ("wait", self.dqfull[s], g // S)
+                if not ok:
+                    break
                 assert self.xslot[s] == ("landed", g), (g, self.xslot[s])
                 assert self.aslot[s] == ("written", g), (g, self.aslot[s])
                 self.mma_q.append(("stage", g))
                 g += 1
+            if not ok:
+                break
             self.mma_q.append(("acc", lt))
         self.mma_q.append(("drain", None))
-        yield ("wait", self.drain, 0)
+        yield ("drain", self.drain, 0)
 
     def dequant_warp(self, wg, q4):
-        S, G, g0 = self.S, self.G, 0
+        S, SW, G, g0 = self.S, self.SW, self.G, 0
         for n in self.units:
             i = (wg + G - g0 % G) % G          # this warpgroup's first stage of the unit
             while i < n:
                 g = g0 + i
-                s = g % S
+                s, sw = g % S, g % SW
                 if self.weights_first:
-                    yield ("wait", self.wfull[s], g // S)
+                    if not (yield ("wait", self.wfull[sw], g // SW)):
+                        return
                     self.w_reads[g] = self.w_reads.get(g, 0) + 1
-                    yield ("arrive", self.wempty[s])
-                    if g >= S:
-                        yield ("wait", self.empty[s], g // S - 1)
+                    yield ("arrive", self.wempty[sw])
+                    if g >= S and not (yield ("wait", self.empty[s], g // S - 1)):
+                        return
                 else:
-                    if g >= S:
-                        yield ("wait", self.empty[s], g // S - 1)
-                    yield ("wait", self.wfull[s], g // S)
-                    assert self.wslot[s] == ("landed", g), (g, self.wslot[s])
+                    if g >= S and not (yield ("wait", self.empty[s], g // S - 1)):
+                        return
+                    if not (yield ("wait", self.wfull[sw], g // SW)):
+                        return
+                    assert self.wslot[sw] == ("landed", g), (g, self.wslot[sw])
                     self.w_reads[g] = self.w_reads.get(g, 0) + 1
-                    yield ("arrive", self.wempty[s])
+                    yield ("arrive", self.wempty[sw])
                 assert g < S or self.mma_done >= g - S, "A slot written before its MMAs completed"
                 if q4 == 0:
                     self.aslot[s] = ("writing", g)
                 yield ("yield",)
-                yield ("wait", self.xfull[s], g // S)
+                if not (yield ("wait", self.xfull[s], g // S)):
+                    return
                 if q4 == 0:
                     self.aslot[s] = ("written", g)
                 yield ("arrive", self.dqfull[s])
@@ -153,7 +190,8 @@ class KernelModel:
     def epilogue_warp(self):
         for lt in range(len(self.units)):
             b = lt % self.kAcc
-            yield ("wait", self.accfull[b], lt // self.kAcc)
+            if not (yield ("wait", self.accfull[b], lt // self.kAcc)):
+                return
             assert self.acc_unit[b] == lt, (lt, self.acc_unit[b])
             yield ("yield",)
             self.epi_done[lt] = self.epi_done.get(lt, 0) + 1
@@ -166,8 +204,10 @@ class KernelModel:
             return False
         if self.rng.choice(kinds) == "tma":
             kind, g = self.tma.pop(self.rng.randrange(len(self.tma)))
-            slots, bars = (self.xslot, self.xfull) if kind == "x" else (self.wslot, self.wfull)
-            s = g % self.S
+            if kind == "x":
+                slots, bars, s = self.xslot, self.xfull, g % self.S
+            else:
+                slots, bars, s = self.wslot, self.wfull, g % self.SW
             assert slots[s] == ("inflight", g)
             slots[s] = ("landed", g)
             bars[s].arrive()
@@ -191,12 +231,24 @@ class KernelModel:
         for ew in range(4):
             gens[f"epi{ew}"] = self.epilogue_warp()
         waiting = {name: None for name in gens}
+        reply = {name: None for name in gens}
         live = set(gens)
         for _ in range(2_000_000):
             if not live:
                 break
-            runnable = [n for n in sorted(live)
-                        if waiting[n] is None or waiting[n][1].try_wait(waiting[n][2])]
+            runnable = []
+            for n in sorted(live):
+                w = waiting[n]
+                if w is None:
+                    runnable.append(n)
+                elif w[1].try_wait(w[2]):
+                    reply[n] = True
+                    runnable.append(n)
+                elif w[0] == "wait" and (self.aborted or self.rng.random() < self.abort_prob):
+                    # the bounded wait gives up: the CTA's abort flag is raised
+                    self.aborted = True
+                    reply[n] = False
+                    runnable.append(n)
             if not runnable or (self.rng.random() < 0.3 and (self.tma or self.mma_q)):
                 if not self.complete_one():
                     assert runnable, f"deadlock: {[(n, waiting[n][1].name) for n in live]}"
@@ -204,32 +256,82 @@ class KernelModel:
             name = self.rng.choice(runnable)
             waiting[name] = None
             try:
-                op = next(gens[name])
+                op = gens[name].send(reply[name])
             except StopIteration:
                 live.discard(name)
                 continue
-            if op[0] == "wait":
+            reply[name] = None
+            if op[0] in ("wait", "drain"):
                 waiting[name] = op
             elif op[0] == "arrive":
                 op[1].arrive()
         assert not live, "no progress"
-        # every copy was consumed: nothing is in flight once all roles finished
-        assert not self.tma and not self.mma_q
+        # every copy and every MMA group has completed once all roles finished
+        # (the CTA's teardown): nothing lands in shared or tensor memory later
+        assert not self.tma and not self.mma_q, (self.tma, self.mma_q)
 
 
-# (X/weight ring stages S, dequantizing warpgroups G, accumulators) per token tile
-KERNEL_CONFIGS = {16: (7, 4, 2), 32: (7, 4, 2), 64: (6, 4, 2), 128: (4, 3, 2),
-                  176: (5, 3, 2), 192: (4, 3, 2), 256: (4, 3, 1)}
+# (X ring stages S, weight ring stages SW, dequantizing warpgroups G,
+# accumulators) per token tile
+KERNEL_CONFIGS = {16: (7, 7, 4, 2), 32: (7, 7, 4, 2), 64: (6, 6, 4, 2), 128: (4, 5, 3, 2),
+                  176: (5, 10, 3, 2), 192: (4, 10, 3, 2), 256: (4, 8, 3, 1)}
 
 
 @pytest.mark.parametrize("tok", sorted(KERNEL_CONFIGS))
 def test_protocol_is_exact_for_every_token_tile(tok):
-    S, G, kAcc = KERNEL_CONFIGS[tok]
+    S, SW, G, kAcc = KERNEL_CONFIGS[tok]
     assert S >= G       # the condition under which the A-slot wait is exact
+    assert SW >= S      # the weight slot's older phase belongs to a stage <= g - S
     for seed in range(60):
         rng = random.Random(tok * 1000 + seed)
-        units = [rng.randint(1, 3 * S) for _ in range(rng.randint(1, 5))]
-        KernelModel(S, G, kAcc, units, seed).run()
+        units = [rng.randint(1, 3 * SW) for _ in range(rng.randint(1, 5))]
+        KernelModel(S, G, kAcc, units, seed, SW=SW).run()
+
+
+@pytest.mark.parametrize("tok", sorted(KERNEL_CONFIGS))
+def test_abort_at_any_wait_leaves_nothing_in_flight(tok):
+    """Any role's wait may give up at any point; every role then leaves its
+    loop, the producers drain the copies they issued, the MMA warp drains its
+    MMAs, and at teardown no copy or MMA is still in flight.  Every parity
+    wait stays exact on the way."""
+    S, SW, G, kAcc = KERNEL_CONFIGS[tok]
+    aborted = 0
+    for seed in range(80):
+        rng = random.Random(tok * 7919 + seed)
+        units = [rng.randint(1, 3 * SW) for _ in range(rng.randint(1, 5))]
+        m = KernelModel(S, G, kAcc, units, seed, SW=SW, abort_prob=0.02)
+        m.run()
+        aborted += m.aborted
+    assert aborted > 10     # the aborts were exercised
+
+
+def test_model_catches_a_producer_that_does_not_drain():
+    """Without the producers' final drain (the older kernel drained only when
+    the producer itself gave up), an abort elsewhere can end the CTA with
+    copies still landing."""
+    class NoDrain(KernelModel):
+        def x_producer(self):
+            S, g = self.S, 0
+            for n in self.units:
+                for _ in range(n):
+                    s = g % S
+                    if g >= S:
+                        if not (yield ("wait", self.empty[s], g // S - 1)):
+                            for j in range(max(0, g - S), g):
+                                yield ("drain", self.xfull[j % S], j // S)
+                            return
+                    self.xslot[s] = ("inflight", g)
+                    self.tma.append(("x", g))
+                    g += 1
+    caught = 0
+    for seed in range(300):
+        rng = random.Random(seed)
+        units = [rng.randint(1, 6) for _ in range(rng.randint(1, 3))]
+        try:
+            NoDrain(4, 3, 2, units, seed, abort_prob=0.05).run()
+        except AssertionError:
+            caught += 1
+    assert caught > 0
 
 
 def test_model_catches_the_older_wait_order():

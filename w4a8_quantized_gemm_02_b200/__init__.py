@@ -22,6 +22,7 @@ QOQ_OK = 0
 QOQ_ERR_INVALID_ARG = 1
 QOQ_ERR_UNSUPPORTED = 2
 QOQ_ERR_CUDA = 3
+QOQ_ERR_WORKSPACE = 4
 
 # Every symbol the public header declares.
 EXPORTS = (

@@ -70,6 +70,7 @@ extern "C" const char* qoq_status_str(int status) {
     case QOQ_ERR_INVALID_ARG: return "invalid argument (pointer, shape or alignment)";
     case QOQ_ERR_UNSUPPORTED: return "unsupported (device, group size or problem size)";
     case QOQ_ERR_CUDA: return "CUDA runtime or driver error";
+    case QOQ_ERR_WORKSPACE: return "split-K workspace too small for the launch plan";
     default: return "unknown status";
   }
 }

@@ -91,6 +91,14 @@ struct Cfg {
   static constexpr int kStageX = kNB * kXBytes;
   static constexpr int kStageRaw = kNB * kRawStageBytes;
   static constexpr int kStages = TOK <= 32 ? 7 : TOK == 64 ? 6 : TOK == 176 ? 5 : 4;
+  // The weight ring may be deeper than the X ring: its slots are small and
+  // its consumers (the dequantizers) have the longest latency.  It must not
+  // be shallower (see the parity note at the dequantizers' waits).
+  static constexpr int kWStages = TOK <= 64 ? kStages : TOK == 128 ? 5 : TOK == 256 ? 8 : 10;
+  static_assert(kWStages >= kStages, "weight ring at least as deep as the X ring");
+  // a dequantizer's A-slot wait is exact only if its own previous stage
+  // (g - kDqGroups) already implied the slot's older phase
+  static_assert(kStages >= kDqGroups, "at least as many stages as dequantizing warpgroups");
   static constexpr int kAcc = TOK <= 192 ? 2 : 1;
   static constexpr int kACols = 32 * kNB;                     // tensor-memory columns of A per stage
   // Tensor-memory columns: up to 128 tokens the A slots come first and the
@@ -103,10 +111,10 @@ struct Cfg {
       kAccFirst ? 0 : ((kStages * kACols + TOK - 1) / TOK) * TOK;   // accumulators
   static constexpr int kOffX = 0;
   static constexpr int kOffRaw = kOffX + kStages * kStageX;
-  static constexpr int kOffEpi = kOffRaw + kStages * kStageRaw;
+  static constexpr int kOffEpi = kOffRaw + kWStages * kStageRaw;
   static constexpr int kOffSx = kOffEpi + 4 * kStageBytesEpi;          // 4 warps x TOK floats
   static constexpr int kOffBar = kOffSx + 4 * TOK * 4;
-  static constexpr int kNumBars = 5 * kStages + 2 * kAcc + 1;
+  static constexpr int kNumBars = 3 * kStages + 2 * kWStages + 2 * kAcc + 1;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 32 + 1024;   // + base alignment slack
   static_assert(kOffRaw % 1024 == 0 && kXBytes % 1024 == 0, "swizzled tiles need 1 KiB alignment");
@@ -279,24 +287,27 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   // warp waits on this one barrier).  The weight ring is released as soon as
   // the blocks are in registers, so the weight stream runs ahead of the MMAs
   // and the weight copy overlaps the previous stages' dequantization.
+  constexpr int SW = C::kWStages;
   const uint32_t bar_xfull = base + C::kOffBar;
   const uint32_t bar_empty = bar_xfull + 8 * S;
-  const uint32_t bar_wfull = bar_empty + 8 * S;
-  const uint32_t bar_wempty = bar_wfull + 8 * S;
-  const uint32_t bar_dqfull = bar_wempty + 8 * S;
-  const uint32_t bar_accfull = bar_dqfull + 8 * S;
+  const uint32_t bar_dqfull = bar_empty + 8 * S;
+  const uint32_t bar_wfull = bar_dqfull + 8 * S;
+  const uint32_t bar_wempty = bar_wfull + 8 * SW;
+  const uint32_t bar_accfull = bar_wempty + 8 * SW;
   const uint32_t bar_accempty = bar_accfull + 8 * C::kAcc;
   const uint32_t bar_drain = bar_accempty + 8 * C::kAcc;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc + 4);
 
   if (warp == 0) {
-    // the barriers are contiguous from bar_xfull: xfull, empty, wfull, wempty,
-    // dqfull (S each), accfull, accempty (kAcc each), drain; the lanes of
-    // warp 0 initialize them in parallel
+    // the barriers are contiguous from bar_xfull: xfull, empty, dqfull (S
+    // each), wfull, wempty (SW each), accfull, accempty (kAcc each), drain;
+    // dqfull, wempty and accempty count the four warps of a warpgroup; the
+    // lanes of warp 0 initialize them in parallel
     for (int i = lane; i < C::kNumBars; i += 32) {
-      const bool four = (i >= 3 * S && i < 5 * S) ||
-                        (i >= 5 * S + C::kAcc && i < 5 * S + 2 * C::kAcc);
+      const int acc0 = 3 * S + 2 * SW;
+      const bool four = (i >= 2 * S && i < 3 * S) || (i >= 3 * S + SW && i < acc0) ||
+                        (i >= acc0 + C::kAcc && i < acc0 + 2 * C::kAcc);
       mbar_init(bar_xfull + 8 * i, four ? 4u : 1u);
     }
     if (lane == 0) {
@@ -342,11 +353,12 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
         __syncwarp();
       }
     }
-    if (aborted) {
-      // the copies already issued must land before the CTA exits
-      for (uint32_t j = (g > S ? g - S : 0); j < g; ++j)
-        drain_wait(bar_xfull + 8 * (j % S), (j / S) & 1);
-    }
+    // the copies already issued must land before the CTA exits, also when
+    // another role gave up a wait after this loop had issued its last stage
+    // (on the normal path they have all landed and every test passes at once)
+    for (uint32_t j = (g > S ? g - S : 0); j < g; ++j)
+      drain_wait(bar_xfull + 8 * (j % S), (j / S) & 1);
+    (void)aborted;
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     // The whole warp runs the loop and waits; one elected lane issues each
@@ -420,24 +432,27 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
         const uint32_t g = g0 + i;
         const int s = g % S;
         const uint32_t ph = (g / S) & 1;
+        const int sw = g % SW;
+        const uint32_t phw = (g / SW) & 1;
         // A parity wait is only exact while the barrier has completed the
         // phase before the awaited one.  This warpgroup first waits for the
         // A columns of slot s (the MMAs of stage g - S completed, in order):
-        // those MMAs read the dequantized weights of stage g - S, so the
-        // weight slot's previous phase has completed before its parity is
-        // tested below.
+        // those MMAs read the dequantized weights of every stage up to
+        // g - S, and the weight slot's previous phase belongs to stage
+        // g - SW <= g - S, so it has completed before its parity is tested
+        // below.
         if (g >= S && !mbar_wait(bar_empty + 8 * s, ph ^ 1, abort_flag, &g_error_word,
                                  kErrDequant)) {
           aborted = true;
           break;
         }
         tc_fence_after_sync();
-        if (!mbar_wait(bar_wfull + 8 * s, ph, abort_flag, &g_error_word, kErrDequant)) {
+        if (!mbar_wait(bar_wfull + 8 * sw, phw, abort_flag, &g_error_word, kErrDequant)) {
           aborted = true;
           break;
         }
         const int nb = min(C::kNB, w.num_kt - i * C::kNB);
-        const uint8_t* stage_raw = smem + C::kOffRaw + s * C::kStageRaw;
+        const uint8_t* stage_raw = smem + C::kOffRaw + sw * C::kStageRaw;
         const uint32_t a_cols = row_tmem + C::kTmemA + C::kACols * s;
         if constexpr (C::kDqGroups == 3) {
           // every block of the stage into registers first, so the weight slot
@@ -449,7 +464,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
           // the weight slot may be refilled once every lane has read it (the
           // arrive releases this warp's reads, ordered by the warp barrier)
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar_wempty + 8 * s);
+          if (lane == 0) mbar_arrive(bar_wempty + 8 * sw);
 #pragma unroll
           for (int q = 0; q < C::kNB; ++q)
             if (q < nb) dequant_store_row_block(rb[q], gpt, a_cols + 32 * q);
@@ -463,7 +478,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
               load_row_block(stage_raw + q * args.blk_bytes, r, gpt, rb);
               if (q == nb - 1) {
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar_wempty + 8 * s);
+                if (lane == 0) mbar_arrive(bar_wempty + 8 * sw);
               }
               dequant_store_row_block(rb, gpt, a_cols + 32 * q);
             }
@@ -627,27 +642,27 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
           args.packed + (static_cast<size_t>(w.nt) * kt_total + w.kt_begin) * args.blk_bytes;
       const int nsteps = (w.num_kt + C::kNB - 1) / C::kNB;
       for (int i = 0; i < nsteps; ++i, ++g) {
-        const int s = g % S;
-        if (g >= S && !__all_sync(0xffffffffu, mbar_wait(bar_wempty + 8 * s, ((g / S) & 1) ^ 1,
-                                                         abort_flag, &g_error_word,
-                                                         kErrProducer))) {
+        const int sw = g % SW;
+        if (g >= SW && !__all_sync(0xffffffffu, mbar_wait(bar_wempty + 8 * sw,
+                                                          ((g / SW) & 1) ^ 1, abort_flag,
+                                                          &g_error_word, kErrProducer))) {
           aborted = true;
           break;
         }
         if (elect_one()) {
           const int nb = min(C::kNB, w.num_kt - i * C::kNB);
-          mbar_arrive_expect_tx(bar_wfull + 8 * s, static_cast<uint32_t>(nb * args.blk_bytes));
-          bulk_load(base + C::kOffRaw + s * C::kStageRaw,
+          mbar_arrive_expect_tx(bar_wfull + 8 * sw, static_cast<uint32_t>(nb * args.blk_bytes));
+          bulk_load(base + C::kOffRaw + sw * C::kStageRaw,
                     src + static_cast<size_t>(i * C::kNB) * args.blk_bytes,
-                    static_cast<uint32_t>(nb * args.blk_bytes), bar_wfull + 8 * s, policy);
+                    static_cast<uint32_t>(nb * args.blk_bytes), bar_wfull + 8 * sw, policy);
         }
         __syncwarp();
       }
     }
-    if (aborted) {
-      for (uint32_t j = (g > S ? g - S : 0); j < g; ++j)
-        drain_wait(bar_wfull + 8 * (j % S), (j / S) & 1);
-    }
+    // as for the X ring: every copy issued lands before the CTA exits
+    for (uint32_t j = (g > SW ? g - SW : 0); j < g; ++j)
+      drain_wait(bar_wfull + 8 * (j % SW), (j / SW) & 1);
+    (void)aborted;
   }
 
   // ------------------------------------------------------------------ teardown
@@ -808,11 +823,19 @@ int launch_tok(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cudaStr
   return QOQ_OK;
 }
 
-}  // namespace
+// Everything one GEMM launch needs, built and checked before anything is
+// enqueued: the plan, the X8 tensor map and the kernel arguments.
+struct GemmLaunch {
+  Plan p;
+  CUtensorMap map;
+  GemmArgs a;
+};
 
-int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* s1, int M, int N,
-              int K, int group, void* Y, int32_t* acc, int tok_req, int splits_req, void* ws,
-              size_t ws_bytes, void* stream, bool pdl) {
+// Validate the arguments, pick the plan and encode the tensor map.  Calls no
+// CUDA API that enqueues work.
+int gemm_prepare(const int8_t* X8, const void* sx, const void* packed, const void* s1, int M,
+                 int N, int K, int group, void* Y, int32_t* acc, int tok_req, int splits_req,
+                 void* ws, size_t ws_bytes, GemmLaunch& L) {
   if (!X8 || !packed) return QOQ_ERR_INVALID_ARG;
   if ((Y == nullptr) == (acc == nullptr)) return QOQ_ERR_INVALID_ARG;
   if (Y && (!sx || !s1)) return QOQ_ERR_INVALID_ARG;
@@ -833,25 +856,26 @@ int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* 
     p.splits = 1;
   }
   if (p.splits > 1 && (ws == nullptr || ws_bytes < ws_bytes_for(p, N))) {
-    if (splits_req) return QOQ_ERR_INVALID_ARG;   // explicit split needs its workspace
-    p.splits = 1;                                  // auto plan: do not split K
+    // an explicit split needs its workspace; so does the automatic plan,
+    // unless the caller passed none (an explicit request not to split K)
+    if (splits_req || ws != nullptr) return QOQ_ERR_WORKSPACE;
+    p.splits = 1;
   }
   finish_plan(p);
   if (int st = check_device()) return st;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return QOQ_ERR_CUDA;
 
-  CUtensorMap map;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileK), static_cast<cuuint32_t>(p.tok)};
   const cuuint32_t estr[2] = {1, 1};
-  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(X8), dims, strides, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  if (enc(&L.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(X8), dims, strides, box,
+          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return QOQ_ERR_CUDA;
 
-  GemmArgs a;
+  GemmArgs& a = L.a;
   a.packed = static_cast<const uint8_t*>(packed);
   a.sx = static_cast<const __half*>(sx);
   a.s1 = static_cast<const __half*>(s1);
@@ -874,17 +898,38 @@ int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* 
   a.blk_bytes = static_cast<int>(block_bytes(group));
   a.rcp_splits = 1.0f / static_cast<float>(p.splits);
   a.rcp_mtiles = 1.0f / static_cast<float>(p.m_tiles);
+  L.p = p;
+  return QOQ_OK;
+}
 
+// Enqueue a prepared launch.  With `clear_counters` the workspace's arrival
+// counters are zeroed on the stream first when the plan splits K.
+int gemm_launch(const GemmLaunch& L, void* stream, bool pdl, bool clear_counters) {
   cudaStream_t s = as_stream(stream);
-  switch (p.tok) {
-    case 16: return launch_tok<16>(map, a, p, s, pdl);
-    case 32: return launch_tok<32>(map, a, p, s, pdl);
-    case 64: return launch_tok<64>(map, a, p, s, pdl);
-    case 128: return launch_tok<128>(map, a, p, s, pdl);
-    case 176: return launch_tok<176>(map, a, p, s, pdl);
-    case 192: return launch_tok<192>(map, a, p, s, pdl);
-    default: return launch_tok<256>(map, a, p, s, pdl);
+  if (clear_counters && L.p.splits > 1 &&
+      cudaMemsetAsync(L.a.ws_count, 0, kCounterBytes, s) != cudaSuccess)
+    return QOQ_ERR_CUDA;
+  switch (L.p.tok) {
+    case 16: return launch_tok<16>(L.map, L.a, L.p, s, pdl);
+    case 32: return launch_tok<32>(L.map, L.a, L.p, s, pdl);
+    case 64: return launch_tok<64>(L.map, L.a, L.p, s, pdl);
+    case 128: return launch_tok<128>(L.map, L.a, L.p, s, pdl);
+    case 176: return launch_tok<176>(L.map, L.a, L.p, s, pdl);
+    case 192: return launch_tok<192>(L.map, L.a, L.p, s, pdl);
+    default: return launch_tok<256>(L.map, L.a, L.p, s, pdl);
   }
+}
+
+}  // namespace
+
+int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* s1, int M, int N,
+              int K, int group, void* Y, int32_t* acc, int tok_req, int splits_req, void* ws,
+              size_t ws_bytes, void* stream, bool pdl, bool clear_counters) {
+  GemmLaunch L;
+  if (int st = gemm_prepare(X8, sx, packed, s1, M, N, K, group, Y, acc, tok_req, splits_req, ws,
+                            ws_bytes, L))
+    return st;
+  return gemm_launch(L, stream, pdl, clear_counters);
 }
 
 size_t gemm_ws_bytes(int M, int N, int K, int tok_req, int splits_req) {
@@ -915,7 +960,7 @@ extern "C" int qoq_w4a8_gemm(const int8_t* X8, const void* sx, const void* packe
                              void* stream) {
   if (!Y) return QOQ_ERR_INVALID_ARG;
   return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, nullptr, 0, 0, ws, ws_bytes, stream,
-                   false);
+                   false, false);
 }
 
 // ---------------------------------------------------------------------------
@@ -962,19 +1007,19 @@ extern "C" int qoq_w4a8_gemm_static_ws(const int8_t* X8, const void* sx, const v
   if (!X8 || !sx || !packed || !s1 || !Y) return QOQ_ERR_INVALID_ARG;
   if (M <= 0) return QOQ_ERR_INVALID_ARG;
   if (int st = check_weight_shape(N, K, group)) return st;
+  if (!aligned16(X8) || !aligned16(sx) || !aligned16(packed) || !aligned16(s1) || !aligned16(Y))
+    return QOQ_ERR_INVALID_ARG;
   const size_t need = gemm_ws_bytes(M, N, K, 0, 0);
   if (need > kStaticWsBytes) return QOQ_ERR_UNSUPPORTED;   // larger than the fixed array
   if (int st = check_device()) return st;
   void* ws = nullptr;
   if (int st = static_ws_ptr(&ws)) return st;
-  if (need > 0) {
-    // the arrival counters must start at zero; a completed call leaves them
-    // so, but the array keeps whatever an interrupted earlier call left
-    if (cudaMemsetAsync(ws, 0, kCounterBytes, as_stream(stream)) != cudaSuccess)
-      return QOQ_ERR_CUDA;
-  }
+  // The arrival counters must start at zero: a completed call leaves them so,
+  // but the array keeps whatever an interrupted earlier call left.  The GEMM
+  // launcher clears them on `stream` after its own checks, only when K is
+  // split, so a rejected call enqueues nothing.
   return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, nullptr, 0, 0, ws, kStaticWsBytes,
-                   stream, false);
+                   stream, false, true);
 }
 
 extern "C" int qoq_w4a8_gemm_i32(const int8_t* X8, const void* packed, int M, int N, int K,
@@ -982,7 +1027,7 @@ extern "C" int qoq_w4a8_gemm_i32(const int8_t* X8, const void* packed, int M, in
                                  void* stream) {
   if (!acc) return QOQ_ERR_INVALID_ARG;
   return gemm_impl(X8, nullptr, packed, nullptr, M, N, K, group, nullptr, acc, 0, 0, ws, ws_bytes,
-                   stream, false);
+                   stream, false, false);
 }
 
 extern "C" int qoq_w4a8_gemm_config(const int8_t* X8, const void* sx, const void* packed,
@@ -990,7 +1035,7 @@ extern "C" int qoq_w4a8_gemm_config(const int8_t* X8, const void* sx, const void
                                     int32_t* acc, int tok_tile, int splits, void* ws,
                                     size_t ws_bytes, void* stream) {
   return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, acc, tok_tile, splits, ws, ws_bytes,
-                   stream, false);
+                   stream, false, false);
 }
 
 extern "C" int qoq_w4a8_linear(const void* X, int M, int K, const void* packed, const void* s1,
@@ -1002,7 +1047,10 @@ extern "C" int qoq_w4a8_linear(const void* X, int M, int K, const void* packed, 
   if (!aligned16(X) || !aligned16(X8) || !aligned16(sx) || !aligned16(Y) || !aligned16(packed) ||
       !aligned16(s1) || (ws && !aligned16(ws)))
     return QOQ_ERR_INVALID_ARG;
-  if (int st = check_device()) return st;
+  // every check of the GEMM runs before the quantizer is launched
+  GemmLaunch L;
+  if (int st = gemm_prepare(X8, sx, packed, s1, M, N, K, group, Y, nullptr, 0, 0, ws, ws_bytes, L))
+    return st;
   // For few rows the quantizer may start while the preceding kernel on the
   // stream drains (it waits for that grid before touching memory); this hides
   // its launch latency.  For many rows that overlap measured slower on B200,
@@ -1011,8 +1059,7 @@ extern "C" int qoq_w4a8_linear(const void* X, int M, int K, const void* packed, 
   if (int st = launch_act_quant(X, M, K, X8, sx, stream, aq_pdl)) return st;
   // both kernels are this library's: the GEMM reads nothing the quantizer
   // writes before its grid-dependency wait, so it may overlap its tail
-  return gemm_impl(X8, sx, packed, s1, M, N, K, group, Y, nullptr, 0, 0, ws, ws_bytes, stream,
-                   true);
+  return gemm_launch(L, stream, true, false);
 }
 
 extern "C" int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int* splits, int* ctas,
