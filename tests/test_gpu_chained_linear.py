@@ -52,3 +52,35 @@ def test_chained_layers_match_synchronized(M):
     assert np.isfinite(y2s).all()
     assert np.array_equal(y1c.view(np.uint16), y1s.view(np.uint16))
     assert np.array_equal(y2c.view(np.uint16), y2s.view(np.uint16))
+
+
+@pytest.mark.parametrize("M", [1, 64, 1024])
+def test_gemm_waits_for_a_preceding_kernel_that_writes_its_weights(oracle, M):
+    """Every GEMM launch may start while the preceding kernel drains; its
+    weight stream must still wait for that kernel when it may have written
+    the weights.  Two code sets are packed in turn into one buffer, each
+    immediately followed by a GEMM on the same stream with no
+    synchronization; every accumulator must be that of its own code set."""
+    N, K, G = 2048, 4096, 128
+    sets = [si.sweep_operands(M, N, K, G, seed=s) for s in (31, 32)]
+    dev_sets = [tuple(torch.from_numpy(a).to(DEV) for a in (o.q, o.s2, o.z)) for o in sets]
+    X8 = torch.from_numpy(sets[0].X8).to(DEV)
+    refs = [oracle.int_gemm(sets[0].X8, oracle.dequant_w(o.q, o.s2, o.z, G)) for o in sets]
+    packed = torch.empty(qoq.packed_weight_bytes(N, K, G), dtype=torch.uint8, device=DEV)
+    accs = [torch.empty((M, N), dtype=torch.int32, device=DEV) for _ in range(6)]
+    L = qoq.lib()
+    import ctypes
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    qoq.device_error(clear=True)
+    for i, acc in enumerate(accs):
+        q, s2, z = dev_sets[i % 2]
+        assert L.qoq_pack_codes(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(s2.data_ptr()),
+                                ctypes.c_void_p(z.data_ptr()), N, K, G,
+                                ctypes.c_void_p(packed.data_ptr()),
+                                ctypes.c_void_p(stream.cuda_stream)) == 0
+        qoq.w4a8_gemm_i32(X8, packed, N, G, out=acc, stream=stream)
+    torch.cuda.synchronize()
+    assert qoq.device_error(clear=True) == 0
+    for i, acc in enumerate(accs):
+        assert np.array_equal(acc.cpu().numpy(), refs[i % 2]), i

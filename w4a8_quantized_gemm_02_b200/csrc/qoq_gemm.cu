@@ -143,6 +143,8 @@ struct GemmArgs {
   int blk_bytes;
   float rcp_splits;     // 1 / splits and 1 / m_tiles, rounded (for small_div)
   float rcp_mtiles;
+  int w_dep_wait;       // the weight producer waits for the preceding grid (it may
+                        // have written the weights) before its first copy
 };
 
 struct Unit {
@@ -263,6 +265,67 @@ __device__ __forceinline__ void dequant_store_row_block(const RowBlock& rb, int 
   tmem_st_32x32b_x32(taddr, out);
 }
 
+// The weight producer's walk over its units' stages, resumable: run() with
+// `prologue` issues stages until the weight ring is full and never waits;
+// without, it continues to the end, waiting for free slots.  The whole warp
+// runs it; one elected lane issues each bulk copy.
+struct WeightStream {
+  int u, i;
+  uint32_t g;
+  Unit w;
+  const uint8_t* src;
+  uint64_t policy;
+
+  __device__ __forceinline__ void load_unit(const GemmArgs& a, int kt_total) {
+    w = unit_of(a, u, kt_total);
+    src = a.packed + (static_cast<size_t>(w.nt) * kt_total + w.kt_begin) * a.blk_bytes;
+    i = 0;
+  }
+
+  __device__ __forceinline__ void begin(const GemmArgs& a, int kt_total) {
+    policy = l2_policy_evict_first();
+    g = 0;
+    u = blockIdx.x;
+    i = 0;
+    if (u < a.units) load_unit(a, kt_total);
+  }
+
+  template <class C>
+  __device__ __forceinline__ bool run(const GemmArgs& a, uint32_t base, uint32_t bar_wfull,
+                                      uint32_t bar_wempty, volatile uint32_t* abort_flag,
+                                      bool prologue) {
+    constexpr int SW = C::kWStages;
+    const int kt_total = a.K / kTileK;
+    while (u < a.units) {
+      const int nsteps = (w.num_kt + C::kNB - 1) / C::kNB;
+      if (i >= nsteps) {
+        u += gridDim.x;
+        if (u >= a.units) break;
+        load_unit(a, kt_total);
+        continue;
+      }
+      const int sw = g % SW;
+      if (g >= SW) {
+        if (prologue) return true;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_wempty + 8 * sw, ((g / SW) & 1) ^ 1,
+                                               abort_flag, &g_error_word, kErrProducer)))
+          return false;
+      }
+      if (elect_one()) {
+        const int nb = min(C::kNB, w.num_kt - i * C::kNB);
+        mbar_arrive_expect_tx(bar_wfull + 8 * sw, static_cast<uint32_t>(nb * a.blk_bytes));
+        bulk_load(base + C::kOffRaw + sw * C::kStageRaw,
+                  src + static_cast<size_t>(i * C::kNB) * a.blk_bytes,
+                  static_cast<uint32_t>(nb * a.blk_bytes), bar_wfull + 8 * sw, policy);
+      }
+      __syncwarp();
+      ++i;
+      ++g;
+    }
+    return true;
+  }
+};
+
 template <int TOK>
 __global__ void __launch_bounds__(Cfg<TOK>::kThreads, 1)
 w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args) {
@@ -303,10 +366,12 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     // the barriers are contiguous from bar_xfull: xfull, empty, dqfull (S
     // each), wfull, wempty (SW each), accfull, accempty (kAcc each), drain;
     // dqfull, wempty and accempty count the four warps of a warpgroup; the
-    // lanes of warp 0 initialize them in parallel
+    // lanes of warp 0 initialize all but the weight ring's, which the weight
+    // producer initializes itself
     for (int i = lane; i < C::kNumBars; i += 32) {
       const int acc0 = 3 * S + 2 * SW;
-      const bool four = (i >= 2 * S && i < 3 * S) || (i >= 3 * S + SW && i < acc0) ||
+      if (i >= 3 * S && i < acc0) continue;
+      const bool four = (i >= 2 * S && i < 3 * S) ||
                         (i >= acc0 + C::kAcc && i < acc0 + 2 * C::kAcc);
       mbar_init(bar_xfull + 8 * i, four ? 4u : 1u);
     }
@@ -319,6 +384,19 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
+  }
+  // The weight producer starts the weight stream before the start-up
+  // barrier: its own barriers, then (once the preceding grid completed, if
+  // that grid may have written the weights) the first SW stages of bulk
+  // copies, all without waiting for a free slot.
+  WeightStream wstream;
+  if (warp == C::kWarpW) {
+    for (int i = lane; i < 2 * SW; i += 32) mbar_init(bar_wfull + 8 * i, i < SW ? 1u : 4u);
+    fence_mbar_init();
+    __syncwarp();
+    wstream.begin(args, kt_total);
+    if (args.w_dep_wait) grid_dependency_wait();
+    wstream.run<C>(args, base, bar_wfull, bar_wempty, abort_flag, /*prologue=*/true);
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -530,9 +608,9 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
                                 &g_error_word, kErrEpilogue);
       if (!__all_sync(0xffffffffu, ok)) break;
       // At this CTA's last accumulator a kernel launched after this one as
-      // its programmatic dependent (the next layer's activation quantizer in
-      // qoq_w4a8_linear) may be scheduled: it waits for this grid to complete
-      // before touching memory, so only its launch overlaps this tail.
+      // its programmatic dependent may be scheduled: it waits for this grid
+      // to complete before it touches memory this grid uses, so only its
+      // launch and set-up overlap this tail.
       if (u + static_cast<int>(gridDim.x) >= args.units) grid_launch_dependents();
       tc_fence_after_sync();
       const uint32_t t_acc = tmem + C::kTmemD + b * TOK + (static_cast<uint32_t>(q4 * 32) << 16);
@@ -631,38 +709,14 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     }
   } else {
     // -------------------------------------------------------------- W producer
-    // Packed weight blocks: independent of the preceding grid, so this warp
-    // starts at once under PDL.
-    const uint64_t policy = l2_policy_evict_first();
-    uint32_t g = 0;
-    bool aborted = false;
-    for (int u = blockIdx.x; u < args.units && !aborted; u += gridDim.x) {
-      const Unit w = unit_of(args, u, kt_total);
-      const uint8_t* src =
-          args.packed + (static_cast<size_t>(w.nt) * kt_total + w.kt_begin) * args.blk_bytes;
-      const int nsteps = (w.num_kt + C::kNB - 1) / C::kNB;
-      for (int i = 0; i < nsteps; ++i, ++g) {
-        const int sw = g % SW;
-        if (g >= SW && !__all_sync(0xffffffffu, mbar_wait(bar_wempty + 8 * sw,
-                                                          ((g / SW) & 1) ^ 1, abort_flag,
-                                                          &g_error_word, kErrProducer))) {
-          aborted = true;
-          break;
-        }
-        if (elect_one()) {
-          const int nb = min(C::kNB, w.num_kt - i * C::kNB);
-          mbar_arrive_expect_tx(bar_wfull + 8 * sw, static_cast<uint32_t>(nb * args.blk_bytes));
-          bulk_load(base + C::kOffRaw + sw * C::kStageRaw,
-                    src + static_cast<size_t>(i * C::kNB) * args.blk_bytes,
-                    static_cast<uint32_t>(nb * args.blk_bytes), bar_wfull + 8 * sw, policy);
-        }
-        __syncwarp();
-      }
-    }
-    // as for the X ring: every copy issued lands before the CTA exits
+    // The stages after the prologue, waiting for free slots.
+    wstream.run<C>(args, base, bar_wfull, bar_wempty, abort_flag, /*prologue=*/false);
+    // every copy issued lands before the CTA exits, also when another role
+    // gave up a wait after this loop had issued its last stage (on the
+    // normal path they have all landed and every test passes at once)
+    const uint32_t g = wstream.g;
     for (uint32_t j = (g > SW ? g - SW : 0); j < g; ++j)
       drain_wait(bar_wfull + 8 * (j % SW), (j / SW) & 1);
-    (void)aborted;
   }
 
   // ------------------------------------------------------------------ teardown
@@ -898,14 +952,22 @@ int gemm_prepare(const int8_t* X8, const void* sx, const void* packed, const voi
   a.blk_bytes = static_cast<int>(block_bytes(group));
   a.rcp_splits = 1.0f / static_cast<float>(p.splits);
   a.rcp_mtiles = 1.0f / static_cast<float>(p.m_tiles);
+  a.w_dep_wait = 1;
   L.p = p;
   return QOQ_OK;
 }
 
 // Enqueue a prepared launch.  With `clear_counters` the workspace's arrival
-// counters are zeroed on the stream first when the plan splits K.
-int gemm_launch(const GemmLaunch& L, void* stream, bool pdl, bool clear_counters) {
+// counters are zeroed on the stream first when the plan splits K.  Every
+// launch may start as a programmatic dependent of the preceding kernel: the
+// kernel touches nothing that kernel may write before its grid-dependency
+// waits.  `weights_independent` says the preceding kernel does not
+// write the weights (the library's own quantizer), so the weight stream
+// need not wait for it.
+int gemm_launch(GemmLaunch L, void* stream, bool weights_independent, bool clear_counters) {
   cudaStream_t s = as_stream(stream);
+  const bool pdl = true;
+  L.a.w_dep_wait = weights_independent ? 0 : 1;
   if (clear_counters && L.p.splits > 1 &&
       cudaMemsetAsync(L.a.ws_count, 0, kCounterBytes, s) != cudaSuccess)
     return QOQ_ERR_CUDA;
@@ -924,12 +986,12 @@ int gemm_launch(const GemmLaunch& L, void* stream, bool pdl, bool clear_counters
 
 int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* s1, int M, int N,
               int K, int group, void* Y, int32_t* acc, int tok_req, int splits_req, void* ws,
-              size_t ws_bytes, void* stream, bool pdl, bool clear_counters) {
+              size_t ws_bytes, void* stream, bool weights_independent, bool clear_counters) {
   GemmLaunch L;
   if (int st = gemm_prepare(X8, sx, packed, s1, M, N, K, group, Y, acc, tok_req, splits_req, ws,
                             ws_bytes, L))
     return st;
-  return gemm_launch(L, stream, pdl, clear_counters);
+  return gemm_launch(L, stream, weights_independent, clear_counters);
 }
 
 size_t gemm_ws_bytes(int M, int N, int K, int tok_req, int splits_req) {
@@ -1059,7 +1121,7 @@ extern "C" int qoq_w4a8_linear(const void* X, int M, int K, const void* packed, 
   if (int st = launch_act_quant(X, M, K, X8, sx, stream, aq_pdl)) return st;
   // both kernels are this library's: the GEMM reads nothing the quantizer
   // writes before its grid-dependency wait, so it may overlap its tail
-  return gemm_launch(L, stream, true, false);
+  return gemm_launch(L, stream, /*weights_independent=*/true, false);
 }
 
 extern "C" int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int* splits, int* ctas,

@@ -43,15 +43,18 @@ int sm_count();
 // cudaGetLastError -> status.
 int launch_status();
 
-// The GEMM launcher shared by the entry points.  With `pdl` the kernel may
-// start while the preceding kernel on the stream is still running: it then
-// streams weights right away and waits for that grid before reading X8 / sx.
-// With `clear_counters` the workspace's arrival counters are zeroed on the
-// stream before the kernel, when the plan splits K (after every argument
-// check, so a rejected call enqueues nothing).
+// The GEMM launcher shared by the entry points.  The kernel may start while
+// the preceding kernel on the stream is still running (programmatic
+// dependent launch): it sets up right away and waits for that grid before
+// reading X8 / sx, writing anything, and (unless
+// `weights_independent`: the preceding kernel cannot have written the
+// weights) before copying weights.  With `clear_counters` the workspace's
+// arrival counters are zeroed on the stream before the kernel, when the
+// plan splits K (after every argument check, so a rejected call enqueues
+// nothing).
 int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* s1, int M, int N,
               int K, int group, void* Y, int32_t* acc, int tok_req, int splits_req, void* ws,
-              size_t ws_bytes, void* stream, bool pdl, bool clear_counters);
+              size_t ws_bytes, void* stream, bool weights_independent, bool clear_counters);
 
 // Launch the per-token activation quantizer (no argument checks).  With
 // `pdl` it may start while the preceding kernel on the stream drains; it
