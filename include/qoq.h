@@ -166,9 +166,13 @@ QOQ_API int qoq_quantize_act_per_token(const void* X, int M, int K, int8_t* X8,
  *   packed : device, packed weights (qoq_quantize_weights / qoq_pack_codes).
  *   s1     : device, FP16[N].
  *   Y      : device, FP16 M x N row-major, written (rows >= M untouched).
- *   ws, ws_bytes : device workspace for splitting K over several CTAs, at
- *            least qoq_gemm_workspace_bytes(M, N, K, group) bytes (0 for
- *            shapes that are not split).  Owned by the caller, who fills it
+ *   ws, ws_bytes : device workspace for splitting K over several CTAs
+ *            through L2, at least qoq_gemm_workspace_bytes(M, N, K, group)
+ *            bytes (0 for shapes that are not split that way: a split of K
+ *            into at most 8 parts for token tiles of 16, or 3 for tiles of
+ *            32, runs on a thread-block cluster whose CTAs add their INT32
+ *            partial tiles up in the leader CTA's shared memory and needs no
+ *            workspace).  Owned by the caller, who fills it
  *            with zeros once before its first use (e.g. cudaMemset); every
  *            call that completes leaves its first 16 KiB (arrival counters,
  *            one per 32-channel slice of an output tile; K is split only when
@@ -186,9 +190,12 @@ QOQ_API int qoq_quantize_act_per_token(const void* X, int M, int K, int8_t* X8,
  * INT8 tensor cores (tcgen05, INT32 accumulators in tensor memory), and the
  * FP16 scaling runs once in the epilogue: Y = fp16_rn(float(acc) *
  * (float(sx[m]) * float(s1[n]))).  The token tile and the number of K splits
- * are chosen per (M, N, K); split partials are added exactly in INT32 by the
- * last CTA of each output tile before its epilogue.  Sources: Methods, 1) and
- * 2); Background.  Asynchronous on `stream`.
+ * are chosen per (M, N, K); split partials are added exactly in INT32 (in a
+ * cluster's leader CTA, or by the last CTA of an output tile to arrive)
+ * before its epilogue.  The kernel may start as a programmatic dependent of
+ * the preceding kernel on `stream`: it reads and writes nothing that kernel
+ * may write before that kernel has completed.  Sources: Methods, 1) and 2);
+ * Background.  Asynchronous on `stream`.
  * ---------------------------------------------------------------------- */
 QOQ_API int qoq_w4a8_gemm(const int8_t* X8, const void* sx, const void* packed,
                           const void* s1, int M, int N, int K, int group, void* Y,
@@ -212,9 +219,11 @@ QOQ_API int qoq_w4a8_gemm(const int8_t* X8, const void* sx, const void* packed,
  *     (qoq_gemm_workspace_bytes(M, N, K, group) > QOQ_STATIC_WS_BYTES) is
  *     rejected with QOQ_ERR_UNSUPPORTED and nothing is launched; use
  *     qoq_w4a8_gemm with a workspace for it.  The automatic plan splits K
- *     only for token tiles of at most 32 and into at most 4 units per SM,
- *     so it needs at most 16 KiB + 4 * SMs * 32 * 128 * 4 bytes (about
- *     9.7 MB with 148 SMs): on such a GPU no valid shape is rejected.
+ *     through this scratch only for token tiles of 32 (more than 3 splits)
+ *     and into at most 4 units per SM, so it needs at most 16 KiB + 4 * SMs
+ *     * 32 * 128 * 4 bytes (about 9.7 MB with 148 SMs): on such a GPU no
+ *     valid shape is rejected.  Plans that split K across a cluster, or do
+ *     not split it, leave the array untouched.
  *   - Every call on a device uses the same array, and it keeps the last
  *     call's contents.  Each call that splits K clears the array's arrival
  *     counters on `stream` before its GEMM, so nothing from an earlier call
@@ -287,8 +296,10 @@ QOQ_API int qoq_w4a8_linear(const void* X, int M, int K, const void* packed, con
                             size_t ws_bytes, void* stream);
 
 /* The launch configuration qoq_w4a8_gemm picks for a shape: token tile,
- * K splits, CTAs in the grid and pipeline stages.  Host only, no CUDA call
- * beyond reading the SM count of the current device (148 if none).  The
+ * K splits, CTAs in the grid and pipeline stages.  Host only: no CUDA call
+ * beyond reading the SM count of the current device and (once per device)
+ * how many thread-block clusters of the kernel fit on it; without a device
+ * 148 SMs and 148 / splits clusters are assumed.  The
  * pages fix no tiling; this reports the library's own choice for the GEMM of
  * Methods, 1) Algorithm: QoQ. */
 QOQ_API int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int* splits,

@@ -57,10 +57,16 @@ def test_plan_is_host_only(L):
         assert p["tok_tile"] >= min(M, 32)
         assert 1 <= p["splits"] <= 8
         # K is split only for small token tiles, at most 4 units per SM
-        assert p["splits"] == 1 or (p["tok_tile"] <= 32 and
-                                    48 * -(-M // p["tok_tile"]) * p["splits"] <= 4 * 148)
-        # persistent grid: one CTA per SM at most (148 without a device)
-        assert p["ctas"] == min(48 * -(-M // p["tok_tile"]) * p["splits"], 148)
+        tiles = 48 * -(-M // p["tok_tile"])
+        assert p["splits"] == 1 or (p["tok_tile"] <= 32 and tiles * p["splits"] <= 4 * 148)
+        cluster_max = 8 if p["tok_tile"] <= 16 else 3 if p["tok_tile"] <= 32 else 1
+        if 1 < p["splits"] <= cluster_max:
+            # K split across clusters of `splits` CTAs, whole clusters only
+            # (148 // splits resident clusters without a device)
+            assert p["ctas"] == min(tiles, 148 // p["splits"]) * p["splits"]
+        else:
+            # persistent grid: one CTA per SM at most (148 without a device)
+            assert p["ctas"] == min(tiles * p["splits"], 148)
     with pytest.raises(qoq.QoQError):
         qoq.gemm_plan(0, 6144, 4096, 128)
     with pytest.raises(qoq.QoQError):
@@ -99,11 +105,16 @@ def test_gemm_argument_validation(L):
     assert c(None, FAKE, 48, 0) == qoq.QOQ_ERR_INVALID_ARG     # bad token tile
     assert c(None, FAKE, 16, 9) == qoq.QOQ_ERR_INVALID_ARG     # too many splits
     assert c(None, FAKE, 16, 5) == qoq.QOQ_ERR_INVALID_ARG     # more splits than k-tiles
-    # an explicit split needs its workspace
-    need = qoq.gemm_workspace_bytes(16, 512, 512, 128, 16, 2)
+    # an explicit split through the workspace needs its workspace
+    need = qoq.gemm_workspace_bytes(16, 512, 512, 128, 64, 2)
     assert need > 0
-    assert c(None, FAKE, 16, 2) == qoq.QOQ_ERR_WORKSPACE
-    assert c(None, FAKE, 16, 2, FAKE, need - 16) == qoq.QOQ_ERR_WORKSPACE
+    assert c(None, FAKE, 64, 2) == qoq.QOQ_ERR_WORKSPACE
+    assert c(None, FAKE, 64, 2, FAKE, need - 16) == qoq.QOQ_ERR_WORKSPACE
+    # a split across a cluster needs none (no GPU here: the call gets as far
+    # as its first CUDA call)
+    assert qoq.gemm_workspace_bytes(16, 512, 512, 128, 16, 2) == 0
+    if not _has_gpu():
+        assert c(None, FAKE, 16, 2) == qoq.QOQ_ERR_CUDA
 
 
 def test_auto_plan_workspace_status(L):
@@ -111,9 +122,10 @@ def test_auto_plan_workspace_status(L):
     given but too small is refused before any CUDA call (on a machine without
     a GPU every CUDA call fails, so QOQ_ERR_WORKSPACE here proves that no call
     was made), while ws == NULL asks for an unsplit launch."""
-    M, N, K = 1, 6144, 4096
+    M, N, K = 32, 4096, 14336
     assert qoq.gemm_plan(M, N, K, 128)["splits"] > 1
     need = qoq.gemm_workspace_bytes(M, N, K, 128)
+    assert need > 0
     assert _gemm(L, M=M, N=N, K=K, ws=FAKE, wsb=need - 16) == qoq.QOQ_ERR_WORKSPACE
     assert _gemm(L, M=M, N=N, K=K, ws=FAKE, wsb=0) == qoq.QOQ_ERR_WORKSPACE
     i32 = L.qoq_w4a8_gemm_i32(P(FAKE), P(FAKE), M, N, K, 128, P(FAKE), P(FAKE), need - 16, None)
@@ -166,14 +178,23 @@ def test_other_entry_validation(L):
 
 def test_workspace_sizes(L):
     assert qoq.gemm_workspace_bytes(16, 512, 512, 128, 16, 1) == 0
-    # 16 KiB of counters + partials [m_tiles][splits][tok][N] int32
-    assert qoq.gemm_workspace_bytes(16, 512, 512, 128, 16, 2) == 16384 + 2 * 16 * 512 * 4
-    assert qoq.gemm_workspace_bytes(40, 512, 512, 128, 16, 4) == \
-        16384 + 3 * 4 * 16 * 512 * 4
+    # 16 KiB of counters + partials [m_tiles][splits][tok][N] int32, for
+    # splits through the workspace (token tiles of 64 and more, or more
+    # splits than a cluster of the tile's kernel reduces)
+    assert qoq.gemm_workspace_bytes(16, 512, 512, 128, 64, 2) == 16384 + 2 * 64 * 512 * 4
+    assert qoq.gemm_workspace_bytes(70, 512, 1024, 128, 32, 4) == \
+        16384 + 3 * 4 * 32 * 512 * 4
+    # splits across a cluster reduce in shared memory: no workspace
+    for tok, sp in ((16, 2), (16, 8), (32, 3)):
+        assert qoq.gemm_workspace_bytes(40, 512, 1024, 128, tok, sp) == 0
     assert qoq.gemm_workspace_bytes(0, 512, 512, 128) == 0
+    # the automatic plan of a decode shape splits K across clusters
     p = qoq.gemm_plan(1, 6144, 4096, 128)
-    ws = qoq.gemm_workspace_bytes(1, 6144, 4096, 128)
-    assert (ws > 0) == (p["splits"] > 1)
+    assert p["splits"] > 1 and qoq.gemm_workspace_bytes(1, 6144, 4096, 128) == 0
+    # one whose split goes through the workspace
+    p = qoq.gemm_plan(32, 4096, 14336, 128)
+    assert p["tok_tile"] == 32 and p["splits"] > 3
+    assert qoq.gemm_workspace_bytes(32, 4096, 14336, 128) > 0
 
 
 def _has_gpu():

@@ -356,3 +356,102 @@ def test_model_catches_fewer_stages_than_warpgroups():
         except AssertionError:
             caught += 1
     assert caught > 0
+
+
+class ClusterReductionModel:
+    """The K split across a cluster: per unit, every non-leader CTA's
+    epilogue warp q waits for red_free[q] (its own barrier, phase lt - 1),
+    writes its INT32 slice into the leader's buffer slot and arrives on the
+    leader's red_full[q] (count cs - 1); the leader's warp q waits for
+    red_full[q] (phase lt), adds the slots up and, if a unit follows, arrives
+    on every non-leader's red_free[q].  Checks parity exactness, that no slot
+    is overwritten before the leader consumed it, that the leader reads every
+    slot of the right unit, and that nothing is left pending at the end."""
+
+    def __init__(self, cs, units, seed):
+        self.cs, self.units = cs, units
+        self.rng = random.Random(seed)
+        self.red_full = [Bar(f"red_full{q}", cs - 1) for q in range(4)]
+        self.red_free = {(r, q): Bar(f"red_free{r}.{q}", 1) for r in range(1, cs) for q in range(4)}
+        self.slot = {}          # (r, q) -> unit whose slice the slot holds
+        self.consumed = {}      # (r, q) -> last unit the leader added up
+
+    def non_leader(self, r, q):
+        for lt in range(self.units):
+            if lt > 0:
+                yield ("wait", self.red_free[(r, q)], lt - 1)
+                assert self.consumed.get((r, q)) == lt - 1, "slot overwritten before it was read"
+            self.slot[(r, q)] = lt
+            yield ("yield",)
+            yield ("arrive", self.red_full[q])
+
+    def leader(self, q):
+        for lt in range(self.units):
+            yield ("wait", self.red_full[q], lt)
+            for r in range(1, self.cs):
+                assert self.slot.get((r, q)) == lt, (r, q, lt, self.slot.get((r, q)))
+                self.consumed[(r, q)] = lt
+            yield ("yield",)
+            if lt + 1 < self.units:
+                for r in range(1, self.cs):
+                    yield ("arrive", self.red_free[(r, q)])
+
+    def run(self):
+        gens = {f"L{q}": self.leader(q) for q in range(4)}
+        for r in range(1, self.cs):
+            for q in range(4):
+                gens[f"N{r}.{q}"] = self.non_leader(r, q)
+        waiting = {n: None for n in gens}
+        live = set(gens)
+        for _ in range(1_000_000):
+            if not live:
+                break
+            runnable = [n for n in sorted(live)
+                        if waiting[n] is None or waiting[n][1].try_wait(waiting[n][2])]
+            assert runnable, f"deadlock: {[(n, waiting[n][1].name) for n in live]}"
+            name = self.rng.choice(runnable)
+            waiting[name] = None
+            try:
+                op = next(gens[name])
+            except StopIteration:
+                live.discard(name)
+                continue
+            if op[0] == "wait":
+                waiting[name] = op
+            elif op[0] == "arrive":
+                op[1].arrive()
+        assert not live
+        # every phase a waiter expects completed, none is left half-arrived
+        for q in range(4):
+            assert self.red_full[q].completed == self.units
+            assert self.red_full[q].pending == self.cs - 1
+        for b in self.red_free.values():
+            assert b.completed == self.units - 1 and b.pending == 1
+
+
+@pytest.mark.parametrize("cs", [2, 3, 4, 8])
+def test_cluster_reduction_protocol(cs):
+    for seed in range(60):
+        units = random.Random(seed).randint(1, 7)
+        ClusterReductionModel(cs, units, seed).run()
+
+
+def test_model_catches_a_leader_that_frees_before_reading():
+    class Early(ClusterReductionModel):
+        def leader(self, q):
+            for lt in range(self.units):
+                yield ("wait", self.red_full[q], lt)
+                if lt + 1 < self.units:
+                    for r in range(1, self.cs):
+                        yield ("arrive", self.red_free[(r, q)])
+                yield ("yield",)
+                for r in range(1, self.cs):
+                    assert self.slot.get((r, q)) == lt, "slot overwritten before it was read"
+                    self.consumed[(r, q)] = lt
+    caught = 0
+    for seed in range(200):
+        try:
+            Early(3, 5, seed).run()
+        except AssertionError:
+            caught += 1
+    assert caught > 0

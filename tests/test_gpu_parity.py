@@ -299,6 +299,29 @@ def test_gemm_shapes_random_codes(oracle, group, M, N, K):
     check_y(host(Y), Y_ref)
 
 
+@pytest.mark.parametrize("tok,splits,M", [(16, 2, 5), (16, 3, 16), (16, 5, 1), (16, 8, 9),
+                                           (32, 2, 30), (32, 3, 17)])
+def test_gemm_cluster_split_persistent(oracle, tok, splits, M):
+    """K split across clusters of `splits` CTAs with more output tiles than
+    resident clusters, so every cluster runs several units and the leader's
+    reduction buffer changes hands between units; uneven K ranges (the split
+    count does not divide the k-tiles), group 64 and 128."""
+    for group in (64, 128):
+        N, K = 8192 if splits > 2 else 24576, 1664
+        ops = si.sweep_operands(M, N, K, group, seed=tok * 100 + splits)
+        acc_ref = oracle.int_gemm(ops.X8, oracle.dequant_w(ops.q, ops.s2, ops.z, group))
+        packed = qoq.pack_codes(to_dev(ops.q), to_dev(ops.s2), to_dev(ops.z), group)
+        X8 = to_dev(ops.X8)
+        assert qoq.gemm_workspace_bytes(M, N, K, group, tok, splits) == 0   # no workspace
+        acc = qoq.w4a8_gemm_config(X8, None, packed, None, N, group, tok_tile=tok,
+                                   splits=splits, int32_out=True, ws=None)
+        Y = qoq.w4a8_gemm_config(X8, to_dev(ops.sx), packed, to_dev(ops.s1), N, group,
+                                 tok_tile=tok, splits=splits, ws=None)
+        torch.cuda.synchronize()
+        assert np.array_equal(host(acc), acc_ref), (tok, splits, M, group)
+        check_y(host(Y), oracle.epilogue(acc_ref, ops.sx, ops.s1))
+
+
 def test_gemm_extreme_values(oracle):
     """Large |dq| (120) and the largest |X8| (127) in every term, over K = 8192:
     accumulators of about +-1.25e8 stay exact on every token tile and split."""

@@ -53,8 +53,10 @@ def _check_against_oracle(oracle, ops, y):
     return acc_ref
 
 
-# (M, N, K): decode shapes that split K (largest scratch last) and one that does not
-SHAPES = [(1, 6144, 4096), (16, 4096, 14336), (256, 6144, 4096), (16, 24576, 8192)]
+# (M, N, K): shapes whose plan splits K through the scratch (largest scratch
+# last), one split across a cluster (no scratch) and one not split at all
+SCRATCH_SHAPES = [(32, 4096, 14336), (24, 2048, 8192), (32, 4096, 24576)]
+SHAPES = SCRATCH_SHAPES + [(1, 6144, 4096), (256, 6144, 4096)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES, ids=[f"M{m}_N{n}_K{k}" for m, n, k in SHAPES])
@@ -62,8 +64,8 @@ def test_static_ws_matches_workspace_entry(oracle, M, N, K):
     ops, (X8, sx, packed, s1) = _operands(M, N, K, seed=M + N + K)
     need = qoq.gemm_workspace_bytes(M, N, K, GROUP)
     assert need <= STATIC_WS_BYTES
-    if M != 256:
-        assert qoq.gemm_plan(M, N, K, GROUP)["splits"] > 1   # the fixed array is used
+    if (M, N, K) in SCRATCH_SHAPES:
+        assert need > 0                                      # the fixed array is used
     qoq.device_error(clear=True)
     y_ref = qoq.w4a8_gemm(X8, sx, packed, s1, N, GROUP)
     acc = qoq.w4a8_gemm_i32(X8, packed, N, GROUP)
@@ -80,14 +82,14 @@ def test_static_ws_matches_workspace_entry(oracle, M, N, K):
 def test_static_ws_back_to_back_shapes(oracle):
     """Consecutive calls with different shapes reuse the array's contents
     from the call before; each result must still be exact."""
-    oa, a = _operands(1, 6144, 4096, seed=7)      # K split
-    ob, b = _operands(16, 4096, 14336, seed=8)    # K split
-    assert qoq.gemm_plan(1, 6144, 4096, GROUP)["splits"] > 1
-    assert qoq.gemm_plan(16, 4096, 14336, GROUP)["splits"] > 1
+    oa, a = _operands(24, 2048, 8192, seed=7)     # K split through the scratch
+    ob, b = _operands(32, 4096, 14336, seed=8)    # K split through the scratch
+    assert qoq.gemm_workspace_bytes(24, 2048, 8192, GROUP) > 0
+    assert qoq.gemm_workspace_bytes(32, 4096, 14336, GROUP) > 0
     qoq.device_error(clear=True)
-    refs = [qoq.w4a8_gemm(*a, 6144, GROUP), qoq.w4a8_gemm(*b, 4096, GROUP)]
-    outs = [qoq.w4a8_gemm_static_ws(*a, 6144, GROUP), qoq.w4a8_gemm_static_ws(*b, 4096, GROUP),
-            qoq.w4a8_gemm_static_ws(*a, 6144, GROUP)]
+    refs = [qoq.w4a8_gemm(*a, 2048, GROUP), qoq.w4a8_gemm(*b, 4096, GROUP)]
+    outs = [qoq.w4a8_gemm_static_ws(*a, 2048, GROUP), qoq.w4a8_gemm_static_ws(*b, 4096, GROUP),
+            qoq.w4a8_gemm_static_ws(*a, 2048, GROUP)]
     torch.cuda.synchronize()
     assert qoq.device_error(clear=True) == 0
     assert torch.equal(outs[0], refs[0])
@@ -101,8 +103,8 @@ def test_static_ws_rejected_call_enqueues_nothing():
     """A misaligned pointer is refused before anything reaches the stream:
     captured into a CUDA graph, the refused call leaves the graph empty."""
     from cuda.bindings import runtime as cudart
-    _, (X8, sx, packed, s1) = _operands(1, 6144, 4096, seed=9)
-    Y = torch.empty((1, 6144), dtype=torch.float16, device=DEV)
+    _, (X8, sx, packed, s1) = _operands(32, 4096, 14336, seed=9)
+    Y = torch.empty((32, 4096), dtype=torch.float16, device=DEV)
     L = qoq.lib()
     P = ctypes.c_void_p
     stream = torch.cuda.Stream(device=DEV)
@@ -111,7 +113,7 @@ def test_static_ws_rejected_call_enqueues_nothing():
         stream.cuda_stream, cudart.cudaStreamCaptureMode.cudaStreamCaptureModeRelaxed)
     assert err == cudart.cudaError_t.cudaSuccess
     st = L.qoq_w4a8_gemm_static_ws(P(X8.data_ptr() + 8), P(sx.data_ptr()), P(packed.data_ptr()),
-                                   P(s1.data_ptr()), 1, 6144, 4096, GROUP, P(Y.data_ptr()),
+                                   P(s1.data_ptr()), 32, 4096, 14336, GROUP, P(Y.data_ptr()),
                                    P(stream.cuda_stream))
     err, graph = cudart.cudaStreamEndCapture(stream.cuda_stream)
     assert err == cudart.cudaError_t.cudaSuccess

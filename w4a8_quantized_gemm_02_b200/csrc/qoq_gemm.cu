@@ -44,6 +44,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "qoq.h"
@@ -67,7 +68,7 @@ constexpr int kSlicesPerTile = 4;
 constexpr int kMaxCounterTiles = 1024;
 constexpr size_t kCounterBytes = kMaxCounterTiles * kSlicesPerTile * 4;
 
-template <int TOK>
+template <int TOK, bool kCluster = false>
 struct Cfg {
   // One ring of kStages stages.  A stage covers kNB consecutive k-tiles of
   // 128 (the last stage of a unit may cover fewer): their X8 tiles and packed
@@ -114,9 +115,19 @@ struct Cfg {
   static constexpr int kOffEpi = kOffRaw + kWStages * kStageRaw;
   static constexpr int kOffSx = kOffEpi + 4 * kStageBytesEpi;          // 4 warps x TOK floats
   static constexpr int kOffBar = kOffSx + 4 * TOK * 4;
-  static constexpr int kNumBars = 3 * kStages + 2 * kWStages + 2 * kAcc + 1;
+  // The kernel variant that splits K across a cluster (token tiles up to 32)
+  // has eight more barriers and the leader CTA's reduction buffer, which
+  // receives the INT32 partial tiles of the other CTAs:
+  // [slot = rank - 1][epilogue warp][token][32 channels].
+  static constexpr int kRedBars = kCluster ? 8 : 0;
+  static constexpr int kNumBars = 3 * kStages + 2 * kWStages + 2 * kAcc + 1 + kRedBars;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
-  static constexpr int kSmemBytes = kOffMisc + 32 + 1024;   // + base alignment slack
+  static constexpr int kMaxClusterSplit = !kCluster ? 1 : TOK <= 16 ? 8 : TOK <= 32 ? 3 : 1;
+  static constexpr int kRedSlotBytes = kTileN * TOK * 4;
+  static constexpr int kOffRed = kCluster ? ((kOffMisc + 32 + 127) / 128) * 128 : kOffMisc + 32;
+  static constexpr int kSmemBytes =
+      kOffRed + (kMaxClusterSplit - 1) * kRedSlotBytes + 1024;   // + base alignment slack
+  static_assert(!kCluster || TOK <= 32, "K split across a cluster for token tiles up to 32");
   static_assert(kOffRaw % 1024 == 0 && kXBytes % 1024 == 0, "swizzled tiles need 1 KiB alignment");
   static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
@@ -145,6 +156,9 @@ struct GemmArgs {
   float rcp_mtiles;
   int w_dep_wait;       // the weight producer waits for the preceding grid (it may
                         // have written the weights) before its first copy
+  int cs;               // K split across a cluster of cs CTAs (1: none); then
+                        // splits == cs and the split partials never leave the
+                        // cluster (no workspace)
 };
 
 struct Unit {
@@ -326,10 +340,10 @@ struct WeightStream {
   }
 };
 
-template <int TOK>
+template <int TOK, bool kCluster>
 __global__ void __launch_bounds__(Cfg<TOK>::kThreads, 1)
 w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args) {
-  using C = Cfg<TOK>;
+  using C = Cfg<TOK, kCluster>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -359,6 +373,14 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   const uint32_t bar_accfull = bar_wempty + 8 * SW;
   const uint32_t bar_accempty = bar_accfull + 8 * C::kAcc;
   const uint32_t bar_drain = bar_accempty + 8 * C::kAcc;
+  // K split across a cluster: red_full[q] (leader CTA) counts the other
+  // CTAs' partial slices of epilogue warp q; red_free[q] (every other CTA)
+  // completes when the leader has added them up and the buffer may be
+  // written again.
+  const uint32_t bar_red_full = bar_drain + 8;
+  const uint32_t bar_red_free = bar_red_full + 8 * 4;
+  const int cs = kCluster ? args.cs : 1;
+  const uint32_t crank = cs > 1 ? cluster_ctarank() : 0u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc + 4);
 
@@ -368,12 +390,16 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     // dqfull, wempty and accempty count the four warps of a warpgroup; the
     // lanes of warp 0 initialize all but the weight ring's, which the weight
     // producer initializes itself
-    for (int i = lane; i < C::kNumBars; i += 32) {
+    for (int i = lane; i < C::kNumBars - C::kRedBars; i += 32) {
       const int acc0 = 3 * S + 2 * SW;
       if (i >= 3 * S && i < acc0) continue;
       const bool four = (i >= 2 * S && i < 3 * S) ||
                         (i >= acc0 + C::kAcc && i < acc0 + 2 * C::kAcc);
       mbar_init(bar_xfull + 8 * i, four ? 4u : 1u);
+    }
+    if (kCluster) {
+      if (lane < 4) mbar_init(bar_red_full + 8 * lane, cs > 1 ? static_cast<uint32_t>(cs - 1) : 1u);
+      else if (lane < 8) mbar_init(bar_red_free + 8 * (lane - 4), 1u);
     }
     if (lane == 0) {
       *abort_flag = 0u;
@@ -400,6 +426,9 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   }
   tc_fence_before_sync();
   __syncthreads();
+  // the leader's reduction barriers must be initialized before another CTA
+  // of the cluster arrives on them
+  if (cs > 1) cluster_sync_all();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
@@ -616,7 +645,38 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
       const uint32_t t_acc = tmem + C::kTmemD + b * TOK + (static_cast<uint32_t>(q4 * 32) << 16);
       const int splits = args.splits;
       bool write_out = true;
-      if (splits > 1) {
+      bool red_ok = true;
+      if (cs > 1 && crank != 0) {
+        // K split across the cluster, not the leader: once the leader has
+        // added up the previous unit's slices, write this warp's INT32 slice
+        // into the leader's reduction buffer and arrive on its barrier
+        if (lt > 0) red_ok = mbar_wait_cluster(bar_red_free + 8 * q4, (lt - 1) & 1, abort_flag,
+                                                &g_error_word, kErrEpilogue);
+        red_ok = __all_sync(0xffffffffu, red_ok);
+        if (red_ok) {
+          const uint32_t dst = map_to_rank(
+              base + C::kOffRed + ((crank - 1) * 4 + q4) * (TOK * 128), 0u) + lane * 4;
+          for (int c0 = 0; c0 < c_end; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(t_acc + c0, v);
+            tmem_ld_wait(v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (c0 + j < c_end) st_cluster_u32(dst + (c0 + j) * 128, v[j]);
+          }
+          // every lane's stores are ordered before lane 0's release
+          asm volatile("fence.acq_rel.cluster;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(map_to_rank(bar_red_full + 8 * q4, 0u));
+        }
+        write_out = false;
+      } else if (cs > 1) {
+        // the leader: wait for the other CTAs' slices of this unit
+        red_ok = __all_sync(0xffffffffu, mbar_wait_cluster(bar_red_full + 8 * q4, lt & 1,
+                                                           abort_flag, &g_error_word,
+                                                           kErrEpilogue));
+        if (!red_ok) write_out = false;
+      } else if (splits > 1) {
         // publish this unit's partial tile (INT32, [token][channel]) ...
         int32_t* part = args.ws_part + (static_cast<size_t>(w.mt * splits + w.split) * TOK) * N;
         for (int c0 = 0; c0 < c_end; c0 += 16) {
@@ -661,7 +721,16 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] = vn[j];
           if (c0 + 16 < c_end) tmem_ld_32x32b_x16(t_acc + c0 + 16, vn);
-          if (splits > 1) {
+          if (cs > 1) {
+            // add the cluster's slices from this CTA's reduction buffer
+            for (int q = 0; q < cs - 1; ++q) {
+              const uint32_t* rp = reinterpret_cast<const uint32_t*>(
+                  smem + C::kOffRed + (q * 4 + q4) * (TOK * 128) + lane * 4);
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                if (c0 + j < c_end) v[j] += rp[(c0 + j) * 32];
+            }
+          } else if (splits > 1) {
             for (int q = 0; q < splits; ++q) {
               if (q == w.split) continue;
               const int32_t* p = parts + (static_cast<size_t>(q) * TOK + c0) * N + nrow0 + lane;
@@ -702,6 +771,14 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
           __syncwarp();
         }
       }
+      if (cs > 1 && crank == 0 && red_ok && u + static_cast<int>(gridDim.x) < args.units) {
+        // the slices are added up: the other CTAs may write the next unit's
+        __syncwarp();
+        if (lane == 0)
+          for (int r = 1; r < cs; ++r)
+            mbar_arrive_remote(map_to_rank(bar_red_free + 8 * q4, static_cast<uint32_t>(r)));
+      }
+      if (!red_ok) break;
       // the accumulator may be overwritten by the unit after next
       tc_fence_before_sync();
       __syncwarp();
@@ -722,6 +799,9 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   // ------------------------------------------------------------------ teardown
   tc_fence_before_sync();
   __syncthreads();
+  // no CTA of the cluster leaves while another may still access its shared
+  // memory (every thread of every CTA reaches this point on every path)
+  if (cs > 1) cluster_sync_all();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after_sync();
@@ -753,7 +833,70 @@ EncodeTiledFn encode_fn() {
 
 struct Plan {
   int tok, splits, m_tiles, n_tiles, stages, units, grid;
+  int cs;   // K split across a cluster of cs CTAs (1: split through the workspace, or none)
 };
+
+// Largest K split a cluster can reduce in the leader's shared memory.
+int max_cluster_split(int tok) { return tok <= 16 ? 8 : tok <= 32 ? 3 : 1; }
+
+template <int TOK, bool kCluster>
+__global__ void __launch_bounds__(Cfg<TOK>::kThreads, 1)
+w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args);
+
+template <int TOK>
+int query_active_clusters(int cs) {
+  using C = Cfg<TOK, true>;
+  if (cudaFuncSetAttribute(w4a8_gemm_kernel<TOK, true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(w4a8_gemm_kernel<TOK, true>,
+                           cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(cs * 64), 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(cs);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, w4a8_gemm_kernel<TOK, true>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+// Clusters of cs CTAs of the `tok` kernel that can be resident at once on the
+// current device (one CTA per SM), cached per device; without a device (or
+// if the query fails) the SM count divided by cs.
+int active_clusters(int tok, int cs) {
+  const int sms = sm_count();
+  if (cs <= 1) return sms;
+  constexpr int kDev = 16;
+  static std::atomic<int> cache[kDev][2][9];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return sms / cs;
+  }
+  const int ti = tok <= 16 ? 0 : 1;
+  if (dev >= 0 && dev < kDev) {
+    const int v = cache[dev][ti][cs].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+  }
+  int n = tok <= 16 ? query_active_clusters<16>(cs) : query_active_clusters<32>(cs);
+  if (n <= 0) n = sms / cs;
+  if (n > sms / cs) n = sms / cs;
+  if (dev >= 0 && dev < kDev) cache[dev][ti][cs].store(n, std::memory_order_relaxed);
+  return n;
+}
 
 bool splittable(const Plan& p) {
   return static_cast<long>(p.m_tiles) * p.n_tiles <= kMaxCounterTiles;   // one counter per slice
@@ -796,29 +939,40 @@ int auto_tok(int M, int n_tiles) {
   return best;
 }
 
-// Cost model for the number of K splits: units are spread over one CTA per
-// SM, a unit costs its k-tiles plus a fixed overhead (pipeline fill and
-// epilogue), a split unit a little more (partial tile out, final sum in).
-// Only small token tiles are split.  The split tail (partial slices written,
-// the last arrival reads the others back) grows with the tokens in the tile:
-// on B200 a 16-token Llama QKV tile (32 k-tiles) ran fastest unsplit, while
-// single tokens, or 64+ k-tiles per unit, gained from splitting.
-int auto_splits(int tiles, int kt, int tok, int M) {
+// Cost model for the number of K splits of a decode plan: units are spread
+// over the CTAs, a unit costs its k-tiles plus a fixed overhead (pipeline
+// fill and epilogue), a split unit a little more.  Up to max_cluster_split
+// splits the partial tiles are added up inside a cluster (through the leader
+// CTA's shared memory); more splits go through the workspace in L2, whose
+// tail (partial slices written, the last arrival reading the others back)
+// grows with the tokens in the tile: on B200 a 16-token Llama QKV tile (32
+// k-tiles) ran fastest unsplit that way, while single tokens, or 64+ k-tiles
+// per unit, gained from splitting.
+int auto_splits(int tiles, int kt, int tok, int M, bool* cluster_out) {
+  *cluster_out = false;
   if (tok > 32) return 1;
-  if ((M < tok ? M : tok) > 4 && kt < 64) return 1;
+  const int tokens = M < tok ? M : tok;
+  // measured on B200: with up to four tokens the workspace split is the
+  // faster of the two (its tail is short, and a cluster waits for all of
+  // its SMs to be free); with more tokens the cluster split is
+  const bool cluster_ok = tokens > 4;
+  const bool l2_ok = tokens <= 4 || kt >= 64;
   const long sms = sm_count();
   int best_s = 1;
   double best = 1e30;
   for (int s = 1; s <= 8 && s <= kt; ++s) {
     if (s > 1 && kt / s < 2) break;
-    if (static_cast<long>(tiles) * s > 4L * sms && s > 1) break;
+    const bool cluster = s > 1 && cluster_ok && s <= max_cluster_split(tok);
+    if (s > 1 && !cluster && (!l2_ok || static_cast<long>(tiles) * s > 4L * sms)) continue;
+    const long slots = cluster ? static_cast<long>(active_clusters(tok, s)) * s : sms;
     const long units = static_cast<long>(tiles) * s;
-    const long rounds = (units + sms - 1) / sms;
-    const double cost =
-        static_cast<double>(rounds) * (static_cast<double>(kt) / s + 3.0 + (s > 1 ? 2.0 : 0.0));
+    const long rounds = (units + slots - 1) / slots;
+    const double ovh = s == 1 ? 0.0 : cluster ? 1.0 : 2.0;
+    const double cost = static_cast<double>(rounds) * (static_cast<double>(kt) / s + 3.0 + ovh);
     if (cost < best - 1e-9) {
       best = cost;
       best_s = s;
+      *cluster_out = cluster;
     }
   }
   return best_s;
@@ -827,7 +981,14 @@ int auto_splits(int tiles, int kt, int tok, int M) {
 void finish_plan(Plan& p) {
   p.units = p.n_tiles * p.m_tiles * p.splits;
   const int sms = sm_count();
-  p.grid = p.units < sms ? p.units : sms;
+  if (p.cs > 1) {
+    // whole clusters, each taking the splits of one output tile
+    const int tiles = p.n_tiles * p.m_tiles;
+    const int ncl = active_clusters(p.tok, p.cs);
+    p.grid = (tiles < ncl ? tiles : ncl) * p.cs;
+  } else {
+    p.grid = p.units < sms ? p.units : sms;
+  }
 }
 
 Plan make_plan(int M, int N, int K, int tok_req, int splits_req) {
@@ -837,28 +998,37 @@ Plan make_plan(int M, int N, int K, int tok_req, int splits_req) {
   p.tok = tok_req ? tok_req : auto_tok(M, p.n_tiles);
   p.m_tiles = (M + p.tok - 1) / p.tok;
   p.stages = stages_for(p.tok);
-  p.splits = splits_req ? splits_req : auto_splits(p.n_tiles * p.m_tiles, kt, p.tok, M);
-  if (!splits_req && !splittable(p)) p.splits = 1;
+  if (splits_req) {
+    // an explicit split runs on a cluster whenever the tile's kernel can
+    // reduce it there
+    p.splits = splits_req;
+    p.cs = (p.splits > 1 && p.splits <= max_cluster_split(p.tok)) ? p.splits : 1;
+  } else {
+    bool cluster = false;
+    p.splits = auto_splits(p.n_tiles * p.m_tiles, kt, p.tok, M, &cluster);
+    p.cs = cluster ? p.splits : 1;
+  }
+  if (!splits_req && p.cs == 1 && !splittable(p)) p.splits = 1;
   finish_plan(p);
   return p;
 }
 
 size_t ws_bytes_for(const Plan& p, int N) {
-  if (p.splits <= 1) return 0;
+  if (p.splits <= 1 || p.cs > 1) return 0;   // a cluster split needs no workspace
   const size_t part = static_cast<size_t>(p.m_tiles) * p.splits * p.tok * N * 4;
   return kCounterBytes + part;
 }
 
-template <int TOK>
-int launch_tok(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cudaStream_t stream,
+template <int TOK, bool kCluster>
+int launch_kernel(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cudaStream_t stream,
                bool pdl) {
-  using C = Cfg<TOK>;
+  using C = Cfg<TOK, kCluster>;
   static int configured_mask = 0;   // one bit per device id < 31
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return QOQ_ERR_CUDA;
   const int bit = dev < 31 ? (1 << dev) : 0;
   if (!bit || !(__atomic_load_n(&configured_mask, __ATOMIC_ACQUIRE) & bit)) {
-    if (cudaFuncSetAttribute(w4a8_gemm_kernel<TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(w4a8_gemm_kernel<TOK, kCluster>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess)
       return QOQ_ERR_CUDA;
     if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_RELEASE);
@@ -868,13 +1038,35 @@ int launch_tok(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cudaStr
   cfg.blockDim = dim3(C::kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (p.cs > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = static_cast<unsigned>(p.cs);
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  if (cudaLaunchKernelEx(&cfg, w4a8_gemm_kernel<TOK>, map, a) != cudaSuccess) return QOQ_ERR_CUDA;
+  cfg.numAttrs = na;
+  if (cudaLaunchKernelEx(&cfg, w4a8_gemm_kernel<TOK, kCluster>, map, a) != cudaSuccess) return QOQ_ERR_CUDA;
   return QOQ_OK;
+}
+
+// The cluster variant of the kernel for token tiles up to 32 when the plan
+// splits K across a cluster, the plain one otherwise.
+template <int TOK>
+int launch_tok(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cudaStream_t stream,
+               bool pdl) {
+  if constexpr (TOK <= 32) {
+    if (p.cs > 1) return launch_kernel<TOK, true>(map, a, p, stream, pdl);
+  }
+  return launch_kernel<TOK, false>(map, a, p, stream, pdl);
 }
 
 // Everything one GEMM launch needs, built and checked before anything is
@@ -905,11 +1097,11 @@ int gemm_prepare(const int8_t* X8, const void* sx, const void* packed, const voi
   Plan p = make_plan(M, N, K, tok_req, splits_req);
   // the kernel divides unit indices below 2^22 by multiplication (small_div)
   if (static_cast<long>(p.n_tiles) * p.m_tiles * p.splits >= (1L << 22)) return QOQ_ERR_UNSUPPORTED;
-  if (p.splits > 1 && !splittable(p)) {
+  if (p.splits > 1 && p.cs == 1 && !splittable(p)) {
     if (splits_req) return QOQ_ERR_UNSUPPORTED;
     p.splits = 1;
   }
-  if (p.splits > 1 && (ws == nullptr || ws_bytes < ws_bytes_for(p, N))) {
+  if (p.splits > 1 && p.cs == 1 && (ws == nullptr || ws_bytes < ws_bytes_for(p, N))) {
     // an explicit split needs its workspace; so does the automatic plan,
     // unless the caller passed none (an explicit request not to split K)
     if (splits_req || ws != nullptr) return QOQ_ERR_WORKSPACE;
@@ -937,10 +1129,11 @@ int gemm_prepare(const int8_t* X8, const void* sx, const void* packed, const voi
   a.acc = acc;
   a.ws_part = nullptr;
   a.ws_count = nullptr;
-  if (p.splits > 1) {
+  if (p.splits > 1 && p.cs == 1) {
     a.ws_count = static_cast<uint32_t*>(ws);
     a.ws_part = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kCounterBytes);
   }
+  a.cs = p.cs;
   a.M = M;
   a.N = N;
   a.K = K;
@@ -968,7 +1161,7 @@ int gemm_launch(GemmLaunch L, void* stream, bool weights_independent, bool clear
   cudaStream_t s = as_stream(stream);
   const bool pdl = true;
   L.a.w_dep_wait = weights_independent ? 0 : 1;
-  if (clear_counters && L.p.splits > 1 &&
+  if (clear_counters && L.a.ws_count != nullptr &&
       cudaMemsetAsync(L.a.ws_count, 0, kCounterBytes, s) != cudaSuccess)
     return QOQ_ERR_CUDA;
   switch (L.p.tok) {
@@ -981,6 +1174,7 @@ int gemm_launch(GemmLaunch L, void* stream, bool weights_independent, bool clear
     default: return launch_tok<256>(L.map, L.a, L.p, s, pdl);
   }
 }
+
 
 }  // namespace
 
