@@ -407,6 +407,22 @@ def layer_per_m(qoq, torch, layer, dev, stream, l2, peaks, int8_peak, packed0=No
         lin_us = graph_us_per_launch(torch, stream, ln)
         extra = {"act_quant_us": aq_us, "linear_us": lin_us,
                  "linear_tops": gemm_ops(M, N, K) / lin_us / 1e6}
+        # the one-kernel linear (activations quantized inside the GEMM), where
+        # it applies (a few decode rows)
+        try:
+            with torch.cuda.stream(stream):
+                qoq.w4a8_linear_fused(xs[0], weights[0], s1s[0], N, G, out=y, scratch=(x8, sx),
+                                      stream=stream)
+            stream.synchronize()
+
+            def lf():
+                for w in range(nw):
+                    qoq.w4a8_linear_fused(xs[w % nx], weights[w], s1s[w], N, G, out=y,
+                                          scratch=(x8, sx), stream=stream)
+                return nw
+            extra["linear_fused_us"] = graph_us_per_launch(torch, stream, lf)
+        except qoq.QoQError:
+            pass
         if isolated:
             times = []
             for i in range(5):

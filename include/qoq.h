@@ -284,16 +284,36 @@ QOQ_API int qoq_w4a8_gemm_config(const int8_t* X8, const void* sx, const void* p
  *            calls on the same stream).
  *   Y      : device, FP16 M x N row-major, written.
  *   ws, ws_bytes : as for qoq_w4a8_gemm.
- * Same results as qoq_quantize_act_per_token followed by qoq_w4a8_gemm; here
- * the GEMM is launched as a programmatic dependent of the quantizer, so it
- * starts streaming weights while the activations are still being quantized.
- * For M <= 2 x SMs the quantizer is itself launched as a programmatic
- * dependent of whatever kernel precedes it on `stream`: it may be scheduled
- * while that kernel drains, but touches no memory before that kernel has
- * completed.  Asynchronous on `stream`. */
+ * Same results (X8, sx and Y, bit for bit) as qoq_quantize_act_per_token
+ * followed by qoq_w4a8_gemm.  Here the GEMM is launched as a programmatic
+ * dependent of the quantizer, so it starts streaming weights while the
+ * activations are still being quantized.  For M <= 2 x SMs the quantizer is
+ * itself launched as a programmatic dependent of whatever kernel precedes
+ * it on `stream`: it may be scheduled while that kernel drains, but touches
+ * no memory before that kernel has completed.
+ * Asynchronous on `stream`. */
 QOQ_API int qoq_w4a8_linear(const void* X, int M, int K, const void* packed, const void* s1,
                             int N, int group, int8_t* X8, void* sx, void* Y, void* ws,
                             size_t ws_bytes, void* stream);
+
+/* qoq_w4a8_linear as one kernel, for a few decode rows: the activation
+ * quantizer fused into the GEMM ("Part5 LLM部署技术", 3. 实践扩展：QServe
+ * （W4A8KV4）, kernel fusion).  Same arguments and the same results (X8, sx
+ * and Y, bit for bit) as qoq_w4a8_linear.  Every CTA copies the FP16 rows
+ * into its shared memory, computes each row's scale with the arithmetic of
+ * qoq_quantize_act_per_token, writes all of X8 (every CTA writes the same
+ * bytes; CTA 0 writes sx) and then runs the GEMM on it.
+ *   - Applies when the rows fit 48 KiB (M * K * 2 <= 49152) and the GEMM's
+ *     plan takes 16-token tiles without a cluster split (up to four rows);
+ *     otherwise QOQ_ERR_UNSUPPORTED and nothing is launched.
+ *   - Measured on B200 in back-to-back decode it is slower than
+ *     qoq_w4a8_linear's two kernels (the quantizer overlaps the GEMM's start,
+ *     while here the rows are quantized inside the GEMM before its first
+ *     MMA), so qoq_w4a8_linear does not use it.
+ * Asynchronous on `stream`. */
+QOQ_API int qoq_w4a8_linear_fused(const void* X, int M, int K, const void* packed,
+                                  const void* s1, int N, int group, int8_t* X8, void* sx,
+                                  void* Y, void* ws, size_t ws_bytes, void* stream);
 
 /* The launch configuration qoq_w4a8_gemm picks for a shape: token tile,
  * K splits, CTAs in the grid and pipeline stages.  Host only: no CUDA call
@@ -312,7 +332,8 @@ QOQ_API int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int* sp
  * current device and, if `clear` is non-zero, resets it to 0.
  * Bits: 1 = producer wait, 2 = MMA wait, 4 = dequantizer wait,
  *       8 = epilogue wait, 16 = split-K arrival counter,
- *       64 = qoq_selftest_wait_timeout.
+ *       64 = qoq_selftest_wait_timeout, 128 = a GEMM kernel launched with
+ *       less shared memory than its layout needs (it did nothing).
  * ---------------------------------------------------------------------- */
 QOQ_API int qoq_device_error(unsigned int* value, int clear);
 

@@ -138,6 +138,20 @@ def test_auto_plan_workspace_status(L):
         assert _gemm(L, M=M, N=N, K=K, ws=FAKE, wsb=need) == qoq.QOQ_ERR_CUDA
 
 
+def test_fused_linear_rejects_rows_that_do_not_fit(L):
+    """The one-kernel linear takes rows of at most 48 KiB; larger ones are
+    refused before any CUDA call."""
+    f = L.qoq_w4a8_linear_fused
+    args = lambda M, K: (P(FAKE), M, K, P(FAKE), P(FAKE), 6144, 128, P(FAKE), P(FAKE), P(FAKE),
+                         None, 0, None)
+    assert f(*args(7, 4096)) == qoq.QOQ_ERR_UNSUPPORTED
+    assert f(*args(2, 14336)) == qoq.QOQ_ERR_UNSUPPORTED
+    assert f(None, 1, 4096, P(FAKE), P(FAKE), 6144, 128, P(FAKE), P(FAKE), P(FAKE), None, 0,
+             None) == qoq.QOQ_ERR_INVALID_ARG
+    if not _has_gpu():
+        assert f(*args(1, 4096)) == qoq.QOQ_ERR_CUDA
+
+
 def _static(L, X8=FAKE, sx=FAKE, packed=FAKE, s1=FAKE, M=1, N=6144, K=4096, G=128, Y=FAKE):
     return L.qoq_w4a8_gemm_static_ws(P(X8), P(sx), P(packed), P(s1), M, N, K, G, P(Y), None)
 
@@ -188,9 +202,12 @@ def test_workspace_sizes(L):
     for tok, sp in ((16, 2), (16, 8), (32, 3)):
         assert qoq.gemm_workspace_bytes(40, 512, 1024, 128, tok, sp) == 0
     assert qoq.gemm_workspace_bytes(0, 512, 512, 128) == 0
-    # the automatic plan of a decode shape splits K across clusters
+    # the automatic plan splits K through the workspace for up to four
+    # tokens and across clusters for more
     p = qoq.gemm_plan(1, 6144, 4096, 128)
-    assert p["splits"] > 1 and qoq.gemm_workspace_bytes(1, 6144, 4096, 128) == 0
+    assert p["splits"] > 1 and qoq.gemm_workspace_bytes(1, 6144, 4096, 128) > 0
+    p = qoq.gemm_plan(16, 6144, 4096, 128)
+    assert p["splits"] > 1 and qoq.gemm_workspace_bytes(16, 6144, 4096, 128) == 0
     # one whose split goes through the workspace
     p = qoq.gemm_plan(32, 4096, 14336, 128)
     assert p["tok_tile"] == 32 and p["splits"] > 3

@@ -32,7 +32,7 @@ EXPORTS = (
     "qoq_quantize_act_per_token", "qoq_w4a8_gemm", "qoq_w4a8_gemm_i32",
     "qoq_w4a8_gemm_config", "qoq_w4a8_linear", "qoq_gemm_plan", "qoq_device_error",
     "qoq_gemm_workspace_bytes", "qoq_gemm_workspace_bytes_config",
-    "qoq_w4a8_gemm_static_ws", "qoq_selftest_wait_timeout",
+    "qoq_w4a8_gemm_static_ws", "qoq_selftest_wait_timeout", "qoq_w4a8_linear_fused",
 )
 
 _lock = threading.Lock()
@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
             L.qoq_w4a8_gemm_config.argtypes = [P, P, P, P, I, I, I, I, P, P, I, I, P, sz, P]
             L.qoq_w4a8_linear.restype = I
             L.qoq_w4a8_linear.argtypes = [P, I, I, P, P, I, I, P, P, P, P, sz, P]
+            L.qoq_w4a8_linear_fused.restype = I
+            L.qoq_w4a8_linear_fused.argtypes = [P, I, I, P, P, I, I, P, P, P, P, sz, P]
             L.qoq_gemm_workspace_bytes.restype = sz
             L.qoq_gemm_workspace_bytes.argtypes = [I, I, I, I]
             L.qoq_gemm_workspace_bytes_config.restype = sz
@@ -392,7 +394,8 @@ def w4a8_gemm_config(X8, sx, packed, s1, N: int, group: int = 128, *, tok_tile=0
 def w4a8_linear(X, packed, s1, N: int, group: int = 128, out=None, scratch=None, ws=_AUTO,
                 stream=None):
     """Y = X . W^T: per-token activation quantization + W4A8 GEMM in one call
-    (the GEMM overlaps the quantizer's tail).  ``scratch`` = (X8, sx)."""
+    (the GEMM overlaps the quantizer's tail).  ``scratch`` = (X8, sx),
+    written."""
     import torch
     _need_cuda(X, "X", torch.float16, 2)
     M, K = X.shape
@@ -410,6 +413,32 @@ def w4a8_linear(X, packed, s1, N: int, group: int = 128, out=None, scratch=None,
     w, wb = _ws_args(_auto_ws(ws, M, N, K, group, dev, stream=stream))
     _check(lib().qoq_w4a8_linear(_ptr(X), M, K, _ptr(packed), _ptr(s1), N, group, _ptr(X8),
                                  _ptr(sx), _ptr(Y), w, wb, _stream(stream)), "qoq_w4a8_linear")
+    return Y
+
+
+def w4a8_linear_fused(X, packed, s1, N: int, group: int = 128, out=None, scratch=None,
+                      ws=_AUTO, stream=None):
+    """w4a8_linear as one kernel that quantizes its own activations (a few
+    decode rows: M * K * 2 <= 49152 and a 16-token plan without a cluster
+    split; else QoQError, unsupported)."""
+    import torch
+    _need_cuda(X, "X", torch.float16, 2)
+    M, K = X.shape
+    dev = X.device
+    _need_cuda(s1, "s1", torch.float16, shape=(N,), device=dev)
+    _need_packed(packed, N, K, group, dev)
+    if scratch is None:
+        X8 = torch.empty((M, K), dtype=torch.int8, device=dev)
+        sx = torch.empty(M, dtype=torch.float16, device=dev)
+    else:
+        X8, sx = scratch
+        _need_cuda(X8, "X8", torch.int8, shape=(M, K), device=dev)
+        _need_cuda(sx, "sx", torch.float16, shape=(M,), device=dev)
+    Y = _out(out, (M, N), torch.float16, dev)
+    w, wb = _ws_args(_auto_ws(ws, M, N, K, group, dev, stream=stream))
+    _check(lib().qoq_w4a8_linear_fused(_ptr(X), M, K, _ptr(packed), _ptr(s1), N, group,
+                                       _ptr(X8), _ptr(sx), _ptr(Y), w, wb, _stream(stream)),
+           "qoq_w4a8_linear_fused")
     return Y
 
 

@@ -18,6 +18,7 @@ enum : uint32_t {
   kErrEpilogue = 8u,
   kErrCounter = 16u,
   kErrSelfTest = 64u,
+  kErrLaunch = 128u,
 };
 
 // Every mbarrier wait gives up after this many SM clock cycles (about two
@@ -30,6 +31,13 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 }
 
 __device__ __forceinline__ long long sm_clock() { return clock64(); }
+
+// Dynamic shared memory the running CTA was launched with.
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+  uint32_t v;
+  asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(v));
+  return v;
+}
 
 // True in exactly one lane of the (converged) calling warp.
 __device__ __forceinline__ bool elect_one() {
@@ -213,6 +221,16 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
+// The same bulk copy with the default L2 policy.
+__device__ __forceinline__ void bulk_load_plain(uint32_t dst, const void* src, uint32_t bytes,
+                                                uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x,
                                             int y, uint32_t bar) {
   asm volatile(
@@ -230,6 +248,12 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
 // (tensor cores, TMA) after this fence.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// The same for global memory: ordinary stores, then tensor copies that read
+// the same bytes.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // ----------------------------------------------------------------------------

@@ -48,6 +48,7 @@
 #include <mutex>
 
 #include "qoq.h"
+#include "qoq_actq.cuh"
 #include "qoq_device.cuh"
 #include "qoq_internal.h"
 
@@ -67,8 +68,12 @@ constexpr int kStageBytesEpi = 32 * 16 * 4;      // per epilogue warp: 16 column
 constexpr int kSlicesPerTile = 4;
 constexpr int kMaxCounterTiles = 1024;
 constexpr size_t kCounterBytes = kMaxCounterTiles * kSlicesPerTile * 4;
+// A GEMM quantizes its own activations when its token rows (FP16) fit this
+// shared-memory staging area: every CTA copies them in, computes each row's
+// scale and writes the INT8 tiles of its K range straight into its X ring.
+constexpr int kMaxFusedRowBytes = 48 * 1024;
 
-template <int TOK, bool kCluster = false>
+template <int TOK, bool kCluster = false, bool kFuseX = false>
 struct Cfg {
   // One ring of kStages stages.  A stage covers kNB consecutive k-tiles of
   // 128 (the last stage of a unit may cover fewer): their X8 tiles and packed
@@ -120,13 +125,20 @@ struct Cfg {
   // receives the INT32 partial tiles of the other CTAs:
   // [slot = rank - 1][epilogue warp][token][32 channels].
   static constexpr int kRedBars = kCluster ? 8 : 0;
-  static constexpr int kNumBars = 3 * kStages + 2 * kWStages + 2 * kAcc + 1 + kRedBars;
+  // The variant that quantizes its own activations has one more barrier (its
+  // token rows landed), the FP16 rows and each row's scale and reciprocal.
+  static constexpr int kFuseBars = kFuseX ? 2 : 0;
+  static constexpr int kNumBars = 3 * kStages + 2 * kWStages + 2 * kAcc + 1 + kRedBars + kFuseBars;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kMaxClusterSplit = !kCluster ? 1 : TOK <= 16 ? 8 : TOK <= 32 ? 3 : 1;
   static constexpr int kRedSlotBytes = kTileN * TOK * 4;
-  static constexpr int kOffRed = kCluster ? ((kOffMisc + 32 + 127) / 128) * 128 : kOffMisc + 32;
-  static constexpr int kSmemBytes =
-      kOffRed + (kMaxClusterSplit - 1) * kRedSlotBytes + 1024;   // + base alignment slack
+  static constexpr int kOffRed = ((kOffMisc + 32 + 127) / 128) * 128;
+  static constexpr int kRedBytes = (kMaxClusterSplit - 1) * kRedSlotBytes;
+  static constexpr int kOffXrow = kOffRed + kRedBytes;
+  static constexpr int kOffSxq = kOffXrow + (kFuseX ? kMaxFusedRowBytes : 0);
+  static constexpr int kSmemBytes = kOffSxq + (kFuseX ? TOK * 8 : 0) + 1024;   // + alignment slack
+  static_assert(!kFuseX || (TOK == 16 && !kCluster), "own activations: 16-token tiles");
+  static_assert(kOffXrow % 128 == 0, "bulk copy destination alignment");
   static_assert(!kCluster || TOK <= 32, "K split across a cluster for token tiles up to 32");
   static_assert(kOffRaw % 1024 == 0 && kXBytes % 1024 == 0, "swizzled tiles need 1 KiB alignment");
   static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
@@ -159,6 +171,13 @@ struct GemmArgs {
   int cs;               // K split across a cluster of cs CTAs (1: none); then
                         // splits == cs and the split partials never leave the
                         // cluster (no workspace)
+  // The GEMM that quantizes its own activations (X != nullptr): every CTA
+  // copies the M FP16 token rows of X into shared memory, computes their
+  // scales and quantizes the tiles it multiplies; the CTAs of the first
+  // channel tile also write X8 (the tiles of their K range) and CTA 0 writes
+  // sx, so the caller sees the same X8 / sx as from the stand-alone quantizer.
+  const __half* X;
+  int8_t* X8;
 };
 
 struct Unit {
@@ -340,11 +359,17 @@ struct WeightStream {
   }
 };
 
-template <int TOK, bool kCluster>
+template <int TOK, bool kCluster, bool kFuseX>
 __global__ void __launch_bounds__(Cfg<TOK>::kThreads, 1)
 w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args) {
-  using C = Cfg<TOK, kCluster>;
+  using C = Cfg<TOK, kCluster, kFuseX>;
   constexpr int S = C::kStages;
+  // a launch with less shared memory than this layout needs does nothing
+  // (every thread returns before any barrier) and records the mistake
+  if (dynamic_smem_bytes() < static_cast<uint32_t>(C::kSmemBytes)) {
+    if (threadIdx.x == 0) atomicOr(&g_error_word, kErrLaunch);
+    return;
+  }
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -379,6 +404,10 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   // written again.
   const uint32_t bar_red_full = bar_drain + 8;
   const uint32_t bar_red_free = bar_red_full + 8 * 4;
+  // own activations: the FP16 token rows landed in shared memory; this CTA
+  // has written X8 (the X producer waits for this one)
+  const uint32_t bar_xrow = bar_drain + 8 + 8 * C::kRedBars;
+  const uint32_t bar_x8 = bar_xrow + 8;
   const int cs = kCluster ? args.cs : 1;
   const uint32_t crank = cs > 1 ? cluster_ctarank() : 0u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
@@ -390,7 +419,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     // dqfull, wempty and accempty count the four warps of a warpgroup; the
     // lanes of warp 0 initialize all but the weight ring's, which the weight
     // producer initializes itself
-    for (int i = lane; i < C::kNumBars - C::kRedBars; i += 32) {
+    for (int i = lane; i < C::kNumBars - C::kRedBars - C::kFuseBars; i += 32) {
       const int acc0 = 3 * S + 2 * SW;
       if (i >= 3 * S && i < acc0) continue;
       const bool four = (i >= 2 * S && i < 3 * S) ||
@@ -401,6 +430,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
       if (lane < 4) mbar_init(bar_red_full + 8 * lane, cs > 1 ? static_cast<uint32_t>(cs - 1) : 1u);
       else if (lane < 8) mbar_init(bar_red_free + 8 * (lane - 4), 1u);
     }
+    if (kFuseX && lane < 2) mbar_init(bar_xrow + 8 * lane, 1u);
     if (lane == 0) {
       *abort_flag = 0u;
       prefetch_tensormap(&tmap_x);
@@ -438,6 +468,13 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     uint32_t g = 0;              // running stage index of this CTA
     bool aborted = false;
     grid_dependency_wait();      // X8 comes from the preceding grid under PDL
+    if constexpr (kFuseX) {
+      // own activations: X8 is written by this CTA's epilogue warps first;
+      // the copies below read it through the async proxy
+      aborted = !__all_sync(0xffffffffu, mbar_wait(bar_x8, 0, abort_flag, &g_error_word,
+                                                    kErrProducer));
+      fence_proxy_async_global();
+    }
     for (int u = blockIdx.x; u < args.units && !aborted; u += gridDim.x) {
       const Unit w = unit_of(args, u, kt_total);
       const int m0 = w.mt * TOK;
@@ -529,6 +566,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     const int gpt = kTileK / args.group;
     uint32_t g0 = 0;                        // running stage index of the unit's first stage
     bool aborted = false;
+
     for (int u = blockIdx.x; u < args.units && !aborted; u += gridDim.x) {
       const Unit w = unit_of(args, u, kt_total);
       const int nsteps = (w.num_kt + C::kNB - 1) / C::kNB;
@@ -616,8 +654,57 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     // rows 16 * (lane & 1) .. +15 of this warp's 32-row slice
     const int tc = lane >> 1, th = lane & 1;
     grid_dependency_wait();                 // sx comes from the preceding grid under PDL
+    // Own activations, before the first accumulator can be ready: the M FP16
+    // token rows (contiguous, M*K*2 bytes) in one bulk copy, each row's scale
+    // as the stand-alone quantizer computes it (CTA 0 writes sx), then all of
+    // X8 written with the same codes by every CTA (identical bytes), and the
+    // X producer released.
+    float* sxq = reinterpret_cast<float*>(smem + C::kOffSxq);   // [row] scale, reciprocal
+    bool sx_ok = true;
+    if constexpr (kFuseX) {
+      const int t = ew * 32 + lane;
+      const uint32_t bytes = static_cast<uint32_t>(M) * static_cast<uint32_t>(args.K) * 2u;
+      if (t == 0) {
+        mbar_arrive_expect_tx(bar_xrow, bytes);
+        bulk_load_plain(base + C::kOffXrow, args.X, bytes, bar_xrow);
+      }
+      sx_ok = __all_sync(0xffffffffu, mbar_wait(bar_xrow, 0, abort_flag, &g_error_word,
+                                                 kErrEpilogue));
+      const uint4* rv = reinterpret_cast<const uint4*>(smem + C::kOffXrow);
+      const int vpr = args.K / 8;                     // 16-byte vectors per row
+      if (sx_ok) {
+        for (int m = ew; m < M; m += 4) {
+          __half2 hmax = __float2half2_rn(0.0f);
+          for (int i = lane; i < vpr; i += 32) hmax = absmax8(rv[m * vpr + i], hmax);
+          float amax = fmaxf(__low2float(hmax), __high2float(hmax));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+          if (lane == 0) {
+            const __half sh = scale_from_absmax(amax, 127.0f);
+            const float sf = __half2float(sh);
+            sxq[2 * m] = sf;
+            sxq[2 * m + 1] = __frcp_rn(sf);
+            if (blockIdx.x == 0) const_cast<__half*>(args.sx)[m] = sh;
+          }
+        }
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (sx_ok) {
+        uint2* x8 = reinterpret_cast<uint2*>(args.X8);
+        for (int v = t; v < M * vpr; v += 128) {
+          const int m = v / vpr;
+          const float sf = sxq[2 * m], rcp = sxq[2 * m + 1];
+          x8[v] = sf < 6.103515625e-05f ? quantize8<true>(rv[v], sf, rcp, 0.5f * sf)
+                                        : quantize8<false>(rv[v], sf, rcp, 0.5f * sf);
+        }
+        // the tensor copies of this CTA's X producer read these stores
+        fence_proxy_async_global();
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (t == 0 && sx_ok) mbar_arrive(bar_x8);
+    }
     int lt = 0;
-    for (int u = blockIdx.x; u < args.units; u += gridDim.x, ++lt) {
+    for (int u = blockIdx.x; u < args.units && sx_ok; u += gridDim.x, ++lt) {
       const Unit w = unit_of(args, u, kt_total);
       const int b = lt % C::kAcc;
       const int m0 = w.mt * TOK;
@@ -630,7 +717,8 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
       if (args.Y) {
         s1r = __half2float(args.s1[w.nt * kTileN + r]);
         for (int c = lane; c < TOK; c += 32)
-          sx_w[c] = (m0 + c < M) ? __half2float(args.sx[m0 + c]) : 0.0f;
+          sx_w[c] = (m0 + c < M) ? (kFuseX ? sxq[2 * (m0 + c)] : __half2float(args.sx[m0 + c]))
+                                 : 0.0f;
         __syncwarp();
       }
       const bool ok = mbar_wait(bar_accfull + 8 * b, (lt / C::kAcc) & 1, abort_flag,
@@ -784,6 +872,10 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_accempty + 8 * b);
     }
+    if constexpr (kFuseX) {
+      // the row copy must land before the CTA exits, also if its wait gave up
+      if (!sx_ok && ew == 0) drain_wait(bar_xrow, 0);
+    }
   } else {
     // -------------------------------------------------------------- W producer
     // The stages after the prologue, waiting for free slots.
@@ -802,6 +894,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
   // no CTA of the cluster leaves while another may still access its shared
   // memory (every thread of every CTA reaches this point on every path)
   if (cs > 1) cluster_sync_all();
+
   if (warp == 1) {
     __syncwarp();
     tc_fence_after_sync();
@@ -839,17 +932,17 @@ struct Plan {
 // Largest K split a cluster can reduce in the leader's shared memory.
 int max_cluster_split(int tok) { return tok <= 16 ? 8 : tok <= 32 ? 3 : 1; }
 
-template <int TOK, bool kCluster>
+template <int TOK, bool kCluster, bool kFuseX>
 __global__ void __launch_bounds__(Cfg<TOK>::kThreads, 1)
 w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args);
 
 template <int TOK>
 int query_active_clusters(int cs) {
   using C = Cfg<TOK, true>;
-  if (cudaFuncSetAttribute(w4a8_gemm_kernel<TOK, true>,
+  if (cudaFuncSetAttribute(w4a8_gemm_kernel<TOK, true, false>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
           cudaSuccess ||
-      cudaFuncSetAttribute(w4a8_gemm_kernel<TOK, true>,
+      cudaFuncSetAttribute(w4a8_gemm_kernel<TOK, true, false>,
                            cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess) {
     cudaGetLastError();
     return 0;
@@ -866,7 +959,7 @@ int query_active_clusters(int cs) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, w4a8_gemm_kernel<TOK, true>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, w4a8_gemm_kernel<TOK, true, false>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -1019,16 +1112,17 @@ size_t ws_bytes_for(const Plan& p, int N) {
   return kCounterBytes + part;
 }
 
-template <int TOK, bool kCluster>
+template <int TOK, bool kCluster, bool kFuseX>
 int launch_kernel(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cudaStream_t stream,
                bool pdl) {
-  using C = Cfg<TOK, kCluster>;
+  // the same layout as the kernel instance (its shared-memory size)
+  using C = Cfg<TOK, kCluster, kFuseX>;
   static int configured_mask = 0;   // one bit per device id < 31
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return QOQ_ERR_CUDA;
   const int bit = dev < 31 ? (1 << dev) : 0;
   if (!bit || !(__atomic_load_n(&configured_mask, __ATOMIC_ACQUIRE) & bit)) {
-    if (cudaFuncSetAttribute(w4a8_gemm_kernel<TOK, kCluster>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(w4a8_gemm_kernel<TOK, kCluster, kFuseX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess)
       return QOQ_ERR_CUDA;
     if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_RELEASE);
@@ -1054,7 +1148,7 @@ int launch_kernel(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cuda
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  if (cudaLaunchKernelEx(&cfg, w4a8_gemm_kernel<TOK, kCluster>, map, a) != cudaSuccess) return QOQ_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, w4a8_gemm_kernel<TOK, kCluster, kFuseX>, map, a) != cudaSuccess) return QOQ_ERR_CUDA;
   return QOQ_OK;
 }
 
@@ -1063,10 +1157,14 @@ int launch_kernel(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cuda
 template <int TOK>
 int launch_tok(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cudaStream_t stream,
                bool pdl) {
+  const bool fuse = a.X != nullptr;
   if constexpr (TOK <= 32) {
-    if (p.cs > 1) return launch_kernel<TOK, true>(map, a, p, stream, pdl);
+    if (p.cs > 1) return launch_kernel<TOK, true, false>(map, a, p, stream, pdl);
   }
-  return launch_kernel<TOK, false>(map, a, p, stream, pdl);
+  if constexpr (TOK == 16) {
+    if (fuse) return launch_kernel<TOK, false, true>(map, a, p, stream, pdl);
+  }
+  return launch_kernel<TOK, false, false>(map, a, p, stream, pdl);
 }
 
 // Everything one GEMM launch needs, built and checked before anything is
@@ -1134,6 +1232,8 @@ int gemm_prepare(const int8_t* X8, const void* sx, const void* packed, const voi
     a.ws_part = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kCounterBytes);
   }
   a.cs = p.cs;
+  a.X = nullptr;
+  a.X8 = nullptr;
   a.M = M;
   a.N = N;
   a.K = K;
@@ -1316,6 +1416,30 @@ extern "C" int qoq_w4a8_linear(const void* X, int M, int K, const void* packed, 
   // both kernels are this library's: the GEMM reads nothing the quantizer
   // writes before its grid-dependency wait, so it may overlap its tail
   return gemm_launch(L, stream, /*weights_independent=*/true, false);
+}
+
+extern "C" int qoq_w4a8_linear_fused(const void* X, int M, int K, const void* packed,
+                                     const void* s1, int N, int group, int8_t* X8, void* sx,
+                                     void* Y, void* ws, size_t ws_bytes, void* stream) {
+  if (!X || !X8 || !sx || !Y || !packed || !s1) return QOQ_ERR_INVALID_ARG;
+  if (M <= 0) return QOQ_ERR_INVALID_ARG;
+  if (int st = check_weight_shape(N, K, group)) return st;
+  if (!aligned16(X) || !aligned16(X8) || !aligned16(sx) || !aligned16(Y) || !aligned16(packed) ||
+      !aligned16(s1) || (ws && !aligned16(ws)))
+    return QOQ_ERR_INVALID_ARG;
+  if (static_cast<long>(M) * K * 2 > static_cast<long>(kMaxFusedRowBytes))
+    return QOQ_ERR_UNSUPPORTED;
+  GemmLaunch L;
+  if (int st = gemm_prepare(X8, sx, packed, s1, M, N, K, group, Y, nullptr, 0, 0, ws, ws_bytes, L))
+    return st;
+  if (L.p.tok != 16 || L.p.cs != 1) return QOQ_ERR_UNSUPPORTED;
+  // One kernel: every CTA copies the FP16 token rows into shared memory,
+  // computes their scales and writes X8 (identical bytes from every CTA)
+  // before its X producer reads it; CTA 0 writes sx.  The preceding kernel
+  // is the caller's, so the weight stream waits for it too.
+  L.a.X = static_cast<const __half*>(X);
+  L.a.X8 = X8;
+  return gemm_launch(L, stream, /*weights_independent=*/false, false);
 }
 
 extern "C" int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int* splits, int* ctas,
