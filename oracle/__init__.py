@@ -14,7 +14,9 @@ full list):
   (protective range, "subtraction after multiplication");
 * the output scaling applied once after the K loop -- same page, Background
   (the partial-sum dequantization that per-group W4A4 needs and W4A8 avoids)
-  and "Part5 LLM部署技术", 3. 实践扩展：QServe（W4A8KV4）.
+  and "Part5 LLM部署技术", 3. 实践扩展：QServe（W4A8KV4）;
+* per-input-channel smoothing (calibration maxima, X / s, W * s) -- "Part5
+  LLM部署技术", 1.1 权重-激活联合量化：SmoothQuant.
 """
 from __future__ import annotations
 
@@ -92,6 +94,9 @@ def _load():
             lib.orc_epilogue.argtypes = [P, P, P, I, I, P]
             lib.orc_w4a8_forward.restype = ctypes.c_long
             lib.orc_w4a8_forward.argtypes = [P, P, P, I, I, I, P, P, P, P]
+            lib.orc_smooth_factors.argtypes = [P, I, P, I, I, P]
+            lib.orc_smooth_weights.argtypes = [P, P, I, I, P]
+            lib.orc_smooth_act.argtypes = [P, P, I, I, P]
             lib.orc_num_threads.restype = I
             _lib = lib
     return _lib
@@ -269,6 +274,43 @@ def w4a8_forward(X, dq, s1):
     if of:
         raise OverflowError(f"{of} accumulator entries exceed INT32")
     return X8, sx.view(np.float16), acc, Y.view(np.float16)
+
+
+# --------------------------------------------------------------------------
+# Per-input-channel smoothing ("Part5 LLM部署技术", 1.1 SmoothQuant):
+# calibration maxima, then X / s and W * s (alpha = 0.5, see qoq_oracle.c)
+# --------------------------------------------------------------------------
+
+def smooth_factors(Xcal, W):
+    """s (float16[K]) from a calibration batch Xcal (Mc, K) and W (N, K)."""
+    Xcal = _as_f16_bits(Xcal)
+    W = _as_f16_bits(W)
+    Mc, K = Xcal.shape
+    N, K2 = W.shape
+    assert K == K2
+    out = np.empty(K, np.uint16)
+    _load().orc_smooth_factors(_p(Xcal), Mc, _p(W), N, K, _p(out))
+    return out.view(np.float16)
+
+
+def smooth_weights(W, s):
+    """W' = fp16(W * s[k]) (float16 (N, K))."""
+    W = _as_f16_bits(W)
+    s = _as_f16_bits(s)
+    N, K = W.shape
+    out = np.empty((N, K), np.uint16)
+    _load().orc_smooth_weights(_p(W), _p(s), N, K, _p(out))
+    return out.view(np.float16)
+
+
+def smooth_act(X, s):
+    """X' = fp16(X / s[k]) (float16 (M, K))."""
+    X = _as_f16_bits(X)
+    s = _as_f16_bits(s)
+    M, K = X.shape
+    out = np.empty((M, K), np.uint16)
+    _load().orc_smooth_act(_p(X), _p(s), M, K, _p(out))
+    return out.view(np.float16)
 
 
 def num_threads() -> int:

@@ -298,6 +298,58 @@ long orc_w4a8_forward(const uint16_t* X, const int8_t* dq, const uint16_t* s1,
     return of;
 }
 
+/* ---------------------------------------------------------------------------
+ * Per-input-channel smoothing, SmoothQuant style ("Part5 LLM部署技术",
+ * 1.1 权重-激活联合量化：SmoothQuant): part of the activations' quantization
+ * difficulty is moved onto the weights, one factor per input channel k.
+ *  1. calibration: the per-channel maxima of the activations (over a
+ *     calibration batch) and of the weights;
+ *  2. smoothing: the activations are divided by the factor, the weights
+ *     multiplied by it, so X . W^T is unchanged up to rounding;
+ *  3. inference: the smoothed operands are quantized as usual.
+ * Readings where the page's formula is lost: migration strength alpha = 0.5
+ * (the default), so s_k = max|X_k|^0.5 / max|W_k|^0.5 = sqrt(max|X_k| /
+ * max|W_k|), formed in IEEE binary32 (a division and a square root, both
+ * correctly rounded), clamped to [2^-14, 2^14] and rounded to FP16; s_k = 1
+ * where either maximum is 0.  The smoothed operands are FP16: W' = fp16(W *
+ * s) (the product of two FP16 values is exact, so it is rounded once) and
+ * X' = fp16(X / s) with the quotient formed in IEEE binary32.
+ * ------------------------------------------------------------------------- */
+void orc_smooth_factors(const uint16_t* Xc, int Mc, const uint16_t* W, int N, int K,
+                        uint16_t* s) {
+    for (int k = 0; k < K; ++k) {
+        float ax = 0.0f, aw = 0.0f;
+        for (int m = 0; m < Mc; ++m) {
+            float v = fabsf(orc_h2f(Xc[(size_t)m * K + k]));
+            if (v > ax) ax = v;
+        }
+        for (int n = 0; n < N; ++n) {
+            float v = fabsf(orc_h2f(W[(size_t)n * K + k]));
+            if (v > aw) aw = v;
+        }
+        if (ax == 0.0f || aw == 0.0f) {
+            s[k] = 0x3c00;                        /* 1.0 */
+            continue;
+        }
+        float r = sqrtf(ax / aw);
+        if (r < 0x1p-14f) r = 0x1p-14f;
+        if (r > 0x1p14f) r = 0x1p14f;
+        s[k] = orc_f2h(r);
+    }
+}
+
+void orc_smooth_weights(const uint16_t* W, const uint16_t* s, int N, int K, uint16_t* Wp) {
+    for (int n = 0; n < N; ++n)
+        for (int k = 0; k < K; ++k)
+            Wp[(size_t)n * K + k] = orc_d2h(orc_h2d(W[(size_t)n * K + k]) * orc_h2d(s[k]));
+}
+
+void orc_smooth_act(const uint16_t* X, const uint16_t* s, int M, int K, uint16_t* Xp) {
+    for (int m = 0; m < M; ++m)
+        for (int k = 0; k < K; ++k)
+            Xp[(size_t)m * K + k] = orc_f2h(orc_h2f(X[(size_t)m * K + k]) / orc_h2f(s[k]));
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
     extern int omp_get_max_threads(void);

@@ -458,3 +458,110 @@ def test_planted_mistakes_are_caught(oracle):
     acc = oracle.int_gemm(X8, Wq["dq"])
     assert np.array_equal(acc, Wq["dq"][:, :8].T.astype(np.int32))
     assert not np.array_equal(acc, Wq["dq"][:8, :].astype(np.int32)[:, :Wq["dq"].shape[0]])
+
+
+# ---------------------------------------------------------------------------
+# Per-input-channel smoothing ("Part5 LLM部署技术", 1.1 权重-激活联合量化：
+# SmoothQuant): calibration maxima, X / s and W * s, migration strength 0.5
+# ---------------------------------------------------------------------------
+
+def _hex16(h):
+    return np.array([int(h, 16)], np.uint16).view(np.float16)
+
+
+def test_smoothing_hand_examples(oracle):
+    for (ax, aw), (sh,) in _golden("smooth_factor"):
+        Xc = np.array([[float(ax)]], np.float16)
+        W = np.array([[float(aw)]], np.float16)
+        s = oracle.smooth_factors(Xc, W)
+        assert s.view(np.uint16)[0] == int(sh, 16), (ax, aw, s)
+    for (wh, sh), (outh,) in _golden("smooth_weight"):
+        got = oracle.smooth_weights(_hex16(wh).reshape(1, 1), _hex16(sh))
+        assert got.view(np.uint16)[0, 0] == int(outh, 16), (wh, sh)
+    for (xh, sh), (outh,) in _golden("smooth_act"):
+        got = oracle.smooth_act(_hex16(xh).reshape(1, 1), _hex16(sh))
+        assert got.view(np.uint16)[0, 0] == int(outh, 16), (xh, sh)
+
+
+def test_smoothing_by_one_is_identity(oracle):
+    """Every finite FP16 value is unchanged by the factor 1."""
+    bits = np.arange(65536, dtype=np.uint16)
+    vals = bits.view(np.float16)
+    vals = vals[np.isfinite(vals)].reshape(1, -1)
+    ones = np.ones(vals.shape[1], np.float16)
+    assert np.array_equal(oracle.smooth_weights(vals, ones).view(np.uint16), vals.view(np.uint16))
+    assert np.array_equal(oracle.smooth_act(vals, ones).view(np.uint16), vals.view(np.uint16))
+
+
+def test_smoothing_by_powers_of_two_is_exact(oracle):
+    """A factor 2^e scales exactly wherever the result stays a normal FP16
+    number: W * 2^e and X / 2^e."""
+    rng = np.random.default_rng(5)
+    vals = rng.uniform(-2.0, 2.0, (7, 64)).astype(np.float16)
+    vals[np.abs(vals) < 2.0 ** -10] = 0.5
+    for e in (-3, -1, 1, 4):
+        s = np.full(64, 2.0 ** e, np.float16)
+        w = oracle.smooth_weights(vals, s).astype(np.float64)
+        x = oracle.smooth_act(vals, s).astype(np.float64)
+        assert np.array_equal(w, vals.astype(np.float64) * 2.0 ** e)
+        assert np.array_equal(x, vals.astype(np.float64) * 2.0 ** -e)
+
+
+def test_smoothing_balances_channel_maxima(oracle):
+    """The factor makes the largest smoothed activation and the largest
+    smoothed weight of each channel equal (both sqrt(ax * aw)), up to the
+    FP16 roundings, and leaves each channel's balance point at the geometric
+    mean -- the migration of difficulty with strength 0.5."""
+    L = si.LLAMA3_8B_QKV
+    Xc = si.activations(L, 16, seed=3)[:, :512]
+    W = si.weights(L, seed=0)[:256, :512]
+    s = oracle.smooth_factors(Xc, W)
+    Xp = oracle.smooth_act(Xc, s).astype(np.float64)
+    Wp = oracle.smooth_weights(W, s).astype(np.float64)
+    mx = np.abs(Xp).max(0)
+    mw = np.abs(Wp).max(0)
+    geo = np.sqrt(np.abs(Xc.astype(np.float64)).max(0) * np.abs(W.astype(np.float64)).max(0))
+    assert np.all(np.abs(np.log(mx / mw)) <= 4 * 2.0 ** -10)
+    assert np.all(np.abs(np.log(mx / geo)) <= 3 * 2.0 ** -10)
+    # the outlier channels of the activation recipe get the largest factors
+    ax = np.abs(Xc.astype(np.float64)).max(0)
+    top = np.argsort(ax)[-5:]
+    assert np.all(s.astype(np.float64)[top] > np.median(s.astype(np.float64)))
+
+
+def test_smoothing_keeps_the_product(oracle):
+    """X' . W'^T equals X . W^T up to the FP16 roundings of the smoothed
+    operands: every term x_k w_k moves by at most 2^-10 of |x_k w_k|
+    (one rounding on each side, each at most 2^-11 relative)."""
+    rng = np.random.default_rng(11)
+    X = rng.standard_normal((5, 96)).astype(np.float16)
+    X[:, 7] *= np.float16(30)
+    W = (rng.standard_normal((6, 96)) * 0.02).astype(np.float16)
+    s = oracle.smooth_factors(X, W)
+    Xp = oracle.smooth_act(X, s).astype(np.float64)
+    Wp = oracle.smooth_weights(W, s).astype(np.float64)
+    Xd, Wd = X.astype(np.float64), W.astype(np.float64)
+    diff = np.abs(Xp @ Wp.T - Xd @ Wd.T)
+    bound = (np.abs(Xd) @ np.abs(Wd).T) * (2.0 ** -10 + 2.0 ** -20)
+    assert np.all(diff <= bound)
+
+
+def test_smoothing_moves_outliers_from_activations_to_weights(oracle):
+    """What the page states the method does: the activations' channel
+    maxima become flatter (the recipe's x20 outlier channels shrink to about
+    sqrt(20) of the typical channel) while the weights' channel maxima
+    spread by the same factor."""
+    L = si.LLAMA3_8B_QKV
+    K, N = 1024, 256
+    W = si.weights(L, seed=0)[:N, :K]
+    X = si.activations(L, 64, seed=4)[:, :K]
+    s = oracle.smooth_factors(X, W)
+
+    def spread(a):
+        m = np.abs(a.astype(np.float64)).max(0)
+        return m.max() / np.median(m)
+    rx, rxs = spread(X), spread(oracle.smooth_act(X, s))
+    rw, rws = spread(W), spread(oracle.smooth_weights(W, s))
+    assert rx > 10 and rxs < rx / 2
+    assert rws > rw
+    assert abs(np.log(rxs / np.sqrt(rx * rw))) < np.log(2)

@@ -152,6 +152,27 @@ MUTANTS = [
      "double v = (double)acc[(size_t)m * N + n] * a * orc_h2d(s1[n]);",
      "double v = (double)((float)acc[(size_t)m * N + n] * (float)a"
      " * (float)orc_h2d(s1[n]));"),
+    # per-input-channel smoothing
+    ("smooth_strength_one",
+     "float r = sqrtf(ax / aw);", "float r = ax / aw;"),
+    ("smooth_factor_inverted",
+     "float r = sqrtf(ax / aw);", "float r = sqrtf(aw / ax);"),
+    ("smooth_zero_guard_zero",
+     "s[k] = 0x3c00;                        /* 1.0 */", "s[k] = 0x0000;"),
+    ("smooth_no_upper_clamp",
+     "if (r > 0x1p14f) r = 0x1p14f;", "if (r > 0x1p20f) r = 0x1p20f;"),
+    ("smooth_activations_multiplied",
+     "orc_f2h(orc_h2f(X[(size_t)m * K + k]) / orc_h2f(s[k]))",
+     "orc_f2h(orc_h2f(X[(size_t)m * K + k]) * orc_h2f(s[k]))"),
+    ("smooth_weights_divided",
+     "orc_d2h(orc_h2d(W[(size_t)n * K + k]) * orc_h2d(s[k]))",
+     "orc_d2h(orc_h2d(W[(size_t)n * K + k]) / orc_h2d(s[k]))"),
+    ("smooth_weights_rounded_twice",
+     "orc_d2h(orc_h2d(W[(size_t)n * K + k]) * orc_h2d(s[k]))",
+     "orc_f2h((float)orc_h2d(W[(size_t)n * K + k]) * (float)orc_h2d(s[k]) + 0x1p-30f)"),
+    ("smooth_factor_row_max_of_weights",
+     "float v = fabsf(orc_h2f(W[(size_t)n * K + k]));\n            if (v > aw) aw = v;",
+     "float v = fabsf(orc_h2f(W[(size_t)n * K + (k % N)]));\n            if (v > aw) aw = v;"),
 ]
 
 
