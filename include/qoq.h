@@ -160,6 +160,33 @@ QOQ_API int qoq_quantize_act_per_token(const void* X, int M, int K, int8_t* X8,
                                void* sx, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Per-input-channel smoothing, SmoothQuant style ("Part5 LLM部署技术",
+ * 1.1 权重-激活联合量化：SmoothQuant): part of the activations' outliers are
+ * moved onto the weights with one factor s[k] per input channel, so that
+ * X . W^T = (X / s) . (W * s)^T.  The factors are folded into the offline
+ * weight quantization (so into s1) and into the per-token quantizer.
+ * Readings where the page's formula is lost: migration strength 0.5 (the
+ * default), s[k] = fp16(clamp(sqrt(max|Xcal[:,k]| / max|W[:,k]|), 2^-14,
+ * 2^14)) with binary32 operations, 1 where either maximum is 0; the smoothed
+ * operands are FP16: W' = fp16(W * s) (one rounding of the exact product),
+ * X' = fp16(X / s) (binary32 quotient, then FP16).
+ *
+ * qoq_smooth_factors: s (device, FP16[K], written) from a calibration batch
+ *   Xcal (device, FP16 Mc x K row-major) and W (device, FP16 N x K).
+ * qoq_quantize_weights_smoothed: qoq_quantize_weights of W' = W * s.
+ * qoq_quantize_act_per_token_smoothed: qoq_quantize_act_per_token of
+ *   X' = X / s; feed X8 / sx to the GEMM with the smoothed weights.
+ * s is 16-byte aligned.  As for every input, the smoothed values must be
+ * finite (X / s overflows FP16 for |X| > 65504 * s).  Asynchronous on `stream`.
+ * ---------------------------------------------------------------------- */
+QOQ_API int qoq_smooth_factors(const void* Xcal, int Mc, const void* W, int N, int K,
+                               void* smooth, void* stream);
+QOQ_API int qoq_quantize_weights_smoothed(const void* W, const void* smooth, int N, int K,
+                                          int group, void* packed, void* s1, void* stream);
+QOQ_API int qoq_quantize_act_per_token_smoothed(const void* X, const void* smooth, int M,
+                                                int K, int8_t* X8, void* sx, void* stream);
+
+/* ------------------------------------------------------------------------
  * The hot path: Y = (X8 . dq^T) * sx[m] * s1[n], FP16 out.
  *   X8     : device, int8 M x K row-major (from qoq_quantize_act_per_token).
  *   sx     : device, FP16[M].

@@ -33,6 +33,7 @@ EXPORTS = (
     "qoq_w4a8_gemm_config", "qoq_w4a8_linear", "qoq_gemm_plan", "qoq_device_error",
     "qoq_gemm_workspace_bytes", "qoq_gemm_workspace_bytes_config",
     "qoq_w4a8_gemm_static_ws", "qoq_selftest_wait_timeout", "qoq_w4a8_linear_fused",
+    "qoq_smooth_factors", "qoq_quantize_weights_smoothed", "qoq_quantize_act_per_token_smoothed",
 )
 
 _lock = threading.Lock()
@@ -75,6 +76,12 @@ def lib() -> ctypes.CDLL:
             L.qoq_unpack_weights.argtypes = [P, I, I, I, P, P, P, P, P]
             L.qoq_quantize_act_per_token.restype = I
             L.qoq_quantize_act_per_token.argtypes = [P, I, I, P, P, P]
+            L.qoq_smooth_factors.restype = I
+            L.qoq_smooth_factors.argtypes = [P, I, P, I, I, P, P]
+            L.qoq_quantize_weights_smoothed.restype = I
+            L.qoq_quantize_weights_smoothed.argtypes = [P, P, I, I, I, P, P, P]
+            L.qoq_quantize_act_per_token_smoothed.restype = I
+            L.qoq_quantize_act_per_token_smoothed.argtypes = [P, P, I, I, P, P, P]
             L.qoq_w4a8_gemm.restype = I
             L.qoq_w4a8_gemm.argtypes = [P, P, P, P, I, I, I, I, P, P, sz, P]
             L.qoq_selftest_wait_timeout.restype = I
@@ -320,6 +327,58 @@ def quantize_act_per_token(X, out=None, stream=None):
         _need_cuda(sx, "sx", torch.float16, shape=(M,), device=X.device)
     _check(lib().qoq_quantize_act_per_token(_ptr(X), M, K, _ptr(X8), _ptr(sx),
                                             _stream(stream)), "qoq_quantize_act_per_token")
+    return X8, sx
+
+
+def smooth_factors(Xcal, W, stream=None):
+    """Per-input-channel smoothing factors (float16[K]) from a calibration
+    batch Xcal (Mc, K) and the weight W (N, K), both float16 CUDA tensors."""
+    import torch
+    _need_cuda(Xcal, "Xcal", torch.float16, 2)
+    Mc, K = Xcal.shape
+    _need_cuda(W, "W", torch.float16, 2, device=Xcal.device)
+    N, K2 = W.shape
+    if K2 != K:
+        raise ValueError("Xcal and W must have the same number of input channels")
+    s = torch.empty(K, dtype=torch.float16, device=W.device)
+    _check(lib().qoq_smooth_factors(_ptr(Xcal), Mc, _ptr(W), N, K, _ptr(s), _stream(stream)),
+           "qoq_smooth_factors")
+    return s
+
+
+def quantize_weights_smoothed(W, smooth, group: int = 128, stream=None):
+    """quantize_weights of W * smooth[k] (the factors folded into s1)."""
+    import torch
+    _need_cuda(W, "W", torch.float16, 2)
+    N, K = W.shape
+    _need_cuda(smooth, "smooth", torch.float16, shape=(K,), device=W.device)
+    nbytes = packed_weight_bytes(N, K, group)
+    if nbytes == 0:
+        raise QoQError(QOQ_ERR_INVALID_ARG, "qoq_packed_weight_bytes")
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    s1 = torch.empty(N, dtype=torch.float16, device=W.device)
+    _check(lib().qoq_quantize_weights_smoothed(_ptr(W), _ptr(smooth), N, K, group, _ptr(packed),
+                                               _ptr(s1), _stream(stream)),
+           "qoq_quantize_weights_smoothed")
+    return packed, s1
+
+
+def quantize_act_per_token_smoothed(X, smooth, out=None, stream=None):
+    """quantize_act_per_token of X / smooth[k]."""
+    import torch
+    _need_cuda(X, "X", torch.float16, 2)
+    M, K = X.shape
+    _need_cuda(smooth, "smooth", torch.float16, shape=(K,), device=X.device)
+    if out is None:
+        X8 = torch.empty((M, K), dtype=torch.int8, device=X.device)
+        sx = torch.empty(M, dtype=torch.float16, device=X.device)
+    else:
+        X8, sx = out
+        _need_cuda(X8, "X8", torch.int8, shape=(M, K), device=X.device)
+        _need_cuda(sx, "sx", torch.float16, shape=(M,), device=X.device)
+    _check(lib().qoq_quantize_act_per_token_smoothed(_ptr(X), _ptr(smooth), M, K, _ptr(X8),
+                                                     _ptr(sx), _stream(stream)),
+           "qoq_quantize_act_per_token_smoothed")
     return X8, sx
 
 

@@ -1412,7 +1412,7 @@ extern "C" int qoq_w4a8_linear(const void* X, int M, int K, const void* packed, 
   // its launch latency.  For many rows that overlap measured slower on B200,
   // so the quantizer is then an ordinary launch.
   const bool aq_pdl = M <= 2 * sm_count();
-  if (int st = launch_act_quant(X, M, K, X8, sx, stream, aq_pdl)) return st;
+  if (int st = launch_act_quant(X, M, K, X8, sx, stream, aq_pdl, nullptr)) return st;
   // both kernels are this library's: the GEMM reads nothing the quantizer
   // writes before its grid-dependency wait, so it may overlap its tail
   return gemm_launch(L, stream, /*weights_independent=*/true, false);

@@ -59,6 +59,9 @@ int gemm_impl(const int8_t* X8, const void* sx, const void* packed, const void* 
 // Launch the per-token activation quantizer (no argument checks).  With
 // `pdl` it may start while the preceding kernel on the stream drains; it
 // waits for that grid before touching memory.
-int launch_act_quant(const void* X, int M, int K, int8_t* X8, void* sx, void* stream, bool pdl);
+// `smooth` (FP16[K] or nullptr): divide each value by its channel's
+// smoothing factor before quantizing.
+int launch_act_quant(const void* X, int M, int K, int8_t* X8, void* sx, void* stream, bool pdl,
+                     const void* smooth);
 
 }  // namespace qoq

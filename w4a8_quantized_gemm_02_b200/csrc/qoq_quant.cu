@@ -17,6 +17,23 @@
 namespace qoq {
 namespace {
 
+// Per-input-channel smoothing of eight FP16 values (the k-th value by the
+// k-th factor): times the factor for weights (one rounding of the exact
+// product), divided by it for activations (binary32 quotient, then FP16).
+template <bool kDivide>
+__device__ __forceinline__ uint4 smooth8(uint4 v, uint4 f) {
+  __half2* h = reinterpret_cast<__half2*>(&v);
+  const __half2* g = reinterpret_cast<const __half2*>(&f);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 x = __half22float2(h[j]);
+    const float2 y = __half22float2(g[j]);
+    h[j] = kDivide ? __floats2half2_rn(__fdiv_rn(x.x, y.x), __fdiv_rn(x.y, y.y))
+                   : __floats2half2_rn(__fmul_rn(x.x, y.x), __fmul_rn(x.y, y.y));
+  }
+  return v;
+}
+
 // Exact round-half-even of a / b for b > 0.
 __device__ __forceinline__ int div_rne(int a, int b) {
   int q = a / b;
@@ -31,10 +48,10 @@ __device__ __forceinline__ int div_rne(int a, int b) {
 // its row in registers (one pass over global memory); longer rows are read
 // twice.  Few vectors per thread keep the register count low, so that many
 // CTAs share an SM and many loads are in flight.
-template <int kWarps, int kWarpsPerRow, int kRegVec>
+template <int kWarps, int kWarpsPerRow, int kRegVec, bool kSmooth>
 __global__ void __launch_bounds__(32 * kWarps)
 act_quant_kernel(const __half* __restrict__ X, int M, int K, int8_t* __restrict__ X8,
-                 __half* __restrict__ sx) {
+                 __half* __restrict__ sx, const __half* __restrict__ smooth) {
   // Launched as a programmatic dependent of the previous kernel on the stream
   // (qoq_w4a8_linear), this CTA may start while that kernel drains: nothing
   // is read or written before that grid has completed and its writes are
@@ -54,13 +71,20 @@ act_quant_kernel(const __half* __restrict__ X, int M, int K, int8_t* __restrict_
   uint2* out = reinterpret_cast<uint2*>(X8 + static_cast<size_t>(active ? m : 0) * K);
   const int nvec = active ? K / 8 : 0;
   const bool in_regs = K / 8 <= kT * kRegVec;
+  // smoothed activations: each value divided by its channel's factor first
+  const uint4* sv = reinterpret_cast<const uint4*>(smooth);
+  auto load = [&](int i) {
+    uint4 x = __ldg(row + i);
+    if constexpr (kSmooth) x = smooth8<true>(x, __ldg(sv + i));
+    return x;
+  };
   uint4 v[kRegVec];
   __half2 hmax = __float2half2_rn(0.0f);
   if (in_regs) {
 #pragma unroll
     for (int u = 0; u < kRegVec; ++u) {
       const int i = t + kT * u;
-      if (i < nvec) v[u] = __ldg(row + i);
+      if (i < nvec) v[u] = load(i);
     }
 #pragma unroll
     for (int u = 0; u < kRegVec; ++u)
@@ -71,7 +95,7 @@ act_quant_kernel(const __half* __restrict__ X, int M, int K, int8_t* __restrict_
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int i = i0 + t + kT * u;
-        if (i < nvec) w[u] = __ldg(row + i);
+        if (i < nvec) w[u] = load(i);
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u)
@@ -112,9 +136,9 @@ act_quant_kernel(const __half* __restrict__ X, int M, int K, int8_t* __restrict_
     }
   } else {
     if (!clamp) {
-      for (int i = t; i < nvec; i += kT) out[i] = quantize8<false>(__ldg(row + i), sf, rcp, half_sf);
+      for (int i = t; i < nvec; i += kT) out[i] = quantize8<false>(load(i), sf, rcp, half_sf);
     } else {
-      for (int i = t; i < nvec; i += kT) out[i] = quantize8<true>(__ldg(row + i), sf, rcp, half_sf);
+      for (int i = t; i < nvec; i += kT) out[i] = quantize8<true>(load(i), sf, rcp, half_sf);
     }
   }
 }
@@ -123,7 +147,8 @@ act_quant_kernel(const __half* __restrict__ X, int M, int K, int8_t* __restrict_
 // Level 1 scale: one warp per output channel.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
-row_scale_kernel(const __half* __restrict__ W, int N, int K, __half* __restrict__ s1) {
+row_scale_kernel(const __half* __restrict__ W, int N, int K, __half* __restrict__ s1,
+                 const __half* __restrict__ smooth) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= N) return;
@@ -131,6 +156,7 @@ row_scale_kernel(const __half* __restrict__ W, int N, int K, __half* __restrict_
   float amax = 0.0f;
   for (int i = lane; i < K / 8; i += 32) {
     uint4 v = __ldg(row + i);
+    if (smooth) v = smooth8<false>(v, __ldg(reinterpret_cast<const uint4*>(smooth) + i));
     const __half2* h = reinterpret_cast<const __half2*>(&v);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -158,7 +184,7 @@ __device__ __forceinline__ int level1_code(float w, float s1f) {
 __global__ void __launch_bounds__(128)
 pack_weights_kernel(const __half* __restrict__ W, int K, int group,
                     const __half* __restrict__ s1, uint8_t* __restrict__ packed,
-                    int blk_bytes) {
+                    int blk_bytes, const __half* __restrict__ smooth) {
   __shared__ __align__(16) uint8_t tile[kTileN * kPackRowBytes];
   const int kt = blockIdx.x, nt = blockIdx.y;
   const int n0 = nt * kTileN, k0 = kt * kTileK;
@@ -166,8 +192,9 @@ pack_weights_kernel(const __half* __restrict__ W, int K, int group,
   // coalesced staging: 128 rows x 256 bytes = 2048 chunks of 16 bytes
   for (int c = threadIdx.x; c < kTileN * 16; c += 128) {
     const int row = c >> 4, col = c & 15;
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(
-                              W + static_cast<size_t>(n0 + row) * K + k0) + col);
+    uint4 v = __ldg(reinterpret_cast<const uint4*>(
+                        W + static_cast<size_t>(n0 + row) * K + k0) + col);
+    if (smooth) v = smooth8<false>(v, __ldg(reinterpret_cast<const uint4*>(smooth + k0) + col));
     *reinterpret_cast<uint4*>(tile + row * kPackRowBytes + col * 16) = v;
   }
   __syncthreads();
@@ -260,6 +287,40 @@ pack_codes_kernel(const uint8_t* __restrict__ q, const int8_t* __restrict__ s2,
 }
 
 // ---------------------------------------------------------------------------
+// Smoothing factors: per input channel k, the largest |X| of the calibration
+// batch (ax) and the largest |W| (aw), then s = fp16(clamp(sqrt(ax / aw),
+// 2^-14, 2^14)) in binary32 (1 where a maximum is 0).  A CTA of 256 threads
+// takes 32 channels; its 8 row lanes stride the rows.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+smooth_factors_kernel(const __half* __restrict__ Xc, int Mc, const __half* __restrict__ W, int N,
+                      int K, __half* __restrict__ s) {
+  __shared__ float red[2][8][32];
+  const int c = threadIdx.x & 31, rl = threadIdx.x >> 5;
+  const int k = blockIdx.x * 32 + c;
+  float ax = 0.0f, aw = 0.0f;
+  if (k < K) {
+    for (int m = rl; m < Mc; m += 8) ax = fmaxf(ax, fabsf(__half2float(Xc[static_cast<size_t>(m) * K + k])));
+    for (int n = rl; n < N; n += 8) aw = fmaxf(aw, fabsf(__half2float(W[static_cast<size_t>(n) * K + k])));
+  }
+  red[0][rl][c] = ax;
+  red[1][rl][c] = aw;
+  __syncthreads();
+  if (rl != 0 || k >= K) return;
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    ax = fmaxf(ax, red[0][i][c]);
+    aw = fmaxf(aw, red[1][i][c]);
+  }
+  if (ax == 0.0f || aw == 0.0f) {
+    s[k] = __ushort_as_half(0x3c00);
+    return;
+  }
+  const float r = fminf(fmaxf(__fsqrt_rn(__fdiv_rn(ax, aw)), 0x1p-14f), 0x1p14f);
+  s[k] = __float2half_rn(r);
+}
+
+// ---------------------------------------------------------------------------
 // Debug unpacker: canonical q / s2 / z and dq via the GEMM's byte-lane path.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128)
@@ -307,7 +368,8 @@ using namespace qoq;
 
 namespace qoq {
 template <int kWarps, int kWarpsPerRow, int kRegVec>
-int launch_aq(const __half* X, int M, int K, int8_t* X8, __half* sx, cudaStream_t st, bool pdl) {
+int launch_aq(const __half* X, int M, int K, int8_t* X8, __half* sx, cudaStream_t st, bool pdl,
+              const __half* smooth) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(M), 1, 1);
   cfg.blockDim = dim3(32 * kWarps, 1, 1);
@@ -317,13 +379,17 @@ int launch_aq(const __half* X, int M, int K, int8_t* X8, __half* sx, cudaStream_
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  if (cudaLaunchKernelEx(&cfg, act_quant_kernel<kWarps, kWarpsPerRow, kRegVec>, X, M, K, X8, sx) !=
-      cudaSuccess)
-    return QOQ_ERR_CUDA;
-  return QOQ_OK;
+  cudaError_t e = smooth
+      ? cudaLaunchKernelEx(&cfg, act_quant_kernel<kWarps, kWarpsPerRow, kRegVec, true>, X, M, K, X8,
+                           sx, smooth)
+      : cudaLaunchKernelEx(&cfg, act_quant_kernel<kWarps, kWarpsPerRow, kRegVec, false>, X, M, K,
+                           X8, sx, smooth);
+  return e == cudaSuccess ? QOQ_OK : QOQ_ERR_CUDA;
 }
 
-int launch_act_quant(const void* X, int M, int K, int8_t* X8, void* sx, void* stream, bool pdl) {
+int launch_act_quant(const void* X, int M, int K, int8_t* X8, void* sx, void* stream, bool pdl,
+                     const void* smooth) {
+  const __half* sm = static_cast<const __half*>(smooth);
   const __half* Xh = static_cast<const __half*>(X);
   __half* sxh = static_cast<__half*>(sx);
   cudaStream_t st = as_stream(stream);
@@ -331,15 +397,15 @@ int launch_act_quant(const void* X, int M, int K, int8_t* X8, void* sx, void* st
   // one row per CTA in every variant
   if (M <= 2 * sm_count()) {
     // few rows: 8 warps per row keep many loads in flight per row
-    return launch_aq<8, 8, 16>(Xh, M, K, X8, sxh, st, pdl);
+    return launch_aq<8, 8, 16>(Xh, M, K, X8, sxh, st, pdl, sm);
   }
   if (nvec <= 128 * 4) {
     // many rows: a CTA of 4 warps per row holding 4 vectors per thread
-    return launch_aq<4, 4, 4>(Xh, M, K, X8, sxh, st, pdl);
+    return launch_aq<4, 4, 4>(Xh, M, K, X8, sxh, st, pdl, sm);
   }
-  if (nvec <= 256 * 4) return launch_aq<8, 8, 4>(Xh, M, K, X8, sxh, st, pdl);
-  if (nvec <= 256 * 8) return launch_aq<8, 8, 8>(Xh, M, K, X8, sxh, st, pdl);
-  return launch_aq<8, 8, 16>(Xh, M, K, X8, sxh, st, pdl);
+  if (nvec <= 256 * 4) return launch_aq<8, 8, 4>(Xh, M, K, X8, sxh, st, pdl, sm);
+  if (nvec <= 256 * 8) return launch_aq<8, 8, 8>(Xh, M, K, X8, sxh, st, pdl, sm);
+  return launch_aq<8, 8, 16>(Xh, M, K, X8, sxh, st, pdl, sm);
 }
 }  // namespace qoq
 
@@ -349,24 +415,62 @@ extern "C" int qoq_quantize_act_per_token(const void* X, int M, int K, int8_t* X
   if (M <= 0 || K <= 0 || K % 8 != 0) return QOQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(X8) || !aligned16(sx)) return QOQ_ERR_INVALID_ARG;
   if (int st = check_device()) return st;
-  return launch_act_quant(X, M, K, X8, sx, stream, false);
+  return launch_act_quant(X, M, K, X8, sx, stream, false, nullptr);
 }
 
-extern "C" int qoq_quantize_weights(const void* W, int N, int K, int group, void* packed,
-                                    void* s1, void* stream) {
+extern "C" int qoq_quantize_act_per_token_smoothed(const void* X, const void* smooth, int M, int K,
+                                                   int8_t* X8, void* sx, void* stream) {
+  if (!X || !smooth || !X8 || !sx) return QOQ_ERR_INVALID_ARG;
+  if (M <= 0 || K <= 0 || K % 8 != 0) return QOQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(smooth) || !aligned16(X8) || !aligned16(sx))
+    return QOQ_ERR_INVALID_ARG;
+  if (int st = check_device()) return st;
+  return launch_act_quant(X, M, K, X8, sx, stream, false, smooth);
+}
+
+extern "C" int qoq_smooth_factors(const void* Xcal, int Mc, const void* W, int N, int K,
+                                  void* smooth, void* stream) {
+  if (!Xcal || !W || !smooth) return QOQ_ERR_INVALID_ARG;
+  if (Mc <= 0 || N <= 0 || K <= 0) return QOQ_ERR_INVALID_ARG;
+  if (int st = check_device()) return st;
+  smooth_factors_kernel<<<(K + 31) / 32, 256, 0, as_stream(stream)>>>(
+      static_cast<const __half*>(Xcal), Mc, static_cast<const __half*>(W), N, K,
+      static_cast<__half*>(smooth));
+  return launch_status();
+}
+
+namespace qoq {
+namespace {
+int quantize_weights_impl(const void* W, const void* smooth, int N, int K, int group,
+                          void* packed, void* s1, void* stream) {
   if (!W || !packed || !s1) return QOQ_ERR_INVALID_ARG;
   if (int st = check_weight_shape(N, K, group)) return st;
-  if (!aligned16(W) || !aligned16(packed) || !aligned16(s1)) return QOQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(s1) || (smooth && !aligned16(smooth)))
+    return QOQ_ERR_INVALID_ARG;
   if (int st = check_device()) return st;
   cudaStream_t s = as_stream(stream);
   const __half* Wh = static_cast<const __half*>(W);
+  const __half* sm = static_cast<const __half*>(smooth);
   __half* s1h = static_cast<__half*>(s1);
-  row_scale_kernel<<<(N + 7) / 8, 256, 0, s>>>(Wh, N, K, s1h);
+  row_scale_kernel<<<(N + 7) / 8, 256, 0, s>>>(Wh, N, K, s1h, sm);
   if (int st = launch_status()) return st;
   dim3 grid(K / kTileK, N / kTileN);
   pack_weights_kernel<<<grid, 128, 0, s>>>(Wh, K, group, s1h, static_cast<uint8_t*>(packed),
-                                           static_cast<int>(block_bytes(group)));
+                                           static_cast<int>(block_bytes(group)), sm);
   return launch_status();
+}
+}  // namespace
+}  // namespace qoq
+
+extern "C" int qoq_quantize_weights(const void* W, int N, int K, int group, void* packed,
+                                    void* s1, void* stream) {
+  return quantize_weights_impl(W, nullptr, N, K, group, packed, s1, stream);
+}
+
+extern "C" int qoq_quantize_weights_smoothed(const void* W, const void* smooth, int N, int K,
+                                             int group, void* packed, void* s1, void* stream) {
+  if (!smooth) return QOQ_ERR_INVALID_ARG;
+  return quantize_weights_impl(W, smooth, N, K, group, packed, s1, stream);
 }
 
 extern "C" int qoq_pack_codes(const uint8_t* q, const int8_t* s2, const uint8_t* z, int N,
