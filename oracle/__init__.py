@@ -16,7 +16,10 @@ full list):
   (the partial-sum dequantization that per-group W4A4 needs and W4A8 avoids)
   and "Part5 LLM部署技术", 3. 实践扩展：QServe（W4A8KV4）;
 * per-input-channel smoothing (calibration maxima, X / s, W * s) -- "Part5
-  LLM部署技术", 1.1 权重-激活联合量化：SmoothQuant.
+  LLM部署技术", 1.1 权重-激活联合量化：SmoothQuant;
+* SiLU(gate) * up between the gate_up and down projections -- the fused
+  output-side step of "Part5 LLM部署技术", 3. 实践扩展：QServe（W4A8KV4）
+  (kernel fusion), for the SwiGLU MLP of the served models.
 """
 from __future__ import annotations
 
@@ -97,6 +100,7 @@ def _load():
             lib.orc_smooth_factors.argtypes = [P, I, P, I, I, P]
             lib.orc_smooth_weights.argtypes = [P, P, I, I, P]
             lib.orc_smooth_act.argtypes = [P, P, I, I, P]
+            lib.orc_silu_mul.argtypes = [P, P, ctypes.c_long, P]
             lib.orc_num_threads.restype = I
             _lib = lib
     return _lib
@@ -311,6 +315,17 @@ def smooth_act(X, s):
     out = np.empty((M, K), np.uint16)
     _load().orc_smooth_act(_p(X), _p(s), M, K, _p(out))
     return out.view(np.float16)
+
+
+def silu_mul(G, U):
+    """H = fp16(silu(G) * U), elementwise, formed in binary64 (float16 in,
+    float16 out): the step between the gate_up and down projections."""
+    G = _as_f16_bits(G)
+    U = _as_f16_bits(U)
+    assert G.shape == U.shape
+    H = np.empty(G.shape, np.uint16)
+    _load().orc_silu_mul(_p(G), _p(U), G.size, _p(H))
+    return H.view(np.float16)
 
 
 def num_threads() -> int:

@@ -350,6 +350,24 @@ void orc_smooth_act(const uint16_t* X, const uint16_t* s, int M, int K, uint16_t
             Xp[(size_t)m * K + k] = orc_f2h(orc_h2f(X[(size_t)m * K + k]) / orc_h2f(s[k]));
 }
 
+/* ---------------------------------------------------------------------------
+ * The output-side step the gate_up GEMM's epilogue takes over ("Part5
+ * LLM部署技术", 3. 实践扩展：QServe（W4A8KV4）, kernel fusion): the MLP of the
+ * served models (Llama-3-8B, Qwen1.5-72B) applies SiLU to the gate half of
+ * the fused gate_up projection and multiplies by the up half; the pages name
+ * the models, not the formula, so this is the reading taken.  G and U are
+ * the FP16 outputs of the two halves (M x I); H = fp16(silu(g) * u) with
+ * silu(x) = x / (1 + exp(-x)), formed in binary64.  H is then quantized per
+ * token (orc_quant_act) for the down projection.
+ * ------------------------------------------------------------------------- */
+void orc_silu_mul(const uint16_t* G, const uint16_t* U, long count, uint16_t* H) {
+    for (long i = 0; i < count; ++i) {
+        double g = orc_h2d(G[i]);
+        double silu = g / (1.0 + exp(-g));
+        H[i] = orc_d2h(silu * orc_h2d(U[i]));
+    }
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
     extern int omp_get_max_threads(void);

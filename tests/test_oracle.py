@@ -565,3 +565,40 @@ def test_smoothing_moves_outliers_from_activations_to_weights(oracle):
     assert rx > 10 and rxs < rx / 2
     assert rws > rw
     assert abs(np.log(rxs / np.sqrt(rx * rw))) < np.log(2)
+
+
+# ---------------------------------------------------------------------------
+# SiLU(gate) * up (the step between the gate_up and down projections)
+# ---------------------------------------------------------------------------
+
+def test_silu_mul_hand_examples(oracle):
+    for (g, u), (hh,) in _golden("silu_mul"):
+        h = oracle.silu_mul(np.array([float(g)], np.float16), np.array([float(u)], np.float16))
+        assert h.view(np.uint16)[0] == int(hh, 16), (g, u, h)
+
+
+def test_silu_odd_part_is_the_identity(oracle):
+    """silu(x) - silu(-x) = x exactly (sigma(x) + sigma(-x) = 1), so with
+    u = 1 the two FP16 results differ by x up to their two roundings."""
+    g = np.random.default_rng(2).uniform(-12, 12, 4000).astype(np.float16)
+    one = np.ones_like(g)
+    hp = oracle.silu_mul(g, one).astype(np.float64)
+    hn = oracle.silu_mul(-g, one).astype(np.float64)
+    ulp = np.spacing(np.abs(hp).astype(np.float16)).astype(np.float64) + \
+        np.spacing(np.abs(hn).astype(np.float16)).astype(np.float64)
+    assert np.all(np.abs((hp - hn) - g.astype(np.float64)) <= ulp)
+
+
+def test_silu_limits_and_linearity_in_up(oracle):
+    g = np.array([30.0, 60.0, -30.0, -60.0], np.float16)
+    u = np.array([1.5, -2.0, 3.0, 1.0], np.float16)
+    h = oracle.silu_mul(g, u).astype(np.float64)
+    assert h[0] == 45.0 and h[1] == -120.0          # silu(x) = x for large x
+    assert abs(h[2]) <= 2.0 ** -24 and h[3] == 0.0  # vanishes for very negative x
+    # scaling up by a power of two scales h exactly (away from under/overflow)
+    g2 = np.random.default_rng(4).uniform(-6, 6, 500).astype(np.float16)
+    u2 = np.random.default_rng(5).uniform(0.5, 2, 500).astype(np.float16)
+    a = oracle.silu_mul(g2, u2).astype(np.float64)
+    b = oracle.silu_mul(g2, (u2.astype(np.float64) * 4).astype(np.float16)).astype(np.float64)
+    keep = np.abs(a) > 2.0 ** -12
+    assert np.array_equal(b[keep], 4 * a[keep])

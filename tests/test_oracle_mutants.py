@@ -173,6 +173,15 @@ MUTANTS = [
     ("smooth_factor_row_max_of_weights",
      "float v = fabsf(orc_h2f(W[(size_t)n * K + k]));\n            if (v > aw) aw = v;",
      "float v = fabsf(orc_h2f(W[(size_t)n * K + (k % N)]));\n            if (v > aw) aw = v;"),
+    # SiLU(gate) * up
+    ("silu_is_sigmoid",
+     "double silu = g / (1.0 + exp(-g));", "double silu = 1.0 / (1.0 + exp(-g));"),
+    ("silu_exponent_sign",
+     "double silu = g / (1.0 + exp(-g));", "double silu = g / (1.0 + exp(g));"),
+    ("silu_gate_and_up_swapped",
+     "double g = orc_h2d(G[i]);", "double g = orc_h2d(U[i]);"),
+    ("silu_without_up",
+     "H[i] = orc_d2h(silu * orc_h2d(U[i]));", "H[i] = orc_d2h(silu);"),
 ]
 
 
