@@ -323,6 +323,34 @@ QOQ_API int qoq_w4a8_linear(const void* X, int M, int K, const void* packed, con
                             int N, int group, int8_t* X8, void* sx, void* Y, void* ws,
                             size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * The MLP's gate_up projection with its output step fused into the GEMM
+ * epilogue (kernel fusion, "Part5 LLM部署技术", 3. 实践扩展：QServe
+ * （W4A8KV4）), for the SwiGLU MLP of the served models: the pages name the
+ * models (Llama-3-8B, Qwen1.5-72B), not the formula, so the step taken is
+ * H = fp16(silu(gate) * up), silu(x) = x / (1 + exp(-x)), and H is then
+ * quantized per token to INT8 for the down projection.
+ *
+ * qoq_quantize_weights_gate_up: offline, the fused weight W (device, FP16,
+ *   2I x K row-major: gate rows 0 .. I-1, then up rows I .. 2I-1; I % 64 ==
+ *   0) quantized as qoq_quantize_weights, packed so that every 128-row tile
+ *   t holds the gate rows 64t .. 64t+63 in its rows 0..63 and the up rows of
+ *   the same channels in rows 64..127; s1 (FP16[2I]) in that packed order.
+ * qoq_w4a8_gate_up_silu: X8 / sx (M x K, from qoq_quantize_act_per_token)
+ *   times that weight; the epilogue writes H (device, FP16 M x I) instead of
+ *   the 2I outputs, gate and up each formed exactly as qoq_w4a8_gemm forms
+ *   an output (fp16 of acc * sx * s1), h = fp16(silu(g) * u) in binary32
+ *   with the C library's expf.  K is not split.  Then H8 / sh (M x I INT8,
+ *   FP16[M]) = qoq_quantize_act_per_token(H), launched as the GEMM's
+ *   programmatic dependent: the operands of the down projection's
+ *   qoq_w4a8_gemm.  Asynchronous on `stream`.
+ * ---------------------------------------------------------------------- */
+QOQ_API int qoq_quantize_weights_gate_up(const void* W, int I, int K, int group, void* packed,
+                                         void* s1, void* stream);
+QOQ_API int qoq_w4a8_gate_up_silu(const int8_t* X8, const void* sx, const void* packed,
+                                  const void* s1, int M, int I, int K, int group, void* H,
+                                  int8_t* H8, void* sh, void* stream);
+
 /* qoq_w4a8_linear as one kernel, for a few decode rows: the activation
  * quantizer fused into the GEMM ("Part5 LLM部署技术", 3. 实践扩展：QServe
  * （W4A8KV4）, kernel fusion).  Same arguments and the same results (X8, sx

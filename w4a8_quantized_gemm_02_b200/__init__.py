@@ -34,6 +34,7 @@ EXPORTS = (
     "qoq_gemm_workspace_bytes", "qoq_gemm_workspace_bytes_config",
     "qoq_w4a8_gemm_static_ws", "qoq_selftest_wait_timeout", "qoq_w4a8_linear_fused",
     "qoq_smooth_factors", "qoq_quantize_weights_smoothed", "qoq_quantize_act_per_token_smoothed",
+    "qoq_quantize_weights_gate_up", "qoq_w4a8_gate_up_silu",
 )
 
 _lock = threading.Lock()
@@ -76,6 +77,10 @@ def lib() -> ctypes.CDLL:
             L.qoq_unpack_weights.argtypes = [P, I, I, I, P, P, P, P, P]
             L.qoq_quantize_act_per_token.restype = I
             L.qoq_quantize_act_per_token.argtypes = [P, I, I, P, P, P]
+            L.qoq_quantize_weights_gate_up.restype = I
+            L.qoq_quantize_weights_gate_up.argtypes = [P, I, I, I, P, P, P]
+            L.qoq_w4a8_gate_up_silu.restype = I
+            L.qoq_w4a8_gate_up_silu.argtypes = [P, P, P, P, I, I, I, I, P, P, P, P]
             L.qoq_smooth_factors.restype = I
             L.qoq_smooth_factors.argtypes = [P, I, P, I, I, P, P]
             L.qoq_quantize_weights_smoothed.restype = I
@@ -328,6 +333,45 @@ def quantize_act_per_token(X, out=None, stream=None):
     _check(lib().qoq_quantize_act_per_token(_ptr(X), M, K, _ptr(X8), _ptr(sx),
                                             _stream(stream)), "qoq_quantize_act_per_token")
     return X8, sx
+
+
+def quantize_weights_gate_up(W, group: int = 128, stream=None):
+    """A fused gate_up weight W (2I, K) float16 (gate rows first) ->
+    (packed, s1 float16[2I]) in the interleaved tile order."""
+    import torch
+    _need_cuda(W, "W", torch.float16, 2)
+    N2, K = W.shape
+    if N2 % 128:
+        raise ValueError("W must have 2I rows with I % 64 == 0")
+    nbytes = packed_weight_bytes(N2, K, group)
+    if nbytes == 0:
+        raise QoQError(QOQ_ERR_INVALID_ARG, "qoq_packed_weight_bytes")
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    s1 = torch.empty(N2, dtype=torch.float16, device=W.device)
+    _check(lib().qoq_quantize_weights_gate_up(_ptr(W), N2 // 2, K, group, _ptr(packed), _ptr(s1),
+                                              _stream(stream)), "qoq_quantize_weights_gate_up")
+    return packed, s1
+
+
+def w4a8_gate_up_silu(X8, sx, packed, s1, I: int, group: int = 128, out=None, stream=None):
+    """H = silu(gate) * up (M, I) float16 from the gate_up weight, and its
+    per-token INT8 quantization (H8, sh) for the down projection."""
+    import torch
+    M, K = _need_gemm_operands(X8, sx, packed, s1, 2 * I, group)
+    dev = X8.device
+    if out is None:
+        H = torch.empty((M, I), dtype=torch.float16, device=dev)
+        H8 = torch.empty((M, I), dtype=torch.int8, device=dev)
+        sh = torch.empty(M, dtype=torch.float16, device=dev)
+    else:
+        H, H8, sh = out
+        _need_cuda(H, "H", torch.float16, shape=(M, I), device=dev)
+        _need_cuda(H8, "H8", torch.int8, shape=(M, I), device=dev)
+        _need_cuda(sh, "sh", torch.float16, shape=(M,), device=dev)
+    _check(lib().qoq_w4a8_gate_up_silu(_ptr(X8), _ptr(sx), _ptr(packed), _ptr(s1), M, I, K, group,
+                                       _ptr(H), _ptr(H8), _ptr(sh), _stream(stream)),
+           "qoq_w4a8_gate_up_silu")
+    return H, H8, sh
 
 
 def smooth_factors(Xcal, W, stream=None):

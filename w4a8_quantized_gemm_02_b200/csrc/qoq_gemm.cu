@@ -359,7 +359,11 @@ struct WeightStream {
   }
 };
 
-template <int TOK, bool kCluster, bool kFuseX>
+// kGateUp: the weight is a fused gate_up projection packed with
+// qoq_quantize_weights_gate_up (tile rows 0..63 gate, 64..127 up of the same
+// 64 channels); the epilogue writes H = fp16(silu(gate) * up), M x (N / 2),
+// instead of Y.
+template <int TOK, bool kCluster, bool kFuseX, bool kGateUp>
 __global__ void __launch_bounds__(Cfg<TOK>::kThreads, 1)
 w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args) {
   using C = Cfg<TOK, kCluster, kFuseX>;
@@ -839,6 +843,39 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
 #pragma unroll
               for (int e = 0; e < 4; ++e) dst[e] = src[e];
             }
+          } else if constexpr (kGateUp) {
+            // every warp's 16 outputs of the chunk in FP16, [column][row], in
+            // its staging buffer; the up warps' (lane quarters 2, 3) reach
+            // the gate warps (quarters 0, 1) of the same channels there
+            __half* st = reinterpret_cast<__half*>(stage);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float scale = __fmul_rn(sx_w[c0 + j], s1r);
+              st[j * 32 + lane] =
+                  __float2half_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(v[j])), scale));
+            }
+            asm volatile("bar.sync 2, 128;" ::: "memory");
+            if (q4 < 2) {
+              const __half* up = reinterpret_cast<const __half*>(
+                  smem + C::kOffEpi + (((q4 + 2) - C::kWarpEpi0) & 3) * kStageBytesEpi);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const float g = __half2float(st[j * 32 + lane]);
+                const float u = __half2float(up[j * 32 + lane]);
+                st[j * 32 + lane] = __float2half_rn(__fmul_rn(__fdiv_rn(g, 1.0f + expf(-g)), u));
+              }
+              __syncwarp();
+              if (c0 + tc < c_end) {
+                const uint4* src = reinterpret_cast<const uint4*>(st + tc * 32 + 16 * th);
+                uint4* dst = reinterpret_cast<uint4*>(
+                    args.Y + static_cast<size_t>(m0 + c0 + tc) * (N / 2) + w.nt * 64 + q4 * 32 +
+                    16 * th);
+                dst[0] = src[0];
+                dst[1] = src[1];
+              }
+            }
+            // the up warps may overwrite their staging buffers afterwards
+            asm volatile("bar.sync 2, 128;" ::: "memory");
           } else {
             __half* st = reinterpret_cast<__half*>(stage);
 #pragma unroll
@@ -932,17 +969,17 @@ struct Plan {
 // Largest K split a cluster can reduce in the leader's shared memory.
 int max_cluster_split(int tok) { return tok <= 16 ? 8 : tok <= 32 ? 3 : 1; }
 
-template <int TOK, bool kCluster, bool kFuseX>
+template <int TOK, bool kCluster, bool kFuseX, bool kGateUp>
 __global__ void __launch_bounds__(Cfg<TOK>::kThreads, 1)
 w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args);
 
 template <int TOK>
 int query_active_clusters(int cs) {
   using C = Cfg<TOK, true>;
-  if (cudaFuncSetAttribute(w4a8_gemm_kernel<TOK, true, false>,
+  if (cudaFuncSetAttribute(w4a8_gemm_kernel<TOK, true, false, false>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
           cudaSuccess ||
-      cudaFuncSetAttribute(w4a8_gemm_kernel<TOK, true, false>,
+      cudaFuncSetAttribute(w4a8_gemm_kernel<TOK, true, false, false>,
                            cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess) {
     cudaGetLastError();
     return 0;
@@ -959,7 +996,7 @@ int query_active_clusters(int cs) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, w4a8_gemm_kernel<TOK, true, false>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, w4a8_gemm_kernel<TOK, true, false, false>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -1112,7 +1149,7 @@ size_t ws_bytes_for(const Plan& p, int N) {
   return kCounterBytes + part;
 }
 
-template <int TOK, bool kCluster, bool kFuseX>
+template <int TOK, bool kCluster, bool kFuseX, bool kGateUp = false>
 int launch_kernel(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cudaStream_t stream,
                bool pdl) {
   // the same layout as the kernel instance (its shared-memory size)
@@ -1122,7 +1159,7 @@ int launch_kernel(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cuda
   if (cudaGetDevice(&dev) != cudaSuccess) return QOQ_ERR_CUDA;
   const int bit = dev < 31 ? (1 << dev) : 0;
   if (!bit || !(__atomic_load_n(&configured_mask, __ATOMIC_ACQUIRE) & bit)) {
-    if (cudaFuncSetAttribute(w4a8_gemm_kernel<TOK, kCluster, kFuseX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(w4a8_gemm_kernel<TOK, kCluster, kFuseX, kGateUp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess)
       return QOQ_ERR_CUDA;
     if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_RELEASE);
@@ -1148,7 +1185,7 @@ int launch_kernel(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cuda
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  if (cudaLaunchKernelEx(&cfg, w4a8_gemm_kernel<TOK, kCluster, kFuseX>, map, a) != cudaSuccess) return QOQ_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, w4a8_gemm_kernel<TOK, kCluster, kFuseX, kGateUp>, map, a) != cudaSuccess) return QOQ_ERR_CUDA;
   return QOQ_OK;
 }
 
@@ -1156,7 +1193,10 @@ int launch_kernel(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cuda
 // splits K across a cluster, the plain one otherwise.
 template <int TOK>
 int launch_tok(const CUtensorMap& map, const GemmArgs& a, const Plan& p, cudaStream_t stream,
-               bool pdl) {
+               bool pdl, bool gate_up) {
+  if constexpr (TOK <= 128 && TOK != 176) {
+    if (gate_up) return launch_kernel<TOK, false, false, true>(map, a, p, stream, pdl);
+  }
   const bool fuse = a.X != nullptr;
   if constexpr (TOK <= 32) {
     if (p.cs > 1) return launch_kernel<TOK, true, false>(map, a, p, stream, pdl);
@@ -1173,6 +1213,7 @@ struct GemmLaunch {
   Plan p;
   CUtensorMap map;
   GemmArgs a;
+  bool gate_up = false;   // the epilogue writes silu(gate) * up (kGateUp kernel)
 };
 
 // Validate the arguments, pick the plan and encode the tensor map.  Calls no
@@ -1265,13 +1306,13 @@ int gemm_launch(GemmLaunch L, void* stream, bool weights_independent, bool clear
       cudaMemsetAsync(L.a.ws_count, 0, kCounterBytes, s) != cudaSuccess)
     return QOQ_ERR_CUDA;
   switch (L.p.tok) {
-    case 16: return launch_tok<16>(L.map, L.a, L.p, s, pdl);
-    case 32: return launch_tok<32>(L.map, L.a, L.p, s, pdl);
-    case 64: return launch_tok<64>(L.map, L.a, L.p, s, pdl);
-    case 128: return launch_tok<128>(L.map, L.a, L.p, s, pdl);
-    case 176: return launch_tok<176>(L.map, L.a, L.p, s, pdl);
-    case 192: return launch_tok<192>(L.map, L.a, L.p, s, pdl);
-    default: return launch_tok<256>(L.map, L.a, L.p, s, pdl);
+    case 16: return launch_tok<16>(L.map, L.a, L.p, s, pdl, L.gate_up);
+    case 32: return launch_tok<32>(L.map, L.a, L.p, s, pdl, L.gate_up);
+    case 64: return launch_tok<64>(L.map, L.a, L.p, s, pdl, L.gate_up);
+    case 128: return launch_tok<128>(L.map, L.a, L.p, s, pdl, L.gate_up);
+    case 176: return launch_tok<176>(L.map, L.a, L.p, s, pdl, L.gate_up);
+    case 192: return launch_tok<192>(L.map, L.a, L.p, s, pdl, L.gate_up);
+    default: return launch_tok<256>(L.map, L.a, L.p, s, pdl, L.gate_up);
   }
 }
 
@@ -1440,6 +1481,27 @@ extern "C" int qoq_w4a8_linear_fused(const void* X, int M, int K, const void* pa
   L.a.X = static_cast<const __half*>(X);
   L.a.X8 = X8;
   return gemm_launch(L, stream, /*weights_independent=*/false, false);
+}
+
+extern "C" int qoq_w4a8_gate_up_silu(const int8_t* X8, const void* sx, const void* packed,
+                                     const void* s1, int M, int I, int K, int group, void* H,
+                                     int8_t* H8, void* sh, void* stream) {
+  if (!X8 || !sx || !packed || !s1 || !H || !H8 || !sh) return QOQ_ERR_INVALID_ARG;
+  if (M <= 0 || I <= 0 || I % 64 != 0) return QOQ_ERR_INVALID_ARG;
+  if (!aligned16(H) || !aligned16(H8) || !aligned16(sh)) return QOQ_ERR_INVALID_ARG;
+  // K is not split (each CTA's epilogue needs the whole sum of both halves)
+  // and the token tile is one the gate_up epilogue is built for
+  int tok = 0;
+  if (M > 64) tok = 128;
+  GemmLaunch L;
+  if (int st = gemm_prepare(X8, sx, packed, s1, M, 2 * I, K, group, H, nullptr, tok, 1, nullptr,
+                            0, L))
+    return st;
+  L.gate_up = true;
+  if (int st = gemm_launch(L, stream, /*weights_independent=*/false, false)) return st;
+  // the per-token INT8 quantization of H for the down projection, launched
+  // as the GEMM's programmatic dependent (it waits for the GEMM to complete)
+  return launch_act_quant(H, M, I, H8, sh, stream, true, nullptr);
 }
 
 extern "C" int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int* splits, int* ctas,

@@ -34,6 +34,17 @@ __device__ __forceinline__ uint4 smooth8(uint4 v, uint4 f) {
   return v;
 }
 
+// Packed row n of a weight -> its row in the caller's matrix.  Plain
+// weights: n.  A fused gate_up weight of 2I rows (gate rows 0 .. I-1, up
+// rows I .. 2I-1, gate_up_i = I): every 128-row tile t holds gate rows
+// 64t .. 64t+63 in its rows 0..63 and the up rows of the same channels in
+// rows 64..127, so one tile of the GEMM holds both halves of 64 outputs.
+__device__ __forceinline__ int source_row(int n, int gate_up_i) {
+  if (gate_up_i == 0) return n;
+  const int t = n >> 7, r = n & 127;
+  return r < 64 ? 64 * t + r : gate_up_i + 64 * t + (r - 64);
+}
+
 // Exact round-half-even of a / b for b > 0.
 __device__ __forceinline__ int div_rne(int a, int b) {
   int q = a / b;
@@ -148,11 +159,12 @@ act_quant_kernel(const __half* __restrict__ X, int M, int K, int8_t* __restrict_
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 row_scale_kernel(const __half* __restrict__ W, int N, int K, __half* __restrict__ s1,
-                 const __half* __restrict__ smooth) {
+                 const __half* __restrict__ smooth, int gate_up_i) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= N) return;
-  const uint4* row = reinterpret_cast<const uint4*>(W + static_cast<size_t>(warp) * K);
+  const uint4* row =
+      reinterpret_cast<const uint4*>(W + static_cast<size_t>(source_row(warp, gate_up_i)) * K);
   float amax = 0.0f;
   for (int i = lane; i < K / 8; i += 32) {
     uint4 v = __ldg(row + i);
@@ -184,7 +196,7 @@ __device__ __forceinline__ int level1_code(float w, float s1f) {
 __global__ void __launch_bounds__(128)
 pack_weights_kernel(const __half* __restrict__ W, int K, int group,
                     const __half* __restrict__ s1, uint8_t* __restrict__ packed,
-                    int blk_bytes, const __half* __restrict__ smooth) {
+                    int blk_bytes, const __half* __restrict__ smooth, int gate_up_i) {
   __shared__ __align__(16) uint8_t tile[kTileN * kPackRowBytes];
   const int kt = blockIdx.x, nt = blockIdx.y;
   const int n0 = nt * kTileN, k0 = kt * kTileK;
@@ -193,7 +205,7 @@ pack_weights_kernel(const __half* __restrict__ W, int K, int group,
   for (int c = threadIdx.x; c < kTileN * 16; c += 128) {
     const int row = c >> 4, col = c & 15;
     uint4 v = __ldg(reinterpret_cast<const uint4*>(
-                        W + static_cast<size_t>(n0 + row) * K + k0) + col);
+                        W + static_cast<size_t>(source_row(n0 + row, gate_up_i)) * K + k0) + col);
     if (smooth) v = smooth8<false>(v, __ldg(reinterpret_cast<const uint4*>(smooth + k0) + col));
     *reinterpret_cast<uint4*>(tile + row * kPackRowBytes + col * 16) = v;
   }
@@ -442,7 +454,7 @@ extern "C" int qoq_smooth_factors(const void* Xcal, int Mc, const void* W, int N
 namespace qoq {
 namespace {
 int quantize_weights_impl(const void* W, const void* smooth, int N, int K, int group,
-                          void* packed, void* s1, void* stream) {
+                          void* packed, void* s1, void* stream, int gate_up_i) {
   if (!W || !packed || !s1) return QOQ_ERR_INVALID_ARG;
   if (int st = check_weight_shape(N, K, group)) return st;
   if (!aligned16(W) || !aligned16(packed) || !aligned16(s1) || (smooth && !aligned16(smooth)))
@@ -452,11 +464,11 @@ int quantize_weights_impl(const void* W, const void* smooth, int N, int K, int g
   const __half* Wh = static_cast<const __half*>(W);
   const __half* sm = static_cast<const __half*>(smooth);
   __half* s1h = static_cast<__half*>(s1);
-  row_scale_kernel<<<(N + 7) / 8, 256, 0, s>>>(Wh, N, K, s1h, sm);
+  row_scale_kernel<<<(N + 7) / 8, 256, 0, s>>>(Wh, N, K, s1h, sm, gate_up_i);
   if (int st = launch_status()) return st;
   dim3 grid(K / kTileK, N / kTileN);
   pack_weights_kernel<<<grid, 128, 0, s>>>(Wh, K, group, s1h, static_cast<uint8_t*>(packed),
-                                           static_cast<int>(block_bytes(group)), sm);
+                                           static_cast<int>(block_bytes(group)), sm, gate_up_i);
   return launch_status();
 }
 }  // namespace
@@ -464,13 +476,19 @@ int quantize_weights_impl(const void* W, const void* smooth, int N, int K, int g
 
 extern "C" int qoq_quantize_weights(const void* W, int N, int K, int group, void* packed,
                                     void* s1, void* stream) {
-  return quantize_weights_impl(W, nullptr, N, K, group, packed, s1, stream);
+  return quantize_weights_impl(W, nullptr, N, K, group, packed, s1, stream, 0);
+}
+
+extern "C" int qoq_quantize_weights_gate_up(const void* W, int I, int K, int group, void* packed,
+                                            void* s1, void* stream) {
+  if (I <= 0 || I % 64 != 0) return QOQ_ERR_INVALID_ARG;
+  return quantize_weights_impl(W, nullptr, 2 * I, K, group, packed, s1, stream, I);
 }
 
 extern "C" int qoq_quantize_weights_smoothed(const void* W, const void* smooth, int N, int K,
                                              int group, void* packed, void* s1, void* stream) {
   if (!smooth) return QOQ_ERR_INVALID_ARG;
-  return quantize_weights_impl(W, smooth, N, K, group, packed, s1, stream);
+  return quantize_weights_impl(W, smooth, N, K, group, packed, s1, stream, 0);
 }
 
 extern "C" int qoq_pack_codes(const uint8_t* q, const int8_t* s2, const uint8_t* z, int N,
