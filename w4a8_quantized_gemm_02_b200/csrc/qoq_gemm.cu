@@ -367,6 +367,7 @@ template <int TOK, bool kCluster, bool kFuseX, bool kGateUp>
 __global__ void __launch_bounds__(Cfg<TOK>::kThreads, 1)
 w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args) {
   using C = Cfg<TOK, kCluster, kFuseX>;
+  static_assert(!kGateUp || (!kCluster && !kFuseX), "gate_up: no cluster split, X8 given");
   constexpr int S = C::kStages;
   // a launch with less shared memory than this layout needs does nothing
   // (every thread returns before any barrier) and records the mistake
@@ -657,6 +658,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
     // transposed read of the staging buffer: lane reads column c = lane / 2,
     // rows 16 * (lane & 1) .. +15 of this warp's 32-row slice
     const int tc = lane >> 1, th = lane & 1;
+    uint32_t gu_seq = 0;                    // gate_up: chunks handed over so far
     grid_dependency_wait();                 // sx comes from the preceding grid under PDL
     // Own activations, before the first accumulator can be ready: the M FP16
     // token rows (contiguous, M*K*2 bytes) in one bulk copy, each row's scale
@@ -725,8 +727,14 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
                                  : 0.0f;
         __syncwarp();
       }
-      const bool ok = mbar_wait(bar_accfull + 8 * b, (lt / C::kAcc) & 1, abort_flag,
-                                &g_error_word, kErrEpilogue);
+      bool ok = mbar_wait(bar_accfull + 8 * b, (lt / C::kAcc) & 1, abort_flag,
+                          &g_error_word, kErrEpilogue);
+      if constexpr (kGateUp) {
+        // the four warps meet at a named barrier in every chunk below: they
+        // decide together whether to run this unit, so that all or none of
+        // them reach each barrier (every wait before this one is bounded)
+        ok = named_barrier_and(3, 128, ok && *abort_flag == 0u);
+      }
       if (!__all_sync(0xffffffffu, ok)) break;
       // At this CTA's last accumulator a kernel launched after this one as
       // its programmatic dependent may be scheduled: it waits for this grid
@@ -801,7 +809,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
         __syncwarp();
         write_out = __shfl_sync(0xffffffffu, last ? 1 : 0, 0) != 0;
       }
-      if (write_out && *abort_flag == 0u) {
+      if (write_out && (kGateUp || *abort_flag == 0u)) {
         const int32_t* parts = args.ws_part + (static_cast<size_t>(w.mt * splits) * TOK) * N;
         // software-pipelined over 16-column chunks: the next chunk's load
         // from tensor memory is in flight while this chunk is scaled and
@@ -812,7 +820,10 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
           tmem_ld_wait(vn);
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] = vn[j];
-          if (c0 + 16 < c_end) tmem_ld_32x32b_x16(t_acc + c0 + 16, vn);
+          // (the gate_up epilogue issues it once this chunk's outputs are in
+          // its staging buffer, which keeps its registers within the
+          // launch's budget)
+          if (!kGateUp && c0 + 16 < c_end) tmem_ld_32x32b_x16(t_acc + c0 + 16, vn);
           if (cs > 1) {
             // add the cluster's slices from this CTA's reduction buffer
             for (int q = 0; q < cs - 1; ++q) {
@@ -823,13 +834,37 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
                 if (c0 + j < c_end) v[j] += rp[(c0 + j) * 32];
             }
           } else if (splits > 1) {
-            for (int q = 0; q < splits; ++q) {
-              if (q == w.split) continue;
-              const int32_t* p = parts + (static_cast<size_t>(q) * TOK + c0) * N + nrow0 + lane;
+            // add the other splits' partials of this chunk's tokens, taken
+            // as a list of (split, token) pairs, 16 pairs per batch: the
+            // batch's loads are unconditional (a pair past the end of the
+            // list reads the last split's row again and is not added), so
+            // all 16 are in flight together and a batch costs one L2 round
+            // trip.  The sums collect in the warp's staging buffer, each
+            // lane in its own column.
+            const int cnt = c_end - c0 < 16 ? c_end - c0 : 16;
+            uint32_t* st = reinterpret_cast<uint32_t*>(stage);
 #pragma unroll
-              for (int j = 0; j < 16; ++j)
-                if (c0 + j < c_end) v[j] += static_cast<uint32_t>(__ldcg(p + static_cast<size_t>(j) * N));
+            for (int j = 0; j < 16; ++j) st[j * 32 + lane] = v[j];
+            int q = 0, jj = 0;
+            while (q < splits) {
+              uint32_t t[16];
+              int qb[16], jb[16];
+#pragma unroll
+              for (int b = 0; b < 16; ++b) {
+                qb[b] = q;
+                jb[b] = jj;
+                const int qc = q < splits ? q : splits - 1;
+                t[b] = static_cast<uint32_t>(
+                    __ldcg(parts + (static_cast<size_t>(qc) * TOK + c0 + jj) * N + nrow0 + lane));
+                jj = jj + 1 == cnt ? 0 : jj + 1;
+                q = jj == 0 ? q + 1 : q;
+              }
+#pragma unroll
+              for (int b = 0; b < 16; ++b)
+                if (qb[b] < splits && qb[b] != w.split) st[jb[b] * 32 + lane] += t[b];
             }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = st[j * 32 + lane];
           }
           if (args.acc) {
             uint32_t* st = reinterpret_cast<uint32_t*>(stage);
@@ -844,38 +879,48 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmArgs args
               for (int e = 0; e < 4; ++e) dst[e] = src[e];
             }
           } else if constexpr (kGateUp) {
-            // every warp's 16 outputs of the chunk in FP16, [column][row], in
-            // its staging buffer; the up warps' (lane quarters 2, 3) reach
-            // the gate warps (quarters 0, 1) of the same channels there
-            __half* st = reinterpret_cast<__half*>(stage);
+            // Every warp's 16 outputs of the chunk in FP16, [column][row], go
+            // to half h of its staging buffer (h alternates chunk by chunk,
+            // across units too, so a half is written again only after every
+            // warp has finished reading it: they all passed the barrier of
+            // the chunk in between).  The four warps pass the same barriers:
+            // they agreed at the unit's start to run its chunks.  Then all four warps form
+            // silu(gate) * up: warp q4 takes the gate rows of lane quarter
+            // q4 & 1 (their up rows are quarter (q4 & 1) + 2) for token
+            // columns 8 (q4 >> 1) .. +7, writes the products over the gate
+            // values it read and stores them to H.
+            const int hb = static_cast<int>(gu_seq & 1u);
+            __half* st = reinterpret_cast<__half*>(stage) + hb * 512;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const float scale = __fmul_rn(sx_w[c0 + j], s1r);
               st[j * 32 + lane] =
                   __float2half_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(v[j])), scale));
             }
+            if (c0 + 16 < c_end) tmem_ld_32x32b_x16(t_acc + c0 + 16, vn);
             asm volatile("bar.sync 2, 128;" ::: "memory");
-            if (q4 < 2) {
-              const __half* up = reinterpret_cast<const __half*>(
-                  smem + C::kOffEpi + (((q4 + 2) - C::kWarpEpi0) & 3) * kStageBytesEpi);
+            ++gu_seq;
+            const int gq = q4 & 1, jb = 8 * (q4 >> 1);
+            __half* gs = reinterpret_cast<__half*>(
+                             smem + C::kOffEpi + ((gq - C::kWarpEpi0) & 3) * kStageBytesEpi) +
+                         hb * 512;
+            const __half* us = reinterpret_cast<const __half*>(
+                                   smem + C::kOffEpi + ((gq + 2 - C::kWarpEpi0) & 3) * kStageBytesEpi) +
+                               hb * 512;
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const float g = __half2float(st[j * 32 + lane]);
-                const float u = __half2float(up[j * 32 + lane]);
-                st[j * 32 + lane] = __float2half_rn(__fmul_rn(__fdiv_rn(g, 1.0f + expf(-g)), u));
-              }
-              __syncwarp();
-              if (c0 + tc < c_end) {
-                const uint4* src = reinterpret_cast<const uint4*>(st + tc * 32 + 16 * th);
-                uint4* dst = reinterpret_cast<uint4*>(
-                    args.Y + static_cast<size_t>(m0 + c0 + tc) * (N / 2) + w.nt * 64 + q4 * 32 +
-                    16 * th);
-                dst[0] = src[0];
-                dst[1] = src[1];
-              }
+            for (int j = jb; j < jb + 8; ++j) {
+              const float g = __half2float(gs[j * 32 + lane]);
+              const float u = __half2float(us[j * 32 + lane]);
+              gs[j * 32 + lane] = __float2half_rn(__fmul_rn(__fdividef(g, 1.0f + __expf(-g)), u));
             }
-            // the up warps may overwrite their staging buffers afterwards
-            asm volatile("bar.sync 2, 128;" ::: "memory");
+            __syncwarp();
+            // lane: token column jb + lane / 4, channels 8 (lane & 3) .. +7
+            const int tq = jb + (lane >> 2), tp = lane & 3;
+            if (c0 + tq < c_end) {
+              *reinterpret_cast<uint4*>(args.Y + static_cast<size_t>(m0 + c0 + tq) * (N / 2) +
+                                        w.nt * 64 + gq * 32 + 8 * tp) =
+                  *reinterpret_cast<const uint4*>(gs + tq * 32 + 8 * tp);
+            }
           } else {
             __half* st = reinterpret_cast<__half*>(stage);
 #pragma unroll
@@ -1071,21 +1116,21 @@ int auto_tok(int M, int n_tiles) {
 
 // Cost model for the number of K splits of a decode plan: units are spread
 // over the CTAs, a unit costs its k-tiles plus a fixed overhead (pipeline
-// fill and epilogue), a split unit a little more.  Up to max_cluster_split
-// splits the partial tiles are added up inside a cluster (through the leader
-// CTA's shared memory); more splits go through the workspace in L2, whose
-// tail (partial slices written, the last arrival reading the others back)
-// grows with the tokens in the tile: on B200 a 16-token Llama QKV tile (32
-// k-tiles) ran fastest unsplit that way, while single tokens, or 64+ k-tiles
-// per unit, gained from splitting.
+// fill and epilogue), a split unit a little more.  A split is added up either
+// inside a cluster (through the leader CTA's shared memory, up to
+// max_cluster_split CTAs) or through the workspace in L2 (partial slices
+// written, the last arrival reading the others back).  Measured on B200 with
+// 16-token tiles: up to four tokens the workspace split is the faster of the
+// two (its tail is one L2 round trip per batch of 16 partial rows, and a
+// cluster waits for all of its SMs to be free); with more tokens the cluster
+// split is, while a 16-token Llama QKV tile (32 k-tiles) ran fastest unsplit
+// through the workspace.  32-token tiles ran faster unsplit than split across
+// a cluster (K = N = 2048 and 4096), so the planner keeps clusters for 16.
 int auto_splits(int tiles, int kt, int tok, int M, bool* cluster_out) {
   *cluster_out = false;
   if (tok > 32) return 1;
   const int tokens = M < tok ? M : tok;
-  // measured on B200: with up to four tokens the workspace split is the
-  // faster of the two (its tail is short, and a cluster waits for all of
-  // its SMs to be free); with more tokens the cluster split is
-  const bool cluster_ok = tokens > 4;
+  const bool cluster_ok = tokens > 4 && tok <= 16;
   const bool l2_ok = tokens <= 4 || kt >= 64;
   const long sms = sm_count();
   int best_s = 1;
