@@ -445,6 +445,72 @@ def layer_per_m(qoq, torch, layer, dev, stream, l2, peaks, int8_peak, packed0=No
     return out
 
 
+def mlp_per_m(qoq, torch, dev, stream, l2):
+    """The Llama-3-8B MLP pair per M: the gate_up projection with SiLU(gate)
+    * up fused into its epilogue plus the per-token re-quantization
+    (qoq_w4a8_gate_up_silu), the plain gate_up GEMM writing all 2I outputs
+    (what the fusion replaces), and the down GEMM on the re-quantized H;
+    each as back-to-back launches in a CUDA graph over rotated weights."""
+    gu, dn = si.LLAMA3_8B_GATE_UP, si.LLAMA3_8B_DOWN
+    I, K, G = dn.K, gu.K, gu.group
+    W = torch.from_numpy(si.weights(gu, seed=0)).to(dev)      # gate rows, then up rows
+    pg, s1g = qoq.quantize_weights_gate_up(W, G, stream=stream)
+    pp, s1p = qoq.quantize_weights(W, G, stream=stream)
+    del W
+    Wd = torch.from_numpy(si.weights(dn, seed=0)).to(dev)
+    pd, s1d = qoq.quantize_weights(Wd, G, stream=stream)
+    del Wd
+    stream.synchronize()
+    nw = copies_for(pg.numel() + pd.numel(), l2, hi=16)
+    gws = [pg] + [pg.clone() for _ in range(nw - 1)]
+    pws = [pp] + [pp.clone() for _ in range(nw - 1)]
+    dws = [pd] + [pd.clone() for _ in range(nw - 1)]
+    out = []
+    for M in gu.ms:
+        X = torch.from_numpy(si.activations(gu, M, seed=0)).to(dev)
+        X8, sx = qoq.quantize_act_per_token(X, stream=stream)
+        H = torch.empty((M, I), dtype=torch.float16, device=dev)
+        H8 = torch.empty((M, I), dtype=torch.int8, device=dev)
+        sh = torch.empty(M, dtype=torch.float16, device=dev)
+        Y2 = torch.empty((M, 2 * I), dtype=torch.float16, device=dev)
+        Yd = torch.empty((M, dn.N), dtype=torch.float16, device=dev)
+        with torch.cuda.stream(stream):
+            qoq.w4a8_gate_up_silu(X8, sx, gws[0], s1g, I, G, out=(H, H8, sh), stream=stream)
+            qoq.w4a8_gemm(X8, sx, pws[0], s1p, 2 * I, G, out=Y2, stream=stream)
+            qoq.w4a8_gemm(H8, sh, dws[0], s1d, dn.N, G, out=Yd, stream=stream)
+        stream.synchronize()
+
+        def fused():
+            for w in range(nw):
+                qoq.w4a8_gate_up_silu(X8, sx, gws[w], s1g, I, G, out=(H, H8, sh), stream=stream)
+            return nw
+
+        def plain():
+            for w in range(nw):
+                qoq.w4a8_gemm(X8, sx, pws[w], s1p, 2 * I, G, out=Y2, stream=stream)
+            return nw
+
+        def down():
+            for w in range(nw):
+                qoq.w4a8_gemm(H8, sh, dws[w], s1d, dn.N, G, out=Yd, stream=stream)
+            return nw
+
+        def pair():
+            for w in range(nw):
+                qoq.w4a8_gate_up_silu(X8, sx, gws[w], s1g, I, G, out=(H, H8, sh), stream=stream)
+                qoq.w4a8_gemm(H8, sh, dws[w], s1d, dn.N, G, out=Yd, stream=stream)
+            return nw
+        out.append({"M": M,
+                    "gate_up_silu_requant_us": graph_us_per_launch(torch, stream, fused),
+                    "gate_up_gemm_us": graph_us_per_launch(torch, stream, plain),
+                    "down_gemm_us": graph_us_per_launch(torch, stream, down),
+                    "mlp_pair_us": graph_us_per_launch(torch, stream, pair)})
+        del X, X8, sx, H, H8, sh, Y2, Yd
+    del gws, pws, dws
+    torch.cuda.synchronize()
+    return out
+
+
 def sweep_per_m(qoq, torch, dev, stream, l2, peaks, int8_peak):
     """The pure-throughput shape sweep: K = N in {2048, 4096, 8192}, group 64
     and 128, M = 1 .. 8192 in powers of two; random UINT4 codes, zeros and
@@ -667,6 +733,9 @@ def run_ours(args):
             if name in (layer.name, si.TINY.name):
                 continue
             layers[name] = layer_per_m(qoq, torch, other, dev, stream, l2, peaks, int8_peak)
+    mlp = None
+    if not args.no_layers and world == 1:
+        mlp = mlp_per_m(qoq, torch, dev, stream, l2)
     sweep = None
     if not args.no_sweep and world == 1:
         sweep = sweep_per_m(qoq, torch, dev, stream, l2, peaks, int8_peak)
@@ -717,6 +786,7 @@ def run_ours(args):
         "roofline": roofline,
         "per_m": per_m,
         "layers": layers,
+        "mlp": mlp,
         "sweep": sweep,
         "clocks": clocks,
         "gpu_launches": 2 * len(ms) * args.steps,
