@@ -19,7 +19,10 @@ full list):
   LLM部署技术", 1.1 权重-激活联合量化：SmoothQuant;
 * SiLU(gate) * up between the gate_up and down projections -- the fused
   output-side step of "Part5 LLM部署技术", 3. 实践扩展：QServe（W4A8KV4）
-  (kernel fusion), for the SwiGLU MLP of the served models.
+  (kernel fusion), for the SwiGLU MLP of the served models;
+* the 4-bit KV cache and decode attention over it -- "QServe: Cuantificación
+  W4A8KV4 y Co-diseño del Sistema ...", abstract (4-bit KV cache), and the
+  velog notes, Insight (memory-bound fused attention).
 """
 from __future__ import annotations
 
@@ -101,6 +104,9 @@ def _load():
             lib.orc_smooth_weights.argtypes = [P, P, I, I, P]
             lib.orc_smooth_act.argtypes = [P, P, I, I, P]
             lib.orc_silu_mul.argtypes = [P, P, ctypes.c_long, P]
+            lib.orc_kv4_quant.argtypes = [P, ctypes.c_long, I, P, P, P]
+            lib.orc_kv4_dequant.argtypes = [P, P, P, ctypes.c_long, I, P]
+            lib.orc_kv4_decode_attention.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, P, P]
             lib.orc_num_threads.restype = I
             _lib = lib
     return _lib
@@ -326,6 +332,54 @@ def silu_mul(G, U):
     H = np.empty(G.shape, np.uint16)
     _load().orc_silu_mul(_p(G), _p(U), G.size, _p(H))
     return H.view(np.float16)
+
+
+def kv4_quant(X):
+    """4-bit KV cache quantization of every length-d vector (last axis) of X
+    (float16): codes q (uint8, one per byte, 0..15), FP16 scale s and FP16
+    offset m per vector, x^ = s * q + m."""
+    X = _as_f16_bits(X)
+    d = X.shape[-1]
+    rows = X.size // d
+    q = np.empty(X.shape, np.uint8)
+    s = np.empty(X.shape[:-1], np.uint16)
+    m = np.empty(X.shape[:-1], np.uint16)
+    _load().orc_kv4_quant(_p(X), rows, d, _p(q), _p(s), _p(m))
+    return q, s.view(np.float16), m.view(np.float16)
+
+
+def kv4_dequant(q, s, m):
+    """x^ = s * q + m in float64 (exact)."""
+    q = np.ascontiguousarray(q, np.uint8)
+    s = _as_f16_bits(s)
+    m = _as_f16_bits(m)
+    d = q.shape[-1]
+    out = np.empty(q.shape, np.float64)
+    _load().orc_kv4_dequant(_p(q), _p(s), _p(m), q.size // d, d, _p(out))
+    return out
+
+
+def kv4_decode_attention(Q, qk, sk, mk, qv, sv, mv, seqlen):
+    """Decode attention of one query token per sequence over the 4-bit cache.
+    Q: (B, Hq, d) float16; qk, qv: (B, Hkv, L, d) uint8 codes; sk, mk, sv,
+    mv: (B, Hkv, L) float16; seqlen: (B,) lengths <= L.  Returns (out
+    float16 (B, Hq, d), out64 float64 before the FP16 rounding)."""
+    Q = _as_f16_bits(Q)
+    B, Hq, d = Q.shape
+    qk = np.ascontiguousarray(qk, np.uint8)
+    qv = np.ascontiguousarray(qv, np.uint8)
+    B2, Hkv, L, d2 = qk.shape
+    assert B2 == B and d2 == d and qv.shape == qk.shape and Hq % Hkv == 0
+    sk, mk, sv, mv = (_as_f16_bits(a) for a in (sk, mk, sv, mv))
+    for a in (sk, mk, sv, mv):
+        assert a.shape == (B, Hkv, L)
+    seqlen = np.ascontiguousarray(seqlen, np.int32)
+    assert seqlen.shape == (B,) and (seqlen >= 0).all() and (seqlen <= L).all()
+    out = np.empty((B, Hq, d), np.uint16)
+    out64 = np.empty((B, Hq, d), np.float64)
+    _load().orc_kv4_decode_attention(_p(Q), _p(qk), _p(sk), _p(mk), _p(qv), _p(sv), _p(mv),
+                                     _p(seqlen), B, Hq, Hkv, L, d, _p(out), _p(out64))
+    return out.view(np.float16), out64
 
 
 def num_threads() -> int:

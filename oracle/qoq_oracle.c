@@ -368,6 +368,115 @@ void orc_silu_mul(const uint16_t* G, const uint16_t* U, long count, uint16_t* H)
     }
 }
 
+/* ---------------------------------------------------------------------------
+ * 4-bit KV cache and decode attention over it ("QServe: Cuantificación
+ * W4A8KV4 y Co-diseño del Sistema ...", abstract: 4-bit KV cache; "QServe:
+ * W4A8KV4 Quantization and System Co-design ..." (velog notes), Insight:
+ * the fused attention is made memory-bound so that KV4 pays off).  The pages
+ * fix no format for the cache; the readings taken:
+ *  - every (token, KV head) vector x of d FP16 values is quantized on its
+ *    own, asymmetrically, to UINT4 codes with an FP16 scale s and an FP16
+ *    offset m (the vector's minimum): x^ = s * q + m;
+ *  - s = fp16(fl32(fl32(max - min) / 15)) and q = clamp(rne(fl32(fl32(x -
+ *    min) / s)), 0, 15), each operation in IEEE binary32 (the kernel's
+ *    precision, so that both sides take every integer decision alike); a
+ *    vector whose s is 0 (constant, or a range below the FP16 resolution)
+ *    gets q = 0 everywhere, so x^ = m;
+ *  - decode attention: one query token per sequence; query head h reads KV
+ *    head h / (Hq / Hkv) (grouped-query attention, as in the served
+ *    Llama-3-8B); score_t = (q . k^_t) / sqrt(d) over the sequence's first
+ *    L_b tokens; p = softmax(score); out = sum_t p_t v^_t, formed in binary64
+ *    and rounded to FP16 once; a sequence of length 0 gives out = 0.
+ * ------------------------------------------------------------------------- */
+void orc_kv4_quant(const uint16_t* X, long rows, int d, uint8_t* q, uint16_t* s, uint16_t* m) {
+    for (long r = 0; r < rows; ++r) {
+        const uint16_t* x = X + r * d;
+        float mn = orc_h2f(x[0]), mx = mn;
+        uint16_t mn_bits = x[0];
+        for (int i = 1; i < d; ++i) {
+            float v = orc_h2f(x[i]);
+            if (v < mn) { mn = v; mn_bits = x[i]; }
+            if (v > mx) mx = v;
+        }
+        float range = mx - mn;
+        uint16_t sh = orc_f2h(range / 15.0f);
+        float sv = orc_h2f(sh);
+        s[r] = sh;
+        m[r] = (mn == 0.0f) ? 0 : mn_bits;   /* -0 and +0 are the same offset */
+        for (int i = 0; i < d; ++i) {
+            int c = 0;
+            if (sv > 0.0f) {
+                float t = (orc_h2f(x[i]) - mn) / sv;
+                c = clampi((int)rne_f(t), 0, 15);
+            }
+            q[r * d + i] = (uint8_t)c;
+        }
+    }
+}
+
+/* x^ = s * q + m, exactly (binary64). */
+void orc_kv4_dequant(const uint8_t* q, const uint16_t* s, const uint16_t* m, long rows, int d,
+                     double* out) {
+    for (long r = 0; r < rows; ++r) {
+        double sv = orc_h2d(s[r]), mv = orc_h2d(m[r]);
+        for (int i = 0; i < d; ++i) out[r * d + i] = sv * (double)q[r * d + i] + mv;
+    }
+}
+
+/* Q: [B][Hq][d] FP16.  Codes qk, qv: [B][Hkv][L][d], one code per byte;
+ * sk, mk, sv, mv: [B][Hkv][L] FP16; seqlen[b] <= L.  out: [B][Hq][d] FP16,
+ * out64 (optional): the same before the FP16 rounding. */
+void orc_kv4_decode_attention(const uint16_t* Q, const uint8_t* qk, const uint16_t* sk,
+                              const uint16_t* mk, const uint8_t* qv, const uint16_t* sv,
+                              const uint16_t* mv, const int* seqlen, int B, int Hq, int Hkv,
+                              int L, int d, uint16_t* out, double* out64) {
+    const int g = Hq / Hkv;
+    double* score = (double*)malloc(sizeof(double) * (L > 0 ? L : 1));
+    double* kh = (double*)malloc(sizeof(double) * d);
+    for (int b = 0; b < B; ++b) {
+        const int Lb = seqlen[b];
+        for (int h = 0; h < Hq; ++h) {
+            const int hk = h / g;
+            const long base = ((long)b * Hkv + hk) * L;      /* first token row of (b, hk) */
+            const uint16_t* qh = Q + ((long)b * Hq + h) * d;
+            double* o64 = out64 ? out64 + ((long)b * Hq + h) * d : NULL;
+            uint16_t* o = out + ((long)b * Hq + h) * d;
+            if (Lb <= 0) {
+                for (int i = 0; i < d; ++i) {
+                    o[i] = 0;
+                    if (o64) o64[i] = 0.0;
+                }
+                continue;
+            }
+            double mx = -INFINITY;
+            for (int t = 0; t < Lb; ++t) {
+                orc_kv4_dequant(qk + (base + t) * d, sk + base + t, mk + base + t, 1, d, kh);
+                double acc = 0.0;
+                for (int i = 0; i < d; ++i) acc += orc_h2d(qh[i]) * kh[i];
+                score[t] = acc / sqrt((double)d);
+                if (score[t] > mx) mx = score[t];
+            }
+            double sum = 0.0;
+            for (int t = 0; t < Lb; ++t) {
+                score[t] = exp(score[t] - mx);
+                sum += score[t];
+            }
+            for (int i = 0; i < d; ++i) {
+                double acc = 0.0;
+                for (int t = 0; t < Lb; ++t) {
+                    const long r = base + t;
+                    acc += score[t] * (orc_h2d(sv[r]) * (double)qv[r * d + i] + orc_h2d(mv[r]));
+                }
+                acc /= sum;
+                if (o64) o64[i] = acc;
+                o[i] = orc_d2h(acc);
+            }
+        }
+    }
+    free(score);
+    free(kh);
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
     extern int omp_get_max_threads(void);

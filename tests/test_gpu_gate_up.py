@@ -43,7 +43,9 @@ def _fp16_step(y):
     return np.spacing(np.abs(y).astype(np.float16)).astype(np.float64)
 
 
-CASES = [(1024, 1024, M) for M in (1, 5, 16, 40, 130)] + [(14336, 4096, 1), (14336, 4096, 200)]
+# M = 400: H is re-quantized by the many-row quantizer
+CASES = [(1024, 1024, M) for M in (1, 5, 16, 40, 130, 400)] + [(14336, 4096, 1),
+                                                                (14336, 4096, 200)]
 
 
 @pytest.mark.parametrize("I,K,M", CASES, ids=[f"I{i}_K{k}_M{m}" for i, k, m in CASES])

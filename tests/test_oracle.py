@@ -7,6 +7,7 @@ Passages pinned: "QServe: W4A8KV4 Quantization and System Co-design for
 Efficient LLM Serving" (velog notes), Methods 1) Algorithm: QoQ and
 2) System: QServe; same page, Background (no partial-sum dequantization).
 """
+import math
 import os
 from fractions import Fraction
 
@@ -602,3 +603,141 @@ def test_silu_limits_and_linearity_in_up(oracle):
     b = oracle.silu_mul(g2, (u2.astype(np.float64) * 4).astype(np.float16)).astype(np.float64)
     keep = np.abs(a) > 2.0 ** -12
     assert np.array_equal(b[keep], 4 * a[keep])
+
+
+# ---------------------------------------------------------------------------
+# 4-bit KV cache and decode attention over it ("QServe: Cuantificación
+# W4A8KV4 ...", abstract: the 4-bit KV cache; velog notes, Insight: the fused,
+# memory-bound attention).  The cache format is a reading: x^ = s * q + m per
+# (token, KV head) vector, q = clamp(rne((x - min) / s), 0, 15).
+# ---------------------------------------------------------------------------
+
+def test_kv4_hand_examples(oracle):
+    for x, q, sm in _golden("kv4_quant"):
+        X = np.array([float(v) for v in x], np.float16)[None, :]
+        qq, s, m = oracle.kv4_quant(X)
+        assert qq[0].tolist() == [int(v) for v in q], x
+        assert int(s.view(np.uint16)[0]) == int(sm[0], 16), x
+        assert int(m.view(np.uint16)[0]) == int(sm[1], 16), x
+
+
+def test_kv4_codes_are_the_nearest_level(oracle):
+    """Brute force over the 16 levels: every code is the level nearest to x
+    (ties aside), the minimum gets code 0, and |x - x^| <= s / 2 where s is
+    a normal FP16 number."""
+    rng = np.random.default_rng(11)
+    X = (rng.standard_normal((400, 8)) * rng.choice([0.01, 1.0, 30.0], (400, 1))).astype(np.float16)
+    q, s, m = oracle.kv4_quant(X)
+    assert q.max() <= 15
+    xh = oracle.kv4_dequant(q, s, m)
+    x = X.astype(np.float64)
+    sv = s.astype(np.float64)[:, None]
+    levels = sv[:, :, None] * np.arange(16)[None, None, :] + m.astype(np.float64)[:, None, None]
+    dist = np.abs(x[:, :, None] - levels)
+    best = dist.min(axis=2)
+    own = np.abs(x - xh)
+    assert np.all(own <= best * (1 + 1e-6) + 1e-30)
+    assert np.all(q[np.arange(400), x.argmin(axis=1)] == 0)
+    normal = sv[:, 0] >= 2.0 ** -14
+    assert np.all(own[normal] <= 0.5 * sv[normal] * (1 + 2.0 ** -10))
+
+
+def _attn_inputs(oracle, rng, B, Hq, Hkv, L, d):
+    Q = rng.standard_normal((B, Hq, d)).astype(np.float16)
+    K = rng.standard_normal((B, Hkv, L, d)).astype(np.float16)
+    V = rng.standard_normal((B, Hkv, L, d)).astype(np.float16)
+    qk, sk, mk = oracle.kv4_quant(K)
+    qv, sv, mv = oracle.kv4_quant(V)
+    return Q, [qk, sk, mk, qv, sv, mv]
+
+
+def test_kv4_attention_single_token_returns_its_value(oracle):
+    """softmax over one token is 1: out = v^ exactly."""
+    rng = np.random.default_rng(1)
+    Q, c = _attn_inputs(oracle, rng, 2, 4, 2, 5, 16)
+    out, out64 = oracle.kv4_decode_attention(Q, *c, np.array([1, 1], np.int32))
+    vh = oracle.kv4_dequant(c[3], c[4], c[5])
+    for h in range(4):
+        assert np.array_equal(out64[:, h], vh[:, h // 2, 0])
+
+
+def test_kv4_attention_equal_keys_average_the_values(oracle):
+    rng = np.random.default_rng(2)
+    Q, c = _attn_inputs(oracle, rng, 1, 2, 1, 7, 16)
+    for a in c[:3]:
+        a[:, :, 1:] = a[:, :, :1]            # every key equal to the first
+    out, out64 = oracle.kv4_decode_attention(Q, *c, np.array([7], np.int32))
+    vh = oracle.kv4_dequant(c[3], c[4], c[5])
+    ref = vh[0, 0].mean(axis=0)
+    for h in range(2):
+        assert np.allclose(out64[0, h], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_kv4_attention_two_tokens_logistic(oracle):
+    """Keys 0 and e_0 (d = 4), values 0 and 3 e_0: the weight of the second
+    token is the logistic function of q_0 / sqrt(4)."""
+    d, L = 4, 2
+    qk = np.zeros((1, 1, L, d), np.uint8)
+    qk[0, 0, 1, 0] = 1
+    qv = np.zeros((1, 1, L, d), np.uint8)
+    qv[0, 0, 1, 0] = 3
+    one = np.full((1, 1, L), 1.0, np.float16)
+    zero = np.zeros((1, 1, L), np.float16)
+    for a in (0.75, -2.0, 5.5):
+        Q = np.array([[[a, 0.3, -1, 2]]], np.float16)
+        out, out64 = oracle.kv4_decode_attention(Q, qk, one, zero, qv, one, zero,
+                                                 np.array([2], np.int32))
+        p1 = 1.0 / (1.0 + math.exp(-float(np.float16(a)) / 2.0))
+        assert abs(out64[0, 0, 0] - 3.0 * p1) <= 1e-12
+        assert np.all(out64[0, 0, 1:] == 0.0)
+
+
+def test_kv4_attention_grouped_heads(oracle):
+    """Query heads 0, 1 read KV head 0 and heads 2, 3 read KV head 1: with
+    every value of a KV head equal to a constant, its query heads return it."""
+    rng = np.random.default_rng(3)
+    Q, c = _attn_inputs(oracle, rng, 1, 4, 2, 6, 16)
+    c[3][:] = 0                                 # codes 0: v^ = m
+    c[5][0, 0, :] = 1.5
+    c[5][0, 1, :] = -0.25
+    out, out64 = oracle.kv4_decode_attention(Q, *c, np.array([6], np.int32))
+    assert np.allclose(out64[0, :2], 1.5, rtol=1e-14, atol=0)
+    assert np.allclose(out64[0, 2:], -0.25, rtol=1e-14, atol=0)
+
+
+def test_kv4_attention_masks_tokens_past_the_length(oracle):
+    rng = np.random.default_rng(4)
+    Q, c = _attn_inputs(oracle, rng, 3, 2, 2, 9, 16)
+    seq = np.array([9, 4, 0], np.int32)
+    out_a, a64 = oracle.kv4_decode_attention(Q, *c, seq)
+    for arr in c:
+        arr[1, :, 4:] = arr[1, :, 4:][..., ::-1] if arr.ndim == 4 else arr[1, :, 4:] * 3
+    out_b, b64 = oracle.kv4_decode_attention(Q, *c, seq)
+    assert np.array_equal(a64, b64)
+    assert np.all(a64[2] == 0.0) and np.all(out_a.view(np.uint16)[2] == 0)
+
+
+def test_kv4_attention_invariances(oracle):
+    """Shifting every key by the same vector t * 1 shifts all scores of a head
+    alike (softmax unchanged); permuting the tokens changes nothing; shifting
+    every value by t shifts the output by t."""
+    rng = np.random.default_rng(5)
+    Q, c = _attn_inputs(oracle, rng, 2, 4, 1, 11, 16)
+    seq = np.array([11, 8], np.int32)
+    _, base = oracle.kv4_decode_attention(Q, *c, seq)
+    c2 = [a.copy() for a in c]
+    c2[2] = (c2[2].astype(np.float64) + 0.5).astype(np.float16)
+    _, shifted = oracle.kv4_decode_attention(Q, *c2, seq)
+    assert np.allclose(shifted, base, rtol=0, atol=1e-9)
+    perm = rng.permutation(8)
+    c3 = [a.copy() for a in c]
+    for a in c3:
+        a[1, :, :8] = a[1][:, perm]
+    _, permuted = oracle.kv4_decode_attention(Q, *c3, seq)
+    assert np.allclose(permuted, base, rtol=0, atol=1e-12)
+    c4 = [a.copy() for a in c]
+    c4[5] = (c4[5].astype(np.float64) + 2.0).astype(np.float16)
+    exact = np.all(c4[5].astype(np.float64) == c[5].astype(np.float64) + 2.0)
+    assert exact
+    _, vshift = oracle.kv4_decode_attention(Q, *c4, seq)
+    assert np.allclose(vshift, base + 2.0, rtol=0, atol=1e-9)

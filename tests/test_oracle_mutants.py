@@ -182,6 +182,31 @@ MUTANTS = [
      "double g = orc_h2d(G[i]);", "double g = orc_h2d(U[i]);"),
     ("silu_without_up",
      "H[i] = orc_d2h(silu * orc_h2d(U[i]));", "H[i] = orc_d2h(silu);"),
+    # 4-bit KV cache and decode attention
+    ("kv4_scale_over_16",
+     "uint16_t sh = orc_f2h(range / 15.0f);", "uint16_t sh = orc_f2h(range / 16.0f);"),
+    ("kv4_codes_truncated",
+     "c = clampi((int)rne_f(t), 0, 15);", "c = clampi((int)t, 0, 15);"),
+    ("kv4_codes_clamped_to_16",
+     "c = clampi((int)rne_f(t), 0, 15);", "c = clampi((int)rne_f(t), 0, 16);"),
+    ("kv4_offset_not_subtracted",
+     "float t = (orc_h2f(x[i]) - mn) / sv;", "float t = orc_h2f(x[i]) / sv;"),
+    ("kv4_dequant_drops_offset",
+     "out[r * d + i] = sv * (double)q[r * d + i] + mv;", "out[r * d + i] = sv * (double)q[r * d + i];"),
+    ("kv4_score_scaled_by_1_over_d",
+     "score[t] = acc / sqrt((double)d);", "score[t] = acc / (double)d;"),
+    ("kv4_grouped_heads_modulo",
+     "const int hk = h / g;", "const int hk = h % Hkv;"),
+    ("kv4_exponent_sign",
+     "score[t] = exp(score[t] - mx);", "score[t] = exp(mx - score[t]);"),
+    ("kv4_values_use_key_scales",
+     "acc += score[t] * (orc_h2d(sv[r]) * (double)qv[r * d + i] + orc_h2d(mv[r]));",
+     "acc += score[t] * (orc_h2d(sk[r]) * (double)qv[r * d + i] + orc_h2d(mv[r]));"),
+    ("kv4_values_drop_offset",
+     "acc += score[t] * (orc_h2d(sv[r]) * (double)qv[r * d + i] + orc_h2d(mv[r]));",
+     "acc += score[t] * (orc_h2d(sv[r]) * (double)qv[r * d + i]);"),
+    ("kv4_not_normalized_by_weights",
+     "acc /= sum;", "acc /= (double)Lb;"),
 ]
 
 
