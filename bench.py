@@ -511,6 +511,66 @@ def mlp_per_m(qoq, torch, dev, stream, l2):
     return out
 
 
+KV4_CONFIGS = [
+    # (model, B, Hq, Hkv, L): Llama-3-8B (32 query heads over 8 KV heads) and
+    # Qwen1.5-72B (64 heads, no grouping), head dimension 128, every
+    # sequence at the full length L
+    ("llama3_8b", 16, 32, 8, 4096),
+    ("llama3_8b", 64, 32, 8, 4096),
+    ("llama3_8b", 256, 32, 8, 1024),
+    ("qwen1.5_72b", 16, 64, 64, 2048),
+]
+
+
+def kv4_attention_bench(qoq, torch, dev, stream, l2, peaks):
+    """Decode attention over the 4-bit KV cache (qoq_kv4_decode_attention,
+    both of its kernels), back to back in a CUDA graph over rotated caches.
+    The caches are quantized by qoq_kv4_quantize from seeded N(0, 1) FP16 K
+    and V drawn on the device.  Algorithmic bytes per call: the cache bytes
+    of the valid tokens (64 + 64 code bytes and 8 scale bytes per token and
+    KV head) plus Q and out."""
+    gen = torch.Generator(device=dev)
+    res = []
+    for model, B, Hq, Hkv, L in KV4_CONFIGS:
+        kb, vb, sb = qoq.kv4_cache_bytes(B, Hkv, L)
+        per = kb + vb + sb
+        n = copies_for(per, l2, lo=2, hi=8)
+        caches = []
+        for i in range(n):
+            cache = qoq.kv4_cache(B, Hkv, L, dev)
+            for t0 in range(0, L, 1024):
+                T = min(1024, L - t0)
+                gen.manual_seed(1000 * i + t0)
+                K = torch.randn((B, Hkv, T, 128), device=dev, generator=gen).half()
+                V = torch.randn((B, Hkv, T, 128), device=dev, generator=gen).half()
+                qoq.kv4_quantize(K, V, cache, t0=t0, stream=stream)
+                stream.synchronize()
+                del K, V
+            caches.append(cache)
+        gen.manual_seed(7)
+        Q = torch.randn((B, Hq, 128), device=dev, generator=gen).half()
+        seq = torch.full((B,), L, dtype=torch.int32, device=dev)
+        out = torch.empty((B, Hq, 128), dtype=torch.float16, device=dev)
+        need = qoq.lib().qoq_kv4_attention_workspace_bytes(B, Hq, Hkv, L, 128)
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        with torch.cuda.stream(stream):
+            qoq.kv4_decode_attention(Q, caches[0], seq, out=out, ws=ws, stream=stream)
+        stream.synchronize()
+
+        def run():
+            for c in caches:
+                qoq.kv4_decode_attention(Q, c, seq, out=out, ws=ws, stream=stream)
+            return len(caches)
+        us = graph_us_per_launch(torch, stream, run, reps=5)
+        nbytes = per + 2 * B * Hq * 128 * 2
+        gbs = nbytes / us / 1e3
+        res.append({"model": model, "B": B, "Hq": Hq, "Hkv": Hkv, "L": L, "us": us,
+                    "algo_bytes": nbytes, "GBs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"]})
+        del caches, Q, seq, out, ws
+        torch.cuda.synchronize()
+    return res
+
+
 def sweep_per_m(qoq, torch, dev, stream, l2, peaks, int8_peak):
     """The pure-throughput shape sweep: K = N in {2048, 4096, 8192}, group 64
     and 128, M = 1 .. 8192 in powers of two; random UINT4 codes, zeros and
@@ -739,6 +799,9 @@ def run_ours(args):
     sweep = None
     if not args.no_sweep and world == 1:
         sweep = sweep_per_m(qoq, torch, dev, stream, l2, peaks, int8_peak)
+    kv4 = None
+    if not args.no_layers and world == 1:
+        kv4 = kv4_attention_bench(qoq, torch, dev, stream, l2, peaks)
     assert qoq.device_error(clear=True) == 0
 
     td = statistics.mean(dom_ms) * 1e-3
@@ -788,6 +851,7 @@ def run_ours(args):
         "layers": layers,
         "mlp": mlp,
         "sweep": sweep,
+        "kv4_attention": kv4,
         "clocks": clocks,
         "gpu_launches": 2 * len(ms) * args.steps,
         "timed_region": "fused qoq_w4a8_linear per M (dominant M: quantizer + qoq_w4a8_gemm)",

@@ -381,6 +381,67 @@ QOQ_API int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int* sp
                   int* ctas, int* stages);
 
 /* ------------------------------------------------------------------------
+ * 4-bit KV cache and decode attention over it.
+ * Source: "QServe: Cuantificación W4A8KV4 y Co-diseño del Sistema para un
+ * Servicio Eficiente de LLM", abstract (W4A8KV4: the KV cache in 4 bits);
+ * "QServe: W4A8KV4 Quantization and System Co-design for Efficient LLM
+ * Serving" (velog notes), Insight (the fused attention made memory-bound).
+ * The pages give no cache format; this library's: every (token, KV head)
+ * vector x of d = 128 FP16 values has UINT4 codes q, an FP16 scale s and an
+ * FP16 offset m (the vector's minimum), x^ = s * q + m, with
+ * s = fp16((max - min) / 15) and q = clamp(rne((x - min) / s), 0, 15)
+ * computed in IEEE binary32 (q = 0 when s = 0).
+ *
+ * A cache of B sequences, Hkv KV heads and L token slots (L % 16 == 0) is
+ * three caller-owned device arrays, 16-byte aligned, sizes from
+ * qoq_kv4_cache_bytes:
+ *   k_codes, v_codes  [B][Hkv][L / 16][1024] bytes each: per block of 16
+ *            tokens, 32 runs of 32 bytes; run r (gid = r >> 2, tig = r & 3),
+ *            32-bit word w (0..7), nibble p (bits 4p..4p+3; j = p & 3,
+ *            e = p >> 2) holds
+ *              K: token gid + 8 (j & 1), dimension 16w + 2 tig + e + 8 (j >> 1)
+ *              V: token 2 tig + e + 8 (j >> 1), dimension 16w + gid + 8 (j & 1)
+ *            of the block;
+ *   scales   [B][Hkv][L][4] FP16: s_K, m_K, s_V, m_V of the token.
+ * (The nibble orders are the operand layouts of the attention kernel's
+ * tensor-core fragments, so each lane loads its 32 bytes in two pieces.)
+ * Only d = 128 is supported (QOQ_ERR_UNSUPPORTED otherwise), and at most
+ * 65535 (B * Hkv) pairs.
+ * ---------------------------------------------------------------------- */
+QOQ_API int qoq_kv4_cache_bytes(int B, int Hkv, int L, int d, size_t* k_bytes, size_t* v_bytes,
+                                size_t* scale_bytes);
+
+/* Quantize T new tokens of every (sequence, KV head) pair into cache slots
+ * t0 .. t0 + T - 1 (0 <= t0, t0 + T <= L).  K, V: [B][Hkv][T][128] FP16
+ * (device, 16-byte aligned).  Slots outside the range keep their codes and
+ * scales (a block of 16 tokens that is written in part is read, merged and
+ * written back).  Asynchronous on `stream`.  Errors: QOQ_ERR_INVALID_ARG for
+ * NULL / misaligned pointers or a range outside the cache,
+ * QOQ_ERR_UNSUPPORTED for d != 128 or L % 16 != 0. */
+QOQ_API int qoq_kv4_quantize(const void* K, const void* V, int B, int Hkv, int T, int d, int L,
+                             int t0, uint8_t* k_codes, uint8_t* v_codes, void* scales,
+                             void* stream);
+
+/* Workspace of qoq_kv4_decode_attention (its per-split partial results);
+ * 0 for an unsupported shape. */
+QOQ_API size_t qoq_kv4_attention_workspace_bytes(int B, int Hq, int Hkv, int L, int d);
+
+/* Decode attention of one query token per sequence over the 4-bit cache:
+ * out[b][h] = softmax_t(Q[b][h] . k^[b][h / g][t] / sqrt(128)) . v^[b][h / g]
+ * over t < seqlen[b], with g = Hq / Hkv query heads per KV head (grouped-query
+ * attention, g <= 8).  Q, out: [B][Hq][128] FP16 (device, 16-byte aligned);
+ * seqlen: B int32 on the device, each clamped to [0, L]; a sequence of length
+ * 0 gives out = 0.  The scores and sums are FP32, the softmax weights enter
+ * the tensor cores as an FP16 pair (high and low part) per weight.  ws: at
+ * least qoq_kv4_attention_workspace_bytes, 16-byte aligned (no zeroing
+ * needed); QOQ_ERR_WORKSPACE when it is NULL or too small.  Two kernels on
+ * `stream` (the attention, then the merge of its splits). */
+QOQ_API int qoq_kv4_decode_attention(const void* Q, const uint8_t* k_codes, const uint8_t* v_codes,
+                                     const void* scales, const int* seqlen, int B, int Hq, int Hkv,
+                                     int L, int d, void* out, void* ws, size_t ws_bytes,
+                                     void* stream);
+
+/* ------------------------------------------------------------------------
  * Device-side error word.  Every wait inside the kernels is bounded; a wait
  * that runs out sets a bit in this word and the kernel returns early
  * instead of hanging.  Synchronous (device-wide): reads the word of the

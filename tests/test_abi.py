@@ -256,3 +256,49 @@ def test_binding_rejects_host_tensors(L):
     for call in calls:
         with pytest.raises(ValueError, match="CUDA tensor"):
             call()
+
+
+def test_kv4_sizes_and_argument_validation(L):
+    """The 4-bit KV cache entries: sizes, and every bad argument refused
+    before a CUDA call (QOQ_ERR_CUDA only where the checks pass and no GPU
+    is there)."""
+    assert qoq.kv4_cache_bytes(2, 8, 64) == (2 * 8 * 4 * 1024, 2 * 8 * 4 * 1024, 2 * 8 * 64 * 8)
+    with pytest.raises(qoq.QoQError) as e:
+        qoq.kv4_cache_bytes(2, 8, 64, d=64)
+    assert e.value.status == qoq.QOQ_ERR_UNSUPPORTED
+    with pytest.raises(qoq.QoQError) as e:
+        qoq.kv4_cache_bytes(2, 8, 40)                       # L % 16
+    assert e.value.status == qoq.QOQ_ERR_UNSUPPORTED
+    ws = L.qoq_kv4_attention_workspace_bytes
+    assert ws(2, 32, 8, 4096, 128) > 0
+    assert ws(2, 32, 8, 4096, 64) == 0
+    assert ws(2, 30, 8, 4096, 128) == 0                     # Hq % Hkv
+    assert ws(1, 18, 2, 4096, 128) == 0                     # 9 query heads per KV head
+
+    def quant(K=FAKE, V=FAKE, B=1, H=2, T=4, d=128, Lc=64, t0=0, kc=FAKE, vc=FAKE, sc=FAKE):
+        return L.qoq_kv4_quantize(P(K), P(V), B, H, T, d, Lc, t0, P(kc), P(vc), P(sc), None)
+    assert quant(K=None) == qoq.QOQ_ERR_INVALID_ARG
+    assert quant(sc=None) == qoq.QOQ_ERR_INVALID_ARG
+    assert quant(T=0) == qoq.QOQ_ERR_INVALID_ARG
+    assert quant(t0=61) == qoq.QOQ_ERR_INVALID_ARG          # past the cache
+    assert quant(t0=-1) == qoq.QOQ_ERR_INVALID_ARG
+    assert quant(kc=FAKE + 8) == qoq.QOQ_ERR_INVALID_ARG
+    assert quant(d=96) == qoq.QOQ_ERR_UNSUPPORTED
+    assert quant(Lc=72) == qoq.QOQ_ERR_UNSUPPORTED
+
+    def attn(Q=FAKE, B=1, Hq=8, Hkv=2, Lc=64, d=128, out=FAKE, seq=FAKE, w=FAKE, wb=1 << 20):
+        return L.qoq_kv4_decode_attention(P(Q), P(FAKE), P(FAKE), P(FAKE), P(seq), B, Hq, Hkv, Lc,
+                                          d, P(out), P(w), wb, None)
+    need = ws(1, 8, 2, 64, 128)
+    assert attn(Q=None) == qoq.QOQ_ERR_INVALID_ARG
+    assert attn(seq=None) == qoq.QOQ_ERR_INVALID_ARG
+    assert attn(seq=FAKE + 2) == qoq.QOQ_ERR_INVALID_ARG   # int32 alignment
+    assert attn(out=FAKE + 8) == qoq.QOQ_ERR_INVALID_ARG
+    assert attn(Hq=6, Hkv=4) == qoq.QOQ_ERR_INVALID_ARG
+    assert attn(Hq=18, Hkv=2) == qoq.QOQ_ERR_UNSUPPORTED   # 9 query heads per KV head
+    assert attn(d=64) == qoq.QOQ_ERR_UNSUPPORTED
+    assert attn(w=None) == qoq.QOQ_ERR_WORKSPACE
+    assert attn(wb=need - 16) == qoq.QOQ_ERR_WORKSPACE
+    if not _has_gpu():
+        assert attn(wb=need) == qoq.QOQ_ERR_CUDA
+        assert quant() == qoq.QOQ_ERR_CUDA

@@ -35,6 +35,8 @@ EXPORTS = (
     "qoq_w4a8_gemm_static_ws", "qoq_selftest_wait_timeout", "qoq_w4a8_linear_fused",
     "qoq_smooth_factors", "qoq_quantize_weights_smoothed", "qoq_quantize_act_per_token_smoothed",
     "qoq_quantize_weights_gate_up", "qoq_w4a8_gate_up_silu",
+    "qoq_kv4_cache_bytes", "qoq_kv4_quantize", "qoq_kv4_attention_workspace_bytes",
+    "qoq_kv4_decode_attention",
 )
 
 _lock = threading.Lock()
@@ -107,6 +109,14 @@ def lib() -> ctypes.CDLL:
             L.qoq_gemm_workspace_bytes_config.argtypes = [I, I, I, I, I, I]
             L.qoq_gemm_plan.restype = I
             L.qoq_gemm_plan.argtypes = [I, I, I, I] + [ctypes.POINTER(I)] * 4
+            L.qoq_kv4_cache_bytes.restype = I
+            L.qoq_kv4_cache_bytes.argtypes = [I, I, I, I] + [ctypes.POINTER(sz)] * 3
+            L.qoq_kv4_quantize.restype = I
+            L.qoq_kv4_quantize.argtypes = [P, P, I, I, I, I, I, I, P, P, P, P]
+            L.qoq_kv4_attention_workspace_bytes.restype = sz
+            L.qoq_kv4_attention_workspace_bytes.argtypes = [I, I, I, I, I]
+            L.qoq_kv4_decode_attention.restype = I
+            L.qoq_kv4_decode_attention.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P, sz, P]
             L.qoq_device_error.restype = I
             L.qoq_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), I]
             _lib = L
@@ -222,19 +232,20 @@ def gemm_workspace_bytes(M: int, N: int, K: int, group: int = 128, tok_tile: int
 _ws_cache = {}
 
 
-def workspace(nbytes: int, device, stream=None):
+def workspace(nbytes: int, device, stream=None, kind: str = "gemm"):
     """A reusable, zero-initialized device workspace of at least `nbytes`
-    bytes.  There is one buffer per (device, stream), grown on demand and
-    allocated and zeroed on that stream: the split-K counters in it assume
-    that the calls sharing it run one after another, which calls on one
-    stream do."""
+    bytes.  There is one buffer per (device, stream, kind), grown on demand
+    and allocated and zeroed on that stream: the split-K counters in the
+    GEMM's assume that the calls sharing it run one after another, which
+    calls on one stream do.  The attention's partial results go to a buffer
+    of their own (kind "kv4"), which leaves the GEMM's counters at zero."""
     import torch
     if nbytes <= 0:
         return None
     device = torch.device(device)
     if stream is None:
         stream = torch.cuda.current_stream(device)
-    key = (device.index, stream.cuda_stream)
+    key = (device.index, stream.cuda_stream, kind)
     with _lock:
         buf = _ws_cache.get(key)
         if buf is None or buf.numel() < nbytes:
@@ -372,6 +383,68 @@ def w4a8_gate_up_silu(X8, sx, packed, s1, I: int, group: int = 128, out=None, st
                                        _ptr(H), _ptr(H8), _ptr(sh), _stream(stream)),
            "qoq_w4a8_gate_up_silu")
     return H, H8, sh
+
+
+def kv4_cache_bytes(B: int, Hkv: int, L: int, d: int = 128):
+    """(k_bytes, v_bytes, scale_bytes) of a 4-bit KV cache."""
+    k, v, sc = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().qoq_kv4_cache_bytes(B, Hkv, L, d, ctypes.byref(k), ctypes.byref(v),
+                                     ctypes.byref(sc)), "qoq_kv4_cache_bytes")
+    return k.value, v.value, sc.value
+
+
+def kv4_cache(B: int, Hkv: int, L: int, device, d: int = 128):
+    """An empty cache: (k_codes uint8, v_codes uint8, scales float16) device
+    tensors, (B, Hkv, L // 16, 1024), (B, Hkv, L // 16, 1024) and
+    (B, Hkv, L, 4)."""
+    import torch
+    kv4_cache_bytes(B, Hkv, L, d)
+    kc = torch.zeros((B, Hkv, L // 16, 1024), dtype=torch.uint8, device=device)
+    vc = torch.zeros((B, Hkv, L // 16, 1024), dtype=torch.uint8, device=device)
+    sc = torch.zeros((B, Hkv, L, 4), dtype=torch.float16, device=device)
+    return kc, vc, sc
+
+
+def kv4_quantize(K, V, cache, t0: int = 0, stream=None):
+    """Write K, V ((B, Hkv, T, 128) float16) into cache slots t0 .. t0+T-1."""
+    import torch
+    kc, vc, sc = cache
+    _need_cuda(K, "K", torch.float16, 4)
+    B, Hkv, T, d = K.shape
+    _need_cuda(V, "V", torch.float16, shape=tuple(K.shape), device=K.device)
+    L = sc.shape[2]
+    _need_cuda(kc, "k_codes", torch.uint8, shape=(B, Hkv, L // 16, 1024), device=K.device)
+    _need_cuda(vc, "v_codes", torch.uint8, shape=(B, Hkv, L // 16, 1024), device=K.device)
+    _need_cuda(sc, "scales", torch.float16, shape=(B, Hkv, L, 4), device=K.device)
+    _check(lib().qoq_kv4_quantize(_ptr(K), _ptr(V), B, Hkv, T, d, L, t0, _ptr(kc), _ptr(vc),
+                                  _ptr(sc), _stream(stream)), "qoq_kv4_quantize")
+
+
+def kv4_decode_attention(Q, cache, seqlen, out=None, ws=None, stream=None):
+    """Decode attention of Q ((B, Hq, 128) float16) over the 4-bit cache for
+    the first seqlen[b] tokens (int32 CUDA tensor (B,)); returns (B, Hq, 128)
+    float16."""
+    import torch
+    kc, vc, sc = cache
+    _need_cuda(Q, "Q", torch.float16, 3)
+    B, Hq, d = Q.shape
+    Hkv, L = sc.shape[1], sc.shape[2]
+    _need_cuda(kc, "k_codes", torch.uint8, shape=(B, Hkv, L // 16, 1024), device=Q.device)
+    _need_cuda(vc, "v_codes", torch.uint8, shape=(B, Hkv, L // 16, 1024), device=Q.device)
+    _need_cuda(sc, "scales", torch.float16, shape=(B, Hkv, L, 4), device=Q.device)
+    _need_cuda(seqlen, "seqlen", torch.int32, shape=(B,), device=Q.device)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float16, device=Q.device)
+    else:
+        _need_cuda(out, "out", torch.float16, shape=(B, Hq, d), device=Q.device)
+    need = int(lib().qoq_kv4_attention_workspace_bytes(B, Hq, Hkv, L, d))
+    if ws is None:
+        ws = workspace(need, Q.device, stream, kind="kv4")
+    _check(lib().qoq_kv4_decode_attention(_ptr(Q), _ptr(kc), _ptr(vc), _ptr(sc), _ptr(seqlen), B,
+                                          Hq, Hkv, L, d, _ptr(out), _ptr(ws),
+                                          ws.numel() * ws.element_size(), _stream(stream)),
+           "qoq_kv4_decode_attention")
+    return out
 
 
 def smooth_factors(Xcal, W, stream=None):
