@@ -992,6 +992,7 @@ def _c_code_only(text):
 
 GEMM_SOURCES = ("w4a8_quantized_gemm_02_b200/csrc/qoq_gemm.cu",
                 "w4a8_quantized_gemm_02_b200/csrc/qoq_device.cuh",
+                "w4a8_quantized_gemm_02_b200/csrc/qoq_actq.cuh",
                 "w4a8_quantized_gemm_02_b200/csrc/qoq_internal.h",
                 "include/qoq.h")
 

@@ -195,9 +195,6 @@ __device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
-}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
@@ -262,7 +259,15 @@ __device__ __forceinline__ float rows_sum(float v) {
   return v + __shfl_xor_sync(0xffffffffu, v, 16);
 }
 
-constexpr int kStageBytes = 32 * 80;   // per warp and stage: K 32, V 32, scales 16 bytes a lane
+// Per warp and stage: the block's K codes (1024 bytes), V codes (1024) and
+// scales (128).  Each copy instruction of the warp moves 512 contiguous bytes
+// (lane l: bytes 16 l .. +15 of the half), so every L2 sector is requested
+// once; the 16-byte chunk c of a code block goes to slot
+// c ^ ((c >> 3) & 1), which lets lane l read chunks 2l and 2l + 1 (its run)
+// without bank conflicts.
+constexpr int kStageBytes = 1024 + 1024 + 128;
+
+__device__ __forceinline__ int chunk_slot(int c) { return c ^ ((c >> 3) & 1); }
 
 // Grid (nsplit, B * Hkv), four warps.  CTA sigma covers the 16-token blocks
 // [sigma * bps, (sigma + 1) * bps) of its pair, warp w every fourth of them
@@ -289,26 +294,28 @@ kv4_decode_kernel(const __half* __restrict__ Q, const uint8_t* __restrict__ kc,
   blk1 = blk1 < nblk ? blk1 : nblk;
   const int niter = blk0 < blk1 ? (blk1 - blk0 + kWarpsPerCta - 1) / kWarpsPerCta : 0;
 
-  // this lane's copies of a block: its K run, its V run, the scales of its
-  // tokens gid and gid + 8
-  // (the next block to copy: pointers advanced by kWarpsPerCta blocks a copy)
-  const uint8_t* kp = kc + (static_cast<size_t>(bh) * (L / 16) + blk0) * 1024 + 32 * lane;
-  const uint8_t* vp = vc + (static_cast<size_t>(bh) * (L / 16) + blk0) * 1024 + 32 * lane;
-  const __half* sp = sc + (static_cast<size_t>(bh) * L + 16 * blk0 + gid) * 4;
+  // the next block to copy (pointers advance by kWarpsPerCta blocks a copy):
+  // lane l moves chunks l and 32 + l of the K and of the V block, and lanes
+  // 0..7 the eight 16-byte chunks of the block's scales
+  const uint8_t* kp = kc + (static_cast<size_t>(bh) * (L / 16) + blk0) * 1024 + 16 * lane;
+  const uint8_t* vp = vc + (static_cast<size_t>(bh) * (L / 16) + blk0) * 1024 + 16 * lane;
+  const uint8_t* sp =
+      reinterpret_cast<const uint8_t*>(sc + (static_cast<size_t>(bh) * L + 16 * blk0) * 4) +
+      16 * (lane & 7);
   uint8_t* wring = smem + warp * kRingStages * kStageBytes;
-  const uint32_t ring0 = static_cast<uint32_t>(__cvta_generic_to_shared(wring)) + 16 * lane;
+  const uint32_t ring0 = static_cast<uint32_t>(__cvta_generic_to_shared(wring));
+  const uint32_t s_lo = 16 * chunk_slot(lane), s_hi = 16 * chunk_slot(32 + lane);
   auto issue = [&](int it) {
     if (it < niter) {
-      const uint32_t dst = ring0 + (it % kRingStages) * kStageBytes;   // pieces of 512 bytes
-      cp_async16(dst, kp);
-      cp_async16(dst + 512, kp + 16);
-      cp_async16(dst + 1024, vp);
-      cp_async16(dst + 1536, vp + 16);
-      cp_async8(dst + 2048, sp);
-      cp_async8(dst + 2056, sp + 8 * 4);
+      const uint32_t dst = ring0 + (it % kRingStages) * kStageBytes;
+      cp_async16(dst + s_lo, kp);
+      cp_async16(dst + s_hi, kp + 512);
+      cp_async16(dst + 1024 + s_lo, vp);
+      cp_async16(dst + 1024 + s_hi, vp + 512);
+      if (lane < 8) cp_async16(dst + 2048 + 16 * lane, sp);
       kp += kWarpsPerCta * 1024;
       vp += kWarpsPerCta * 1024;
-      sp += kWarpsPerCta * 16 * 4;
+      sp += kWarpsPerCta * 16 * 8;
     }
     cp_async_commit();   // an empty group past the end keeps the counting uniform
   };
@@ -343,27 +350,38 @@ kv4_decode_kernel(const __half* __restrict__ Q, const uint8_t* __restrict__ kc,
   float mrun[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.0f, 0.0f}, msum[2] = {0.0f, 0.0f};
 
   for (int it = 0; it < niter; ++it) {
-    issue(it + kRingStages - 1);
-    cp_async_wait<kRingStages - 1>();
+    // the block's copies landed (this lane's), then the whole warp's
+    cp_async_wait<kRingStages - 2>();
+    __syncwarp();
     const int blk = blk0 + it * kWarpsPerCta;
-    const int st = it % kRingStages;
-    const uint8_t* slot = wring + st * kStageBytes + 16 * lane;
-    const uint4 kq0 = *reinterpret_cast<const uint4*>(slot);
-    const uint4 kq1 = *reinterpret_cast<const uint4*>(slot + 512);
-    const uint4 vq0 = *reinterpret_cast<const uint4*>(slot + 1024);
-    const uint4 vq1 = *reinterpret_cast<const uint4*>(slot + 1536);
-    const uint4 sq = *reinterpret_cast<const uint4*>(slot + 2048);
+    const uint8_t* stage = wring + (it % kRingStages) * kStageBytes;
+    const uint4 kq0 = *reinterpret_cast<const uint4*>(stage + 16 * chunk_slot(2 * lane));
+    const uint4 kq1 = *reinterpret_cast<const uint4*>(stage + 16 * chunk_slot(2 * lane + 1));
+    const uint4 vq0 = *reinterpret_cast<const uint4*>(stage + 1024 + 16 * chunk_slot(2 * lane));
+    const uint4 vq1 = *reinterpret_cast<const uint4*>(stage + 1024 + 16 * chunk_slot(2 * lane + 1));
+    uint4 sq;
+    *reinterpret_cast<uint2*>(&sq.x) = *reinterpret_cast<const uint2*>(stage + 2048 + 8 * gid);
+    *reinterpret_cast<uint2*>(&sq.z) = *reinterpret_cast<const uint2*>(stage + 2048 + 64 + 8 * gid);
+    // every lane has read the stage before any lane copies into it again
+    __syncwarp();
+    issue(it + kRingStages - 1);
 
     // S^T = C_K Q^T: rows tokens (gid, gid + 8), columns heads (2 tig, +1)
+    // (two accumulators, even and odd k-steps, halve the dependent chain)
     float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     {
+      float s2[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       const uint32_t wk[8] = {kq0.x, kq0.y, kq0.z, kq0.w, kq1.x, kq1.y, kq1.z, kq1.w};
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        uint32_t a[4];
+      for (int ks = 0; ks < 8; ks += 2) {
+        uint32_t a[4], a2[4];
         a_frag(wk[ks], a);
+        a_frag(wk[ks + 1], a2);
         mma_16816(s, a, qb[ks][0], qb[ks][1]);
+        mma_16816(s2, a2, qb[ks + 1][0], qb[ks + 1][1]);
       }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) s[i] += s2[i];
     }
     // scales of tokens gid (first 8 bytes) and gid + 8
     const __half* hs = reinterpret_cast<const __half*>(&sq);
@@ -560,14 +578,15 @@ struct AttnPlan {
 };
 
 // Splits of the sequence axis: about four waves of CTAs (four resident per
-// SM), each warp keeping at least two blocks of 16 tokens, at most 64 splits
-// (the merge reads every split).
+// SM), each warp keeping at least eight blocks of 16 tokens (fewer, longer
+// CTAs measured faster than more, shorter ones), at most 64 splits (the
+// merge reads every split).
 AttnPlan attn_plan(int B, int Hkv, int L) {
   const long pairs = static_cast<long>(B) * Hkv;
   const int nblk = L / 16;
   const long want = 4L * 4 * sm_count();
   long ns = (want + pairs - 1) / pairs;
-  long cap = nblk / (2 * kWarpsPerCta);
+  long cap = nblk / (8 * kWarpsPerCta);
   if (cap > 64) cap = 64;
   if (ns > cap) ns = cap;
   if (ns < 1) ns = 1;
