@@ -1101,7 +1101,9 @@ bool valid_tok(int t) {
 // the wide tiles 176 / 192 (one k-tile per stage, so more control work per
 // K but fewer output tiles): the cost of a shape is the number of rounds of
 // units over the SMs times the time a unit takes per k-tile, measured on B200
-// with every SM busy as about 272, 393 and 445 ns for 128, 176 and 192 tokens.
+// with every SM busy as about 277, 363 and 377 ns for 128, 176 and 192 tokens
+// (Llama-3-8B QKV at 4096 tokens; the wide tiles gained from the deeper
+// weight ring).
 int auto_tok(int M, int n_tiles) {
   const long sms = sm_count();
   if (M <= 16) return 16;
@@ -1111,7 +1113,7 @@ int auto_tok(int M, int n_tiles) {
     return static_cast<long>((M + 31) / 32) * n_tiles <= sms ? 32 : 64;
   }
   const int cand[3] = {128, 176, 192};
-  const double per_kt[3] = {272.0, 393.0, 445.0};
+  const double per_kt[3] = {277.0, 363.0, 377.0};
   int best = 128;
   double best_cost = 1e30;
   for (int i = 0; i < 3; ++i) {
