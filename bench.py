@@ -59,6 +59,9 @@ def parse_args(argv=None):
     p.add_argument("--profile-gemm", type=int, default=0, metavar="M",
                    help="only launch the GEMM for this M a few times (for ncu)")
     p.add_argument("--profile-launches", type=int, default=3)
+    p.add_argument("--profile-kv4", action="store_true",
+                   help="run a few KV4 decode attention calls (Llama-3-8B heads, 64 sequences "
+                        "of 4096 tokens) and exit: the command line for an ncu capture")
     p.add_argument("--no-layers", action="store_true",
                    help="skip the per-M timing of the other layer workloads")
     p.add_argument("--no-sweep", action="store_true",
@@ -318,6 +321,31 @@ def run_profile(args, qoq, torch):
     assert qoq.device_error(clear=True) == 0
     print(json.dumps({"profile": layer.name, "M": M, "plan": qoq.gemm_plan(
         M, layer.N, layer.K, layer.group), "y_absmax": float(Y.abs().max())}))
+    return 0
+
+
+def run_profile_kv4(args, qoq, torch):
+    """A few launches of the KV4 decode attention on the first KV4_CONFIGS
+    workload with 4096 tokens (Llama-3-8B heads, 64 sequences): the command
+    line for an ncu capture of its kernels."""
+    model, B, Hq, Hkv, L = KV4_CONFIGS[1]
+    dev = torch.device("cuda")
+    gen = torch.Generator(device=dev)
+    cache = qoq.kv4_cache(B, Hkv, L, dev)
+    for t0 in range(0, L, 1024):
+        gen.manual_seed(t0)
+        K = torch.randn((B, Hkv, 1024, 128), device=dev, generator=gen).half()
+        V = torch.randn((B, Hkv, 1024, 128), device=dev, generator=gen).half()
+        qoq.kv4_quantize(K, V, cache, t0=t0)
+        del K, V
+    Q = torch.randn((B, Hq, 128), device=dev, generator=gen).half()
+    seq = torch.full((B,), L, dtype=torch.int32, device=dev)
+    for _ in range(args.profile_launches):
+        out = qoq.kv4_decode_attention(Q, cache, seq)
+    torch.cuda.synchronize()
+    assert qoq.device_error(clear=True) == 0
+    print(json.dumps({"profile_kv4": model, "B": B, "Hq": Hq, "Hkv": Hkv, "L": L,
+                      "out_absmax": float(out.abs().max())}))
     return 0
 
 
@@ -656,6 +684,8 @@ def run_ours(args):
     qoq.lib()
     if args.profile_gemm:
         return run_profile(args, qoq, torch)
+    if args.profile_kv4:
+        return run_profile_kv4(args, qoq, torch)
 
     layer = si.LAYERS[args.workload]
     ms = list(layer.ms)
