@@ -203,11 +203,17 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Codes enter the tensor cores as the FP16 subnormals c * 2^-24 (one shift
-// and one AND per pair); with kCodesAsSubnormals false they are made exact
-// normal FP16 integers instead (0x6400 | c is 1024 + c, minus 1024).
+// Codes enter the tensor cores as FP16 subnormals: the pairs masked from
+// bits 0..3 of each half are c * 2^-24, those masked from bits 4..7 are
+// c * 2^-20 (no shift needed).  In both products the latter land on rows 8..15
+// of the 16-row operand (tokens gid + 8 of S^T, dimensions gid + 8 of O^T),
+// so each accumulator row has one factor: kRowScale0 for rows 0..7,
+// kRowScale1 for rows 8..15.  With kCodesAsSubnormals false the codes are
+// made exact normal FP16 integers instead (0x6400 | c is 1024 + c, minus
+// 1024) and both factors are 1.
 constexpr bool kCodesAsSubnormals = true;
-constexpr float kCodeScale = kCodesAsSubnormals ? 16777216.0f : 1.0f;
+constexpr float kRowScale0 = kCodesAsSubnormals ? 16777216.0f : 1.0f;
+constexpr float kRowScale1 = kCodesAsSubnormals ? 1048576.0f : 1.0f;
 
 // Two codes (nibbles j and j + 4 of `word`) as an FP16 pair.
 __device__ __forceinline__ uint32_t codes_h2(uint32_t word, int j) {
@@ -221,25 +227,27 @@ __device__ __forceinline__ uint32_t codes_h2(uint32_t word, int j) {
   }
 }
 
-// The A fragment (16 rows x 16 k) held in one word of a run.  As
-// subnormals, the pairs j = 1 and 3 are masked in place (bits 4..7 of each
-// half: c * 2^-20) and brought to c * 2^-24 by an exact FP16 multiply, which
-// runs on the FMA pipe instead of the integer pipe that the masks use.
+// The A fragment (16 rows x 16 k) held in one word of a run: one shift and
+// four masks.  The pairs j = 1 and 3 (rows 8..15) stay at c * 2^-20.
 __device__ __forceinline__ void a_frag(uint32_t word, uint32_t (&a)[4]) {
   if constexpr (kCodesAsSubnormals) {
     const uint32_t hi = word >> 8;
-    const __half2 k16 = __float2half2_rn(0.0625f);
-    uint32_t m1 = word & 0x00f000f0u, m3 = hi & 0x00f000f0u;
-    const __half2 h1 = __hmul2(*reinterpret_cast<const __half2*>(&m1), k16);
-    const __half2 h3 = __hmul2(*reinterpret_cast<const __half2*>(&m3), k16);
     a[0] = word & 0x000f000fu;
-    a[1] = *reinterpret_cast<const uint32_t*>(&h1);
+    a[1] = word & 0x00f000f0u;
     a[2] = hi & 0x000f000fu;
-    a[3] = *reinterpret_cast<const uint32_t*>(&h3);
+    a[3] = hi & 0x00f000f0u;
   } else {
 #pragma unroll
     for (int j = 0; j < 4; ++j) a[j] = codes_h2(word, j);
   }
+}
+
+// 2^x by the SFU's approximation (relative error ~2^-22, far inside the
+// attention's tolerance); 2^-inf = 0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
@@ -339,11 +347,10 @@ kv4_decode_kernel(const __half* __restrict__ Q, const uint8_t* __restrict__ kc,
   }
   qs += __shfl_xor_sync(0xffffffffu, qs, 1);
   qs += __shfl_xor_sync(0xffffffffu, qs, 2);                    // Q_gid in lanes 4 gid ..
-  const float qh[2] = {__shfl_sync(0xffffffffu, qs, 8 * tig),        // Q of head 2 tig
-                       __shfl_sync(0xffffffffu, qs, 8 * tig + 4)};   // and 2 tig + 1
-
   // scores in log2 units: (q . k^) * log2(e) / sqrt(128)
   const float kScale = 1.4426950408889634f / 11.313708498984761f;
+  const float qh[2] = {__shfl_sync(0xffffffffu, qs, 8 * tig) * kScale,       // Q of head 2 tig
+                       __shfl_sync(0xffffffffu, qs, 8 * tig + 4) * kScale};  // and 2 tig + 1
   float acc[8][4];
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.0f;
@@ -389,7 +396,8 @@ kv4_decode_kernel(const __half* __restrict__ Q, const uint8_t* __restrict__ kc,
     bool valid[2];
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      skt[r] = __half2float(hs[4 * r + 0]) * kCodeScale;   // the codes carry 1 / kCodeScale
+      // row r of S^T is token gid + 8 r: its codes carry 1 / kRowScale<r>
+      skt[r] = __half2float(hs[4 * r + 0]) * ((r ? kRowScale1 : kRowScale0) * kScale);
       mkt[r] = __half2float(hs[4 * r + 1]);
       svt[r] = __half2float(hs[4 * r + 2]);
       mvt[r] = __half2float(hs[4 * r + 3]);
@@ -400,7 +408,7 @@ kv4_decode_kernel(const __half* __restrict__ Q, const uint8_t* __restrict__ kc,
     for (int r = 0; r < 2; ++r) {
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        const float v = valid[r] ? (skt[r] * s[2 * r + c] + mkt[r] * qh[c]) * kScale : -INFINITY;
+        const float v = valid[r] ? skt[r] * s[2 * r + c] + mkt[r] * qh[c] : -INFINITY;
         s[2 * r + c] = v;
         bm[c] = fmaxf(bm[c], v);
       }
@@ -409,7 +417,7 @@ kv4_decode_kernel(const __half* __restrict__ Q, const uint8_t* __restrict__ kc,
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const float mn = fmaxf(mrun[c], rows_max(bm[c]));
-      al[c] = mn == -INFINITY ? 1.0f : exp2f(mrun[c] - mn);
+      al[c] = mn == -INFINITY ? 1.0f : fast_exp2(mrun[c] - mn);
       mrun[c] = mn;
       lsum[c] *= al[c];
       msum[c] *= al[c];
@@ -430,7 +438,7 @@ kv4_decode_kernel(const __half* __restrict__ Q, const uint8_t* __restrict__ kc,
     for (int r = 0; r < 2; ++r) {
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        const float p = mrun[c] == -INFINITY ? 0.0f : exp2f(s[2 * r + c] - mrun[c]);
+        const float p = mrun[c] == -INFINITY ? 0.0f : fast_exp2(s[2 * r + c] - mrun[c]);
         lsum[c] += p;
         wt[2 * r + c] = valid[r] ? p * svt[r] : 0.0f;
         msum[c] += valid[r] ? p * mvt[r] : 0.0f;
@@ -470,8 +478,8 @@ kv4_decode_kernel(const __half* __restrict__ Q, const uint8_t* __restrict__ kc,
     }
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
-      row[4 + 16 * mt + gid] = acc[mt][c] * kCodeScale + mo;
-      row[4 + 16 * mt + gid + 8] = acc[mt][2 + c] * kCodeScale + mo;
+      row[4 + 16 * mt + gid] = acc[mt][c] * kRowScale0 + mo;
+      row[4 + 16 * mt + gid + 8] = acc[mt][2 + c] * kRowScale1 + mo;
     }
   }
   __syncthreads();
