@@ -552,7 +552,7 @@ KV4_CONFIGS = [
 
 def kv4_attention_bench(qoq, torch, dev, stream, l2, peaks):
     """Decode attention over the 4-bit KV cache (qoq_kv4_decode_attention,
-    both of its kernels), back to back in a CUDA graph over rotated caches.
+    with the merge of its splits), back to back in a CUDA graph over rotated caches.
     The caches are quantized by qoq_kv4_quantize from seeded N(0, 1) FP16 K
     and V drawn on the device.  Algorithmic bytes per call: the cache bytes
     of the valid tokens (64 + 64 code bytes and 8 scale bytes per token and
@@ -580,7 +580,7 @@ def kv4_attention_bench(qoq, torch, dev, stream, l2, peaks):
         seq = torch.full((B,), L, dtype=torch.int32, device=dev)
         out = torch.empty((B, Hq, 128), dtype=torch.float16, device=dev)
         need = qoq.lib().qoq_kv4_attention_workspace_bytes(B, Hq, Hkv, L, 128)
-        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        ws = torch.zeros(need, dtype=torch.uint8, device=dev)
         with torch.cuda.stream(stream):
             qoq.kv4_decode_attention(Q, caches[0], seq, out=out, ws=ws, stream=stream)
         stream.synchronize()

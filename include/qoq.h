@@ -434,8 +434,9 @@ QOQ_API size_t qoq_kv4_attention_workspace_bytes(int B, int Hq, int Hkv, int L, 
  * 0 gives out = 0.  The scores and sums are FP32, the softmax weights enter
  * the tensor cores as an FP16 pair (high and low part) per weight.  ws: at
  * least qoq_kv4_attention_workspace_bytes, 16-byte aligned (no zeroing
- * needed); QOQ_ERR_WORKSPACE when it is NULL or too small.  Two kernels on
- * `stream` (the attention, then the merge of its splits). */
+ * needed); QOQ_ERR_WORKSPACE when it is NULL or too small.  On `stream`: the
+ * attention kernel, then a kernel that merges its splits of the sequence
+ * when there is more than one. */
 QOQ_API int qoq_kv4_decode_attention(const void* Q, const uint8_t* k_codes, const uint8_t* v_codes,
                                      const void* scales, const int* seqlen, int B, int Hq, int Hkv,
                                      int L, int d, void* out, void* ws, size_t ws_bytes,

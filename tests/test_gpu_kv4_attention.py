@@ -161,7 +161,8 @@ CASES = [
     (2, 16, 2, 128, [0, 33]),                 # g = 8, an empty sequence
     (1, 8, 1, 96, [95]),                      # g = 8, a single KV head
     (4, 8, 2, 48, [15, 16, 31, 48]),          # lengths at block edges
-    (1, 32, 8, 4096, [4096]),                 # one sequence over many splits
+    (1, 32, 8, 4096, [4096]),                 # one sequence over 8 splits
+    (1, 16, 4, 8192, [8190]),                 # 16 splits
 ]
 
 
@@ -213,6 +214,29 @@ def test_attention_ignores_slots_past_the_length(oracle):
     out = qoq.kv4_decode_attention(_dev(Q), cache, _dev(seqlen))
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
+
+
+def test_repeated_calls_share_the_workspace(oracle):
+    """Calls of different shapes on one workspace, in a row (one split and
+    several), give the same results as calls on fresh ones."""
+    shapes = [(4, 16, 4, 256, [256, 1, 100, 0]), (2, 8, 2, 512, [512, 300]),
+              (4, 16, 4, 256, [256, 1, 100, 0])]
+    need = max(qoq.lib().qoq_kv4_attention_workspace_bytes(B, Hq, Hkv, L, D)
+               for B, Hq, Hkv, L, _ in shapes)
+    shared = torch.zeros(need, dtype=torch.uint8, device=DEV)
+    for i, (B, Hq, Hkv, L, seq) in enumerate(shapes):
+        rng = np.random.default_rng(i)
+        K, V = _kv(rng, B, Hkv, L)
+        Q = _dev(rng.standard_normal((B, Hq, D)).astype(np.float16))
+        cache = qoq.kv4_cache(B, Hkv, L, DEV)
+        qoq.kv4_quantize(_dev(K), _dev(V), cache, t0=0)
+        s = _dev(np.array(seq, np.int32))
+        a = qoq.kv4_decode_attention(Q, cache, s, ws=shared)
+        b = qoq.kv4_decode_attention(Q, cache, s, ws=shared)
+        fresh = torch.zeros(need, dtype=torch.uint8, device=DEV)
+        c = qoq.kv4_decode_attention(Q, cache, s, ws=fresh)
+        torch.cuda.synchronize()
+        assert torch.equal(a, c) and torch.equal(b, c)
 
 
 def test_more_than_eight_heads_per_kv_head_unsupported():

@@ -283,12 +283,13 @@ __device__ __forceinline__ int chunk_slot(int c) { return c ^ ((c >> 3) & 1); }
 // <= 8), the running maximum (log2 units), the sum of 2^(score - max), the
 // offset term sum p m_V, and O^T in 8 accumulator tiles; at the end the four
 // warps' results are merged in shared memory and the CTA leaves one partial
-// result per head: ws[pair][sigma][head] = (max, sum, 128 outputs).
+// result per head: ws[pair][sigma][head] = (max, sum, 128 outputs), or, when
+// it covers the whole sequence (nsplit = 1), the output itself.
 __global__ void __launch_bounds__(32 * kWarpsPerCta)
 kv4_decode_kernel(const __half* __restrict__ Q, const uint8_t* __restrict__ kc,
                   const uint8_t* __restrict__ vc, const __half* __restrict__ sc,
                   const int* __restrict__ seqlen, int Hq, int Hkv, int L, int g, int bps,
-                  float* __restrict__ ws) {
+                  float* __restrict__ ws, __half* __restrict__ out) {
   __shared__ __align__(16) uint8_t smem[kWarpsPerCta * kRingStages * kStageBytes];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
@@ -498,18 +499,32 @@ kv4_decode_kernel(const __half* __restrict__ Q, const uint8_t* __restrict__ kc,
         f[w] = M == -INFINITY ? 0.0f : exp2f(row[0] - M);
         den += f[w] * row[1];
       }
-      float* out = ws + ((static_cast<size_t>(bh) * gridDim.x + blockIdx.x) * g + h) * kPartFloats;
-      if ((threadIdx.x & 15) == 0) {
-        out[0] = M;
-        out[1] = den;
-      }
+      float v[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        float v = 0.0f;
+        v[u] = 0.0f;
 #pragma unroll
         for (int w = 0; w < kWarpsPerCta; ++w)
-          v += f[w] == 0.0f ? 0.0f : f[w] * mrg[(w * 8 + h) * kPartFloats + 4 + d0 + u];
-        out[4 + d0 + u] = v;
+          v[u] += f[w] == 0.0f ? 0.0f : f[w] * mrg[(w * 8 + h) * kPartFloats + 4 + d0 + u];
+      }
+      if (gridDim.x == 1) {
+        // the whole sequence in this CTA: the output directly
+        __half2 o[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          o[u] = __floats2half2_rn(den > 0.0f ? __fdiv_rn(v[2 * u], den) : 0.0f,
+                                   den > 0.0f ? __fdiv_rn(v[2 * u + 1], den) : 0.0f);
+        *reinterpret_cast<uint4*>(out + (static_cast<size_t>(b) * Hq + hk * g + h) * kHeadDim +
+                                  d0) = *reinterpret_cast<const uint4*>(o);
+      } else {
+        float* part =
+            ws + ((static_cast<size_t>(bh) * gridDim.x + blockIdx.x) * g + h) * kPartFloats;
+        if ((threadIdx.x & 15) == 0) {
+          part[0] = M;
+          part[1] = den;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) part[4 + d0 + u] = v[u];
       }
     }
   }
@@ -584,6 +599,8 @@ kv4_combine_kernel(const float* __restrict__ ws, int Hq, int Hkv, int g, int nsp
 struct AttnPlan {
   int nsplit, bps;
 };
+
+
 
 // Splits of the sequence axis: about four waves of CTAs (four resident per
 // SM), each warp keeping at least eight blocks of 16 tokens (fewer, longer
@@ -668,11 +685,15 @@ extern "C" int qoq_kv4_decode_attention(const void* Q, const uint8_t* k_codes,
   const int g = Hq / Hkv;
   cudaStream_t s = as_stream(stream);
   dim3 grid(static_cast<unsigned>(p.nsplit), static_cast<unsigned>(B * Hkv));
+  float* parts = static_cast<float*>(ws);
   kv4_decode_kernel<<<grid, 32 * kWarpsPerCta, 0, s>>>(
       static_cast<const __half*>(Q), k_codes, v_codes, static_cast<const __half*>(scales), seqlen,
-      Hq, Hkv, L, g, p.bps, static_cast<float*>(ws));
+      Hq, Hkv, L, g, p.bps, parts, static_cast<__half*>(out));
   if (int st = launch_status()) return st;
-  kv4_combine_kernel<<<B * Hq, 256, 0, s>>>(static_cast<const float*>(ws), Hq, Hkv, g, p.nsplit,
-                                            static_cast<__half*>(out));
-  return launch_status();
+  if (p.nsplit > 1) {
+    kv4_combine_kernel<<<B * Hq, 256, 0, s>>>(parts, Hq, Hkv, g, p.nsplit,
+                                              static_cast<__half*>(out));
+    return launch_status();
+  }
+  return QOQ_OK;
 }
