@@ -44,6 +44,8 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "qoq.h"
 #include "qoq_internal.h"
 
@@ -374,93 +376,106 @@ kv4_decode_kernel(const __half* __restrict__ Q, const uint8_t* __restrict__ kc,
     __syncwarp();
     issue(it + kRingStages - 1);
 
-    // S^T = C_K Q^T: rows tokens (gid, gid + 8), columns heads (2 tig, +1)
-    // (two accumulators, even and odd k-steps, halve the dependent chain)
-    float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    {
-      float s2[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      const uint32_t wk[8] = {kq0.x, kq0.y, kq0.z, kq0.w, kq1.x, kq1.y, kq1.z, kq1.w};
+    // the block's work; only a block that reaches past the sequence's end
+    // masks its tokens (kMasked), the others skip the selects
+    auto step = [&](auto masked) {
+      constexpr bool kMasked = decltype(masked)::value;
+      // S^T = C_K Q^T: rows tokens (gid, gid + 8), columns heads (2 tig, +1)
+      // (two accumulators, even and odd k-steps, halve the dependent chain)
+      float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      {
+        float s2[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        const uint32_t wk[8] = {kq0.x, kq0.y, kq0.z, kq0.w, kq1.x, kq1.y, kq1.z, kq1.w};
 #pragma unroll
-      for (int ks = 0; ks < 8; ks += 2) {
-        uint32_t a[4], a2[4];
-        a_frag(wk[ks], a);
-        a_frag(wk[ks + 1], a2);
-        mma_16816(s, a, qb[ks][0], qb[ks][1]);
-        mma_16816(s2, a2, qb[ks + 1][0], qb[ks + 1][1]);
+        for (int ks = 0; ks < 8; ks += 2) {
+          uint32_t a[4], a2[4];
+          a_frag(wk[ks], a);
+          a_frag(wk[ks + 1], a2);
+          mma_16816(s, a, qb[ks][0], qb[ks][1]);
+          mma_16816(s2, a2, qb[ks + 1][0], qb[ks + 1][1]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) s[i] += s2[i];
       }
+      // scales of tokens gid (first 8 bytes) and gid + 8
+      const __half* hs = reinterpret_cast<const __half*>(&sq);
+      float skt[2], mkt[2], svt[2], mvt[2];
+      bool valid[2];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) s[i] += s2[i];
-    }
-    // scales of tokens gid (first 8 bytes) and gid + 8
-    const __half* hs = reinterpret_cast<const __half*>(&sq);
-    float skt[2], mkt[2], svt[2], mvt[2];
-    bool valid[2];
+      for (int r = 0; r < 2; ++r) {
+        // row r of S^T is token gid + 8 r: its codes carry 1 / kRowScale<r>
+        skt[r] = __half2float(hs[4 * r + 0]) * ((r ? kRowScale1 : kRowScale0) * kScale);
+        mkt[r] = __half2float(hs[4 * r + 1]);
+        svt[r] = __half2float(hs[4 * r + 2]);
+        mvt[r] = __half2float(hs[4 * r + 3]);
+        valid[r] = !kMasked || blk * 16 + gid + 8 * r < Lb;
+      }
+      float bm[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      // row r of S^T is token gid + 8 r: its codes carry 1 / kRowScale<r>
-      skt[r] = __half2float(hs[4 * r + 0]) * ((r ? kRowScale1 : kRowScale0) * kScale);
-      mkt[r] = __half2float(hs[4 * r + 1]);
-      svt[r] = __half2float(hs[4 * r + 2]);
-      mvt[r] = __half2float(hs[4 * r + 3]);
-      valid[r] = blk * 16 + gid + 8 * r < Lb;
-    }
-    float bm[2] = {-INFINITY, -INFINITY};
+      for (int r = 0; r < 2; ++r) {
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
+        for (int c = 0; c < 2; ++c) {
+          const float v =
+              !kMasked || valid[r] ? skt[r] * s[2 * r + c] + mkt[r] * qh[c] : -INFINITY;
+          s[2 * r + c] = v;
+          bm[c] = fmaxf(bm[c], v);
+        }
+      }
+      float al[2];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        const float v = valid[r] ? skt[r] * s[2 * r + c] + mkt[r] * qh[c] : -INFINITY;
-        s[2 * r + c] = v;
-        bm[c] = fmaxf(bm[c], v);
+        const float mn = fmaxf(mrun[c], rows_max(bm[c]));
+        al[c] = mn == -INFINITY ? 1.0f : fast_exp2(mrun[c] - mn);
+        mrun[c] = mn;
+        lsum[c] *= al[c];
+        msum[c] *= al[c];
       }
-    }
-    float al[2];
+      if (al[0] != 1.0f || al[1] != 1.0f) {
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const float mn = fmaxf(mrun[c], rows_max(bm[c]));
-      al[c] = mn == -INFINITY ? 1.0f : fast_exp2(mrun[c] - mn);
-      mrun[c] = mn;
-      lsum[c] *= al[c];
-      msum[c] *= al[c];
-    }
-    if (al[0] != 1.0f || al[1] != 1.0f) {
+        for (int mt = 0; mt < 8; ++mt) {
+          acc[mt][0] *= al[0];
+          acc[mt][1] *= al[1];
+          acc[mt][2] *= al[0];
+          acc[mt][3] *= al[1];
+        }
+      }
+      // the weights w = p s_V (a token past the length has p = 0 and scales
+      // that were never written: its terms are left out, not multiplied by 0)
+      float wt[4];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const float p = mrun[c] == -INFINITY ? 0.0f : fast_exp2(s[2 * r + c] - mrun[c]);
+          lsum[c] += p;
+          if constexpr (kMasked) {
+            wt[2 * r + c] = valid[r] ? p * svt[r] : 0.0f;
+            msum[c] += valid[r] ? p * mvt[r] : 0.0f;
+          } else {
+            wt[2 * r + c] = p * svt[r];
+            msum[c] += p * mvt[r];
+          }
+        }
+      }
+      // P^T as the B fragment, in an FP16 high part and the FP16 rest
+      const uint32_t top = pack_h2(wt[0], wt[1]), bot = pack_h2(wt[2], wt[3]);
+      const float2 ft = __half22float2(*reinterpret_cast<const __half2*>(&top));
+      const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&bot));
+      const uint32_t b0h = transpose8x8(top), b1h = transpose8x8(bot);
+      const uint32_t b0l = transpose8x8(pack_h2(wt[0] - ft.x, wt[1] - ft.y));
+      const uint32_t b1l = transpose8x8(pack_h2(wt[2] - fb.x, wt[3] - fb.y));
+      // O^T += C_V^T P^T, dimension tile mt from V word mt
+      const uint32_t wv[8] = {vq0.x, vq0.y, vq0.z, vq0.w, vq1.x, vq1.y, vq1.z, vq1.w};
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
-        acc[mt][0] *= al[0];
-        acc[mt][1] *= al[1];
-        acc[mt][2] *= al[0];
-        acc[mt][3] *= al[1];
+        uint32_t a[4];
+        a_frag(wv[mt], a);
+        mma_16816(acc[mt], a, b0h, b1h);
+        mma_16816(acc[mt], a, b0l, b1l);
       }
-    }
-    // the weights w = p s_V (a token past the length has p = 0 and scales
-    // that were never written: its terms are left out, not multiplied by 0)
-    float wt[4];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const float p = mrun[c] == -INFINITY ? 0.0f : fast_exp2(s[2 * r + c] - mrun[c]);
-        lsum[c] += p;
-        wt[2 * r + c] = valid[r] ? p * svt[r] : 0.0f;
-        msum[c] += valid[r] ? p * mvt[r] : 0.0f;
-      }
-    }
-    // P^T as the B fragment, in an FP16 high part and the FP16 rest
-    const uint32_t top = pack_h2(wt[0], wt[1]), bot = pack_h2(wt[2], wt[3]);
-    const float2 ft = __half22float2(*reinterpret_cast<const __half2*>(&top));
-    const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&bot));
-    const uint32_t b0h = transpose8x8(top), b1h = transpose8x8(bot);
-    const uint32_t b0l = transpose8x8(pack_h2(wt[0] - ft.x, wt[1] - ft.y));
-    const uint32_t b1l = transpose8x8(pack_h2(wt[2] - fb.x, wt[3] - fb.y));
-    // O^T += C_V^T P^T, dimension tile mt from V word mt
-    const uint32_t wv[8] = {vq0.x, vq0.y, vq0.z, vq0.w, vq1.x, vq1.y, vq1.z, vq1.w};
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      uint32_t a[4];
-      a_frag(wv[mt], a);
-      mma_16816(acc[mt], a, b0h, b1h);
-      mma_16816(acc[mt], a, b0l, b1l);
-    }
+    };
+    if (blk * 16 + 16 <= Lb) step(std::false_type{});
+    else step(std::true_type{});
   }
   cp_async_wait<0>();
   __syncthreads();   // the ring becomes the merge area
