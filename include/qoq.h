@@ -359,8 +359,11 @@ QOQ_API int qoq_w4a8_gate_up_silu(const int8_t* X8, const void* sx, const void* 
  * qoq_quantize_act_per_token, writes all of X8 (every CTA writes the same
  * bytes; CTA 0 writes sx) and then runs the GEMM on it.
  *   - Applies when the rows fit 48 KiB (M * K * 2 <= 49152) and the GEMM's
- *     plan takes 16-token tiles without a cluster split (up to four rows);
- *     otherwise QOQ_ERR_UNSUPPORTED and nothing is launched.
+ *     plan takes 16-token tiles without a cluster split; for one to four rows
+ *     (where the automatic plan is the CUDA-core GEMV) it runs its own
+ *     16-token plan, whose workspace size is
+ *     qoq_gemm_workspace_bytes_config(M, N, K, group, 16, 0).  Otherwise
+ *     QOQ_ERR_UNSUPPORTED and nothing is launched.
  *   - Measured on B200 in back-to-back decode it is slower than
  *     qoq_w4a8_linear's two kernels (the quantizer overlaps the GEMM's start,
  *     while here the rows are quantized inside the GEMM before its first
@@ -376,7 +379,11 @@ QOQ_API int qoq_w4a8_linear_fused(const void* X, int M, int K, const void* packe
  * how many thread-block clusters of the kernel fit on it; without a device
  * 148 SMs and 148 / splits clusters are assumed.  The
  * pages fix no tiling; this reports the library's own choice for the GEMM of
- * Methods, 1) Algorithm: QoQ. */
+ * Methods, 1) Algorithm: QoQ.  For one to four tokens (when their INT8 rows
+ * fit 200 KiB) the product runs on the CUDA cores as a matrix-vector product
+ * with the same integer sums and epilogue: tok_tile = 0, stages = 0, a CTA
+ * per 32 output channels and K range (ctas = N / 32 * splits); a K split
+ * keeps an INT32 slice per range in the workspace. */
 QOQ_API int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int* splits,
                   int* ctas, int* stages);
 

@@ -51,7 +51,18 @@ def test_sizes(L):
 
 
 def test_plan_is_host_only(L):
-    for M in (1, 16, 17, 64, 100, 256, 1024, 4096):
+    for M in (1, 4):
+        # one to four tokens: the CUDA-core GEMV, a CTA per 32 channels and
+        # K range; a split keeps an INT32 slice per range in the workspace
+        p = qoq.gemm_plan(M, 4096, 14336, 128)               # fewer groups than SMs: split
+        assert (p["tok_tile"], p["stages"]) == (0, 0)
+        assert p["splits"] > 1 and p["ctas"] == 4096 // 32 * p["splits"]
+        assert qoq.gemm_workspace_bytes(M, 4096, 14336, 128) == \
+            16384 + p["splits"] * M * 4096 * 4
+        p = qoq.gemm_plan(M, 6144, 4096, 128)                # enough groups: no split
+        assert (p["tok_tile"], p["splits"], p["ctas"]) == (0, 1, 6144 // 32)
+        assert qoq.gemm_workspace_bytes(M, 6144, 4096, 128) == 0
+    for M in (5, 16, 17, 64, 100, 256, 1024, 4096):
         p = qoq.gemm_plan(M, 6144, 4096, 128)
         assert p["tok_tile"] in (16, 32, 64, 128, 176, 192, 256)
         assert p["tok_tile"] >= min(M, 32)
@@ -204,9 +215,9 @@ def test_workspace_sizes(L):
         assert qoq.gemm_workspace_bytes(40, 512, 1024, 128, tok, sp) == 0
     assert qoq.gemm_workspace_bytes(0, 512, 512, 128) == 0
     # the automatic plan splits K through the workspace for up to four
-    # tokens and across clusters for more
-    p = qoq.gemm_plan(1, 6144, 4096, 128)
-    assert p["splits"] > 1 and qoq.gemm_workspace_bytes(1, 6144, 4096, 128) > 0
+    # tokens (the GEMV, few channels) and across clusters for more
+    p = qoq.gemm_plan(1, 4096, 14336, 128)
+    assert p["splits"] > 1 and qoq.gemm_workspace_bytes(1, 4096, 14336, 128) > 0
     p = qoq.gemm_plan(16, 6144, 4096, 128)
     assert p["splits"] > 1 and qoq.gemm_workspace_bytes(16, 6144, 4096, 128) == 0
     # one whose split goes through the workspace

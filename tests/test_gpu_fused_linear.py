@@ -33,9 +33,16 @@ def _dev(a):
 
 
 def fused(M, N, K):
+    """The fused kernel runs a 16-token tile without a cluster split: for up
+    to four tokens (where the automatic plan is the CUDA-core GEMV) its own
+    16-token plan never splits across a cluster."""
+    if M * K * 2 > 49152:
+        return False
+    if M <= 4:
+        return True
     p = qoq.gemm_plan(M, N, K, G)
     cluster = 1 < p["splits"] <= 8 and min(M, 16) > 4
-    return p["tok_tile"] == 16 and not cluster and M * K * 2 <= 49152
+    return p["tok_tile"] == 16 and not cluster
 
 
 _LAYERS = {}
@@ -125,7 +132,10 @@ def test_kernel_count(oracle, entry, N, K, M):
     sx = torch.empty(M, dtype=torch.float16, device=DEV)
     Y = torch.empty((M, N), dtype=torch.float16, device=DEV)
     stream = torch.cuda.Stream(device=DEV)
-    ws = qoq.workspace(qoq.gemm_workspace_bytes(M, N, K, G), DEV, stream)
+    # the fused kernel runs its 16-token plan: its workspace is that plan's
+    need = (qoq.gemm_workspace_bytes(M, N, K, G, tok_tile=16) if entry == "fused"
+            else qoq.gemm_workspace_bytes(M, N, K, G))
+    ws = qoq.workspace(need, DEV, stream)
     call = qoq.w4a8_linear_fused if entry == "fused" else qoq.w4a8_linear
     assert entry != "fused" or fused(M, N, K)
     call(X, packed, s1, N, G, out=Y, scratch=(X8, sx), ws=ws, stream=stream)

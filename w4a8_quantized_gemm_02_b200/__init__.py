@@ -611,7 +611,10 @@ def w4a8_linear_fused(X, packed, s1, N: int, group: int = 128, out=None, scratch
         _need_cuda(X8, "X8", torch.int8, shape=(M, K), device=dev)
         _need_cuda(sx, "sx", torch.float16, shape=(M,), device=dev)
     Y = _out(out, (M, N), torch.float16, dev)
-    w, wb = _ws_args(_auto_ws(ws, M, N, K, group, dev, stream=stream))
+    # up to four rows the kernel runs its own 16-token plan (the automatic
+    # plan would be the GEMV): the workspace is that plan's
+    tok = 16 if M <= 4 else 0
+    w, wb = _ws_args(_auto_ws(ws, M, N, K, group, dev, tok_tile=tok, stream=stream))
     _check(lib().qoq_w4a8_linear_fused(_ptr(X), M, K, _ptr(packed), _ptr(s1), N, group,
                                        _ptr(X8), _ptr(sx), _ptr(Y), w, wb, _stream(stream)),
            "qoq_w4a8_linear_fused")

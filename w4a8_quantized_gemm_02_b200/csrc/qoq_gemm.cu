@@ -1021,6 +1021,8 @@ EncodeTiledFn encode_fn() {
 struct Plan {
   int tok, splits, m_tiles, n_tiles, stages, units, grid;
   int cs;   // K split across a cluster of cs CTAs (1: split through the workspace, or none)
+  bool gemv = false;   // one to four tokens on the CUDA cores (qoq_gemv.cu): tok = 0
+  int rows = 0;        // the GEMV's tokens
 };
 
 // Largest K split a cluster can reduce in the leader's shared memory.
@@ -1168,6 +1170,7 @@ int auto_splits(int tiles, int kt, int tok, int M, bool* cluster_out) {
 }
 
 void finish_plan(Plan& p) {
+  if (p.gemv) return;   // a CTA per 32 channels, set by make_plan
   p.units = p.n_tiles * p.m_tiles * p.splits;
   const int sms = sm_count();
   if (p.cs > 1) {
@@ -1184,6 +1187,28 @@ Plan make_plan(int M, int N, int K, int tok_req, int splits_req) {
   Plan p;
   p.n_tiles = N / kTileN;
   const int kt = K / kTileK;
+  if (!tok_req && !splits_req && M <= kGemvMaxTokens && gemv_smem_bytes(M, K) <= kGemvMaxSmem) {
+    // a matrix-vector product: the packed weights streamed through the CUDA
+    // cores (measured faster than a 16-token tensor-core tile on B200)
+    p.gemv = true;
+    p.rows = M;
+    p.tok = 0;
+    p.cs = 1;
+    p.m_tiles = 1;
+    p.stages = 0;
+    // K split only when there are fewer 32-channel groups than SMs (the
+    // partial sums go through the workspace and the last arrival adds them:
+    // measured slower than no split for Llama-3-8B QKV, faster for down),
+    // each warp keeping at least two k-tiles
+    const long groups = N / 32;
+    const long want = sm_count();
+    long ks = (want + groups - 1) / groups;
+    const long cap = kt / (2 * 8) > 1 ? kt / (2 * 8) : 1;
+    if (ks > cap) ks = cap;
+    p.splits = static_cast<int>(ks);
+    p.units = p.grid = static_cast<int>(groups * ks);
+    return p;
+  }
   p.tok = tok_req ? tok_req : auto_tok(M, p.n_tiles);
   p.m_tiles = (M + p.tok - 1) / p.tok;
   p.stages = stages_for(p.tok);
@@ -1204,6 +1229,8 @@ Plan make_plan(int M, int N, int K, int tok_req, int splits_req) {
 
 size_t ws_bytes_for(const Plan& p, int N) {
   if (p.splits <= 1 || p.cs > 1) return 0;   // a cluster split needs no workspace
+  if (p.gemv)   // a slice of INT32 sums per split
+    return kCounterBytes + static_cast<size_t>(p.splits) * p.rows * N * 4;
   const size_t part = static_cast<size_t>(p.m_tiles) * p.splits * p.tok * N * 4;
   return kCounterBytes + part;
 }
@@ -1272,6 +1299,7 @@ struct GemmLaunch {
   Plan p;
   CUtensorMap map;
   GemmArgs a;
+  GemvArgs g;             // the plan is a GEMV (p.gemv)
   bool gate_up = false;   // the epilogue writes silu(gate) * up (kGateUp kernel)
 };
 
@@ -1307,6 +1335,32 @@ int gemm_prepare(const int8_t* X8, const void* sx, const void* packed, const voi
   }
   finish_plan(p);
   if (int st = check_device()) return st;
+  if (p.gemv) {
+    p.units = p.grid = (N / 32) * p.splits;   // the split may have been dropped above
+    GemvArgs& g = L.g;
+    g.packed = static_cast<const uint8_t*>(packed);
+    g.X8 = X8;
+    g.sx = static_cast<const __half*>(sx);
+    g.s1 = static_cast<const __half*>(s1);
+    g.Y = static_cast<__half*>(Y);
+    g.acc = acc;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.group = group;
+    g.blk_bytes = static_cast<int>(block_bytes(group));
+    g.w_dep_wait = 1;
+    g.ks = p.splits;
+    g.kt_per = (K / kTileK + p.splits - 1) / p.splits;
+    g.ws_count = nullptr;
+    g.ws_acc = nullptr;
+    if (p.splits > 1) {
+      g.ws_count = static_cast<uint32_t*>(ws);
+      g.ws_acc = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kCounterBytes);
+    }
+    L.p = p;
+    return QOQ_OK;
+  }
   EncodeTiledFn enc = encode_fn();
   if (!enc) return QOQ_ERR_CUDA;
 
@@ -1360,6 +1414,13 @@ int gemm_prepare(const int8_t* X8, const void* sx, const void* packed, const voi
 int gemm_launch(GemmLaunch L, void* stream, bool weights_independent, bool clear_counters) {
   cudaStream_t s = as_stream(stream);
   const bool pdl = true;
+  if (L.p.gemv) {
+    L.g.w_dep_wait = weights_independent ? 0 : 1;
+    if (clear_counters && L.g.ws_count != nullptr &&
+        cudaMemsetAsync(L.g.ws_count, 0, kCounterBytes, s) != cudaSuccess)
+      return QOQ_ERR_CUDA;
+    return launch_gemv(L.g, s);
+  }
   L.a.w_dep_wait = weights_independent ? 0 : 1;
   if (clear_counters && L.a.ws_count != nullptr &&
       cudaMemsetAsync(L.a.ws_count, 0, kCounterBytes, s) != cudaSuccess)
@@ -1530,7 +1591,10 @@ extern "C" int qoq_w4a8_linear_fused(const void* X, int M, int K, const void* pa
   if (static_cast<long>(M) * K * 2 > static_cast<long>(kMaxFusedRowBytes))
     return QOQ_ERR_UNSUPPORTED;
   GemmLaunch L;
-  if (int st = gemm_prepare(X8, sx, packed, s1, M, N, K, group, Y, nullptr, 0, 0, ws, ws_bytes, L))
+  // the kernel's own 16-token tile also where the automatic plan would take
+  // the CUDA-core GEMV (one to four tokens)
+  const int tok = M <= kGemvMaxTokens ? 16 : 0;
+  if (int st = gemm_prepare(X8, sx, packed, s1, M, N, K, group, Y, nullptr, tok, 0, ws, ws_bytes, L))
     return st;
   if (L.p.tok != 16 || L.p.cs != 1) return QOQ_ERR_UNSUPPORTED;
   // One kernel: every CTA copies the FP16 token rows into shared memory,

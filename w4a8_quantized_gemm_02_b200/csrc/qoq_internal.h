@@ -1,6 +1,7 @@
 // Host-side helpers shared by the library's translation units.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -42,6 +43,27 @@ int check_device();
 int sm_count();
 // cudaGetLastError -> status.
 int launch_status();
+
+// The CUDA-core GEMV for one to four tokens (qoq_gemv.cu): same integer
+// product and epilogue as the tensor-core GEMM.  Launched as a programmatic
+// dependent; with w_dep_wait == 0 its first weight loads may precede the
+// preceding grid's completion.
+struct GemvArgs {
+  const uint8_t* packed;
+  const int8_t* X8;
+  const __half* sx;
+  const __half* s1;
+  __half* Y;        // FP16 output, or
+  int32_t* acc;     // the INT32 accumulators (exactly one of the two)
+  int M, N, K, group, blk_bytes, w_dep_wait;
+  int ks, kt_per;           // K split into ks ranges of kt_per k-tiles
+  uint32_t* ws_count;       // ks > 1: an arrival counter per 32 channels (zero between calls)
+  int32_t* ws_acc;          // ks > 1: [split][M][N] INT32 partial sums
+};
+constexpr int kGemvMaxTokens = 4;
+constexpr size_t kGemvMaxSmem = 200 * 1024;
+size_t gemv_smem_bytes(int M, int K);
+int launch_gemv(const GemvArgs& a, cudaStream_t s);
 
 // The GEMM launcher shared by the entry points.  The kernel may start while
 // the preceding kernel on the stream is still running (programmatic
