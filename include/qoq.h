@@ -290,7 +290,10 @@ QOQ_API int qoq_w4a8_gemm_i32(const int8_t* X8, const void* packed, int M, int N
                               size_t ws_bytes, void* stream);
 
 /* The same GEMM with an explicit launch configuration (tuning and tests).
- *   tok_tile : token tile (MMA N): 16, 32, 64, 128 or 256, or 0 for auto;
+ *   tok_tile : token tile (MMA N): 16, 32, 64, 128, 176, 192 or 256, or 0
+ *              for auto; 1 asks for the CUDA-core matrix-vector product
+ *              (M <= 4 and the token rows within its shared memory, else
+ *              QOQ_ERR_UNSUPPORTED), with `splits` its K ranges;
  *   splits   : K splits per output tile, 1..8 (at most K/128), or 0 for auto.
  * Exactly one of Y (FP16 output, needs sx and s1) and acc (INT32 output) is
  * non-NULL.  An explicit split count > 1 needs its workspace
@@ -380,10 +383,14 @@ QOQ_API int qoq_w4a8_linear_fused(const void* X, int M, int K, const void* packe
  * 148 SMs and 148 / splits clusters are assumed.  The
  * pages fix no tiling; this reports the library's own choice for the GEMM of
  * Methods, 1) Algorithm: QoQ.  For one to four tokens (when their INT8 rows
- * fit 200 KiB) the product runs on the CUDA cores as a matrix-vector product
- * with the same integer sums and epilogue: tok_tile = 0, stages = 0, a CTA
- * per 32 output channels and K range (ctas = N / 32 * splits); a K split
- * keeps an INT32 slice per range in the workspace. */
+ * fit, with the per-warp copy rings, 227 KiB of shared memory) the product
+ * may run on the CUDA cores as a matrix-vector product
+ * with the same integer sums and epilogue: tok_tile = 0, stages = the
+ * depth of each warp's weight copy ring (2 or 4), a CTA per 32 output
+ * channels and K range (ctas = N / 32 * splits); a K split keeps an INT32
+ * slice per range in the workspace.  It is taken for one token, and for two
+ * to four when a launch-time model fitted on B200 prefers it to the 16-token
+ * tensor-core tile (small weights). */
 QOQ_API int qoq_gemm_plan(int M, int N, int K, int group, int* tok_tile, int* splits,
                   int* ctas, int* stages);
 

@@ -51,17 +51,25 @@ def test_sizes(L):
 
 
 def test_plan_is_host_only(L):
-    for M in (1, 4):
-        # one to four tokens: the CUDA-core GEMV, a CTA per 32 channels and
-        # K range; a split keeps an INT32 slice per range in the workspace
-        p = qoq.gemm_plan(M, 4096, 14336, 128)               # fewer groups than SMs: split
-        assert (p["tok_tile"], p["stages"]) == (0, 0)
-        assert p["splits"] > 1 and p["ctas"] == 4096 // 32 * p["splits"]
-        assert qoq.gemm_workspace_bytes(M, 4096, 14336, 128) == \
-            16384 + p["splits"] * M * 4096 * 4
-        p = qoq.gemm_plan(M, 6144, 4096, 128)                # enough groups: no split
+    # one token: the CUDA-core GEMV, a CTA per 32 channels and K range; a
+    # split (only when fewer than half the SMs would get a CTA) keeps an INT32
+    # slice per range in the workspace; stages = the copy ring's depth
+    p = qoq.gemm_plan(1, 4096, 14336, 128)                   # 128 CTAs: no split
+    assert (p["tok_tile"], p["splits"], p["ctas"], p["stages"]) == (0, 1, 128, 2)
+    assert qoq.gemm_workspace_bytes(1, 4096, 14336, 128) == 0
+    p = qoq.gemm_plan(1, 512, 14336, 128)                    # 16 groups: split 7 ways
+    assert (p["tok_tile"], p["splits"], p["ctas"]) == (0, 7, 16 * 7)
+    assert qoq.gemm_workspace_bytes(1, 512, 14336, 128) == 16384 + 7 * 1 * 512 * 4
+    p = qoq.gemm_plan(1, 8192, 24576, 128)                   # 24 k-tiles per warp: deep ring
+    assert (p["tok_tile"], p["splits"], p["stages"]) == (0, 1, 4)
+    # two to four tokens: the GEMV for small weights, else the tensor cores
+    for M in (2, 3, 4):
+        p = qoq.gemm_plan(M, 6144, 4096, 128)
         assert (p["tok_tile"], p["splits"], p["ctas"]) == (0, 1, 6144 // 32)
         assert qoq.gemm_workspace_bytes(M, 6144, 4096, 128) == 0
+        assert qoq.gemm_plan(M, 49152, 8192, 128)["tok_tile"] == 16
+    # an explicit request (token tile 1) sizes its slices the same way
+    assert qoq.gemm_workspace_bytes(3, 4096, 14336, 128, 1, 5) == 16384 + 5 * 3 * 4096 * 4
     for M in (5, 16, 17, 64, 100, 256, 1024, 4096):
         p = qoq.gemm_plan(M, 6144, 4096, 128)
         assert p["tok_tile"] in (16, 32, 64, 128, 176, 192, 256)
@@ -117,6 +125,10 @@ def test_gemm_argument_validation(L):
     assert c(None, FAKE, 48, 0) == qoq.QOQ_ERR_INVALID_ARG     # bad token tile
     assert c(None, FAKE, 16, 9) == qoq.QOQ_ERR_INVALID_ARG     # too many splits
     assert c(None, FAKE, 16, 5) == qoq.QOQ_ERR_INVALID_ARG     # more splits than k-tiles
+    assert c(None, FAKE, 1, 0) == qoq.QOQ_ERR_UNSUPPORTED      # the GEMV: at most 4 tokens
+    # an explicit GEMV split needs its workspace too
+    assert cfg(P(FAKE), P(FAKE), P(FAKE), P(FAKE), 2, 512, 512, 128, None, P(FAKE), 1, 2, None, 0,
+               None) == qoq.QOQ_ERR_WORKSPACE
     # an explicit split through the workspace needs its workspace
     need = qoq.gemm_workspace_bytes(16, 512, 512, 128, 64, 2)
     assert need > 0
@@ -216,8 +228,8 @@ def test_workspace_sizes(L):
     assert qoq.gemm_workspace_bytes(0, 512, 512, 128) == 0
     # the automatic plan splits K through the workspace for up to four
     # tokens (the GEMV, few channels) and across clusters for more
-    p = qoq.gemm_plan(1, 4096, 14336, 128)
-    assert p["splits"] > 1 and qoq.gemm_workspace_bytes(1, 4096, 14336, 128) > 0
+    p = qoq.gemm_plan(1, 512, 14336, 128)
+    assert p["splits"] > 1 and qoq.gemm_workspace_bytes(1, 512, 14336, 128) > 0
     p = qoq.gemm_plan(16, 6144, 4096, 128)
     assert p["splits"] > 1 and qoq.gemm_workspace_bytes(16, 6144, 4096, 128) == 0
     # one whose split goes through the workspace

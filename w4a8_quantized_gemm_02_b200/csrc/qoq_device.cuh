@@ -434,6 +434,20 @@ __device__ __forceinline__ uint32_t dq_lanes(uint32_t codes, uint32_t s2, uint32
   return (codes * s2 + bias) ^ 0x80808080u;
 }
 
+// 16-byte asynchronous copy global -> shared, cached in L2 only; groups of
+// such copies are committed and waited for per thread.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Wait until at most N of this thread's committed groups are still pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Low and high nibbles of a packed word: codes k0..k0+3 and k0+4..k0+7.
 __device__ __forceinline__ uint32_t lo_codes(uint32_t w) { return w & 0x0F0F0F0Fu; }
 __device__ __forceinline__ uint32_t hi_codes(uint32_t w) { return (w >> 4) & 0x0F0F0F0Fu; }

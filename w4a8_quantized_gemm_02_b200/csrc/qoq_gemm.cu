@@ -1093,8 +1093,39 @@ bool splittable(const Plan& p) {
 
 int stages_for(int tok) { return tok <= 32 ? 7 : tok == 64 ? 6 : tok == 176 ? 5 : 4; }
 
+// Token tiles a caller may request; 1 asks for the CUDA-core GEMV.
 bool valid_tok(int t) {
-  return t == 16 || t == 32 || t == 64 || t == 128 || t == 176 || t == 192 || t == 256;
+  return t == 1 || t == 16 || t == 32 || t == 64 || t == 128 || t == 176 || t == 192 || t == 256;
+}
+
+// The CUDA-core GEMV's copy ring: 4 slots per warp when each warp has at
+// least 16 k-tiles of its K range (and the larger ring fits beside the token
+// rows), else 2.  On B200 the deeper ring made Qwen1.5-72B down (K = 24576,
+// 24 k-tiles per warp) 18% faster and the layers with 4 to 8 k-tiles per
+// warp 9-17% slower (fewer CTAs per SM).
+int gemv_ring(int M, int K, int kt_per) {
+  const bool long_k = (kt_per + 7) / 8 >= 16;
+  return long_k && gemv_smem_bytes(M, K, 4) <= kGemvMaxSmem ? 4 : 2;
+}
+
+bool gemv_fits(int M, int K, int stages) {
+  return M <= kGemvMaxTokens && gemv_smem_bytes(M, K, stages) <= kGemvMaxSmem;
+}
+
+// For two to four tokens, GEMV or tensor cores: modelled launch times in us
+// against the packed weight megabytes, fitted to back-to-back launches on
+// B200 over the six Llama-3-8B and Qwen1.5-72B layers (the GEMV at one and
+// four tokens, the 16-token tensor-core tile).  The GEMV turns
+// compute-bound as tokens are added; the tensor-core kernel costs the same
+// for one to sixteen tokens but has the larger fixed cost.  One token always
+// takes the GEMV; two to four take it when its modelled time is at least 5%
+// lower (the per-layer slopes scatter around the fit).
+bool gemv_preferred(int M, int N, int K) {
+  if (M == 1) return true;
+  const double mb = static_cast<double>(N) * K * 0.5e-6;
+  const double t_gemv = 3.4 + 0.27 * M + (0.122 + 0.034 * M) * mb;
+  const double t_mma = 6.2 + 0.169 * mb;
+  return t_gemv < 0.95 * t_mma;
 }
 
 // Token tile for a shape.  Up to 32 tokens the smallest tile that holds M; up
@@ -1187,27 +1218,36 @@ Plan make_plan(int M, int N, int K, int tok_req, int splits_req) {
   Plan p;
   p.n_tiles = N / kTileN;
   const int kt = K / kTileK;
-  if (!tok_req && !splits_req && M <= kGemvMaxTokens && gemv_smem_bytes(M, K) <= kGemvMaxSmem) {
+  const bool want_gemv =
+      tok_req == 1 || (!tok_req && !splits_req && M <= kGemvMaxTokens && gemv_preferred(M, N, K));
+  if (want_gemv) {
     // a matrix-vector product: the packed weights streamed through the CUDA
-    // cores (measured faster than a 16-token tensor-core tile on B200)
-    p.gemv = true;
-    p.rows = M;
-    p.tok = 0;
-    p.cs = 1;
-    p.m_tiles = 1;
-    p.stages = 0;
-    // K split only when there are fewer 32-channel groups than SMs (the
-    // partial sums go through the workspace and the last arrival adds them:
-    // measured slower than no split for Llama-3-8B QKV, faster for down),
-    // each warp keeping at least two k-tiles
+    // cores.  K is split only when fewer than half the SMs would get a CTA
+    // (the partial sums go through the workspace and the last arrival adds
+    // them; with the copy rings every split measured slower on the six
+    // Llama-3-8B / Qwen1.5-72B layers), each warp keeping two k-tiles.
     const long groups = N / 32;
-    const long want = sm_count();
-    long ks = (want + groups - 1) / groups;
-    const long cap = kt / (2 * 8) > 1 ? kt / (2 * 8) : 1;
-    if (ks > cap) ks = cap;
-    p.splits = static_cast<int>(ks);
-    p.units = p.grid = static_cast<int>(groups * ks);
-    return p;
+    long ks = splits_req;
+    if (!ks) {
+      const long sms = sm_count();
+      ks = 2 * groups < sms ? (sms + groups - 1) / groups : 1;
+      const long cap = kt / (2 * 8) > 1 ? kt / (2 * 8) : 1;
+      if (ks > cap) ks = cap;
+    }
+    const int stages = gemv_ring(M, K, (kt + static_cast<int>(ks) - 1) / static_cast<int>(ks));
+    // an explicit request that cannot run is refused by gemm_prepare; the
+    // automatic plan takes the tensor cores instead
+    if (tok_req == 1 || gemv_fits(M, K, stages)) {
+      p.gemv = true;
+      p.rows = M;
+      p.tok = 0;
+      p.cs = 1;
+      p.m_tiles = 1;
+      p.stages = stages;
+      p.splits = static_cast<int>(ks);
+      p.units = p.grid = static_cast<int>(groups * ks);
+      return p;
+    }
   }
   p.tok = tok_req ? tok_req : auto_tok(M, p.n_tiles);
   p.m_tiles = (M + p.tok - 1) / p.tok;
@@ -1321,6 +1361,7 @@ int gemm_prepare(const int8_t* X8, const void* sx, const void* packed, const voi
     return QOQ_ERR_INVALID_ARG;
 
   Plan p = make_plan(M, N, K, tok_req, splits_req);
+  if (p.gemv && !gemv_fits(M, K, p.stages)) return QOQ_ERR_UNSUPPORTED;
   // the kernel divides unit indices below 2^22 by multiplication (small_div)
   if (static_cast<long>(p.n_tiles) * p.m_tiles * p.splits >= (1L << 22)) return QOQ_ERR_UNSUPPORTED;
   if (p.splits > 1 && p.cs == 1 && !splittable(p)) {
@@ -1352,6 +1393,7 @@ int gemm_prepare(const int8_t* X8, const void* sx, const void* packed, const voi
     g.w_dep_wait = 1;
     g.ks = p.splits;
     g.kt_per = (K / kTileK + p.splits - 1) / p.splits;
+    g.stages = gemv_ring(M, K, g.kt_per);   // the split may have been dropped above
     g.ws_count = nullptr;
     g.ws_acc = nullptr;
     if (p.splits > 1) {

@@ -10,17 +10,21 @@
 // weight is used by at most four multiply-adds, so the work is the stream of
 // packed weights through the SM, and a 128 x TOK tensor-core tile would carry
 // over 97% padding.  Here lane l of a warp owns channel 32 c + l of its CTA's
-// 32 channels; per k-tile it loads its row's four 16-byte code chunks (the
-// warp reads 512 contiguous bytes per load), turns four codes into four INT8
-// weights per 32-bit multiply-add (the same byte-lane arithmetic as the GEMM),
-// and multiplies them with the tokens' INT8 codes four at a time (dp4a,
-// exact INT32).  A CTA covers 32 channels over one of ks ranges of K; its
-// eight warps take every eighth k-tile of the range and their sums are added
-// in shared memory.  With ks > 1 each CTA stores its INT32 partial sums in
-// the workspace and counts its arrival at its 32 channels (acquire-release at
-// GPU scope); the last arrival adds the ks slices.  Warp 0 of the CTA holding
-// the whole sum applies Y = fp16(float(acc) * (sx * s1)), the GEMM's
-// epilogue, bit for bit.
+// 32 channels.  A CTA covers 32 channels over one of ks ranges of K; its
+// eight warps take every eighth k-tile of the range.  Each warp streams its
+// k-tiles through its own ring of S shared-memory slots with asynchronous
+// 16-byte copies (per k-tile every lane copies its row's four code chunks,
+// the warp 512 contiguous bytes per chunk, and six lanes the group scales and
+// zero points), so S k-tiles per warp are in flight while one is multiplied.
+// S is 2, or 4 for long K ranges (measured on B200: the deeper ring holds more
+// bytes in flight, the shallower one more CTAs per SM).  The multiply turns four codes into four
+// INT8 weights per 32-bit multiply-add (the same byte-lane arithmetic as the
+// GEMM) and multiplies them with the tokens' INT8 codes four at a time (dp4a,
+// exact INT32).  The warps' sums are added in shared memory.  With ks > 1
+// each CTA stores its INT32 partial sums in the workspace and counts its
+// arrival at its 32 channels (acquire-release at GPU scope); the last arrival
+// adds the ks slices.  Warp 0 of the CTA holding the whole sum applies
+// Y = fp16(float(acc) * (sx * s1)), the GEMM's epilogue, bit for bit.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -33,24 +37,51 @@ namespace {
 
 constexpr int kGemvWarps = 8;
 constexpr int kGemvRows = 32;          // channels per CTA (one per lane)
+// A ring slot: the 32 rows' code chunks (chunk j of lane l at 512 j + 16 l),
+// then s2 of up to two groups ([group][row], 32 bytes each) and their zero
+// points ([group][row / 2], two nibbles per byte, 16 bytes each).
+constexpr int kSlotCodes = 4 * 512;
+constexpr int kSlotS2 = kSlotCodes;
+constexpr int kSlotZ = kSlotCodes + 64;
+constexpr int kSlotBytes = kSlotCodes + 64 + 32;
+constexpr size_t ring_bytes(int S) { return static_cast<size_t>(kGemvWarps) * S * kSlotBytes; }
 
-// One k-tile of one row: four 16-byte chunks of codes (chunk j holds codes
-// 32 j .. 32 j + 31) and the group scale / bias of its one or two groups.
+// One k-tile of one row in registers: four 16-byte chunks of codes (chunk j
+// holds codes 32 j .. 32 j + 31) and the group scale / bias of its one or
+// two groups.
 struct GemvTile {
   uint4 c[4];
   uint32_t s2[2], bias[2];
 };
 
-__device__ __forceinline__ void gemv_load(const uint8_t* blk, int rr, int gpt, GemvTile& t) {
+// Copy one k-tile of the CTA's 32 rows (rows rr0 .. rr0 + 31 of the packed
+// block blk) into a ring slot.  Every source is 16-byte aligned: blocks are
+// multiples of 16 bytes, rr0 is a multiple of 32.
+__device__ __forceinline__ void gemv_issue(const uint8_t* blk, int rr0, int gpt, int lane,
+                                           uint32_t slot) {
+  const uint8_t* src = blk + (rr0 + lane) * 16;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) t.c[j] = __ldg(reinterpret_cast<const uint4*>(blk + j * 2048 + rr * 16));
+  for (int j = 0; j < 4; ++j) cp_async16(slot + j * 512 + lane * 16, src + j * 2048);
   const uint8_t* scl = blk + kCodesBytes;
+  if (lane < 2 * gpt) {            // s2 of group lane / 2, half lane % 2
+    const int g = lane >> 1, h = lane & 1;
+    cp_async16(slot + kSlotS2 + g * 32 + h * 16, scl + g * 128 + rr0 + h * 16);
+  } else if (lane < 3 * gpt) {     // the zero points of group lane - 2 gpt
+    const int g = lane - 2 * gpt;
+    cp_async16(slot + kSlotZ + g * 16, scl + gpt * 128 + g * 64 + (rr0 >> 1));
+  }
+}
+
+// This lane's row of a landed slot into registers.
+__device__ __forceinline__ void gemv_read(const uint8_t* slot, int lane, int gpt, GemvTile& t) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) t.c[j] = *reinterpret_cast<const uint4*>(slot + j * 512 + lane * 16);
 #pragma unroll
   for (int g = 0; g < 2; ++g) {
     const int gg = g < gpt ? g : 0;          // one group: both entries alike
-    const uint32_t s2 = __ldg(scl + gg * 128 + rr);
-    const uint32_t zb = __ldg(scl + gpt * 128 + gg * 64 + (rr >> 1));
-    const uint32_t z = (rr & 1) ? (zb >> 4) : (zb & 15u);
+    const uint32_t s2 = slot[kSlotS2 + gg * 32 + lane];
+    const uint32_t zb = slot[kSlotZ + gg * 16 + (lane >> 1)];
+    const uint32_t z = (lane & 1) ? (zb >> 4) : (zb & 15u);
     t.s2[g] = s2;
     t.bias[g] = dq_bias(z, s2);
   }
@@ -87,30 +118,47 @@ __device__ __forceinline__ void gemv_accumulate(const GemvTile& t, int gpt, cons
   }
 }
 
-template <int MT>
+template <int MT, int S>
 __global__ void __launch_bounds__(32 * kGemvWarps)
 w4a8_gemv_kernel(const GemvArgs a) {
   extern __shared__ __align__(16) uint8_t gsm[];
-  int8_t* xs = reinterpret_cast<int8_t*>(gsm);                                // [MT][K]
-  int* red = reinterpret_cast<int*>(gsm + ((MT * a.K + 15) & ~15));          // [warps][MT][32]
+  constexpr size_t kRing = ring_bytes(S);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* ring = gsm + static_cast<size_t>(warp) * S * kSlotBytes;            // this warp's
+  int8_t* xs = reinterpret_cast<int8_t*>(gsm + kRing);                         // [MT][K]
+  int* red = reinterpret_cast<int*>(gsm + kRing + ((MT * a.K + 15) & ~15));    // [warps][MT][32]
   const int grp = blockIdx.x / a.ks, split = blockIdx.x - grp * a.ks;
   const int r = grp * kGemvRows + lane;                                       // output channel
-  const int nt = r >> 7, rr = r & 127;
+  const int nt = r >> 7, rr0 = (grp * kGemvRows) & 127;
   const int kt_total = a.K / kTileK;
   const int gpt = kTileK / a.group;
   const uint8_t* wrow = a.packed + static_cast<size_t>(nt) * kt_total * a.blk_bytes;
 
-  // The first k-tile's weights may be read before the preceding grid
+  // this warp's k-tiles: kt0, kt0 + 8, ... below kt_end
+  const int kt0 = split * a.kt_per + warp;
+  const int kt_end = min(kt_total, (split + 1) * a.kt_per);
+  const int n = kt0 < kt_end ? (kt_end - kt0 + kGemvWarps - 1) / kGemvWarps : 0;
+  // k-tile i goes to slot i mod S; one commit group per k-tile
+  // index, empty past the end, keeps the group count uniform
+  auto issue = [&](int i) {
+    if (i < n)
+      gemv_issue(wrow + static_cast<size_t>(kt0 + i * kGemvWarps) * a.blk_bytes, rr0, gpt, lane,
+                 smem_u32(ring + (i % S) * kSlotBytes));
+    cp_async_commit();
+  };
+
+  // The first k-tiles' weights may be read before the preceding grid
   // completes when that grid cannot have written them (programmatic
   // dependent launch); everything else waits for it.
-  const int kt_end = min(kt_total, (split + 1) * a.kt_per);
-  GemvTile cur;
-  int kt = split * a.kt_per + warp;
-  const bool have = kt < kt_end;
-  if (!a.w_dep_wait && have) gemv_load(wrow + static_cast<size_t>(kt) * a.blk_bytes, rr, gpt, cur);
+  if (!a.w_dep_wait) {
+#pragma unroll
+    for (int i = 0; i < S; ++i) issue(i);
+  }
   grid_dependency_wait();
-  if (a.w_dep_wait && have) gemv_load(wrow + static_cast<size_t>(kt) * a.blk_bytes, rr, gpt, cur);
+  if (a.w_dep_wait) {
+#pragma unroll
+    for (int i = 0; i < S; ++i) issue(i);
+  }
   // the tokens' codes, M x K bytes, into shared memory
   {
     const uint4* src = reinterpret_cast<const uint4*>(a.X8);
@@ -124,15 +172,19 @@ w4a8_gemv_kernel(const GemvArgs a) {
   int acc[MT];
 #pragma unroll
   for (int m = 0; m < MT; ++m) acc[m] = 0;
-  // software-pipelined: the next k-tile's loads are in flight while this one
-  // is multiplied
-  for (; kt < kt_end; kt += kGemvWarps) {
-    GemvTile nxt;
-    const int kn = kt + kGemvWarps;
-    if (kn < kt_end) gemv_load(wrow + static_cast<size_t>(kn) * a.blk_bytes, rr, gpt, nxt);
-    gemv_accumulate<MT>(cur, gpt, xs, a.K, kt * kTileK, acc);
-    if (kn < kt_end) cur = nxt;
+  for (int i = 0; i < n; ++i) {
+    // groups 0 .. i have landed (S + i committed so far); the
+    // warp-wide sync makes the scales other lanes copied visible, and the
+    // second one keeps the slot's refill behind every lane's read
+    cp_async_wait<S - 1>();
+    __syncwarp();
+    GemvTile t;
+    gemv_read(ring + (i % S) * kSlotBytes, lane, gpt, t);
+    __syncwarp();
+    issue(i + S);
+    gemv_accumulate<MT>(t, gpt, xs, a.K, (kt0 + i * kGemvWarps) * kTileK, acc);
   }
+  cp_async_wait<0>();
 #pragma unroll
   for (int m = 0; m < MT; ++m) red[(warp * MT + m) * 32 + lane] = acc[m];
   __syncthreads();
@@ -187,16 +239,15 @@ w4a8_gemv_kernel(const GemvArgs a) {
   }
 }
 
-template <int MT>
+template <int MT, int S>
 int launch_mt(const GemvArgs& a, cudaStream_t s) {
-  const size_t smem = ((static_cast<size_t>(MT) * a.K + 15) & ~static_cast<size_t>(15)) +
-                      static_cast<size_t>(kGemvWarps) * MT * 32 * sizeof(int);
+  const size_t smem = gemv_smem_bytes(MT, a.K, S);
   static int configured_mask = 0;   // one bit per device id < 31
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return QOQ_ERR_CUDA;
   const int bit = dev < 31 ? (1 << dev) : 0;
   if (!bit || !(__atomic_load_n(&configured_mask, __ATOMIC_ACQUIRE) & bit)) {
-    if (cudaFuncSetAttribute(w4a8_gemv_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(w4a8_gemv_kernel<MT, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kGemvMaxSmem)) != cudaSuccess)
       return QOQ_ERR_CUDA;
     if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_RELEASE);
@@ -211,23 +262,28 @@ int launch_mt(const GemvArgs& a, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, w4a8_gemv_kernel<MT>, a) != cudaSuccess) return QOQ_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, w4a8_gemv_kernel<MT, S>, a) != cudaSuccess) return QOQ_ERR_CUDA;
   return QOQ_OK;
+}
+
+template <int MT>
+int launch_stages(const GemvArgs& a, cudaStream_t s) {
+  return a.stages == 4 ? launch_mt<MT, 4>(a, s) : launch_mt<MT, 2>(a, s);
 }
 
 }  // namespace
 
-size_t gemv_smem_bytes(int M, int K) {
-  return ((static_cast<size_t>(M) * K + 15) & ~static_cast<size_t>(15)) +
+size_t gemv_smem_bytes(int M, int K, int stages) {
+  return ring_bytes(stages) + ((static_cast<size_t>(M) * K + 15) & ~static_cast<size_t>(15)) +
          static_cast<size_t>(kGemvWarps) * M * 32 * sizeof(int);
 }
 
 int launch_gemv(const GemvArgs& a, cudaStream_t s) {
   switch (a.M) {
-    case 1: return launch_mt<1>(a, s);
-    case 2: return launch_mt<2>(a, s);
-    case 3: return launch_mt<3>(a, s);
-    default: return launch_mt<4>(a, s);
+    case 1: return launch_stages<1>(a, s);
+    case 2: return launch_stages<2>(a, s);
+    case 3: return launch_stages<3>(a, s);
+    default: return launch_stages<4>(a, s);
   }
 }
 

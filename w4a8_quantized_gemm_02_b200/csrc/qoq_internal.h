@@ -57,12 +57,13 @@ struct GemvArgs {
   int32_t* acc;     // the INT32 accumulators (exactly one of the two)
   int M, N, K, group, blk_bytes, w_dep_wait;
   int ks, kt_per;           // K split into ks ranges of kt_per k-tiles
+  int stages;               // copy-ring slots per warp: 2 or 4
   uint32_t* ws_count;       // ks > 1: an arrival counter per 32 channels (zero between calls)
   int32_t* ws_acc;          // ks > 1: [split][M][N] INT32 partial sums
 };
 constexpr int kGemvMaxTokens = 4;
-constexpr size_t kGemvMaxSmem = 200 * 1024;
-size_t gemv_smem_bytes(int M, int K);
+constexpr size_t kGemvMaxSmem = 227 * 1024;   // the opt-in maximum per block on sm_100
+size_t gemv_smem_bytes(int M, int K, int stages);
 int launch_gemv(const GemvArgs& a, cudaStream_t s);
 
 // The GEMM launcher shared by the entry points.  The kernel may start while

@@ -47,6 +47,7 @@
 #include <type_traits>
 
 #include "qoq.h"
+#include "qoq_device.cuh"
 #include "qoq_internal.h"
 
 namespace qoq {
@@ -192,17 +193,6 @@ __device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
   uint32_t y;
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
   return y;
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // Codes enter the tensor cores as FP16 subnormals: the pairs masked from
