@@ -70,6 +70,15 @@ def test_plan_is_host_only(L):
         assert qoq.gemm_plan(M, 49152, 8192, 128)["tok_tile"] == 16
     # an explicit request (token tile 1) sizes its slices the same way
     assert qoq.gemm_workspace_bytes(3, 4096, 14336, 128, 1, 5) == 16384 + 5 * 3 * 4096 * 4
+    # the GEMV choice shrinks with the token count: if the plan takes it for
+    # M tokens it takes it for fewer; one token takes it whenever it fits
+    import synthetic_inputs as si
+    shapes = [(L.N, L.K, L.group) for L in si.LAYERS.values()] + [
+        (n, n, g) for n in si.SWEEP_KN for g in si.SWEEP_GROUPS]
+    for N, K, G in shapes:
+        gemv = [qoq.gemm_plan(M, N, K, G)["tok_tile"] == 0 for M in (1, 2, 3, 4)]
+        assert gemv[0]
+        assert all(a or not b for a, b in zip(gemv, gemv[1:]))
     for M in (5, 16, 17, 64, 100, 256, 1024, 4096):
         p = qoq.gemm_plan(M, 6144, 4096, 128)
         assert p["tok_tile"] in (16, 32, 64, 128, 176, 192, 256)
