@@ -381,7 +381,10 @@ def per_m_entry(M, N, K, G, t_us, peaks, int8_peak, plan, extra=None):
          "weight_gbs": weight_bytes(N, K, G) / t / 1e9,
          "hbm_frac": algo_bytes(M, N, K, G) / t / 1e9 / peaks["hbm_gbs"],
          "int8_frac": gemm_ops(M, N, K) / t / 1e12 / int8_peak,
-         "tok_tile": plan["tok_tile"], "splits": plan["splits"], "ctas": plan["ctas"]}
+         "tok_tile": plan["tok_tile"], "splits": plan["splits"], "ctas": plan["ctas"],
+         # tok_tile 0: the CUDA-core GEMV (stages = its copy-ring depth per warp);
+         # otherwise the tcgen05 GEMM (stages = its X ring depth)
+         "kernel": "gemv" if plan["tok_tile"] == 0 else "tcgen05", "stages": plan["stages"]}
     if extra:
         d.update(extra)
     return d
