@@ -16,11 +16,11 @@
 // 16-byte copies (per k-tile every lane copies its row's four code chunks,
 // the warp 512 contiguous bytes per chunk, and six lanes the group scales and
 // zero points), so S k-tiles per warp are in flight while one is multiplied.
-// S is 2, or 4 for long K ranges (measured on B200: the deeper ring holds more
-// bytes in flight, the shallower one more CTAs per SM).  The multiply turns four codes into four
-// INT8 weights per 32-bit multiply-add (the same byte-lane arithmetic as the
-// GEMM) and multiplies them with the tokens' INT8 codes four at a time (dp4a,
-// exact INT32).  The warps' sums are added in shared memory.  With ks > 1
+// S is 2, or 4 for long K ranges (measured on B200: the deeper ring holds
+// more bytes in flight, the shallower one more CTAs per SM).  The multiply
+// turns four codes into four INT8 weights per 32-bit multiply-add (the same
+// byte-lane arithmetic as the GEMM) and multiplies them with the tokens' INT8
+// codes four at a time (dp4a, exact INT32).  The warps' sums are added in shared memory.  With ks > 1
 // each CTA stores its INT32 partial sums in the workspace and counts its
 // arrival at its 32 channels (acquire-release at GPU scope); the last arrival
 // adds the ks slices.  Warp 0 of the CTA holding the whole sum applies
